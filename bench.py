@@ -1,0 +1,409 @@
+"""Benchmark of the Flash PD-SSM forward pass on B200 (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload lm]
+
+A step is one pdssm_forward call (selection + dictionary preparation + the
+whole chunked scan) over one batch of the LM-layer workload (batch 8, L 2048,
+heads 32, N = P = 64, K = 16; bf16 inputs, fp32 state, bf16 y). Under
+torchrun every rank runs its own batch (weak scaling; the batch shards need no
+collective), the timed region is bracketed by a barrier and a device
+synchronise on every rank, and the slowest rank's time is reported.
+
+Rank 0 prints one JSON line. ``--impl reference`` times the dense CPU oracle
+on the host cores on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "PD-SSM forward scan tokens·heads/s at LM shape; achieved HBM GB/s vs B200 peak"
+UNIT = "token·heads/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Largest value over all ranks (the slowest rank's time)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def shard_seed(rank: int) -> int:
+    """Each rank draws its own batch of the workload (independent problems)."""
+    return 1000 + rank
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {  # NVML clocks-event-reason bits
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.idx = device_index
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        self.error = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            # NVML enumerates physical devices; map through CUDA_VISIBLE_DEVICES
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            phys = self.idx
+            if vis:
+                ids = [v for v in vis.split(",") if v.strip()]
+                if self.idx < len(ids) and ids[self.idx].strip().isdigit():
+                    phys = int(ids[self.idx])
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(phys)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._nv = pynvml
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.error = repr(e)
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception as e:
+                self.error = repr(e)
+                return
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+        return False
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0, "error": self.error}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ peaks
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]), "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# ------------------------------------------------------------ workload
+
+def workload_config(sp: workloads.Spec, chunk: int, world: int):
+    return {
+        "workload": (f"{sp.recipe}: batch {sp.batch}, L {sp.seqlen}, heads {sp.heads}, N {sp.N}, P {sp.P}, "
+                     f"K {sp.K}; logits/d/B/C/x {str(sp.in_dtype).replace('torch.', '')}, "
+                     f"state {'complex64' if sp.state_complex else 'float32'}, "
+                     f"y {str(sp.out_dtype).replace('torch.', '')}"),
+        "batch_per_gpu": sp.batch, "seqlen": sp.seqlen, "heads": sp.heads, "N": sp.N, "P": sp.P,
+        "K": sp.K, "chunk": chunk,
+        "l2": "inputs larger than L2 (%.0f MB per step vs 126 MB) and an L2 flush between timed steps"
+              % (sp.token_heads * sp.algorithmic_bytes_per_token_head() / 1e6),
+        "parallelism": f"dp{world} (independent batch shards, no collective)",
+    }
+
+
+def cpu_baseline(sp: workloads.Spec, target_s: float = 12.0):
+    """The oracle as it stands, on the host cores, on whole (batch, head) slices of the workload."""
+    import oracle
+    cores = oracle.threads()
+    idx = workloads.generate_idx(sp)
+    picks = []
+    total = 0.0
+    n = max(1, cores)
+    # one calibration slice, then enough slices for ~target_s of work
+    sl = [workloads.generate_slice(sp, 0, 0)]
+    t0 = time.perf_counter()
+    oracle.scan_slices(sl[0]["logits"][None], idx, sl[0]["d"][None], sl[0]["B"][None], sl[0]["C"][None],
+                       sl[0]["x"][None], want_prod=False)
+    one = time.perf_counter() - t0
+    n = int(max(1, min(sp.batch * sp.heads, round(target_s / max(one, 1e-3) * cores))))
+    n = max(1, (n // cores) * cores) if n >= cores else n
+    for i in range(n):
+        picks.append((i // sp.heads % sp.batch, i % sp.heads))
+    sls = [workloads.generate_slice(sp, b, h) for b, h in picks]
+    stack = {k: torch.stack([s[k] for s in sls]) for k in sls[0]}
+    t0 = time.perf_counter()
+    oracle.scan_slices(stack["logits"], idx, stack["d"], stack["B"], stack["C"], stack["x"], want_prod=False)
+    total = time.perf_counter() - t0
+    units = n * sp.seqlen
+    return {"value": units / total, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} whole (batch, head) slices x L={sp.seqlen} of the {sp.recipe} workload "
+                      f"({units} token-heads), dense fp64 oracle, {total:.1f} s wall"}
+
+
+# ------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local):
+    import structured_sparse_selective_b200 as pd
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    sp = workloads.spec(args.workload)
+    inp = workloads.generate(sp, seed=shard_seed(rank), device=device)
+    pb = pd.make_problem(inp["logits"], inp["d"], inp["B"], inp["x"], chunk=args.chunk)
+    Bt, L, H, N = inp["B"].shape
+    P = inp["x"].shape[-1]
+    sdt = torch.float32 if not sp.state_complex else torch.complex64
+    out = {
+        "y": torch.empty(Bt, L, H, P, dtype=sp.out_dtype, device=device),
+        "h_final": torch.empty(Bt, H, N, P, dtype=sdt, device=device),
+        "prod_idx": torch.empty(Bt, H, N, dtype=torch.int32, device=device),
+        "prod_val": torch.empty(Bt, H, N, dtype=sdt, device=device),
+    }
+    ws = pd.alloc_workspace(pb, device)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        pd.pdssm_forward(pb, inp["logits"], inp["idx"], inp["d"], inp["B"], inp["C"], inp["x"], None,
+                         out["y"], out["h_final"], out["prod_idx"], out["prod_val"], None, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+
+    # ---- headline: K device-timed steps, L2 flushed between steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    traces = [pd.KernelTrace(max_launches=16) for _ in range(args.steps)]
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            with traces[i]:
+                step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(device)
+    barrier(world, device)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms_local = sum(step_ms) / len(step_ms)
+    ms = max_over_ranks(ms_local, world, device)
+    per_kernel = {}
+    launches = 0
+    for tr in traces:
+        for name, t in tr.timings():
+            per_kernel.setdefault(name, []).append(t)
+            launches += 1
+    totals = {k: sum(v) for k, v in per_kernel.items()}
+    dominant = max(totals, key=totals.get)
+    dom_ms = sum(per_kernel[dominant]) / len(per_kernel[dominant])
+    units = sp.token_heads
+    value = units * world / (ms / 1e3)
+
+    # ---- algorithmic bytes of the dominant kernel (per launch)
+    with_logits = sp.K * torch.empty((), dtype=sp.logits_dtype).element_size()
+    bytes_fwd = units * sp.algorithmic_bytes_per_token_head(with_logits=True)
+    alg_bytes = {
+        "fused_forward": bytes_fwd,
+        # phase A reads s, d, B, C and x of every token-head (its y_loc and
+        # chunk-state writes are workspace traffic, not algorithmic)
+        "chunked_phase_a": units * (4 + sp.algorithmic_bytes_per_token_head(with_logits=False) - 4
+                                    - sp.P * torch.empty((), dtype=sp.out_dtype).element_size()),
+        "chunked_phase_c": units * (4 + sp.N * (torch.empty((), dtype=sp.d_dtype).element_size()
+                                                + torch.empty((), dtype=sp.in_dtype).element_size())
+                                    + sp.P * torch.empty((), dtype=sp.out_dtype).element_size()),
+        "select": units * (with_logits + 4),
+    }.get(dominant)
+    peaks = load_peaks()
+    roofline = None
+    if alg_bytes is not None:
+        achieved = alg_bytes / (dom_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1),
+                    "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
+                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                    "algorithmic_bytes_per_launch": int(alg_bytes), "launch_ms": round(dom_ms, 4)}
+
+    # ---- end to end through the public API with host buffers
+    host_in = {k: v.cpu().pin_memory() for k, v in inp.items()}
+    host_y = torch.empty_like(out["y"], device="cpu").pin_memory()
+    host_h = torch.empty_like(out["h_final"], device="cpu").pin_memory()
+    dev_in = {k: torch.empty_like(v) for k, v in inp.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = host_y.numel() * host_y.element_size() + host_h.numel() * host_h.element_size()
+
+    def e2e_step():
+        for k in dev_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        pd.pdssm_forward(pb, dev_in["logits"], dev_in["idx"], dev_in["d"], dev_in["B"], dev_in["C"],
+                         dev_in["x"], None, out["y"], out["h_final"], out["prod_idx"], out["prod_val"],
+                         None, ws, stream)
+        host_y.copy_(out["y"], non_blocking=True)
+        host_h.copy_(out["h_final"], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    e_s = torch.cuda.Event(enable_timing=True)
+    e_e = torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    e_s.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_e.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / args.steps, world, device)
+
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(sp, args.chunk, world),
+            "roofline": roofline,
+            "kernels_ms_per_step": {k: round(sum(v) / args.steps, 5) for k, v in per_kernel.items()},
+            "e2e": {"value": round(units * world / (e2e_ms / 1e3), 1), "unit": UNIT,
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+        }
+    return result
+
+
+# ------------------------------------------------------------ reference arm
+
+def run_reference(args, rank, world):
+    """The dense CPU oracle on the host cores; each step a bounded slice sample."""
+    if rank != 0:
+        return None
+    import oracle
+    sp = workloads.spec(args.workload)
+    cores = oracle.threads()
+    idx = workloads.generate_idx(sp)
+    n = max(1, cores)
+    picks = [(i // sp.heads % sp.batch, i % sp.heads) for i in range(n)]
+    sls = [workloads.generate_slice(sp, b, h) for b, h in picks]
+    stack = {k: torch.stack([s[k] for s in sls]) for k in sls[0]}
+
+    def step():
+        oracle.scan_slices(stack["logits"], idx, stack["d"], stack["B"], stack["C"], stack["x"], want_prod=False)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    sec = (time.perf_counter() - t0) / args.steps
+    units = n * sp.seqlen
+    value = units / sec
+    sample = (f"each step: {n} whole (batch, head) slices x L={sp.seqlen} of the {sp.recipe} workload "
+              f"({units} token-heads), dense fp64 oracle")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(sp, args.chunk, world),
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="lm", choices=list(workloads.RECIPES))
+    ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    init_dist(world, "nccl")
+    try:
+        res = run_ours(args, rank, world, local)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(workloads.spec(args.workload))
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

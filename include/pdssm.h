@@ -1,0 +1,194 @@
+/*
+ * pdssm.h -- C ABI of libpdssm.so, the B200 (sm_100a) forward pass of Flash PD-SSM.
+ *
+ * Method: "Flash PD-SSM: Memory-Optimized Structured Sparse State-Space Models"
+ * (gist.science explainer of arXiv 2605.19150), Technical Summary:
+ *   - Methodology 1 ("Novel Selection Mechanism"): the input gives K scores; the
+ *     single highest-scoring matrix of a dictionary of K sparse matrices is
+ *     used directly. Each is a one-hot column selector, so memory is O(L*N),
+ *     not the O(L*N^2) of the original PD-SSM.
+ *   - Methodology 2: the forward pass uses hard argmax.
+ *   - Methodology 3 ("Hardware-Aware Implementation"): a three-phase chunked
+ *     scan -- A: independent sequential recurrences inside chunks; B: a prefix
+ *     scan over the chunks' dependencies gives the carry states; C: the carry
+ *     corrections are applied.
+ * The page prints no formula. This library computes the PD (one-hot-column
+ * matrix times diagonal) recurrence those passages describe:
+ *     s_t = argmax_k logits_t[k]          (lowest k on ties, first NaN wins)
+ *     H_t = P_{s_t} diag(d_t) H_{t-1} + B_t x_t^T,   H_{-1} = h0 (or 0)
+ *     y_t = H_t^T C_t                     (plain transpose, also for complex H)
+ * where P_k[idx[k][j]][j] = 1 is the only nonzero of column j. Chunks are
+ * combined with the associative composition of (index, value) pairs
+ *     (idx, val) o (idx', val') = (idx[idx'], val[idx'] * val')
+ * which is the pair of the matrix product A * A' (A' applied first); the
+ * prefix-scan framing follows the abstract of "Sequential-Parallel Duality in
+ * Prefix Scannable Models" (state updates by a parallel prefix scan with a
+ * custom associative operator). No N x N matrix is ever formed.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Ownership: the caller allocates every buffer, inputs, outputs and the
+ *   workspace, in device memory of the device that owns `stream`. The library
+ *   never allocates, frees or synchronises (pdssm_read_device_check and the
+ *   PDSSM_FLAG_DEVICE_CHECK flag are the documented exceptions: they
+ *   synchronise the stream).
+ * Streams: every call only enqueues work on `stream` and returns. A NULL
+ *   stream is the legacy default stream of the calling thread's current
+ *   device. Outputs are valid once the stream has reached the call.
+ * Layouts (row-major, contiguous, element-aligned):
+ *   logits [batch][seqlen][heads][K]          s    [batch][seqlen][heads] int32
+ *   idx    [K][N] int32, shared by all heads  (idx[k][j] = row of the nonzero
+ *                                              of column j of P_k, in [0, N))
+ *   d, B, C [batch][seqlen][heads][N]         x, y [batch][seqlen][heads][P]
+ *   h0, h_final [batch][heads][N][P]          prod_idx, prod_val [batch][heads][N]
+ *   Complex values (PDSSM_C64) are interleaved (re, im) float pairs, the
+ *   layout of torch.complex64 / std::complex<float>.
+ * Errors: argument errors are reported before anything is enqueued; a
+ *   non-PDSSM_OK return means nothing was launched. Launch failures return
+ *   PDSSM_ERR_CUDA. Index values that the host cannot see (idx entries outside
+ *   [0, N), s entries outside [0, K)) never cause an out-of-bounds access: the
+ *   kernels substitute 0, set a bit in the workspace's error word and carry
+ *   on; pdssm_read_device_check reports it.
+ */
+#ifndef PDSSM_H_
+#define PDSSM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+struct CUstream_st;
+typedef struct CUstream_st *pdssm_stream_t;
+
+typedef enum {
+  PDSSM_OK = 0,
+  PDSSM_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misalignment */
+  PDSSM_ERR_UNSUPPORTED = 2,  /* N, P or K above the limits, dtype combination */
+  PDSSM_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+  PDSSM_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+  PDSSM_ERR_DEVICE_CHECK = 5, /* a kernel met an out-of-range idx or s */
+  PDSSM_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up */
+} pdssm_status;
+
+typedef enum { PDSSM_F32 = 0, PDSSM_BF16 = 1, PDSSM_C64 = 2 } pdssm_dtype;
+
+#define PDSSM_MAX_N 128
+#define PDSSM_MAX_P 128
+#define PDSSM_MAX_K 64
+
+/* flags */
+#define PDSSM_FLAG_DEVICE_CHECK 1u   /* synchronise and return PDSSM_ERR_DEVICE_CHECK on bad idx/s */
+#define PDSSM_FLAG_REFERENCE_PATH 2u /* use the plain three-kernel chunked path (no fused kernel) */
+
+/*
+ * Problem description. Supported dtype combinations:
+ *   real state:    state_t = F32; d_t in {F32, BF16}; in_t (B, C, x) in {F32, BF16};
+ *                  out_t (y) in {F32, BF16}; logits_t in {F32, BF16};
+ *                  h0 / h_final / prod_val are F32.
+ *   complex state: state_t = C64; d_t = C64; in_t in {F32, BF16}; out_t = C64;
+ *                  logits_t in {F32, BF16}; h0 / h_final / prod_val are C64.
+ * Sizes: batch, seqlen, heads >= 0 (zero is an empty problem);
+ *        1 <= N <= PDSSM_MAX_N, 1 <= P <= PDSSM_MAX_P, 1 <= K <= PDSSM_MAX_K.
+ * chunk: the chunk length T of the three-phase scan; 0 picks a default. The
+ *        results do not depend on T beyond floating-point rounding.
+ */
+typedef struct {
+  int64_t batch, seqlen, heads, N, P, K;
+  int32_t chunk;
+  int32_t logits_t, in_t, d_t, state_t, out_t; /* pdssm_dtype values */
+  uint32_t flags;
+} pdssm_problem;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *pdssm_status_string(int32_t status);
+
+/* Library version as "major.minor.patch" (static string). */
+const char *pdssm_version(void);
+
+/*
+ * Workspace bytes that pdssm_scan_fwd / pdssm_forward need for `pb`
+ * (written to *bytes). The size grows as O(batch*heads*seqlen*(N+P)) -- the
+ * O(L*N) memory of Methodology 1 -- and never with N*N.
+ * Errors: PDSSM_ERR_INVALID_ARG / PDSSM_ERR_UNSUPPORTED as for the calls.
+ */
+pdssm_status pdssm_workspace_size(const pdssm_problem *pb, size_t *bytes);
+
+/*
+ * Hard selection, Methodology 1 and 2: s[b][t][h] = the lowest k with
+ * logits[b][t][h][k] == max_k' logits[b][t][h][k']. +0 and -0 compare equal;
+ * a NaN counts as the maximum and the first NaN wins. Bit-exact.
+ * logits: device, logits_t; s: device int32 output. No workspace.
+ */
+pdssm_status pdssm_select(const pdssm_problem *pb, const void *logits, int32_t *s,
+                          pdssm_stream_t stream);
+
+/*
+ * The PD scan (Methodology 3) for given selections s.
+ *   s        device int32 [batch][seqlen][heads], each in [0, K)
+ *   idx      device int32 [K][N]
+ *   d        device d_t    [batch][seqlen][heads][N]
+ *   B, C     device in_t   [batch][seqlen][heads][N]
+ *   x        device in_t   [batch][seqlen][heads][P]
+ *   h0       device state  [batch][heads][N][P], or NULL for a zero state
+ *   y        device out_t  [batch][seqlen][heads][P]            (output)
+ *   h_final  device state  [batch][heads][N][P], or NULL         (output)
+ *   prod_idx device int32  [batch][heads][N], or NULL            (output)
+ *   prod_val device state  [batch][heads][N], or NULL            (output)
+ *            (prod_idx, prod_val) is the pair of P_{s_{L-1}} diag(d_{L-1}) ...
+ *            P_{s_0} diag(d_0): column j has its only nonzero, prod_val[j], at
+ *            row prod_idx[j]. prod_idx is exact; prod_val may underflow to 0.
+ *   workspace device, >= pdssm_workspace_size bytes, 16-byte aligned. Its
+ *            contents are scratch, except the error word that
+ *            pdssm_read_device_check reads after the call.
+ * The output buffers must not overlap the inputs or each other.
+ */
+pdssm_status pdssm_scan_fwd(const pdssm_problem *pb, const int32_t *s, const int32_t *idx,
+                            const void *d, const void *B, const void *C, const void *x,
+                            const void *h0, void *y, void *h_final, int32_t *prod_idx,
+                            void *prod_val, void *workspace, size_t workspace_bytes,
+                            pdssm_stream_t stream);
+
+/*
+ * Selection and scan in one call: pdssm_select followed by pdssm_scan_fwd,
+ * with the selection fused into the scan's input read where the fused path
+ * applies. `logits` replaces `s`; `s_out` (device int32
+ * [batch][seqlen][heads], or NULL) receives the selections.
+ */
+pdssm_status pdssm_forward(const pdssm_problem *pb, const void *logits, const int32_t *idx,
+                           const void *d, const void *B, const void *C, const void *x,
+                           const void *h0, void *y, void *h_final, int32_t *prod_idx,
+                           void *prod_val, int32_t *s_out, void *workspace,
+                           size_t workspace_bytes, pdssm_stream_t stream);
+
+/*
+ * Synchronises `stream` and reads the error word that the last pdssm_scan_fwd
+ * or pdssm_forward call on `workspace` left: PDSSM_OK, PDSSM_ERR_DEVICE_CHECK
+ * (an idx or s value was out of range) or PDSSM_ERR_TIMEOUT.
+ */
+pdssm_status pdssm_read_device_check(const void *workspace, pdssm_stream_t stream);
+
+/*
+ * Kernel tracing (observability; the pages describe none).
+ * Between pdssm_trace_begin and pdssm_trace_end, every kernel the calling
+ * thread's pdssm_* calls enqueue is bracketed by cudaEventRecord of
+ * events[2*i] (before) and events[2*i+1] (after) on the launch stream, for
+ * the first n_events/2 launches. `events` holds cudaEvent_t handles the caller
+ * created (with timing enabled) and keeps alive until it has read them; the
+ * library only records them.
+ * pdssm_trace_end returns the number of launches recorded and stops tracing;
+ * pdssm_trace_kernel_name(i) names launch i of the last trace (static
+ * string, or NULL when i is out of range).
+ */
+pdssm_status pdssm_trace_begin(void *const *events, int32_t n_events);
+int32_t pdssm_trace_end(void);
+const char *pdssm_trace_kernel_name(int32_t i);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PDSSM_H_ */

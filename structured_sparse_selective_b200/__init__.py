@@ -1,0 +1,247 @@
+"""Python binding of libpdssm.so, the B200 forward pass of Flash PD-SSM.
+
+Argument marshalling only: every step of the forward pass runs in the CUDA
+kernels behind the C ABI declared in ``include/pdssm.h``. PyTorch supplies
+device memory and the current stream. There is no CPU fallback: if the
+library is missing, importing this package raises.
+
+The functions keep the C names:
+
+    pdssm_workspace_size(problem) -> int
+    pdssm_select(problem, logits, s, stream=None)
+    pdssm_scan_fwd(problem, s, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val, workspace, stream=None)
+    pdssm_forward(problem, logits, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val, s_out, workspace, stream=None)
+    pdssm_read_device_check(workspace, stream=None)
+
+``forward(...)`` is a convenience wrapper that allocates the outputs and the
+workspace with torch and calls ``pdssm_forward``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+__all__ = [
+    "PdssmError", "Problem", "F32", "BF16", "C64", "FLAG_DEVICE_CHECK", "FLAG_REFERENCE_PATH",
+    "library_path", "make_problem", "pdssm_workspace_size", "pdssm_select", "pdssm_scan_fwd",
+    "pdssm_forward", "pdssm_read_device_check", "pdssm_status_string", "forward", "EXPORTED_SYMBOLS",
+    "KernelTrace", "alloc_workspace",
+]
+
+F32, BF16, C64 = 0, 1, 2
+FLAG_DEVICE_CHECK = 1
+FLAG_REFERENCE_PATH = 2
+MAX_N, MAX_P, MAX_K = 128, 128, 64
+
+EXPORTED_SYMBOLS = (
+    "pdssm_status_string", "pdssm_version", "pdssm_workspace_size", "pdssm_select",
+    "pdssm_scan_fwd", "pdssm_forward", "pdssm_read_device_check", "pdssm_trace_begin",
+    "pdssm_trace_end", "pdssm_trace_kernel_name",
+)
+
+_DIR = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_DIR, "libpdssm.so")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+class Problem(ctypes.Structure):
+    """Mirror of ``pdssm_problem``."""
+
+    _fields_ = [
+        ("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("heads", ctypes.c_int64),
+        ("N", ctypes.c_int64), ("P", ctypes.c_int64), ("K", ctypes.c_int64),
+        ("chunk", ctypes.c_int32), ("logits_t", ctypes.c_int32), ("in_t", ctypes.c_int32),
+        ("d_t", ctypes.c_int32), ("state_t", ctypes.c_int32), ("out_t", ctypes.c_int32),
+        ("flags", ctypes.c_uint32),
+    ]
+
+
+class PdssmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {pdssm_status_string(status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is missing; build it with `python structured_sparse_selective_b200/build.py`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32p, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t
+    pb = ctypes.POINTER(Problem)
+    lib.pdssm_status_string.argtypes = [ctypes.c_int32]
+    lib.pdssm_status_string.restype = ctypes.c_char_p
+    lib.pdssm_version.restype = ctypes.c_char_p
+    lib.pdssm_workspace_size.argtypes = [pb, ctypes.POINTER(sz)]
+    lib.pdssm_workspace_size.restype = ctypes.c_int
+    lib.pdssm_select.argtypes = [pb, vp, i32p, vp]
+    lib.pdssm_select.restype = ctypes.c_int
+    lib.pdssm_scan_fwd.argtypes = [pb, i32p, i32p, vp, vp, vp, vp, vp, vp, vp, i32p, vp, vp, sz, vp]
+    lib.pdssm_scan_fwd.restype = ctypes.c_int
+    lib.pdssm_forward.argtypes = [pb, vp, i32p, vp, vp, vp, vp, vp, vp, vp, i32p, vp, i32p, vp, sz, vp]
+    lib.pdssm_forward.restype = ctypes.c_int
+    lib.pdssm_read_device_check.argtypes = [vp, vp]
+    lib.pdssm_read_device_check.restype = ctypes.c_int
+    lib.pdssm_trace_begin.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
+    lib.pdssm_trace_begin.restype = ctypes.c_int
+    lib.pdssm_trace_end.argtypes = []
+    lib.pdssm_trace_end.restype = ctypes.c_int32
+    lib.pdssm_trace_kernel_name.argtypes = [ctypes.c_int32]
+    lib.pdssm_trace_kernel_name.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+_DT = {torch.float32: F32, torch.bfloat16: BF16, torch.complex64: C64}
+
+
+def pdssm_status_string(status: int) -> str:
+    return _lib.pdssm_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return _lib.pdssm_version().decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise PdssmError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor], device: Optional[torch.device] = None):
+    """Device address of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError("libpdssm takes device memory only; got a CPU tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"tensor on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr()) if t.numel() > 0 else ctypes.c_void_p(t.data_ptr() or 0)
+
+
+def _stream(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    return ctypes.c_void_p(handle)
+
+
+def make_problem(logits: torch.Tensor, d: torch.Tensor, B: torch.Tensor, x: torch.Tensor,
+                 out_dtype: Optional[torch.dtype] = None, chunk: int = 0, flags: int = 0,
+                 K: Optional[int] = None) -> Problem:
+    """Problem description from tensor shapes and dtypes (logits may be None if K is given)."""
+    Bt, L, H, N = B.shape
+    P = x.shape[-1]
+    cplx = d.dtype == torch.complex64
+    if out_dtype is None:
+        out_dtype = torch.complex64 if cplx else B.dtype
+    return Problem(
+        batch=Bt, seqlen=L, heads=H, N=N, P=P, K=(logits.shape[-1] if logits is not None else K),
+        chunk=chunk, logits_t=_DT[logits.dtype] if logits is not None else F32, in_t=_DT[B.dtype],
+        d_t=_DT[d.dtype], state_t=C64 if cplx else F32, out_t=_DT[out_dtype], flags=flags)
+
+
+def pdssm_workspace_size(pb: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.pdssm_workspace_size(ctypes.byref(pb), ctypes.byref(n)), "pdssm_workspace_size")
+    return int(n.value)
+
+
+def pdssm_select(pb: Problem, logits: torch.Tensor, s: torch.Tensor, stream=None) -> None:
+    dev = logits.device
+    _check(_lib.pdssm_select(ctypes.byref(pb), _ptr(logits, dev), _ptr(s, dev), _stream(stream, dev)),
+           "pdssm_select")
+
+
+def pdssm_scan_fwd(pb: Problem, s, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val, workspace,
+                   stream=None) -> None:
+    dev = idx.device
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pdssm_scan_fwd(
+        ctypes.byref(pb), _ptr(s, dev), _ptr(idx, dev), _ptr(d, dev), _ptr(B, dev), _ptr(C, dev),
+        _ptr(x, dev), _ptr(h0, dev), _ptr(y, dev), _ptr(h_final, dev), _ptr(prod_idx, dev),
+        _ptr(prod_val, dev), _ptr(workspace, dev), ws_bytes, _stream(stream, dev)), "pdssm_scan_fwd")
+
+
+def pdssm_forward(pb: Problem, logits, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val, s_out,
+                  workspace, stream=None) -> None:
+    dev = idx.device
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pdssm_forward(
+        ctypes.byref(pb), _ptr(logits, dev), _ptr(idx, dev), _ptr(d, dev), _ptr(B, dev), _ptr(C, dev),
+        _ptr(x, dev), _ptr(h0, dev), _ptr(y, dev), _ptr(h_final, dev), _ptr(prod_idx, dev),
+        _ptr(prod_val, dev), _ptr(s_out, dev), _ptr(workspace, dev), ws_bytes, _stream(stream, dev)),
+        "pdssm_forward")
+
+
+def pdssm_read_device_check(workspace: torch.Tensor, stream=None) -> int:
+    """Status left in the workspace's error word by the last scan (synchronises)."""
+    return int(_lib.pdssm_read_device_check(_ptr(workspace), _stream(stream, workspace.device)))
+
+
+class KernelTrace:
+    """Times each kernel the library launches inside a ``with`` block (CUDA events).
+
+        with KernelTrace(max_launches=16) as tr:
+            pdssm_forward(...)
+        torch.cuda.synchronize(); tr.timings() -> [(kernel_name, ms), ...]
+    """
+
+    def __init__(self, max_launches: int = 16):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * max_launches)]
+        self._arr = (ctypes.c_void_p * len(self.events))(*[ctypes.c_void_p(e.cuda_event) for e in self.events])
+        self.names = []
+
+    def __enter__(self):
+        _check(_lib.pdssm_trace_begin(self._arr, len(self.events)), "pdssm_trace_begin")
+        return self
+
+    def __exit__(self, *exc):
+        n = int(_lib.pdssm_trace_end())
+        self.names = [_lib.pdssm_trace_kernel_name(i).decode() for i in range(n)]
+        return False
+
+    def timings(self):
+        return [(nm, self.events[2 * i].elapsed_time(self.events[2 * i + 1])) for i, nm in enumerate(self.names)]
+
+
+def alloc_workspace(pb: Problem, device) -> torch.Tensor:
+    return torch.empty(max(1, pdssm_workspace_size(pb)), dtype=torch.uint8, device=device)
+
+
+def forward(logits: torch.Tensor, idx: torch.Tensor, d: torch.Tensor, B: torch.Tensor,
+            C: torch.Tensor, x: torch.Tensor, h0: Optional[torch.Tensor] = None,
+            out_dtype: Optional[torch.dtype] = None, chunk: int = 0, flags: int = 0,
+            want_prod: bool = True, want_s: bool = False, workspace: Optional[torch.Tensor] = None,
+            stream=None) -> Dict[str, torch.Tensor]:
+    """Allocates the outputs (torch) and runs ``pdssm_forward`` on the inputs' device."""
+    pb = make_problem(logits, d, B, x, out_dtype=out_dtype, chunk=chunk, flags=flags)
+    dev = B.device
+    Bt, L, H, N = B.shape
+    P = x.shape[-1]
+    sdt = torch.complex64 if pb.state_t == C64 else torch.float32
+    ydt = {F32: torch.float32, BF16: torch.bfloat16, C64: torch.complex64}[pb.out_t]
+    out = {
+        "y": torch.empty(Bt, L, H, P, dtype=ydt, device=dev),
+        "h_final": torch.empty(Bt, H, N, P, dtype=sdt, device=dev),
+    }
+    if want_prod:
+        out["prod_idx"] = torch.empty(Bt, H, N, dtype=torch.int32, device=dev)
+        out["prod_val"] = torch.empty(Bt, H, N, dtype=sdt, device=dev)
+    if want_s:
+        out["s"] = torch.empty(Bt, L, H, dtype=torch.int32, device=dev)
+    ws = workspace if workspace is not None else alloc_workspace(pb, dev)
+    pdssm_forward(pb, logits, idx, d, B, C, x, h0, out["y"], out["h_final"], out.get("prod_idx"),
+                  out.get("prod_val"), out.get("s"), ws, stream)
+    return out

@@ -1,0 +1,320 @@
+// C-ABI entry points of libpdssm.so: argument validation, workspace layout,
+// device binding and dispatch. See include/pdssm.h for the contract.
+#include <string.h>
+
+#include <algorithm>
+
+#include "launch.h"
+#include "pdssm.h"
+
+using namespace pdssm;
+
+namespace {
+
+size_t dtype_size(int dt) {
+  switch (dt) {
+    case PDSSM_F32: return 4;
+    case PDSSM_BF16: return 2;
+    case PDSSM_C64: return 8;
+    default: return 0;
+  }
+}
+
+bool mul_ok(int64_t a, int64_t b, int64_t *out) { return !__builtin_mul_overflow(a, b, out); }
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct Plan {
+  int64_t Bt, L, H, N, P, K, T, nC, rows;
+  bool cplx;
+  size_t state_size;  // bytes per state element (4 or 8)
+  // workspace offsets
+  size_t o_err, o_idx, o_off, o_src, o_s, o_cstate, o_cidx, o_cval, o_yloc, total;
+};
+
+int64_t default_chunk(const pdssm_problem *pb) {
+  // Long enough that chunk-end states stay O(L*N) (T >= P), short enough
+  // that every SM gets several (batch, head, chunk) blocks.
+  return std::max<int64_t>(64, pb->P);
+}
+
+pdssm_status make_plan(const pdssm_problem *pb, Plan *pl) {
+  if (!pb) return PDSSM_ERR_INVALID_ARG;
+  if (pb->batch < 0 || pb->seqlen < 0 || pb->heads < 0 || pb->N < 1 || pb->P < 1 || pb->K < 1 ||
+      pb->chunk < 0)
+    return PDSSM_ERR_INVALID_ARG;
+  if (pb->N > PDSSM_MAX_N || pb->P > PDSSM_MAX_P || pb->K > PDSSM_MAX_K) return PDSSM_ERR_UNSUPPORTED;
+  if (pb->batch > 65535 || pb->heads > 65535) return PDSSM_ERR_UNSUPPORTED;
+  if (pb->logits_t != PDSSM_F32 && pb->logits_t != PDSSM_BF16) return PDSSM_ERR_UNSUPPORTED;
+  if (pb->in_t != PDSSM_F32 && pb->in_t != PDSSM_BF16) return PDSSM_ERR_UNSUPPORTED;
+  if (pb->state_t == PDSSM_F32) {
+    if (pb->d_t != PDSSM_F32 && pb->d_t != PDSSM_BF16) return PDSSM_ERR_UNSUPPORTED;
+    if (pb->out_t != PDSSM_F32 && pb->out_t != PDSSM_BF16) return PDSSM_ERR_UNSUPPORTED;
+  } else if (pb->state_t == PDSSM_C64) {
+    if (pb->d_t != PDSSM_C64 || pb->out_t != PDSSM_C64) return PDSSM_ERR_UNSUPPORTED;
+  } else {
+    return PDSSM_ERR_UNSUPPORTED;
+  }
+  if (pb->flags & ~(PDSSM_FLAG_DEVICE_CHECK | PDSSM_FLAG_REFERENCE_PATH)) return PDSSM_ERR_INVALID_ARG;
+
+  Plan p;
+  p.Bt = pb->batch; p.L = pb->seqlen; p.H = pb->heads; p.N = pb->N; p.P = pb->P; p.K = pb->K;
+  p.cplx = pb->state_t == PDSSM_C64;
+  p.state_size = p.cplx ? 8 : 4;
+  p.T = pb->chunk ? pb->chunk : default_chunk(pb);
+  p.nC = p.L > 0 ? (p.L + p.T - 1) / p.T : 0;
+  int64_t bh, rows, tmp;
+  if (!mul_ok(p.Bt, p.H, &bh) || !mul_ok(bh, p.L, &rows)) return PDSSM_ERR_UNSUPPORTED;
+  if (!mul_ok(rows, std::max(std::max(p.N, p.P), p.K) * 8, &tmp)) return PDSSM_ERR_UNSUPPORTED;
+  if (p.nC > INT32_MAX) return PDSSM_ERR_UNSUPPORTED;
+  p.rows = rows;
+  int64_t nchunks = bh * p.nC;
+  size_t o = 0;
+  p.o_err = o; o = align256(o + 4);
+  p.o_idx = o; o = align256(o + (size_t)(p.K * p.N) * 4);
+  p.o_off = o; o = align256(o + (size_t)(p.K * (p.N + 1)) * 4);
+  p.o_src = o; o = align256(o + (size_t)(p.K * p.N) * 4);
+  p.o_s = o; o = align256(o + (size_t)rows * 4);
+  p.o_cstate = o; o = align256(o + (size_t)nchunks * p.N * p.P * p.state_size);
+  p.o_cidx = o; o = align256(o + (size_t)nchunks * p.N * 4);
+  p.o_cval = o; o = align256(o + (size_t)nchunks * p.N * p.state_size);
+  p.o_yloc = o; o = align256(o + (size_t)rows * p.P * p.state_size);
+  p.total = o;
+  *pl = p;
+  return PDSSM_OK;
+}
+
+Workspace carve(const Plan &p, void *ws) {
+  char *base = static_cast<char *>(ws);
+  Workspace w;
+  w.err = reinterpret_cast<uint32_t *>(base + p.o_err);
+  w.idx = reinterpret_cast<int32_t *>(base + p.o_idx);
+  w.csr_off = reinterpret_cast<int32_t *>(base + p.o_off);
+  w.csr_src = reinterpret_cast<int32_t *>(base + p.o_src);
+  w.s = reinterpret_cast<int32_t *>(base + p.o_s);
+  w.chunk_state = base + p.o_cstate;
+  w.chunk_idx = reinterpret_cast<int32_t *>(base + p.o_cidx);
+  w.chunk_val = base + p.o_cval;
+  w.y_loc = base + p.o_yloc;
+  return w;
+}
+
+bool aligned(const void *ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+// Makes the device that owns `stream` current for this library's runtime.
+pdssm_status bind_device(cudaStream_t stream) {
+  if (stream == nullptr) return PDSSM_OK;
+  int dev = -1;
+  if (cudaStreamGetDevice(stream, &dev) != cudaSuccess) return PDSSM_ERR_CUDA;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return PDSSM_ERR_CUDA;
+  if (cur != dev && cudaSetDevice(dev) != cudaSuccess) return PDSSM_ERR_CUDA;
+  return PDSSM_OK;
+}
+
+pdssm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PDSSM_OK : PDSSM_ERR_CUDA; }
+
+pdssm_status check_scan_args(const pdssm_problem *pb, const Plan &p, const int32_t *idx,
+                             const void *d, const void *B, const void *C, const void *x,
+                             const void *h0, const void *y, const void *h_final,
+                             const int32_t *prod_idx, const void *prod_val, const void *ws,
+                             size_t ws_bytes) {
+  if (!idx) return PDSSM_ERR_INVALID_ARG;
+  if (p.rows > 0 && (!d || !B || !C || !x || !y)) return PDSSM_ERR_INVALID_ARG;
+  const size_t es_in = dtype_size(pb->in_t), es_d = dtype_size(pb->d_t), es_o = dtype_size(pb->out_t);
+  if (!aligned(idx, 4) || !aligned(d, es_d) || !aligned(B, es_in) || !aligned(C, es_in) ||
+      !aligned(x, es_in) || !aligned(y, es_o) || !aligned(h0, p.state_size) ||
+      !aligned(h_final, p.state_size) || !aligned(prod_idx, 4) || !aligned(prod_val, p.state_size))
+    return PDSSM_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < p.total) return PDSSM_ERR_WORKSPACE;
+  if (!aligned(ws, 16)) return PDSSM_ERR_INVALID_ARG;
+  return PDSSM_OK;
+}
+
+pdssm_status finish(const pdssm_problem *pb, const Workspace &w, cudaStream_t stream) {
+  if (cudaGetLastError() != cudaSuccess) return PDSSM_ERR_CUDA;
+  if (pb->flags & PDSSM_FLAG_DEVICE_CHECK) return pdssm_read_device_check(w.err, stream);
+  return PDSSM_OK;
+}
+
+pdssm_status run_scan(const pdssm_problem *pb, const Plan &p, const int32_t *s,
+                      const void *logits, int32_t *s_out, const int32_t *idx, const void *d,
+                      const void *B, const void *C, const void *x, const void *h0, void *y,
+                      void *h_final, int32_t *prod_idx, void *prod_val, void *workspace,
+                      cudaStream_t stream) {
+  Workspace w = carve(p, workspace);
+  if (cudaMemsetAsync(w.err, 0, 4, stream) != cudaSuccess) return PDSSM_ERR_CUDA;
+  pdssm_status st = cuda_status(launch_prep_dict(idx, (int)p.K, (int)p.N, w, stream));
+  if (st != PDSSM_OK) return st;
+
+  ScanArgs a;
+  a.Bt = p.Bt; a.L = p.L; a.H = p.H; a.N = p.N; a.P = p.P; a.K = p.K; a.T = p.T; a.nC = p.nC;
+  a.d_t = pb->d_t; a.in_t = pb->in_t; a.out_t = pb->out_t; a.logits_t = pb->logits_t;
+  a.cplx = p.cplx;
+  a.s = s; a.logits = logits; a.s_out = s_out;
+  a.d = d; a.B = B; a.C = C; a.x = x; a.h0 = h0; a.y = y; a.h_final = h_final;
+  a.prod_idx = prod_idx; a.prod_val = prod_val; a.ws = w;
+
+  if (p.Bt * p.H == 0) return finish(pb, w, stream);
+  if (p.L == 0) {
+    st = cuda_status(launch_empty_outputs(a, stream));
+    return st != PDSSM_OK ? st : finish(pb, w, stream);
+  }
+  if (!a.s) {
+    // unfused selection into s_out (or the workspace)
+    int32_t *sbuf = s_out ? s_out : w.s;
+    st = cuda_status(launch_select(pb->logits_t, logits, p.rows, (int)p.K, sbuf, stream));
+    if (st != PDSSM_OK) return st;
+    a.s = sbuf;
+  }
+  st = cuda_status(launch_chunked_scan(a, stream));
+  if (st != PDSSM_OK) return st;
+  return finish(pb, w, stream);
+}
+
+constexpr int kMaxTraced = 64;
+struct TraceState {
+  void *const *events = nullptr;
+  int32_t n_events = 0;
+  int32_t used = 0;
+  bool on = false;
+  const char *names[kMaxTraced] = {};
+};
+thread_local TraceState g_trace;
+
+}  // namespace
+
+namespace pdssm {
+
+cudaError_t trace_before(cudaStream_t st, const char *kernel_name) {
+  TraceState &t = g_trace;
+  if (!t.on || 2 * (t.used + 1) > t.n_events || t.used >= kMaxTraced) return cudaSuccess;
+  t.names[t.used] = kernel_name;
+  return cudaEventRecord(static_cast<cudaEvent_t>(t.events[2 * t.used]), st);
+}
+
+cudaError_t trace_after(cudaStream_t st) {
+  TraceState &t = g_trace;
+  if (!t.on || 2 * (t.used + 1) > t.n_events || t.used >= kMaxTraced) return cudaSuccess;
+  cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(t.events[2 * t.used + 1]), st);
+  ++t.used;
+  return e;
+}
+
+}  // namespace pdssm
+
+extern "C" {
+
+pdssm_status pdssm_trace_begin(void *const *events, int32_t n_events) {
+  if (n_events < 0 || (n_events > 0 && !events)) return PDSSM_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n_events; ++i)
+    if (!events[i]) return PDSSM_ERR_INVALID_ARG;
+  g_trace.events = events;
+  g_trace.n_events = n_events;
+  g_trace.used = 0;
+  g_trace.on = true;
+  for (int i = 0; i < kMaxTraced; ++i) g_trace.names[i] = nullptr;
+  return PDSSM_OK;
+}
+
+int32_t pdssm_trace_end(void) {
+  g_trace.on = false;
+  g_trace.events = nullptr;
+  g_trace.n_events = 0;
+  return g_trace.used;
+}
+
+const char *pdssm_trace_kernel_name(int32_t i) {
+  if (i < 0 || i >= g_trace.used || i >= kMaxTraced) return nullptr;
+  return g_trace.names[i];
+}
+
+
+const char *pdssm_status_string(int32_t status) {
+  switch (status) {
+    case PDSSM_OK: return "PDSSM_OK";
+    case PDSSM_ERR_INVALID_ARG: return "PDSSM_ERR_INVALID_ARG: invalid argument";
+    case PDSSM_ERR_UNSUPPORTED: return "PDSSM_ERR_UNSUPPORTED: size or dtype combination not supported";
+    case PDSSM_ERR_WORKSPACE: return "PDSSM_ERR_WORKSPACE: workspace missing or too small";
+    case PDSSM_ERR_CUDA: return "PDSSM_ERR_CUDA: CUDA launch or runtime error";
+    case PDSSM_ERR_DEVICE_CHECK: return "PDSSM_ERR_DEVICE_CHECK: idx or s value out of range";
+    case PDSSM_ERR_TIMEOUT: return "PDSSM_ERR_TIMEOUT: bounded device wait gave up";
+    default: return "PDSSM_ERR_UNKNOWN";
+  }
+}
+
+const char *pdssm_version(void) { return "0.1.0"; }
+
+pdssm_status pdssm_workspace_size(const pdssm_problem *pb, size_t *bytes) {
+  if (!bytes) return PDSSM_ERR_INVALID_ARG;
+  Plan p;
+  pdssm_status st = make_plan(pb, &p);
+  if (st != PDSSM_OK) return st;
+  *bytes = p.total;
+  return PDSSM_OK;
+}
+
+pdssm_status pdssm_select(const pdssm_problem *pb, const void *logits, int32_t *s,
+                          pdssm_stream_t stream) {
+  Plan p;
+  pdssm_status st = make_plan(pb, &p);
+  if (st != PDSSM_OK) return st;
+  if (p.rows == 0) return PDSSM_OK;
+  if (!logits || !s) return PDSSM_ERR_INVALID_ARG;
+  if (!aligned(logits, dtype_size(pb->logits_t)) || !aligned(s, 4)) return PDSSM_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = bind_device(cs)) != PDSSM_OK) return st;
+  return cuda_status(launch_select(pb->logits_t, logits, p.rows, (int)p.K, s, cs));
+}
+
+pdssm_status pdssm_scan_fwd(const pdssm_problem *pb, const int32_t *s, const int32_t *idx,
+                            const void *d, const void *B, const void *C, const void *x,
+                            const void *h0, void *y, void *h_final, int32_t *prod_idx,
+                            void *prod_val, void *workspace, size_t workspace_bytes,
+                            pdssm_stream_t stream) {
+  Plan p;
+  pdssm_status st = make_plan(pb, &p);
+  if (st != PDSSM_OK) return st;
+  if (p.rows > 0 && (!s || !aligned(s, 4))) return PDSSM_ERR_INVALID_ARG;
+  st = check_scan_args(pb, p, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val, workspace,
+                       workspace_bytes);
+  if (st != PDSSM_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = bind_device(cs)) != PDSSM_OK) return st;
+  return run_scan(pb, p, s, nullptr, nullptr, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val,
+                  workspace, cs);
+}
+
+pdssm_status pdssm_forward(const pdssm_problem *pb, const void *logits, const int32_t *idx,
+                           const void *d, const void *B, const void *C, const void *x,
+                           const void *h0, void *y, void *h_final, int32_t *prod_idx,
+                           void *prod_val, int32_t *s_out, void *workspace,
+                           size_t workspace_bytes, pdssm_stream_t stream) {
+  Plan p;
+  pdssm_status st = make_plan(pb, &p);
+  if (st != PDSSM_OK) return st;
+  if (p.rows > 0 && (!logits || !aligned(logits, dtype_size(pb->logits_t)))) return PDSSM_ERR_INVALID_ARG;
+  if (!aligned(s_out, 4)) return PDSSM_ERR_INVALID_ARG;
+  st = check_scan_args(pb, p, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val, workspace,
+                       workspace_bytes);
+  if (st != PDSSM_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = bind_device(cs)) != PDSSM_OK) return st;
+  return run_scan(pb, p, nullptr, logits, s_out, idx, d, B, C, x, h0, y, h_final, prod_idx,
+                  prod_val, workspace, cs);
+}
+
+pdssm_status pdssm_read_device_check(const void *workspace, pdssm_stream_t stream) {
+  if (!workspace) return PDSSM_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  pdssm_status st = bind_device(cs);
+  if (st != PDSSM_OK) return st;
+  uint32_t word = 0;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return PDSSM_ERR_CUDA;
+  if (cudaMemcpy(&word, workspace, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return PDSSM_ERR_CUDA;
+  if (word & kErrTimeout) return PDSSM_ERR_TIMEOUT;
+  if (word & (kErrIdxRange | kErrSRange)) return PDSSM_ERR_DEVICE_CHECK;
+  return PDSSM_OK;
+}
+
+}  // extern "C"

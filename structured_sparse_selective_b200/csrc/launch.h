@@ -1,0 +1,40 @@
+// Host-side launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace pdssm {
+
+// Everything a scan launch needs; validated and laid out by the C-ABI layer.
+struct ScanArgs {
+  int64_t Bt, L, H, N, P, K;
+  int64_t T, nC;  // chunk length and chunk count
+  int d_t, in_t, out_t, logits_t;
+  bool cplx;
+  const int32_t *s;        // selections (device)
+  const void *logits;      // logits when the scan selects by itself (may be null)
+  int32_t *s_out;          // where a fused select stores s (may be null)
+  const void *d, *B, *C, *x, *h0;
+  void *y, *h_final;
+  int32_t *prod_idx;
+  void *prod_val;
+  Workspace ws;
+};
+
+// Records the caller's trace events around a launch (no-op unless tracing).
+cudaError_t trace_before(cudaStream_t st, const char *kernel_name);
+cudaError_t trace_after(cudaStream_t st);
+
+cudaError_t launch_select(int logits_t, const void *logits, int64_t rows, int K, int32_t *s,
+                          cudaStream_t st);
+cudaError_t launch_prep_dict(const int32_t *idx, int K, int N, const Workspace &ws,
+                             cudaStream_t st);
+// The plain three-kernel chunked scan (phases A, B, C as separate launches).
+cudaError_t launch_chunked_scan(const ScanArgs &a, cudaStream_t st);
+// Outputs of an empty sequence (L == 0): h_final = h0 (or 0), prod = identity.
+cudaError_t launch_empty_outputs(const ScanArgs &a, cudaStream_t st);
+
+}  // namespace pdssm

@@ -1,0 +1,179 @@
+"""The C-ABI boundary on a machine without a GPU.
+
+Checks that libpdssm.so loads, exports every function include/pdssm.h
+declares, that the Python mirror of ``pdssm_problem`` has the C layout, and
+that argument errors come back as status codes before anything touches CUDA.
+No test here passes a pointer that could reach a kernel launch.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import structured_sparse_selective_b200 as pd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pdssm.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pdssm_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert set(_declared_functions()) == set(pd.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(pd.library_path())
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", pd.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    assert exported == set(_declared_functions()), "only the C ABI may be exported"
+
+
+def test_problem_struct_layout_matches_c(tmp_path):
+    src = tmp_path / "layout.c"
+    fields = [f for f, _ in pd.Problem._fields_]
+    body = "\n".join(f'  printf("{f} %zu\\n", offsetof(pdssm_problem, {f}));' for f in fields)
+    src.write_text(f'#include <stdio.h>\n#include <stddef.h>\n#include "pdssm.h"\nint main(void){{\n'
+                   f'{body}\n  printf("sizeof %zu\\n", sizeof(pdssm_problem));\n  return 0;\n}}\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                       check=True).stdout.splitlines())
+    for f in fields:
+        assert int(got[f]) == getattr(pd.Problem, f).offset, f
+    assert int(got["sizeof"]) == ctypes.sizeof(pd.Problem)
+
+
+def test_status_strings():
+    for code in range(7):
+        assert pd.pdssm_status_string(code).startswith("PDSSM_")
+    assert pd.pdssm_status_string(99) == "PDSSM_ERR_UNKNOWN"
+    assert re.match(r"^\d+\.\d+\.\d+$", pd.version())
+
+
+def _pb(**kw):
+    base = dict(batch=2, seqlen=100, heads=3, N=16, P=8, K=4, chunk=0, logits_t=pd.F32, in_t=pd.F32,
+                d_t=pd.F32, state_t=pd.F32, out_t=pd.F32, flags=0)
+    base.update(kw)
+    return pd.Problem(**base)
+
+
+def _ws(pb):
+    n = ctypes.c_size_t(0)
+    rc = pd._lib.pdssm_workspace_size(ctypes.byref(pb), ctypes.byref(n))
+    return rc, n.value
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(), OK),
+    (dict(N=0), INVALID), (dict(P=0), INVALID), (dict(K=0), INVALID), (dict(batch=-1), INVALID),
+    (dict(seqlen=-5), INVALID), (dict(chunk=-1), INVALID), (dict(flags=1 << 7), INVALID),
+    (dict(N=129), UNSUPPORTED), (dict(P=129), UNSUPPORTED), (dict(K=65), UNSUPPORTED),
+    (dict(N=128, P=128, K=64), OK), (dict(batch=0), OK), (dict(seqlen=0), OK),
+    (dict(logits_t=pd.C64), UNSUPPORTED), (dict(in_t=pd.C64), UNSUPPORTED),
+    (dict(d_t=pd.C64), UNSUPPORTED), (dict(out_t=pd.C64), UNSUPPORTED), (dict(state_t=pd.BF16), UNSUPPORTED),
+    (dict(state_t=pd.C64, d_t=pd.F32, out_t=pd.C64), UNSUPPORTED),
+    (dict(state_t=pd.C64, d_t=pd.C64, out_t=pd.F32), UNSUPPORTED),
+    (dict(state_t=pd.C64, d_t=pd.C64, out_t=pd.C64, in_t=pd.BF16, logits_t=pd.BF16), OK),
+    (dict(d_t=pd.BF16, in_t=pd.BF16, out_t=pd.BF16, logits_t=pd.BF16), OK),
+    (dict(heads=70000), UNSUPPORTED),
+])
+def test_workspace_size_validation(kw, code):
+    assert _ws(_pb(**kw))[0] == code
+
+
+def test_workspace_null_arguments():
+    n = ctypes.c_size_t(0)
+    assert pd._lib.pdssm_workspace_size(None, ctypes.byref(n)) == INVALID
+    pb = _pb()
+    assert pd._lib.pdssm_workspace_size(ctypes.byref(pb), None) == INVALID
+
+
+def test_workspace_is_linear_in_length_and_never_quadratic_in_N():
+    """O(L*N) memory (Flash PD-SSM page, Methodology 1): no term grows with N*N."""
+    def ws(**kw):
+        rc, n = _ws(_pb(**kw))
+        assert rc == OK
+        return n
+    base = dict(batch=4, heads=8, P=32, K=8, chunk=64)
+    for N in (16, 32, 64, 128):
+        for L in (64, 1000, 18000):
+            n = ws(N=N, seqlen=L, **base)
+            units = base["batch"] * base["heads"] * L
+            # y_loc (P per step) + chunk states (N*P per chunk, T >= P) + pairs + selections + dictionary
+            assert n <= units * (2 * N + 2 * base["P"] + 8) * 4 + 8 * 128 * 129 * 4 + 4096, (N, L, n)
+    # doubling N at fixed everything else at most doubles the N-dependent part
+    a, b = ws(N=64, seqlen=4096, **base), ws(N=128, seqlen=4096, **base)
+    assert b < 2.2 * a
+    # doubling L doubles it (up to alignment)
+    a, b = ws(N=64, seqlen=4096, **base), ws(N=64, seqlen=8192, **base)
+    assert abs(b - 2 * a) < 2 * 4096
+
+
+def _call_scan(pb, ws_bytes, **ptrs):
+    null = None
+    fake = ctypes.c_void_p(4096)  # never reaches a launch: every call below fails validation first
+    args = dict(s=fake, idx=fake, d=fake, B=fake, C=fake, x=fake, h0=null, y=fake, h_final=null,
+                prod_idx=null, prod_val=null, ws=fake)
+    args.update(ptrs)
+    return pd._lib.pdssm_scan_fwd(ctypes.byref(pb), args["s"], args["idx"], args["d"], args["B"], args["C"],
+                                  args["x"], args["h0"], args["y"], args["h_final"], args["prod_idx"],
+                                  args["prod_val"], args["ws"], ws_bytes, None)
+
+
+@pytest.mark.parametrize("missing", ["s", "idx", "d", "B", "C", "x", "y"])
+def test_scan_rejects_null_inputs(missing):
+    pb = _pb()
+    _, need = _ws(pb)
+    assert _call_scan(pb, need, **{missing: None}) == INVALID
+
+
+def test_scan_rejects_small_or_missing_workspace():
+    pb = _pb()
+    _, need = _ws(pb)
+    assert _call_scan(pb, need - 1) == WORKSPACE
+    assert _call_scan(pb, need, ws=None) == WORKSPACE
+
+
+def test_scan_rejects_misaligned_pointers():
+    pb = _pb()
+    _, need = _ws(pb)
+    assert _call_scan(pb, need, d=ctypes.c_void_p(4098)) == INVALID
+    assert _call_scan(pb, need, ws=ctypes.c_void_p(4104)) == INVALID
+    assert _call_scan(pb, need, h0=ctypes.c_void_p(4097)) == INVALID
+
+
+def test_scan_rejects_bad_problem_before_pointers():
+    assert _call_scan(_pb(N=200), 1 << 30) == UNSUPPORTED
+    assert pd._lib.pdssm_scan_fwd(None, *([None] * 12), 0, None) == INVALID
+
+
+def test_select_and_forward_validation():
+    pb = _pb()
+    fake = ctypes.c_void_p(4096)
+    assert pd._lib.pdssm_select(ctypes.byref(pb), None, fake, None) == INVALID
+    assert pd._lib.pdssm_select(ctypes.byref(pb), fake, None, None) == INVALID
+    assert pd._lib.pdssm_select(ctypes.byref(_pb(K=100)), fake, fake, None) == UNSUPPORTED
+    _, need = _ws(pb)
+    args = [fake] * 6 + [None] * 5 + [fake]  # logits..x, h0/y/h_final/prod_idx/prod_val, s_out
+    args[7] = None  # y missing
+    assert pd._lib.pdssm_forward(ctypes.byref(pb), *args[:11], None, fake, need, None) == INVALID
+    assert pd._lib.pdssm_read_device_check(None, None) == INVALID
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    t = torch.zeros(4)
+    with pytest.raises(ValueError):
+        pd._ptr(t)
