@@ -210,7 +210,7 @@ def run_ours(args, rank, world, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     sp = workloads.spec(args.workload)
-    inp = workloads.generate(sp, seed=shard_seed(rank), device=device)
+    inp = {k: v.to(device) for k, v in workloads.generate(sp, seed=shard_seed(rank)).items()}
     pb = pd.make_problem(inp["logits"], inp["d"], inp["B"], inp["x"], chunk=args.chunk)
     Bt, L, H, N = inp["B"].shape
     P = inp["x"].shape[-1]

@@ -200,6 +200,8 @@ class KernelTrace:
 
     def __init__(self, max_launches: int = 16):
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * max_launches)]
+        for e in self.events:  # torch creates the CUDA event on first record
+            e.record()
         self._arr = (ctypes.c_void_p * len(self.events))(*[ctypes.c_void_p(e.cuda_event) for e in self.events])
         self.names = []
 
