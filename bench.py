@@ -267,7 +267,7 @@ def run_ours(args, rank, world, local):
     with_logits = sp.K * torch.empty((), dtype=sp.logits_dtype).element_size()
     bytes_fwd = units * sp.algorithmic_bytes_per_token_head(with_logits=True)
     alg_bytes = {
-        "fused_forward": bytes_fwd,
+        "fused_scan": bytes_fwd,
         # phase A reads s, d, B, C and x of every token-head (its y_loc and
         # chunk-state writes are workspace traffic, not algorithmic)
         "chunked_phase_a": units * (4 + sp.algorithmic_bytes_per_token_head(with_logits=False) - 4

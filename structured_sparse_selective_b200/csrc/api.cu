@@ -144,14 +144,13 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &p, const int32_t *s,
                       cudaStream_t stream) {
   Workspace w = carve(p, workspace);
   if (cudaMemsetAsync(w.err, 0, 4, stream) != cudaSuccess) return PDSSM_ERR_CUDA;
-  pdssm_status st = cuda_status(launch_prep_dict(idx, (int)p.K, (int)p.N, w, stream));
-  if (st != PDSSM_OK) return st;
+  pdssm_status st = PDSSM_OK;
 
   ScanArgs a;
   a.Bt = p.Bt; a.L = p.L; a.H = p.H; a.N = p.N; a.P = p.P; a.K = p.K; a.T = p.T; a.nC = p.nC;
   a.d_t = pb->d_t; a.in_t = pb->in_t; a.out_t = pb->out_t; a.logits_t = pb->logits_t;
   a.cplx = p.cplx;
-  a.s = s; a.logits = logits; a.s_out = s_out;
+  a.s = s; a.logits = logits; a.s_out = s_out; a.idx = idx;
   a.d = d; a.B = B; a.C = C; a.x = x; a.h0 = h0; a.y = y; a.h_final = h_final;
   a.prod_idx = prod_idx; a.prod_val = prod_val; a.ws = w;
 
@@ -160,6 +159,14 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &p, const int32_t *s,
     st = cuda_status(launch_empty_outputs(a, stream));
     return st != PDSSM_OK ? st : finish(pb, w, stream);
   }
+  const bool fused_chunk = pb->chunk == 0 || pb->chunk == 16;
+  if (!(pb->flags & PDSSM_FLAG_REFERENCE_PATH) && fused_chunk && fused_scan_supported(a)) {
+    // the fused kernel validates idx itself and needs no preimage lists
+    st = cuda_status(launch_fused_scan(a, stream));
+    return st != PDSSM_OK ? st : finish(pb, w, stream);
+  }
+  st = cuda_status(launch_prep_dict(idx, (int)p.K, (int)p.N, w, stream));
+  if (st != PDSSM_OK) return st;
   if (!a.s) {
     // unfused selection into s_out (or the workspace)
     int32_t *sbuf = s_out ? s_out : w.s;

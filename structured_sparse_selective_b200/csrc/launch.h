@@ -14,7 +14,8 @@ struct ScanArgs {
   int64_t T, nC;  // chunk length and chunk count
   int d_t, in_t, out_t, logits_t;
   bool cplx;
-  const int32_t *s;        // selections (device)
+  const int32_t *s;        // selections (device; null when the scan selects from logits)
+  const int32_t *idx;      // caller's dictionary [K][N]
   const void *logits;      // logits when the scan selects by itself (may be null)
   int32_t *s_out;          // where a fused select stores s (may be null)
   const void *d, *B, *C, *x, *h0;
@@ -34,6 +35,9 @@ cudaError_t launch_prep_dict(const int32_t *idx, int K, int N, const Workspace &
                              cudaStream_t st);
 // The plain three-kernel chunked scan (phases A, B, C as separate launches).
 cudaError_t launch_chunked_scan(const ScanArgs &a, cudaStream_t st);
+// The fused single-kernel forward pass (real state, N = P = 64, bf16 d/B/C/x).
+bool fused_scan_supported(const ScanArgs &a);
+cudaError_t launch_fused_scan(const ScanArgs &a, cudaStream_t st);
 // Outputs of an empty sequence (L == 0): h_final = h0 (or 0), prod = identity.
 cudaError_t launch_empty_outputs(const ScanArgs &a, cudaStream_t st);
 

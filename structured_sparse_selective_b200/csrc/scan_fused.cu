@@ -1,0 +1,773 @@
+// Fused forward pass on sm_100a: selection, the three phases of the chunked
+// scan and the output, in one kernel per (batch, head) sequence.
+//
+// Flash PD-SSM page, Technical Summary: Methodology 1 (hard selection of one
+// one-hot-column dictionary matrix per step), Methodology 3 (phase A:
+// recurrences inside chunks; phase B: prefix over chunk dependencies gives the
+// carry states; phase C: carry corrections). This kernel runs the three
+// phases as a software pipeline over 16-token sub-chunks of one sequence, with
+// the dense contractions of the chunked form on the 5th-generation tensor
+// cores and the carry state resident in tensor memory.
+//
+// Notation for one sub-chunk a of T = 16 steps (tau, sigma in [0, T)):
+//   A_t = P_{s_t} diag(d_t)                   one-hot-column transition
+//   Phi_tau = A_tau ... A_0                   prefix from the sub-chunk start
+//   Psi_sigma = A_{T-1} ... A_{sigma+1}       suffix to the sub-chunk end
+//   Ct_tau = Phi_tau^T C_tau      (gather)    readout seen from the start
+//   Bh_sigma = Psi_sigma B_sigma  (scatter)   input seen at the end
+//   G[tau][sigma] = C_tau^T A_tau...A_{sigma+1} B_sigma  (sigma <= tau)
+// With S_a the state entering the sub-chunk (N x P):
+//   y_tau   = S_a^T Ct_tau + sum_sigma G[tau][sigma] x_sigma        (phase A + C)
+//   S_{a+1} = Phi_{T-1} S_a + sum_sigma Bh_sigma x_sigma^T          (phase B)
+// Only S_{a+1} depends on S_a through a sparse map; everything else is dense:
+//   U^T   = X^T Bh        (64 x 64, K = 16)  bf16 x bf16 (X exact, Bh = hi + lo)
+//   Y^T   = X^T G^T       (64 x 16, K = 16)  bf16 x bf16 (G = hi + lo)
+//   Y^T  += S^T Ct^T      (64 x 16, K = 64)  tf32, S and Ct split hi + lo
+// The tensor core truncates fp32 to tf32 (checked on B200), so with
+// S_lo = S - trunc_tf32(S) the three products hi*hi + hi*lo + lo*hi carry
+// about 21 bits. No N x N matrix is formed.
+//
+// Roles (288 threads): warps 0-3 prepare sub-chunk operands, warp 8 (one
+// thread) issues the MMAs, warps 4-7 (one per tensor-memory quarter) advance
+// the carry state and write y. Every wait is bounded; a timeout sets an error
+// bit, makes every role leave its loop, drains outstanding MMAs and copies,
+// and frees tensor memory.
+#include <algorithm>
+
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace pdssm {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kN = 64;   // state rows
+constexpr int kP = 64;   // state columns
+constexpr int kT = 16;   // sub-chunk length
+constexpr int kNW = 4;   // prep warps; warp w prepares sub-chunks w, w + 4, ...
+constexpr int kNS = kNW; // operand stages (one per prep warp)
+constexpr int kNY = 4;   // output accumulator slots
+constexpr int kThreads = 256;  // 4 prep warps + 4 carry warps (warp 4 also issues the MMAs)
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
+
+// tensor-memory columns
+constexpr uint32_t kColState0 = 0;    // two 64-column state regions
+constexpr uint32_t kColSlo = 128;     // tf32 low part of the state read by the readout
+constexpr uint32_t kColY = 192;       // kNY slots of kT columns
+constexpr uint32_t kTmemCols = 256;
+
+// operand stage layout (bytes)
+constexpr int kOffCtHi = 0;                   // tf32 K-major [T][N]: 4 KB
+constexpr int kOffCtLo = kOffCtHi + 4096;
+constexpr int kOffBhHi = kOffCtLo + 4096;     // bf16 K-major (n = i, k = sigma): 2 KB
+constexpr int kOffBhLo = kOffBhHi + 2048;
+constexpr int kOffGtHi = kOffBhLo + 2048;     // bf16 K-major (n = tau, k = sigma): 512 B
+constexpr int kOffGtLo = kOffGtHi + 512;
+constexpr int kOffX = kOffGtLo + 512;         // bf16 MN-major (mn = p, k = tau): 2 KB
+constexpr int kOffCsrMeta = kOffX + 2048;     // int [N]: src | dst << 8 | first << 16 | last << 17
+constexpr int kOffCsrNu = kOffCsrMeta + 256;  // float [N]: value of the source column
+constexpr int kOffPhiIdx = kOffCsrNu + 256;   // int [N]: Phi_{T-1} index of source j
+constexpr int kOffPhiVal = kOffPhiIdx + 256;  // float [N]: Phi_{T-1} value of source j
+constexpr int kOpStage = kOffPhiVal + 256;    // 16384 B
+
+// per-prep-warp scratch (bytes)
+constexpr int kScrBins = 0;                   // int [N] fixed-point accumulators
+constexpr int kScrCnt = 256;                  // int [N]
+constexpr int kScrCntLo = 512;                // int [N]
+constexpr int kScrOffs = 768;                 // int [N]
+constexpr int kScrBytes = 1024;
+
+// input stage layout: logits [T][K] raw, d/B/C [T][N] bf16, x canonical
+struct InLayout {
+  int logits, d, B, C, x, bytes;
+};
+
+struct FParams {
+  int64_t L, H;
+  int K, logit_size;
+  int nsub;
+  const void *logits;   // null when the selections are given
+  const int32_t *s_in;  // selections [Bt][L][H] (when logits is null)
+  const int32_t *idx;
+  const __nv_bfloat16 *d, *B, *C, *x;
+  const float *h0;
+  void *y;
+  float *h_final;
+  int32_t *prod_idx;
+  float *prod_val;
+  int32_t *s_out;
+  uint32_t *err;
+  InLayout in;
+  int off_in, off_op, off_dict, off_scr, off_bar;
+};
+
+struct Bars {
+  uint64_t full[kNS], opfree[kNS], yfull[kNY], yfree[kNY];
+  uint64_t ufull, gdone, sready, slofree, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait shared by every role: false (and the abort flag set) on timeout.
+__device__ __forceinline__ bool wait_bar(Bars *bars, uint64_t *bar, uint32_t parity, uint32_t *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*(volatile int *)&bars->abort) return false;
+    if (now_ns() - t0 > kTimeoutNs) {
+      *(volatile int *)&bars->abort = 1;
+      flag_error(err, kErrTimeout);
+      return false;
+    }
+  }
+}
+
+// The same bounded wait, with one decision for the whole warp.
+__device__ __forceinline__ bool wait_bar_warp(Bars *bars, uint64_t *bar, uint32_t parity, uint32_t *err) {
+  const bool ok = wait_bar(bars, bar, parity, err);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ float tf32_trunc(float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); }
+
+__device__ __forceinline__ float ld_bf16(const uint8_t *base, int idx) {
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[idx]);
+}
+
+template <typename TL>
+__device__ __forceinline__ float ld_logit(const uint8_t *base, int idx) {
+  return to_f32(reinterpret_cast<const TL *>(base)[idx]);
+}
+
+// 2^e as a float, e clamped to the normal range
+__device__ __forceinline__ float exp2i(int e) {
+  e = max(-126, min(127, e));
+  return __int_as_float((127 + e) << 23);
+}
+
+// operand element offsets
+__device__ __forceinline__ int off_ct(int tau, int j) {  // tf32 K-major, SBO = (N/4)*128
+  return (tau & 7) * 16 + (tau >> 3) * 2048 + (j >> 2) * 128 + (j & 3) * 4;
+}
+__device__ __forceinline__ int off_bh(int i, int sigma) {  // bf16 K-major, SBO = (T/8)*128
+  return (i & 7) * 16 + (i >> 3) * 256 + (sigma >> 3) * 128 + (sigma & 7) * 2;
+}
+__device__ __forceinline__ int off_gt(int tau, int sigma) { return off_bh(tau, sigma); }
+
+__device__ __forceinline__ void store_out(float *p, float v) { *p = v; }
+__device__ __forceinline__ void store_out(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ void st_bf16_split(uint8_t *hi, uint8_t *lo, int off, float v) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  *reinterpret_cast<__nv_bfloat16 *>(hi + off) = h;
+  *reinterpret_cast<__nv_bfloat16 *>(lo + off) = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
+// ---------------------------------------------------------------- loads
+
+// cp.async of one sub-chunk's inputs into an input stage by one warp; tail
+// tokens are zero-filled.
+template <typename TL>
+__device__ __forceinline__ void load_inputs(const FParams &a, uint8_t *st, int64_t b, int64_t h, int sub,
+                                            int lane) {
+  const int t0 = sub * kT;
+  const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
+  const int lchunks = a.logits ? a.K * a.logit_size / 16 : 0;  // 16-byte chunks per logits row
+  const int per_tok = lchunks + 8 * 4;          // logits + d, B, C, x rows of 128 B
+  for (int e = lane; e < kT * per_tok; e += 32) {
+    const int tau = e / per_tok, c = e % per_tok;
+    uint8_t *dst;
+    const uint8_t *src = nullptr;
+    const int64_t row = (b * a.L + t0 + tau) * a.H + h;
+    if (c < lchunks) {
+      dst = st + a.in.logits + (tau * lchunks + c) * 16;
+      if (tau < nvalid) src = static_cast<const uint8_t *>(a.logits) + (row * lchunks + c) * 16;
+    } else {
+      const int cc = c - lchunks, which = cc >> 3, ch = cc & 7;
+      if (which < 3) {
+        const int off = which == 0 ? a.in.d : which == 1 ? a.in.B : a.in.C;
+        const __nv_bfloat16 *g = which == 0 ? a.d : which == 1 ? a.B : a.C;
+        dst = st + off + tau * 128 + ch * 16;
+        if (tau < nvalid) src = reinterpret_cast<const uint8_t *>(g + row * kN) + ch * 16;
+      } else {  // x into the MN-major canonical layout: (tau%8)*16 + (tau/8)*1024 + (p/8)*128
+        dst = st + a.in.x + (tau & 7) * 16 + (tau >> 3) * 1024 + ch * 128;
+        if (tau < nvalid) src = reinterpret_cast<const uint8_t *>(a.x + row * kP) + ch * 16;
+      }
+    }
+    if (src)
+      cp_async16(dst, src);
+    else
+      *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// ------------------------------------------------------------- the kernel
+
+template <typename TL, typename TO>
+__global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t *in_base = smem + a.off_in;
+  uint8_t *op_base = smem + a.off_op;
+  uint8_t *dict = smem + a.off_dict;     // uint8 [K][N]
+  uint8_t *scr = smem + a.off_scr;       // prep scratch
+  Bars *bars = reinterpret_cast<Bars *>(smem + a.off_bar);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+  const int nsub = a.nsub;
+
+  // ---- setup
+  if (tid == 0) {
+    for (int i = 0; i < kNS; ++i) {
+      mbar_init(&bars->full[i], 1);
+      mbar_init(&bars->opfree[i], 1 + 4);  // MMA commit + one arrival per carry warp
+    }
+    for (int i = 0; i < kNY; ++i) {
+      mbar_init(&bars->yfull[i], 1);
+      mbar_init(&bars->yfree[i], 4);
+    }
+    mbar_init(&bars->ufull, 1);
+    mbar_init(&bars->gdone, 4);
+    mbar_init(&bars->sready, 4);
+    mbar_init(&bars->slofree, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    mbar_fence_init();
+  }
+  for (int e = tid; e < a.K * kN; e += kThreads) {
+    int v = a.idx[e];
+    if (v < 0 || v >= kN) {
+      flag_error(a.err, kErrIdxRange);
+      v = 0;
+    }
+    dict[e] = (uint8_t)v;
+  }
+  if (warp == kNW) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = bars->tmem_base;
+
+  if (warp < kNW) {
+    // ================================================================ prep
+    // Warp w prepares sub-chunks w, w + kNW, ... into operand stage w. Per
+    // sub-chunk one loop runs three independent 16-step chains side by side:
+    // the prefix Phi_tau (forward), the suffix Psi_sigma and the readouts
+    // R_sigma (both backward). Lanes own rows j0 = lane and j1 = lane + 32.
+    uint8_t *in = in_base + warp * a.in.bytes;
+    uint8_t *op = op_base + warp * kOpStage;
+    uint8_t *ws = scr + warp * kScrBytes;
+    int *bins = reinterpret_cast<int *>(ws + kScrBins);
+    if (warp < nsub) load_inputs<TL>(a, in, b, h, warp, lane);
+    cp_async_commit();
+    bins[lane] = 0;
+    bins[lane + 32] = 0;
+    const int j0 = lane, j1 = lane + 32;
+    for (int sub = warp, use = 0; sub < nsub; sub += kNW, ++use) {
+      const int t0 = sub * kT;
+      const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
+      if (!wait_bar_warp(bars, &bars->opfree[warp], (use & 1) ^ 1, a.err)) break;
+      cp_async_wait<0>();
+      __syncwarp();
+
+      // selections, one lane per token
+      int s_lane = 0;
+      if (lane < nvalid && !a.logits) {
+        s_lane = a.s_in[(b * a.L + t0 + lane) * a.H + h];
+        if (s_lane < 0 || s_lane >= a.K) {
+          flag_error(a.err, kErrSRange);
+          s_lane = 0;
+        }
+      } else if (lane < nvalid) {
+        const uint8_t *row = in + a.in.logits + lane * a.K * a.logit_size;
+        float best = ld_logit<TL>(row, 0);
+        if (!(best != best))
+          for (int k = 1; k < a.K; ++k) {
+            const float v = ld_logit<TL>(row, k);
+            if (v != v) {
+              s_lane = k;
+              break;
+            }
+            if (v > best) {
+              best = v;
+              s_lane = k;
+            }
+          }
+      }
+      if (lane < nvalid && a.s_out) a.s_out[(b * a.L + t0 + lane) * a.H + h] = s_lane;
+
+      // x into the operand stage (2 KB)
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        reinterpret_cast<uint4 *>(op + kOffX)[lane + 32 * c] = reinterpret_cast<const uint4 *>(in + a.in.x)[lane + 32 * c];
+
+      const uint8_t *din = in + a.in.d, *Bin = in + a.in.B, *Cin = in + a.in.C;
+      uint8_t *cthi = op + kOffCtHi, *ctlo = op + kOffCtLo;
+      int i0 = j0, i1 = j1;          // Phi_tau (forward)
+      float v0 = 1.f, v1 = 1.f;
+      int k0 = j0, k1 = j1;          // Psi_sigma (backward)
+      float m0 = 1.f, m1 = 1.f;
+      float R0[kT], R1[kT];          // R_sigma[j][tau], tau > sigma (backward)
+#pragma unroll
+      for (int c = 0; c < kT; ++c) R0[c] = R1[c] = 0.f;
+
+      for (int k = 0; k < kT; ++k) {
+        // ---- forward step tau = k: Ct_tau = Phi_tau^T C_tau, split tf32 hi + lo
+        {
+          const int tau = k;
+          float c0 = 0.f, c1 = 0.f;
+          if (tau < nvalid) {
+            const int s = __shfl_sync(0xffffffffu, s_lane, tau);
+            const uint8_t *dk = dict + s * kN;
+            v0 *= ld_bf16(din, tau * kN + i0);
+            v1 *= ld_bf16(din, tau * kN + i1);
+            i0 = dk[i0];
+            i1 = dk[i1];
+            c0 = v0 * ld_bf16(Cin, tau * kN + i0);
+            c1 = v1 * ld_bf16(Cin, tau * kN + i1);
+          }
+          const float h0 = tf32_trunc(c0), h1 = tf32_trunc(c1);
+          *reinterpret_cast<float *>(cthi + off_ct(tau, j0)) = h0;
+          *reinterpret_cast<float *>(cthi + off_ct(tau, j1)) = h1;
+          *reinterpret_cast<float *>(ctlo + off_ct(tau, j0)) = c0 - h0;
+          *reinterpret_cast<float *>(ctlo + off_ct(tau, j1)) = c1 - h1;
+        }
+        const int sg = kT - 1 - k;
+        const bool sv = sg < nvalid;
+        const float bs0 = sv ? ld_bf16(Bin, sg * kN + j0) : 0.f;
+        const float bs1 = sv ? ld_bf16(Bin, sg * kN + j1) : 0.f;
+        // ---- backward step sigma = sg: Bh_sigma = Psi_sigma B_sigma as an exact
+        //      fixed-point sum (integer adds are order-independent)
+        {
+          const float w0 = m0 * bs0, w1 = m1 * bs1;
+          const unsigned mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(w0), fabsf(w1))));
+          // |w| < 2^ex; 64 terms of magnitude < 2^24 stay below 2^30
+          const int ex = (int)((mb >> 23) & 0xff) - 126;
+          const int e = mb ? 24 - ex : 0;
+          const float up = exp2i(e), dn = exp2i(-e);
+          if (sv) {
+            atomicAdd(&bins[k0], __float2int_rn(w0 * up));
+            atomicAdd(&bins[k1], __float2int_rn(w1 * up));
+          }
+          __syncwarp();
+          const float bh0 = (float)bins[j0] * dn, bh1 = (float)bins[j1] * dn;
+          bins[j0] = 0;
+          bins[j1] = 0;
+          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(j0, sg), bh0);
+          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(j1, sg), bh1);
+          if (sv && sg > 0) {  // Psi_{sg-1} = Psi_sg A_sg: column j <- d[j] * column idx[j]
+            const int s = __shfl_sync(0xffffffffu, s_lane, sg);
+            const uint8_t *dk = dict + s * kN;
+            const int r0 = dk[j0], r1 = dk[j1];
+            const int ka = __shfl_sync(0xffffffffu, k0, r0 & 31), kb = __shfl_sync(0xffffffffu, k1, r0 & 31);
+            const float ma = __shfl_sync(0xffffffffu, m0, r0 & 31), mb2 = __shfl_sync(0xffffffffu, m1, r0 & 31);
+            const int kc = __shfl_sync(0xffffffffu, k0, r1 & 31), kd = __shfl_sync(0xffffffffu, k1, r1 & 31);
+            const float mc = __shfl_sync(0xffffffffu, m0, r1 & 31), md = __shfl_sync(0xffffffffu, m1, r1 & 31);
+            const float d0 = ld_bf16(din, sg * kN + j0), d1 = ld_bf16(din, sg * kN + j1);
+            k0 = r0 < 32 ? ka : kb;
+            m0 = (r0 < 32 ? ma : mb2) * d0;
+            k1 = r1 < 32 ? kc : kd;
+            m1 = (r1 < 32 ? mc : md) * d1;
+          }
+        }
+        // ---- readout step sigma = sg: R_sg = A_{sg+1}^T R_{sg+1} (tau > sg), R_sg[:, sg] = C_sg,
+        //      G[tau][sg] = sum_j B_sg[j] R_sg[j][tau]
+        {
+          if (sg + 1 < nvalid) {
+            const int s = __shfl_sync(0xffffffffu, s_lane, sg + 1);
+            const uint8_t *dk = dict + s * kN;
+            const int r0 = dk[j0], r1 = dk[j1];
+            const float d0 = ld_bf16(din, (sg + 1) * kN + j0), d1 = ld_bf16(din, (sg + 1) * kN + j1);
+#pragma unroll
+            for (int tau = 0; tau < kT; ++tau) {
+              if (tau > sg) {
+                const float a0 = __shfl_sync(0xffffffffu, R0[tau], r0 & 31);
+                const float a1 = __shfl_sync(0xffffffffu, R1[tau], r0 & 31);
+                const float c0 = __shfl_sync(0xffffffffu, R0[tau], r1 & 31);
+                const float c1 = __shfl_sync(0xffffffffu, R1[tau], r1 & 31);
+                R0[tau] = d0 * (r0 < 32 ? a0 : a1);
+                R1[tau] = d1 * (r1 < 32 ? c0 : c1);
+              }
+            }
+          }
+          if (sv) {
+            const float c0 = ld_bf16(Cin, sg * kN + j0), c1 = ld_bf16(Cin, sg * kN + j1);
+#pragma unroll
+            for (int tau = 0; tau < kT; ++tau)
+              if (tau == sg) {
+                R0[tau] = c0;
+                R1[tau] = c1;
+              }
+          }
+          // G[tau][sg] for tau in [8 * rnd, 8 * rnd + 8): partials, then a reduce-scatter
+          // of 8 values over 32 lanes (two rounds keep the register count down)
+#pragma unroll
+          for (int rnd = 0; rnd < 2; ++rnd) {
+            float g[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int tau = 8 * rnd + c;
+              g[c] = (tau >= sg) ? bs0 * R0[tau] + bs1 * R1[tau] : 0.f;
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const bool upr = lane & 16;
+              const float send = upr ? g[c] : g[c + 4];
+              const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+              g[c] = (upr ? g[c + 4] : g[c]) + recv;
+            }
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const bool upr = lane & 8;
+              const float send = upr ? g[c] : g[c + 2];
+              const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
+              g[c] = (upr ? g[c + 2] : g[c]) + recv;
+            }
+            {
+              const bool upr = lane & 4;
+              const float send = upr ? g[0] : g[1];
+              const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
+              g[0] = (upr ? g[1] : g[0]) + recv;
+            }
+            g[0] += __shfl_xor_sync(0xffffffffu, g[0], 2);
+            g[0] += __shfl_xor_sync(0xffffffffu, g[0], 1);
+            if ((lane & 3) == 0) {
+              const int tau = 8 * rnd + ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+              st_bf16_split(op + kOffGtHi, op + kOffGtLo, off_gt(tau, sg), g[0]);
+            }
+          }
+        }
+      }
+
+      // ---- Phi_{T-1}: its pair, and its sources grouped by target (increasing j)
+      {
+        int *cnt = reinterpret_cast<int *>(ws + kScrCnt);
+        int *cntlo = reinterpret_cast<int *>(ws + kScrCntLo);
+        int *offs = reinterpret_cast<int *>(ws + kScrOffs);
+        reinterpret_cast<int *>(op + kOffPhiIdx)[j0] = i0;
+        reinterpret_cast<int *>(op + kOffPhiIdx)[j1] = i1;
+        reinterpret_cast<float *>(op + kOffPhiVal)[j0] = v0;
+        reinterpret_cast<float *>(op + kOffPhiVal)[j1] = v1;
+        cnt[j0] = 0;
+        cnt[j1] = 0;
+        cntlo[j0] = 0;
+        cntlo[j1] = 0;
+        __syncwarp();
+        atomicAdd(&cnt[i0], 1);
+        atomicAdd(&cntlo[i0], 1);
+        atomicAdd(&cnt[i1], 1);
+        __syncwarp();
+        const int ca = cnt[2 * lane], cb = cnt[2 * lane + 1];
+        int incl = ca + cb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += n;
+        }
+        const int excl = incl - ca - cb;
+        offs[2 * lane] = excl;
+        offs[2 * lane + 1] = excl + ca;
+        __syncwarp();
+        const unsigned lt = (1u << lane) - 1u;
+        const unsigned mm0 = __match_any_sync(0xffffffffu, i0);
+        const unsigned mm1 = __match_any_sync(0xffffffffu, i1);
+        const int pos0 = offs[i0] + __popc(mm0 & lt);
+        const int pos1 = offs[i1] + cntlo[i1] + __popc(mm1 & lt);
+        int *meta = reinterpret_cast<int *>(op + kOffCsrMeta);
+        float *cnu = reinterpret_cast<float *>(op + kOffCsrNu);
+        meta[pos0] = j0 | (i0 << 8) | ((pos0 == offs[i0]) << 16) | ((pos0 == offs[i0] + cnt[i0] - 1) << 17);
+        cnu[pos0] = v0;
+        meta[pos1] = j1 | (i1 << 8) | ((pos1 == offs[i1]) << 16) | ((pos1 == offs[i1] + cnt[i1] - 1) << 17);
+        cnu[pos1] = v1;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->full[warp]);
+      // prefetch this warp's next sub-chunk into its (now free) input stage
+      const int nxt = sub + kNW;
+      if (nxt < nsub) load_inputs<TL>(a, in, b, h, nxt, lane);
+      cp_async_commit();
+    }
+    cp_async_wait<0>();
+  } else {
+    // ============================================ carry state, output, and the MMA issue (warp 4, lane 0)
+    const int q = warp & 3;                 // tensor-memory quarter
+    const bool act = lane < 16;
+    const int p = 16 * q + lane;            // state column owned by this lane
+    const uint32_t lanebase = (uint32_t)(32 * q) << 16;
+    const bool issuer = (q == 0) && (lane == 0);
+    const uint32_t id_u = idesc_bf16_f32(64, kN, true, false);
+    const uint32_t id_g = idesc_bf16_f32(64, kT, true, false);
+    const uint32_t id_c = idesc_tf32_f32(64, kT);
+    // U and the intra-sub-chunk part of Y: need the operands and a free state region
+    auto issue_u = [&](int sub) -> bool {
+      const int st = sub % kNS;
+      if (!wait_bar(bars, &bars->full[st], (sub / kNS) & 1, a.err)) return false;
+      if (sub >= 1 && !wait_bar(bars, &bars->gdone, (sub - 1) & 1, a.err)) return false;
+      if (sub >= kNY && !wait_bar(bars, &bars->yfree[sub % kNY], ((sub / kNY) - 1) & 1, a.err)) return false;
+      tc_fence_after();
+      const uint32_t op = smem_u32(op_base + st * kOpStage);
+      const uint32_t dU = tbase + kColState0 + ((sub + 1) & 1) * 64;
+      const uint32_t dY = tbase + kColY + (sub % kNY) * kT;
+      const uint64_t ax = smem_desc(op + kOffX, (kP / 8) * 128, 128);
+      mma_bf16(dU, ax, smem_desc(op + kOffBhHi, 128, 256), id_u, 0);
+      mma_bf16(dU, ax, smem_desc(op + kOffBhLo, 128, 256), id_u, 1);
+      mma_bf16(dY, ax, smem_desc(op + kOffGtHi, 128, 256), id_g, 0);
+      mma_bf16(dY, ax, smem_desc(op + kOffGtLo, 128, 256), id_g, 1);
+      mma_commit(&bars->ufull);
+      return true;
+    };
+    // readout of the entering state S_sub: A operand from tensor memory, tf32 x3
+    auto issue_y = [&](int sub) -> bool {
+      const int st = sub % kNS;
+      if (!wait_bar(bars, &bars->sready, sub & 1, a.err)) return false;
+      tc_fence_after();
+      const uint32_t op = smem_u32(op_base + st * kOpStage);
+      const uint32_t dY = tbase + kColY + (sub % kNY) * kT;
+      const uint32_t aS = tbase + kColState0 + (sub & 1) * 64;
+      const uint32_t aL = tbase + kColSlo;
+#pragma unroll
+      for (int ks = 0; ks < kN / 8; ++ks) {
+        const uint64_t bhi = smem_desc(op + kOffCtHi + ks * 256, 128, 2048);
+        const uint64_t blo = smem_desc(op + kOffCtLo + ks * 256, 128, 2048);
+        mma_tf32_ts(dY, aS + ks * 8, bhi, id_c, 1);
+        mma_tf32_ts(dY, aS + ks * 8, blo, id_c, 1);
+        mma_tf32_ts(dY, aL + ks * 8, bhi, id_c, 1);
+      }
+      mma_commit(&bars->yfull[sub % kNY]);
+      mma_commit(&bars->opfree[st]);
+      mma_commit(&bars->slofree);
+      return true;
+    };
+    bool ok = true;
+    if (issuer && nsub > 0) ok = issue_u(0);
+    __syncwarp();
+    // S_0 = h0 (or 0) and its tf32 low part
+    {
+      float v[16];
+      for (int c0 = 0; c0 < kN; c0 += 16) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          v[i] = (act && a.h0) ? a.h0[((b * a.H + h) * kN + c0 + i) * kP + p] : 0.f;
+        tmem_st16(tbase + lanebase + kColState0 + c0, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] -= tf32_trunc(v[i]);
+        tmem_st16(tbase + lanebase + kColSlo + c0, v);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->sready);
+    }
+    if (issuer && ok && nsub > 0) ok = issue_y(0);
+    TO *yout = static_cast<TO *>(a.y);
+    int pidx0 = lane, pidx1 = lane + 32;
+    float pval0 = 1.f, pval1 = 1.f;
+    for (int sub = 0; sub < nsub; ++sub) {
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int st = sub % kNS;
+      const uint8_t *op = op_base + st * kOpStage;
+      const int t0 = sub * kT;
+      const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
+      if (!wait_bar_warp(bars, &bars->ufull, sub & 1, a.err)) break;
+      if (!wait_bar_warp(bars, &bars->full[st], (sub / kNS) & 1, a.err)) break;
+      tc_fence_after();
+      const uint32_t RS = tbase + lanebase + kColState0 + (sub & 1) * 64;
+      const uint32_t RU = tbase + lanebase + kColState0 + ((sub + 1) & 1) * 64;
+      const int4 *meta4 = reinterpret_cast<const int4 *>(op + kOffCsrMeta);
+      const float4 *nu4 = reinterpret_cast<const float4 *>(op + kOffCsrNu);
+      // running whole-sequence product (warp 4 keeps it; sub-chunks arrive in order)
+      if (q == 0) {
+        const int *pi = reinterpret_cast<const int *>(op + kOffPhiIdx);
+        const float *pv = reinterpret_cast<const float *>(op + kOffPhiVal);
+        pval0 *= pv[pidx0];
+        pval1 *= pv[pidx1];
+        pidx0 = pi[pidx0];
+        pidx1 = pi[pidx1];
+      }
+      // S_{a+1}[i] = U[i] + sum_{j: Phi[j] = i} nu_j S_a[j], in place over U
+      float run = 0.f;
+#pragma unroll
+      for (int part = 0; part < 4; ++part) {
+        float v[16], u[16], nu[16];
+        int mt[16];
+#pragma unroll
+        for (int r4 = 0; r4 < 4; ++r4) {
+          const int4 m4 = meta4[4 * part + r4];
+          const float4 n4 = nu4[4 * part + r4];
+          mt[4 * r4 + 0] = m4.x; mt[4 * r4 + 1] = m4.y; mt[4 * r4 + 2] = m4.z; mt[4 * r4 + 3] = m4.w;
+          nu[4 * r4 + 0] = n4.x; nu[4 * r4 + 1] = n4.y; nu[4 * r4 + 2] = n4.z; nu[4 * r4 + 3] = n4.w;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          tmem_ld1(RS + (mt[r] & 0xff), v[r]);
+          if (mt[r] & (1 << 16)) tmem_ld1(RU + ((mt[r] >> 8) & 0xff), u[r]);
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          if (mt[r] & (1 << 16)) run = u[r];
+          run = fmaf(nu[r], v[r], run);
+          if (mt[r] & (1 << 17)) tmem_st1(RU + ((mt[r] >> 8) & 0xff), run);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->gdone);
+      if (issuer && sub + 1 < nsub) ok = issue_u(sub + 1);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      // tf32 low part of S_{a+1} for the next readout, once this readout is done
+      if (!wait_bar_warp(bars, &bars->slofree, sub & 1, a.err)) break;
+      tc_fence_after();
+      for (int c0 = 0; c0 < kN; c0 += 16) {
+        float v[16];
+        tmem_ld16(RU + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] -= tf32_trunc(v[i]);
+        tmem_st16(tbase + lanebase + kColSlo + c0, v);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars->sready);
+        mbar_arrive(&bars->opfree[st]);
+      }
+      if (issuer && sub + 1 < nsub) ok = issue_y(sub + 1);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      // output of this sub-chunk
+      if (!wait_bar_warp(bars, &bars->yfull[sub % kNY], (sub / kNY) & 1, a.err)) break;
+      tc_fence_after();
+      {
+        float v[16];
+        tmem_ld16(tbase + lanebase + kColY + (sub % kNY) * kT, v);
+        tmem_wait_ld();
+        if (act) {
+#pragma unroll
+          for (int tau = 0; tau < kT; ++tau)
+            if (tau < nvalid) store_out(yout + ((b * a.L + t0 + tau) * a.H + h) * kP + p, v[tau]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->yfree[sub % kNY]);
+    }
+    const bool clean = !*(volatile int *)&bars->abort;
+    if (q == 0 && clean) {
+      const int64_t o = (b * a.H + h) * kN;
+      if (a.prod_idx) {
+        a.prod_idx[o + lane] = pidx0;
+        a.prod_idx[o + lane + 32] = pidx1;
+      }
+      if (a.prod_val) {
+        a.prod_val[o + lane] = pval0;
+        a.prod_val[o + lane + 32] = pval1;
+      }
+    }
+    if (clean && a.h_final) {
+      const uint32_t RF = tbase + lanebase + kColState0 + (nsub & 1) * 64;
+      for (int c0 = 0; c0 < kN; c0 += 16) {
+        float v[16];
+        tmem_ld16(RF + c0, v);
+        tmem_wait_ld();
+        if (act)
+          for (int i = 0; i < 16; ++i) a.h_final[((b * a.H + h) * kN + c0 + i) * kP + p] = v[i];
+      }
+    }
+    if (issuer) {
+      // every MMA issued so far has completed once this arrives
+      mma_commit(&bars->drain);
+      const uint64_t t0 = now_ns();
+      while (!mbar_try_wait(&bars->drain, 0) && now_ns() - t0 < kTimeoutNs) {
+      }
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kNW) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+}  // namespace
+
+bool fused_scan_supported(const ScanArgs &s) {
+  if (s.cplx || s.N != kN || s.P != kP) return false;
+  if (s.d_t != PDSSM_BF16 || s.in_t != PDSSM_BF16) return false;
+  const int lsz = s.logits_t == PDSSM_BF16 ? 2 : 4;
+  if ((s.K * lsz) % 16 != 0) return false;
+  if (!s.logits && !s.s) return false;
+  auto al16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  return (!s.logits || al16(s.logits)) && al16(s.d) && al16(s.B) && al16(s.C) && al16(s.x);
+}
+
+cudaError_t launch_fused_scan(const ScanArgs &s, cudaStream_t st) {
+  FParams a;
+  a.L = s.L;
+  a.H = s.H;
+  a.K = (int)s.K;
+  a.logit_size = s.logits_t == PDSSM_BF16 ? 2 : 4;
+  a.nsub = (int)((s.L + kT - 1) / kT);
+  a.logits = s.logits;
+  a.s_in = s.logits ? nullptr : s.s;
+  a.idx = s.idx;
+  a.d = static_cast<const __nv_bfloat16 *>(s.d);
+  a.B = static_cast<const __nv_bfloat16 *>(s.B);
+  a.C = static_cast<const __nv_bfloat16 *>(s.C);
+  a.x = static_cast<const __nv_bfloat16 *>(s.x);
+  a.h0 = static_cast<const float *>(s.h0);
+  a.y = s.y;
+  a.h_final = static_cast<float *>(s.h_final);
+  a.prod_idx = s.prod_idx;
+  a.prod_val = static_cast<float *>(s.prod_val);
+  a.s_out = s.s_out;
+  a.err = s.ws.err;
+  // input stage
+  int o = 0;
+  a.in.logits = o; o += s.logits ? kT * a.K * a.logit_size : 0; o = (o + 127) & ~127;
+  a.in.d = o; o += kT * kN * 2;
+  a.in.B = o; o += kT * kN * 2;
+  a.in.C = o; o += kT * kN * 2;
+  a.in.x = o; o += kT * kP * 2;
+  a.in.bytes = (o + 127) & ~127;
+  // smem
+  int off = 0;
+  a.off_op = off; off += kNS * kOpStage; off = (off + 1023) & ~1023;
+  a.off_in = off; off += kNW * a.in.bytes;
+  a.off_dict = off; off += (int)((s.K * kN + 127) & ~127);
+  a.off_scr = off; off += kNW * kScrBytes;
+  off = (off + 127) & ~127;
+  a.off_bar = off; off += (int)sizeof(Bars);
+
+  cudaError_t e;
+  auto kern = (s.logits_t == PDSSM_BF16)
+                  ? (s.out_t == PDSSM_BF16 ? fused_scan_kernel<__nv_bfloat16, __nv_bfloat16>
+                                           : fused_scan_kernel<__nv_bfloat16, float>)
+                  : (s.out_t == PDSSM_BF16 ? fused_scan_kernel<float, __nv_bfloat16>
+                                           : fused_scan_kernel<float, float>);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, off);
+  if (e != cudaSuccess) return e;
+  if ((e = trace_before(st, "fused_scan")) != cudaSuccess) return e;
+  kern<<<(unsigned)(s.Bt * s.H), kThreads, off, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return trace_after(st);
+}
+
+}  // namespace pdssm

@@ -218,3 +218,71 @@ def test_full_size_workload(cuda_device, recipe):
         ep = slice_rel_err(to_np(out["prod_val"][b, h])[None], r["prod_val"][i:i + 1])
         assert np.array_equal(to_np(out["prod_idx"][b, h]), r["prod_idx"][i])
         assert ey <= tol and eh <= 1e-4 and ep <= 1e-4, (b, h, ey, eh, ep)
+
+
+# ------------------------------------------- fused single-kernel path (N = P = 64, bf16)
+
+FUSED = [
+    dict(batch=1, seqlen=1, heads=1),
+    dict(batch=1, seqlen=15, heads=2),
+    dict(batch=1, seqlen=16, heads=1),
+    dict(batch=2, seqlen=17, heads=1),
+    dict(batch=1, seqlen=100, heads=3),
+    dict(batch=3, seqlen=257, heads=2),
+]
+
+
+@pytest.mark.parametrize("kw", FUSED)
+def test_fused_path_matches_oracle(cuda_device, kw):
+    sp = workloads.spec("lm", **kw)
+    inp = workloads.generate(sp, seed=11)
+    compare_full(inp, run_gpu(inp, cuda_device, chunk=0))
+
+
+def test_fused_path_with_initial_state_and_selection_entry(cuda_device):
+    sp = workloads.spec("lm", batch=2, seqlen=99, heads=2)
+    inp = workloads.generate(sp, seed=12)
+    h0 = torch.randn(sp.batch, sp.heads, sp.N, sp.P, generator=torch.Generator().manual_seed(3))
+    a = run_gpu(inp, cuda_device, chunk=0, h0=h0)
+    compare_full(inp, a, h0=h0)
+    b = run_gpu(inp, cuda_device, chunk=0, h0=h0, via_scan=True)  # selections given
+    for k in ("y", "h_final", "prod_idx", "prod_val", "s"):
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_fused_path_is_deterministic_and_agrees_with_reference_path(cuda_device):
+    sp = workloads.spec("lm", batch=2, seqlen=200, heads=2)
+    inp = workloads.generate(sp, seed=13)
+    a = run_gpu(inp, cuda_device, chunk=0)
+    b = run_gpu(inp, cuda_device, chunk=0)
+    for k in ("y", "h_final", "prod_idx", "prod_val", "s"):
+        assert torch.equal(a[k], b[k]), k
+    r = run_gpu(inp, cuda_device, chunk=0, flags=pd.FLAG_REFERENCE_PATH)
+    assert torch.equal(a["s"], r["s"]) and torch.equal(a["prod_idx"], r["prod_idx"])
+    assert slice_rel_err(to_np(a["h_final"]).reshape(4, -1), to_np(r["h_final"]).reshape(4, -1)) < 1e-5
+
+
+@pytest.mark.parametrize("dictionary", ["permutation", "identity", "constant"])
+def test_fused_path_dictionary_shapes(cuda_device, dictionary):
+    sp = workloads.spec("lm", batch=1, seqlen=150, heads=2)
+    inp = workloads.generate(sp, seed=14)
+    g = torch.Generator().manual_seed(5)
+    if dictionary == "permutation":
+        inp["idx"] = torch.stack([torch.randperm(64, generator=g) for _ in range(sp.K)]).to(torch.int32)
+    elif dictionary == "identity":
+        inp["idx"] = torch.arange(64, dtype=torch.int32).repeat(sp.K, 1)
+    else:  # every column into one row: maximal collisions
+        inp["idx"] = torch.full((sp.K, 64), 7, dtype=torch.int32)
+    compare_full(inp, run_gpu(inp, cuda_device, chunk=0))
+
+
+@pytest.mark.parametrize("ldt,odt", [(torch.float32, torch.bfloat16), (torch.bfloat16, torch.float32),
+                                     (torch.float32, torch.float32)])
+def test_fused_path_logit_and_output_dtypes(cuda_device, ldt, odt):
+    sp = workloads.spec("lm", batch=1, seqlen=70, heads=2)
+    inp = workloads.generate(sp, seed=15)
+    inp["logits"] = inp["logits"].to(ldt)
+    g = {k: v.to(cuda_device) for k, v in inp.items()}
+    out = pd.forward(g["logits"], g["idx"], g["d"], g["B"], g["C"], g["x"], out_dtype=odt, want_s=True)
+    torch.cuda.synchronize()
+    compare_full(inp, out)
