@@ -165,6 +165,31 @@ pdssm_status pdssm_forward(const pdssm_problem *pb, const void *logits, const in
                            size_t workspace_bytes, pdssm_stream_t stream);
 
 /*
+ * pdssm_forward without a caller workspace, for callers that cannot allocate
+ * device memory on their call path (a plug-in whose host application already
+ * owns all device memory, or a latency-critical loop that cannot afford
+ * cudaMalloc's implicit synchronisation). The paper has no counterpart to
+ * this entry point.
+ *   Arguments are those of pdssm_forward minus workspace / workspace_bytes.
+ *   The workspace is a 32 MiB array inside this library's device image,
+ *   held by every GPU that loads the library until the process exits.
+ *   Problems whose pdssm_workspace_size exceeds 32 MiB return
+ *   PDSSM_ERR_WORKSPACE before anything is enqueued.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture.
+ *   All calls on a device share the array and it keeps the last call's
+ *   contents: calls that overlap on the GPU race and must be ordered by the
+ *   caller (one stream, or events). pdssm_read_device_check cannot read this
+ *   workspace; PDSSM_FLAG_DEVICE_CHECK still reports out-of-range values.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+pdssm_status pdssm_forward_noalloc(const pdssm_problem *pb, const void *logits, const int32_t *idx,
+                                   const void *d, const void *B, const void *C, const void *x,
+                                   const void *h0, void *y, void *h_final, int32_t *prod_idx,
+                                   void *prod_val, int32_t *s_out, pdssm_stream_t stream);
+
+/*
  * Synchronises `stream` and reads the error word that the last pdssm_scan_fwd
  * or pdssm_forward call on `workspace` left: PDSSM_OK, PDSSM_ERR_DEVICE_CHECK
  * (an idx or s value was out of range) or PDSSM_ERR_TIMEOUT.

@@ -28,7 +28,7 @@ __all__ = [
     "PdssmError", "Problem", "F32", "BF16", "C64", "FLAG_DEVICE_CHECK", "FLAG_REFERENCE_PATH",
     "library_path", "make_problem", "pdssm_workspace_size", "pdssm_select", "pdssm_scan_fwd",
     "pdssm_forward", "pdssm_read_device_check", "pdssm_status_string", "forward", "EXPORTED_SYMBOLS",
-    "KernelTrace", "alloc_workspace",
+    "KernelTrace", "alloc_workspace", "pdssm_forward_noalloc",
 ]
 
 F32, BF16, C64 = 0, 1, 2
@@ -39,7 +39,7 @@ MAX_N, MAX_P, MAX_K = 128, 128, 64
 EXPORTED_SYMBOLS = (
     "pdssm_status_string", "pdssm_version", "pdssm_workspace_size", "pdssm_select",
     "pdssm_scan_fwd", "pdssm_forward", "pdssm_read_device_check", "pdssm_trace_begin",
-    "pdssm_trace_end", "pdssm_trace_kernel_name",
+    "pdssm_trace_end", "pdssm_trace_kernel_name", "pdssm_forward_noalloc",
 )
 
 _DIR = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +86,8 @@ def _load() -> ctypes.CDLL:
     lib.pdssm_scan_fwd.restype = ctypes.c_int
     lib.pdssm_forward.argtypes = [pb, vp, i32p, vp, vp, vp, vp, vp, vp, vp, i32p, vp, i32p, vp, sz, vp]
     lib.pdssm_forward.restype = ctypes.c_int
+    lib.pdssm_forward_noalloc.argtypes = [pb, vp, i32p, vp, vp, vp, vp, vp, vp, vp, i32p, vp, i32p, vp]
+    lib.pdssm_forward_noalloc.restype = ctypes.c_int
     lib.pdssm_read_device_check.argtypes = [vp, vp]
     lib.pdssm_read_device_check.restype = ctypes.c_int
     lib.pdssm_trace_begin.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
@@ -183,6 +185,16 @@ def pdssm_forward(pb: Problem, logits, idx, d, B, C, x, h0, y, h_final, prod_idx
         _ptr(x, dev), _ptr(h0, dev), _ptr(y, dev), _ptr(h_final, dev), _ptr(prod_idx, dev),
         _ptr(prod_val, dev), _ptr(s_out, dev), _ptr(workspace, dev), ws_bytes, _stream(stream, dev)),
         "pdssm_forward")
+
+
+def pdssm_forward_noalloc(pb: Problem, logits, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val,
+                          s_out, stream=None) -> None:
+    """pdssm_forward with the library's built-in 32 MiB device workspace (no caller workspace)."""
+    dev = idx.device
+    _check(_lib.pdssm_forward_noalloc(
+        ctypes.byref(pb), _ptr(logits, dev), _ptr(idx, dev), _ptr(d, dev), _ptr(B, dev), _ptr(C, dev),
+        _ptr(x, dev), _ptr(h0, dev), _ptr(y, dev), _ptr(h_final, dev), _ptr(prod_idx, dev),
+        _ptr(prod_val, dev), _ptr(s_out, dev), _stream(stream, dev)), "pdssm_forward_noalloc")
 
 
 def pdssm_read_device_check(workspace: torch.Tensor, stream=None) -> int:

@@ -3,6 +3,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "launch.h"
 #include "pdssm.h"
@@ -325,3 +326,67 @@ pdssm_status pdssm_read_device_check(const void *workspace, pdssm_stream_t strea
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// Allocation-free variant of pdssm_forward.
+//
+// Some callers cannot call cudaMalloc on their call path: plug-ins whose host
+// application already owns all device memory (a framework's caching
+// allocator has reserved it), and latency-critical loops where cudaMalloc's
+// implicit device synchronisation is not acceptable. For them the workspace
+// lives in a fixed-size array in this library's device image instead of a
+// caller buffer. Every GPU that loads the library holds the array until the
+// process exits. All calls on a device share it, and it keeps the last call's
+// contents; calls that overlap on the GPU (different streams, or different
+// threads without ordering) race on it.
+
+namespace {
+
+constexpr size_t kStaticWorkspaceBytes = size_t(32) << 20;  // 32 MiB
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+std::once_flag g_static_ws_once[kMaxDevices];
+void *g_static_ws_ptr[kMaxDevices] = {};
+cudaError_t g_static_ws_err[kMaxDevices] = {};
+
+// Device address of the static workspace on the current device. In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+pdssm_status static_workspace(void **ptr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PDSSM_ERR_CUDA;
+  std::call_once(g_static_ws_once[dev], [dev] {
+    void *p = nullptr;
+    g_static_ws_err[dev] = cudaGetSymbolAddress(&p, g_static_workspace);
+    g_static_ws_ptr[dev] = p;
+  });
+  if (g_static_ws_err[dev] != cudaSuccess || !g_static_ws_ptr[dev]) return PDSSM_ERR_CUDA;
+  *ptr = g_static_ws_ptr[dev];
+  return PDSSM_OK;
+}
+
+}  // namespace
+
+extern "C" pdssm_status pdssm_forward_noalloc(const pdssm_problem *pb, const void *logits,
+                                              const int32_t *idx, const void *d, const void *B,
+                                              const void *C, const void *x, const void *h0, void *y,
+                                              void *h_final, int32_t *prod_idx, void *prod_val,
+                                              int32_t *s_out, pdssm_stream_t stream) {
+  Plan p;
+  pdssm_status st = make_plan(pb, &p);
+  if (st != PDSSM_OK) return st;
+  if (p.total > kStaticWorkspaceBytes) return PDSSM_ERR_WORKSPACE;
+  if (p.rows > 0 && (!logits || !aligned(logits, dtype_size(pb->logits_t)))) return PDSSM_ERR_INVALID_ARG;
+  if (!aligned(s_out, 4)) return PDSSM_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = bind_device(cs)) != PDSSM_OK) return st;
+  void *ws = nullptr;
+  if ((st = static_workspace(&ws)) != PDSSM_OK) return st;
+  st = check_scan_args(pb, p, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val, ws,
+                       kStaticWorkspaceBytes);
+  if (st != PDSSM_OK) return st;
+  return run_scan(pb, p, nullptr, logits, s_out, idx, d, B, C, x, h0, y, h_final, prod_idx,
+                  prod_val, ws, cs);
+}
