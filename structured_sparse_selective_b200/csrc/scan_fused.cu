@@ -27,9 +27,17 @@
 // S_lo = S - trunc_tf32(S) the three products hi*hi + hi*lo + lo*hi carry
 // about 21 bits. No N x N matrix is formed.
 //
-// Roles (288 threads): warps 0-3 prepare sub-chunk operands, warp 8 (one
-// thread) issues the MMAs, warps 4-7 (one per tensor-memory quarter) advance
-// the carry state and write y. Every wait is bounded; a timeout sets an error
+// State order. S_a lives in tensor memory with its rows in the source order of
+// Phi_{T-1} of sub-chunk a: sources grouped by target row, increasing source
+// row inside a group. A carry step then needs one 64-column load of S_a, a
+// segmented sum in registers and one read-modify-write per target row. The
+// prep warp of sub-chunk a composes sub-chunk a+1's indices as well, so it
+// writes Bh (hence U and S_{a+1}) in sub-chunk a+1's order and Ct in its own.
+// The state after the last sub-chunk is in natural order.
+//
+// Roles (256 threads): warps 0-3 each prepare every fourth sub-chunk's
+// operands; warps 4-7 (one per tensor-memory quarter) advance the carry state
+// and write y, and one thread of warp 4 issues the MMAs. Every wait is bounded; a timeout sets an error
 // bit, makes every role leave its loop, drains outstanding MMAs and copies,
 // and frees tensor memory.
 #include <algorithm>
@@ -59,29 +67,35 @@ constexpr uint32_t kColY = 192;       // kNY slots of kT columns
 constexpr uint32_t kTmemCols = 256;
 
 // operand stage layout (bytes)
-constexpr int kOffCtHi = 0;                   // tf32 K-major [T][N]: 4 KB
+constexpr int kOffCtHi = 0;                   // tf32 K-major (n = tau, k = state position): 4 KB
 constexpr int kOffCtLo = kOffCtHi + 4096;
-constexpr int kOffBhHi = kOffCtLo + 4096;     // bf16 K-major (n = i, k = sigma): 2 KB
+constexpr int kOffBhHi = kOffCtLo + 4096;     // bf16 K-major (n = state position, k = sigma): 2 KB
 constexpr int kOffBhLo = kOffBhHi + 2048;
 constexpr int kOffGtHi = kOffBhLo + 2048;     // bf16 K-major (n = tau, k = sigma): 512 B
 constexpr int kOffGtLo = kOffGtHi + 512;
 constexpr int kOffX = kOffGtLo + 512;         // bf16 MN-major (mn = p, k = tau): 2 KB
-constexpr int kOffCsrMeta = kOffX + 2048;     // int [N]: src | dst << 8 | first << 16 | last << 17
-constexpr int kOffCsrNu = kOffCsrMeta + 256;  // float [N]: value of the source column
-constexpr int kOffPhiIdx = kOffCsrNu + 256;   // int [N]: Phi_{T-1} index of source j
-constexpr int kOffPhiVal = kOffPhiIdx + 256;  // float [N]: Phi_{T-1} value of source j
-constexpr int kOpStage = kOffPhiVal + 256;    // 16384 B
+constexpr int kOffMeta = kOffX + 2048;        // int [N] by position: carry-step record (below)
+constexpr int kOffNu = kOffMeta + 256;        // float [N] by position: Phi_{T-1} value of the source
+constexpr int kOffPhiIdx = kOffNu + 256;      // int [N] by source row: Phi_{T-1} index
+constexpr int kOffPhiVal = kOffPhiIdx + 256;  // float [N] by source row: Phi_{T-1} value
+constexpr int kOffSrc = kOffPhiVal + 256;     // int [N] by position: source row
+constexpr int kOpStage = kOffSrc + 256;       // 16640 B
+
+// carry-step record of a position: the target's column in the next order, and
+// whether the position continues a target group (else it starts one) and ends it
+constexpr int kMetaKeep = 1 << 8;
+constexpr int kMetaEnd = 1 << 9;
 
 // per-prep-warp scratch (bytes)
 constexpr int kScrBins = 0;                   // int [N] fixed-point accumulators
-constexpr int kScrCnt = 256;                  // int [N]
-constexpr int kScrCntLo = 512;                // int [N]
-constexpr int kScrOffs = 768;                 // int [N]
+constexpr int kScrCnt = 256;                  // int [N] sources per target
+constexpr int kScrCntLo = 512;                // int [N] sources j < 32 per target
+constexpr int kScrOffs = 768;                 // int [N] first position of each target's group
 constexpr int kScrBytes = 1024;
 
 // input stage layout: logits [T][K] raw, d/B/C [T][N] bf16, x canonical
 struct InLayout {
-  int logits, d, B, C, x, bytes;
+  int logits, nlogits, d, B, C, x, bytes;  // nlogits: the next sub-chunk's logits
 };
 
 struct FParams {
@@ -174,15 +188,16 @@ __device__ __forceinline__ void st_bf16_split(uint8_t *hi, uint8_t *lo, int off,
 
 // ---------------------------------------------------------------- loads
 
-// cp.async of one sub-chunk's inputs into an input stage by one warp; tail
-// tokens are zero-filled.
+// cp.async of one sub-chunk's inputs (and the next sub-chunk's logits) into an
+// input stage by one warp; rows past the end of the sequence are zero-filled.
 template <typename TL>
 __device__ __forceinline__ void load_inputs(const FParams &a, uint8_t *st, int64_t b, int64_t h, int sub,
                                             int lane) {
   const int t0 = sub * kT;
   const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
+  const int nnext = (int)(a.L - t0 - kT < kT ? (a.L - t0 - kT > 0 ? a.L - t0 - kT : 0) : kT);
   const int lchunks = a.logits ? a.K * a.logit_size / 16 : 0;  // 16-byte chunks per logits row
-  const int per_tok = lchunks + 8 * 4;          // logits + d, B, C, x rows of 128 B
+  const int per_tok = 2 * lchunks + 8 * 4;  // logits, next logits, and d, B, C, x rows of 128 B
   for (int e = lane; e < kT * per_tok; e += 32) {
     const int tau = e / per_tok, c = e % per_tok;
     uint8_t *dst;
@@ -191,8 +206,13 @@ __device__ __forceinline__ void load_inputs(const FParams &a, uint8_t *st, int64
     if (c < lchunks) {
       dst = st + a.in.logits + (tau * lchunks + c) * 16;
       if (tau < nvalid) src = static_cast<const uint8_t *>(a.logits) + (row * lchunks + c) * 16;
+    } else if (c < 2 * lchunks) {
+      const int cc = c - lchunks;
+      dst = st + a.in.nlogits + (tau * lchunks + cc) * 16;
+      if (tau < nnext)
+        src = static_cast<const uint8_t *>(a.logits) + ((row + (int64_t)kT * a.H) * lchunks + cc) * 16;
     } else {
-      const int cc = c - lchunks, which = cc >> 3, ch = cc & 7;
+      const int cc = c - 2 * lchunks, which = cc >> 3, ch = cc & 7;
       if (which < 3) {
         const int off = which == 0 ? a.in.d : which == 1 ? a.in.B : a.in.C;
         const __nv_bfloat16 *g = which == 0 ? a.d : which == 1 ? a.B : a.C;
@@ -208,6 +228,57 @@ __device__ __forceinline__ void load_inputs(const FParams &a, uint8_t *st, int64
     else
       *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
   }
+}
+
+// Hard selection of one token from its logits row (lowest k on ties, first NaN wins).
+template <typename TL>
+__device__ __forceinline__ int argmax_row(const uint8_t *row, int K) {
+  float best = ld_logit<TL>(row, 0);
+  if (best != best) return 0;
+  int bi = 0;
+  for (int k = 1; k < K; ++k) {
+    const float v = ld_logit<TL>(row, k);
+    if (v != v) return k;
+    if (v > best) {
+      best = v;
+      bi = k;
+    }
+  }
+  return bi;
+}
+
+// Positions of the 64 sources j0 = lane, j1 = lane + 32 of an index map when the
+// sources are grouped by target row (targets ascending, sources ascending in a
+// group). Leaves per-target counts and first positions in the warp's scratch.
+__device__ __forceinline__ void group_positions(int t0, int t1, uint8_t *ws, int lane, int &pos0, int &pos1) {
+  int *cnt = reinterpret_cast<int *>(ws + kScrCnt);
+  int *cntlo = reinterpret_cast<int *>(ws + kScrCntLo);
+  int *offs = reinterpret_cast<int *>(ws + kScrOffs);
+  cnt[lane] = 0;
+  cnt[lane + 32] = 0;
+  cntlo[lane] = 0;
+  cntlo[lane + 32] = 0;
+  __syncwarp();
+  atomicAdd(&cnt[t0], 1);
+  atomicAdd(&cntlo[t0], 1);
+  atomicAdd(&cnt[t1], 1);
+  __syncwarp();
+  const int ca = cnt[2 * lane], cb = cnt[2 * lane + 1];
+  int incl = ca + cb;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  const int excl = incl - ca - cb;
+  offs[2 * lane] = excl;
+  offs[2 * lane + 1] = excl + ca;
+  __syncwarp();
+  const unsigned lt = (1u << lane) - 1u;
+  const unsigned m0 = __match_any_sync(0xffffffffu, t0);
+  const unsigned m1 = __match_any_sync(0xffffffffu, t1);
+  pos0 = offs[t0] + __popc(m0 & lt);
+  pos1 = offs[t1] + cntlo[t1] + __popc(m1 & lt);
 }
 
 // ------------------------------------------------------------- the kernel
@@ -262,10 +333,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
 
   if (warp < kNW) {
     // ================================================================ prep
-    // Warp w prepares sub-chunks w, w + kNW, ... into operand stage w. Per
-    // sub-chunk one loop runs three independent 16-step chains side by side:
-    // the prefix Phi_tau (forward), the suffix Psi_sigma and the readouts
-    // R_sigma (both backward). Lanes own rows j0 = lane and j1 = lane + 32.
+    // Warp w prepares sub-chunks w, w + kNW, ... into operand stage w. Lanes own
+    // rows j0 = lane and j1 = lane + 32.
     uint8_t *in = in_base + warp * a.in.bytes;
     uint8_t *op = op_base + warp * kOpStage;
     uint8_t *ws = scr + warp * kScrBytes;
@@ -278,33 +347,24 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     for (int sub = warp, use = 0; sub < nsub; sub += kNW, ++use) {
       const int t0 = sub * kT;
       const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
+      const int nnext = (int)(a.L - t0 - kT < kT ? (a.L - t0 - kT > 0 ? a.L - t0 - kT : 0) : kT);
       if (!wait_bar_warp(bars, &bars->opfree[warp], (use & 1) ^ 1, a.err)) break;
       cp_async_wait<0>();
       __syncwarp();
 
-      // selections, one lane per token
-      int s_lane = 0;
-      if (lane < nvalid && !a.logits) {
-        s_lane = a.s_in[(b * a.L + t0 + lane) * a.H + h];
-        if (s_lane < 0 || s_lane >= a.K) {
+      // selections of this sub-chunk and of the next one, one lane per token
+      int s_lane = 0, sn_lane = 0;
+      if (!a.logits) {
+        if (lane < nvalid) s_lane = a.s_in[(b * a.L + t0 + lane) * a.H + h];
+        if (lane < nnext) sn_lane = a.s_in[(b * a.L + t0 + kT + lane) * a.H + h];
+        if (s_lane < 0 || s_lane >= a.K || sn_lane < 0 || sn_lane >= a.K) {
           flag_error(a.err, kErrSRange);
-          s_lane = 0;
+          if (s_lane < 0 || s_lane >= a.K) s_lane = 0;
+          if (sn_lane < 0 || sn_lane >= a.K) sn_lane = 0;
         }
-      } else if (lane < nvalid) {
-        const uint8_t *row = in + a.in.logits + lane * a.K * a.logit_size;
-        float best = ld_logit<TL>(row, 0);
-        if (!(best != best))
-          for (int k = 1; k < a.K; ++k) {
-            const float v = ld_logit<TL>(row, k);
-            if (v != v) {
-              s_lane = k;
-              break;
-            }
-            if (v > best) {
-              best = v;
-              s_lane = k;
-            }
-          }
+      } else {
+        if (lane < nvalid) s_lane = argmax_row<TL>(in + a.in.logits + lane * a.K * a.logit_size, a.K);
+        if (lane < nnext) sn_lane = argmax_row<TL>(in + a.in.nlogits + lane * a.K * a.logit_size, a.K);
       }
       if (lane < nvalid && a.s_out) a.s_out[(b * a.L + t0 + lane) * a.H + h] = s_lane;
 
@@ -314,23 +374,71 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         reinterpret_cast<uint4 *>(op + kOffX)[lane + 32 * c] = reinterpret_cast<const uint4 *>(in + a.in.x)[lane + 32 * c];
 
       const uint8_t *din = in + a.in.d, *Bin = in + a.in.B, *Cin = in + a.in.C;
+
+      // ---- the next sub-chunk's composite (indices only) -> the order of S_{a+1}
+      int posB0, posB1;
+      {
+        int n0 = j0, n1 = j1;
+        for (int tau = 0; tau < nnext; ++tau) {
+          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, sn_lane, tau) * kN;
+          n0 = dk[n0];
+          n1 = dk[n1];
+        }
+        group_positions(n0, n1, ws, lane, posB0, posB1);
+      }
+      __syncwarp();
+      // ---- this sub-chunk's composite Phi_{T-1} -> the order of S_a, target groups
+      int ia0 = j0, ia1 = j1;
+      float va0 = 1.f, va1 = 1.f;
+      for (int tau = 0; tau < nvalid; ++tau) {
+        const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
+        va0 *= ld_bf16(din, tau * kN + ia0);
+        va1 *= ld_bf16(din, tau * kN + ia1);
+        ia0 = dk[ia0];
+        ia1 = dk[ia1];
+      }
+      int posA0, posA1;
+      group_positions(ia0, ia1, ws, lane, posA0, posA1);
+      {
+        const int *cnt = reinterpret_cast<const int *>(ws + kScrCnt);
+        const int *offs = reinterpret_cast<const int *>(ws + kScrOffs);
+        // the target's column in the next order: posB of row ia (held by lane ia & 31)
+        const int pb0a = __shfl_sync(0xffffffffu, posB0, ia0 & 31), pb0b = __shfl_sync(0xffffffffu, posB1, ia0 & 31);
+        const int pb1a = __shfl_sync(0xffffffffu, posB0, ia1 & 31), pb1b = __shfl_sync(0xffffffffu, posB1, ia1 & 31);
+        const int f0 = offs[ia0], f1 = offs[ia1];
+        int *meta = reinterpret_cast<int *>(op + kOffMeta);
+        meta[posA0] = (ia0 < 32 ? pb0a : pb0b) | (posA0 != f0 ? kMetaKeep : 0) |
+                      (posA0 == f0 + cnt[ia0] - 1 ? kMetaEnd : 0);
+        meta[posA1] = (ia1 < 32 ? pb1a : pb1b) | (posA1 != f1 ? kMetaKeep : 0) |
+                      (posA1 == f1 + cnt[ia1] - 1 ? kMetaEnd : 0);
+        reinterpret_cast<float *>(op + kOffNu)[posA0] = va0;
+        reinterpret_cast<float *>(op + kOffNu)[posA1] = va1;
+        reinterpret_cast<int *>(op + kOffSrc)[posA0] = j0;
+        reinterpret_cast<int *>(op + kOffSrc)[posA1] = j1;
+        reinterpret_cast<int *>(op + kOffPhiIdx)[j0] = ia0;
+        reinterpret_cast<int *>(op + kOffPhiIdx)[j1] = ia1;
+        reinterpret_cast<float *>(op + kOffPhiVal)[j0] = va0;
+        reinterpret_cast<float *>(op + kOffPhiVal)[j1] = va1;
+      }
+
+      // ---- three 16-step chains side by side: the prefix Phi_tau (forward), the
+      //      suffix Psi_sigma and the readouts R_sigma (both backward)
       uint8_t *cthi = op + kOffCtHi, *ctlo = op + kOffCtLo;
-      int i0 = j0, i1 = j1;          // Phi_tau (forward)
+      int i0 = j0, i1 = j1;          // Phi_tau
       float v0 = 1.f, v1 = 1.f;
-      int k0 = j0, k1 = j1;          // Psi_sigma (backward)
+      int k0 = j0, k1 = j1;          // Psi_sigma
       float m0 = 1.f, m1 = 1.f;
-      float R0[kT], R1[kT];          // R_sigma[j][tau], tau > sigma (backward)
+      float R0[kT], R1[kT];          // R_sigma[j][tau], tau >= sigma
 #pragma unroll
       for (int c = 0; c < kT; ++c) R0[c] = R1[c] = 0.f;
 
       for (int k = 0; k < kT; ++k) {
-        // ---- forward step tau = k: Ct_tau = Phi_tau^T C_tau, split tf32 hi + lo
+        // ---- forward step tau = k: Ct_tau = Phi_tau^T C_tau at the source's position in S_a's order
         {
           const int tau = k;
           float c0 = 0.f, c1 = 0.f;
           if (tau < nvalid) {
-            const int s = __shfl_sync(0xffffffffu, s_lane, tau);
-            const uint8_t *dk = dict + s * kN;
+            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
             v0 *= ld_bf16(din, tau * kN + i0);
             v1 *= ld_bf16(din, tau * kN + i1);
             i0 = dk[i0];
@@ -339,17 +447,18 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
             c1 = v1 * ld_bf16(Cin, tau * kN + i1);
           }
           const float h0 = tf32_trunc(c0), h1 = tf32_trunc(c1);
-          *reinterpret_cast<float *>(cthi + off_ct(tau, j0)) = h0;
-          *reinterpret_cast<float *>(cthi + off_ct(tau, j1)) = h1;
-          *reinterpret_cast<float *>(ctlo + off_ct(tau, j0)) = c0 - h0;
-          *reinterpret_cast<float *>(ctlo + off_ct(tau, j1)) = c1 - h1;
+          *reinterpret_cast<float *>(cthi + off_ct(tau, posA0)) = h0;
+          *reinterpret_cast<float *>(cthi + off_ct(tau, posA1)) = h1;
+          *reinterpret_cast<float *>(ctlo + off_ct(tau, posA0)) = c0 - h0;
+          *reinterpret_cast<float *>(ctlo + off_ct(tau, posA1)) = c1 - h1;
         }
         const int sg = kT - 1 - k;
         const bool sv = sg < nvalid;
         const float bs0 = sv ? ld_bf16(Bin, sg * kN + j0) : 0.f;
         const float bs1 = sv ? ld_bf16(Bin, sg * kN + j1) : 0.f;
         // ---- backward step sigma = sg: Bh_sigma = Psi_sigma B_sigma as an exact
-        //      fixed-point sum (integer adds are order-independent)
+        //      fixed-point sum (integer adds are order-independent), written at
+        //      the target's position in S_{a+1}'s order
         {
           const float w0 = m0 * bs0, w1 = m1 * bs1;
           const unsigned mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(w0), fabsf(w1))));
@@ -365,11 +474,10 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           const float bh0 = (float)bins[j0] * dn, bh1 = (float)bins[j1] * dn;
           bins[j0] = 0;
           bins[j1] = 0;
-          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(j0, sg), bh0);
-          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(j1, sg), bh1);
+          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB0, sg), bh0);
+          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB1, sg), bh1);
           if (sv && sg > 0) {  // Psi_{sg-1} = Psi_sg A_sg: column j <- d[j] * column idx[j]
-            const int s = __shfl_sync(0xffffffffu, s_lane, sg);
-            const uint8_t *dk = dict + s * kN;
+            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, sg) * kN;
             const int r0 = dk[j0], r1 = dk[j1];
             const int ka = __shfl_sync(0xffffffffu, k0, r0 & 31), kb = __shfl_sync(0xffffffffu, k1, r0 & 31);
             const float ma = __shfl_sync(0xffffffffu, m0, r0 & 31), mb2 = __shfl_sync(0xffffffffu, m1, r0 & 31);
@@ -451,47 +559,6 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         }
       }
 
-      // ---- Phi_{T-1}: its pair, and its sources grouped by target (increasing j)
-      {
-        int *cnt = reinterpret_cast<int *>(ws + kScrCnt);
-        int *cntlo = reinterpret_cast<int *>(ws + kScrCntLo);
-        int *offs = reinterpret_cast<int *>(ws + kScrOffs);
-        reinterpret_cast<int *>(op + kOffPhiIdx)[j0] = i0;
-        reinterpret_cast<int *>(op + kOffPhiIdx)[j1] = i1;
-        reinterpret_cast<float *>(op + kOffPhiVal)[j0] = v0;
-        reinterpret_cast<float *>(op + kOffPhiVal)[j1] = v1;
-        cnt[j0] = 0;
-        cnt[j1] = 0;
-        cntlo[j0] = 0;
-        cntlo[j1] = 0;
-        __syncwarp();
-        atomicAdd(&cnt[i0], 1);
-        atomicAdd(&cntlo[i0], 1);
-        atomicAdd(&cnt[i1], 1);
-        __syncwarp();
-        const int ca = cnt[2 * lane], cb = cnt[2 * lane + 1];
-        int incl = ca + cb;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int n = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += n;
-        }
-        const int excl = incl - ca - cb;
-        offs[2 * lane] = excl;
-        offs[2 * lane + 1] = excl + ca;
-        __syncwarp();
-        const unsigned lt = (1u << lane) - 1u;
-        const unsigned mm0 = __match_any_sync(0xffffffffu, i0);
-        const unsigned mm1 = __match_any_sync(0xffffffffu, i1);
-        const int pos0 = offs[i0] + __popc(mm0 & lt);
-        const int pos1 = offs[i1] + cntlo[i1] + __popc(mm1 & lt);
-        int *meta = reinterpret_cast<int *>(op + kOffCsrMeta);
-        float *cnu = reinterpret_cast<float *>(op + kOffCsrNu);
-        meta[pos0] = j0 | (i0 << 8) | ((pos0 == offs[i0]) << 16) | ((pos0 == offs[i0] + cnt[i0] - 1) << 17);
-        cnu[pos0] = v0;
-        meta[pos1] = j1 | (i1 << 8) | ((pos1 == offs[i1]) << 16) | ((pos1 == offs[i1] + cnt[i1] - 1) << 17);
-        cnu[pos1] = v1;
-      }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->full[warp]);
@@ -554,13 +621,17 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     bool ok = true;
     if (issuer && nsub > 0) ok = issue_u(0);
     __syncwarp();
-    // S_0 = h0 (or 0) and its tf32 low part
-    {
+    // S_0 = h0 (or 0) in the source order of sub-chunk 0's composite, and its tf32 low part
+    if (nsub > 0 && !wait_bar_warp(bars, &bars->full[0], 0, a.err)) ok = false;
+    if (__all_sync(0xffffffffu, ok)) {
+      const int *src0 = reinterpret_cast<const int *>(op_base + kOffSrc);
       float v[16];
       for (int c0 = 0; c0 < kN; c0 += 16) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          v[i] = (act && a.h0) ? a.h0[((b * a.H + h) * kN + c0 + i) * kP + p] : 0.f;
+        for (int i = 0; i < 16; ++i) {
+          const int row = nsub > 0 ? src0[c0 + i] : c0 + i;
+          v[i] = (act && a.h0) ? a.h0[((b * a.H + h) * kN + row) * kP + p] : 0.f;
+        }
         tmem_st16(tbase + lanebase + kColState0 + c0, v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] -= tf32_trunc(v[i]);
@@ -586,8 +657,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       tc_fence_after();
       const uint32_t RS = tbase + lanebase + kColState0 + (sub & 1) * 64;
       const uint32_t RU = tbase + lanebase + kColState0 + ((sub + 1) & 1) * 64;
-      const int4 *meta4 = reinterpret_cast<const int4 *>(op + kOffCsrMeta);
-      const float4 *nu4 = reinterpret_cast<const float4 *>(op + kOffCsrNu);
+      const int4 *meta4 = reinterpret_cast<const int4 *>(op + kOffMeta);
+      const float4 *nu4 = reinterpret_cast<const float4 *>(op + kOffNu);
       // running whole-sequence product (warp 4 keeps it; sub-chunks arrive in order)
       if (q == 0) {
         const int *pi = reinterpret_cast<const int *>(op + kOffPhiIdx);
@@ -597,7 +668,9 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         pidx0 = pi[pidx0];
         pidx1 = pi[pidx1];
       }
-      // S_{a+1}[i] = U[i] + sum_{j: Phi[j] = i} nu_j S_a[j], in place over U
+      // S_{a+1}[i] = U[i] + sum_{j: Phi[j] = i} nu_j S_a[j], in place over U: the
+      // sources of a target are adjacent in S_a, so a segmented sum over the
+      // positions yields each target's total at its group's last position
       float run = 0.f;
 #pragma unroll
       for (int part = 0; part < 4; ++part) {
@@ -610,17 +683,16 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           mt[4 * r4 + 0] = m4.x; mt[4 * r4 + 1] = m4.y; mt[4 * r4 + 2] = m4.z; mt[4 * r4 + 3] = m4.w;
           nu[4 * r4 + 0] = n4.x; nu[4 * r4 + 1] = n4.y; nu[4 * r4 + 2] = n4.z; nu[4 * r4 + 3] = n4.w;
         }
+        tmem_ld16(RS + 16 * part, v);
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          tmem_ld1(RS + (mt[r] & 0xff), v[r]);
-          if (mt[r] & (1 << 16)) tmem_ld1(RU + ((mt[r] >> 8) & 0xff), u[r]);
-        }
+        for (int r = 0; r < 16; ++r)
+          if (mt[r] & kMetaEnd) tmem_ld1(RU + (mt[r] & 0xff), u[r]);
         tmem_wait_ld();
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-          if (mt[r] & (1 << 16)) run = u[r];
+          run = (mt[r] & kMetaKeep) ? run : 0.f;
           run = fmaf(nu[r], v[r], run);
-          if (mt[r] & (1 << 17)) tmem_st1(RU + ((mt[r] >> 8) & 0xff), run);
+          if (mt[r] & kMetaEnd) tmem_st1(RU + (mt[r] & 0xff), u[r] + run);
         }
       }
       tmem_wait_st();
@@ -742,6 +814,7 @@ cudaError_t launch_fused_scan(const ScanArgs &s, cudaStream_t st) {
   // input stage
   int o = 0;
   a.in.logits = o; o += s.logits ? kT * a.K * a.logit_size : 0; o = (o + 127) & ~127;
+  a.in.nlogits = o; o += s.logits ? kT * a.K * a.logit_size : 0; o = (o + 127) & ~127;
   a.in.d = o; o += kT * kN * 2;
   a.in.B = o; o += kT * kN * 2;
   a.in.C = o; o += kT * kN * 2;
