@@ -22,10 +22,14 @@
 // Only S_{a+1} depends on S_a through a sparse map; everything else is dense:
 //   U^T   = X^T Bh        (64 x 64, K = 16)  bf16 x bf16 (X exact, Bh = hi + lo)
 //   Y^T   = X^T G^T       (64 x 16, K = 16)  bf16 x bf16 (G = hi + lo)
-//   Y^T  += S^T Ct^T      (64 x 16, K = 64)  tf32, S and Ct split hi + lo
-// The tensor core truncates fp32 to tf32 (checked on B200), so with
-// S_lo = S - trunc_tf32(S) the three products hi*hi + hi*lo + lo*hi carry
-// about 21 bits. No N x N matrix is formed.
+//   Y^T  += S^T Ct^T      (64 x 16, K = 64)  tf32 (S read from tensor memory)
+// The tensor core reads S as tf32 (it drops the low 13 mantissa bits). The
+// readout precision follows the output type:
+//   bf16 y: Ct rounded to tf32, one product, relative error below 2^-10 per
+//           term (the rounding of y to bf16 is 2^-9);
+//   fp32 y: S_lo = S - tf32(S) kept in tensor memory and Ct split hi + lo, three
+//           products hi*hi + hi*lo + lo*hi, about 21 bits.
+// The state itself is accumulated in fp32. No N x N matrix is formed.
 //
 // State order. S_a lives in tensor memory with its rows in the source order of
 // Phi_{T-1} of sub-chunk a: sources grouped by target row, increasing source
@@ -35,11 +39,16 @@
 // writes Bh (hence U and S_{a+1}) in sub-chunk a+1's order and Ct in its own.
 // The state after the last sub-chunk is in natural order.
 //
+// Tensor memory holds a ring of 64-column state regions (S_a in region a mod R;
+// U_a, the input term of S_{a+1}, is accumulated into region (a+1) mod R ahead
+// of time) and four 16-column output slots. R = 3 for bf16 output; for fp32
+// output R = 2 and the third region holds S_lo.
+//
 // Roles (256 threads): warps 0-3 each prepare every fourth sub-chunk's
 // operands; warps 4-7 (one per tensor-memory quarter) advance the carry state
-// and write y, and one thread of warp 4 issues the MMAs. Every wait is bounded; a timeout sets an error
-// bit, makes every role leave its loop, drains outstanding MMAs and copies,
-// and frees tensor memory.
+// and write y, and one thread of warp 4 issues the MMAs. Every wait is
+// bounded; a timeout sets an error bit, makes every role leave its loop,
+// drains outstanding MMAs and copies, and frees tensor memory.
 #include <algorithm>
 
 #include "launch.h"
@@ -60,26 +69,32 @@ constexpr int kNY = 4;   // output accumulator slots
 constexpr int kThreads = 256;  // 4 prep warps + 4 carry warps (warp 4 also issues the MMAs)
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
 
-// tensor-memory columns
-constexpr uint32_t kColState0 = 0;    // two 64-column state regions
-constexpr uint32_t kColSlo = 128;     // tf32 low part of the state read by the readout
-constexpr uint32_t kColY = 192;       // kNY slots of kT columns
+// tensor-memory columns: 64-column state regions (a ring of 3, or 2 plus S_lo
+// at column 128), then the output slots
+constexpr uint32_t kColSlo = 128;
+constexpr uint32_t kColY = 192;
 constexpr uint32_t kTmemCols = 256;
+__device__ __forceinline__ uint32_t col_state(int region) { return 64u * (uint32_t)region; }
 
-// operand stage layout (bytes)
-constexpr int kOffCtHi = 0;                   // tf32 K-major (n = tau, k = state position): 4 KB
-constexpr int kOffCtLo = kOffCtHi + 4096;
-constexpr int kOffBhHi = kOffCtLo + 4096;     // bf16 K-major (n = state position, k = sigma): 2 KB
-constexpr int kOffBhLo = kOffBhHi + 2048;
-constexpr int kOffGtHi = kOffBhLo + 2048;     // bf16 K-major (n = tau, k = sigma): 512 B
+// Operand stage layout (bytes). Strides are padded so that the prep warp's
+// stores of one column spread over all shared-memory banks.
+constexpr int kCtLbo = 144;                   // Ct, tf32 K-major (n = tau, k = position)
+constexpr int kCtSbo = 16 * kCtLbo;           //   2 row groups of 2304 B
+constexpr int kBhSbo = 144;                   // Bh, bf16 MN-major (n = position, k = sigma)
+constexpr int kBhLbo = 8 * kBhSbo;            //   2 k groups of 1152 B
+constexpr int kOffCt = 0;
+constexpr int kOffBhHi = kOffCt + 2 * kCtSbo;
+constexpr int kOffBhLo = kOffBhHi + 2 * kBhLbo;
+constexpr int kOffGtHi = kOffBhLo + 2 * kBhLbo;  // G^T, bf16 K-major (n = tau, k = sigma): 512 B
 constexpr int kOffGtLo = kOffGtHi + 512;
-constexpr int kOffX = kOffGtLo + 512;         // bf16 MN-major (mn = p, k = tau): 2 KB
-constexpr int kOffMeta = kOffX + 2048;        // int [N] by position: carry-step record (below)
-constexpr int kOffNu = kOffMeta + 256;        // float [N] by position: Phi_{T-1} value of the source
-constexpr int kOffPhiIdx = kOffNu + 256;      // int [N] by source row: Phi_{T-1} index
-constexpr int kOffPhiVal = kOffPhiIdx + 256;  // float [N] by source row: Phi_{T-1} value
-constexpr int kOffSrc = kOffPhiVal + 256;     // int [N] by position: source row
-constexpr int kOpStage = kOffSrc + 256;       // 16640 B
+constexpr int kOffX = kOffGtLo + 512;            // x, bf16 MN-major (mn = p, k = tau): 2 KB
+constexpr int kOffMeta = kOffX + 2048;           // int [N] by position: carry-step record (below)
+constexpr int kOffNu = kOffMeta + 256;           // float [N] by position: Phi_{T-1} value of the source
+constexpr int kOffPhiIdx = kOffNu + 256;         // int [N] by source row: Phi_{T-1} index
+constexpr int kOffPhiVal = kOffPhiIdx + 256;     // float [N] by source row: Phi_{T-1} value
+constexpr int kOffSrc = kOffPhiVal + 256;        // int [N] by position: source row
+constexpr int kOffCtLo = kOffSrc + 256;          // low part of Ct (fp32 output only), as kOffCt
+__host__ __device__ constexpr int op_stage_bytes(bool precise) { return kOffCtLo + (precise ? 2 * kCtSbo : 0); }
 
 // carry-step record of a position: the target's column in the next order, and
 // whether the position continues a target group (else it starts one) and ends it
@@ -119,7 +134,7 @@ struct FParams {
 
 struct Bars {
   uint64_t full[kNS], opfree[kNS], yfull[kNY], yfree[kNY];
-  uint64_t ufull, gdone, sready, slofree, drain;
+  uint64_t ufull[3], sready, slofree, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -153,13 +168,15 @@ __device__ __forceinline__ bool wait_bar_warp(Bars *bars, uint64_t *bar, uint32_
 
 __device__ __forceinline__ float tf32_trunc(float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); }
 
-__device__ __forceinline__ float ld_bf16(const uint8_t *base, int idx) {
-  return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[idx]);
+// fp32 -> tf32, round to nearest (ties away from zero), as a 32-bit pattern
+__device__ __forceinline__ float tf32_rn(float v) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(v));
+  return __uint_as_float(r);
 }
 
-template <typename TL>
-__device__ __forceinline__ float ld_logit(const uint8_t *base, int idx) {
-  return to_f32(reinterpret_cast<const TL *>(base)[idx]);
+__device__ __forceinline__ float ld_bf16(const uint8_t *base, int idx) {
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[idx]);
 }
 
 // 2^e as a float, e clamped to the normal range
@@ -169,13 +186,14 @@ __device__ __forceinline__ float exp2i(int e) {
 }
 
 // operand element offsets
-__device__ __forceinline__ int off_ct(int tau, int j) {  // tf32 K-major, SBO = (N/4)*128
-  return (tau & 7) * 16 + (tau >> 3) * 2048 + (j >> 2) * 128 + (j & 3) * 4;
+__device__ __forceinline__ int off_ct_pos(int pos) { return (pos >> 2) * kCtLbo + (pos & 3) * 4; }
+__device__ __forceinline__ int off_ct_tau(int tau) { return (tau & 7) * 16 + (tau >> 3) * kCtSbo; }
+__device__ __forceinline__ int off_bh(int pos, int sigma) {
+  return (sigma & 7) * 16 + (sigma >> 3) * kBhLbo + (pos >> 3) * kBhSbo + (pos & 7) * 2;
 }
-__device__ __forceinline__ int off_bh(int i, int sigma) {  // bf16 K-major, SBO = (T/8)*128
-  return (i & 7) * 16 + (i >> 3) * 256 + (sigma >> 3) * 128 + (sigma & 7) * 2;
+__device__ __forceinline__ int off_gt(int tau, int sigma) {  // SBO = 256, LBO = 128
+  return (tau & 7) * 16 + (tau >> 3) * 256 + (sigma >> 3) * 128 + (sigma & 7) * 2;
 }
-__device__ __forceinline__ int off_gt(int tau, int sigma) { return off_bh(tau, sigma); }
 
 __device__ __forceinline__ void store_out(float *p, float v) { *p = v; }
 __device__ __forceinline__ void store_out(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
@@ -196,55 +214,69 @@ __device__ __forceinline__ void load_inputs(const FParams &a, uint8_t *st, int64
   const int t0 = sub * kT;
   const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
   const int nnext = (int)(a.L - t0 - kT < kT ? (a.L - t0 - kT > 0 ? a.L - t0 - kT : 0) : kT);
-  const int lchunks = a.logits ? a.K * a.logit_size / 16 : 0;  // 16-byte chunks per logits row
-  const int per_tok = 2 * lchunks + 8 * 4;  // logits, next logits, and d, B, C, x rows of 128 B
-  for (int e = lane; e < kT * per_tok; e += 32) {
-    const int tau = e / per_tok, c = e % per_tok;
-    uint8_t *dst;
-    const uint8_t *src = nullptr;
-    const int64_t row = (b * a.L + t0 + tau) * a.H + h;
-    if (c < lchunks) {
-      dst = st + a.in.logits + (tau * lchunks + c) * 16;
-      if (tau < nvalid) src = static_cast<const uint8_t *>(a.logits) + (row * lchunks + c) * 16;
-    } else if (c < 2 * lchunks) {
-      const int cc = c - lchunks;
-      dst = st + a.in.nlogits + (tau * lchunks + cc) * 16;
-      if (tau < nnext)
-        src = static_cast<const uint8_t *>(a.logits) + ((row + (int64_t)kT * a.H) * lchunks + cc) * 16;
+  const int64_t row0 = (b * a.L + t0) * a.H + h;  // row of token t0 in [Bt][L][H]
+  // d, B, C, x: 16 rows of 128 B each (8 chunks of 16 B), 4 chunks per lane and array
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int e = lane + 32 * c;
+    const int tau = e >> 3, ch = e & 7;
+    const int64_t row = row0 + (int64_t)tau * a.H;
+    uint8_t *dd = st + a.in.d + tau * 128 + ch * 16;
+    uint8_t *db = st + a.in.B + tau * 128 + ch * 16;
+    uint8_t *dc = st + a.in.C + tau * 128 + ch * 16;
+    // x into the MN-major canonical layout: (tau%8)*16 + (tau/8)*1024 + (p/8)*128
+    uint8_t *dx = st + a.in.x + (tau & 7) * 16 + (tau >> 3) * 1024 + ch * 128;
+    if (tau < nvalid) {
+      cp_async16(dd, a.d + row * kN + ch * 8);
+      cp_async16(db, a.B + row * kN + ch * 8);
+      cp_async16(dc, a.C + row * kN + ch * 8);
+      cp_async16(dx, a.x + row * kP + ch * 8);
     } else {
-      const int cc = c - 2 * lchunks, which = cc >> 3, ch = cc & 7;
-      if (which < 3) {
-        const int off = which == 0 ? a.in.d : which == 1 ? a.in.B : a.in.C;
-        const __nv_bfloat16 *g = which == 0 ? a.d : which == 1 ? a.B : a.C;
-        dst = st + off + tau * 128 + ch * 16;
-        if (tau < nvalid) src = reinterpret_cast<const uint8_t *>(g + row * kN) + ch * 16;
-      } else {  // x into the MN-major canonical layout: (tau%8)*16 + (tau/8)*1024 + (p/8)*128
-        dst = st + a.in.x + (tau & 7) * 16 + (tau >> 3) * 1024 + ch * 128;
-        if (tau < nvalid) src = reinterpret_cast<const uint8_t *>(a.x + row * kP) + ch * 16;
-      }
+      const uint4 z = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4 *>(dd) = z;
+      *reinterpret_cast<uint4 *>(db) = z;
+      *reinterpret_cast<uint4 *>(dc) = z;
+      *reinterpret_cast<uint4 *>(dx) = z;
     }
-    if (src)
-      cp_async16(dst, src);
-    else
-      *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+  }
+  if (a.logits) {
+    const int lchunks = a.K * a.logit_size / 16;  // 16-byte chunks per logits row
+    const uint8_t *lg = static_cast<const uint8_t *>(a.logits);
+    for (int e = lane; e < 2 * kT * lchunks; e += 32) {
+      const int nx = e >= kT * lchunks;
+      const int f = e - nx * kT * lchunks;
+      const int tau = f / lchunks, c = f - tau * lchunks;
+      uint8_t *dst = st + (nx ? a.in.nlogits : a.in.logits) + f * 16;
+      if (tau < (nx ? nnext : nvalid))
+        cp_async16(dst, lg + ((row0 + (int64_t)(tau + nx * kT) * a.H) * lchunks + c) * 16);
+      else
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+    }
   }
 }
 
-// Hard selection of one token from its logits row (lowest k on ties, first NaN wins).
+// Hard selection of one token from its logits row: the largest value, the lowest
+// k among ties, and the first NaN if there is one. Reads 16-byte chunks.
 template <typename TL>
 __device__ __forceinline__ int argmax_row(const uint8_t *row, int K) {
-  float best = ld_logit<TL>(row, 0);
-  if (best != best) return 0;
-  int bi = 0;
-  for (int k = 1; k < K; ++k) {
-    const float v = ld_logit<TL>(row, k);
-    if (v != v) return k;
-    if (v > best) {
-      best = v;
-      bi = k;
+  constexpr int kPer = 16 / (int)sizeof(TL);
+  float best = 0.f;
+  int bi = 0, nan_at = -1;
+  for (int c = 0; c < K; c += kPer) {
+    const uint4 q = *reinterpret_cast<const uint4 *>(row + c * sizeof(TL));
+    const TL *e = reinterpret_cast<const TL *>(&q);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const float v = to_f32(e[u]);
+      const int k = c + u;
+      if (v != v && nan_at < 0) nan_at = k;
+      if (k == 0 || v > best) {
+        best = v;
+        bi = k;
+      }
     }
   }
-  return bi;
+  return nan_at >= 0 ? nan_at : bi;
 }
 
 // Positions of the 64 sources j0 = lane, j1 = lane + 32 of an index map when the
@@ -283,8 +315,10 @@ __device__ __forceinline__ void group_positions(int t0, int t1, uint8_t *ws, int
 
 // ------------------------------------------------------------- the kernel
 
-template <typename TL, typename TO>
+template <typename TL, typename TO, bool kPrecise>
 __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
+  constexpr int kRing = kPrecise ? 2 : 3;
+  constexpr int kOpStage = op_stage_bytes(kPrecise);
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t *in_base = smem + a.off_in;
   uint8_t *op_base = smem + a.off_op;
@@ -306,8 +340,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       mbar_init(&bars->yfull[i], 1);
       mbar_init(&bars->yfree[i], 4);
     }
-    mbar_init(&bars->ufull, 1);
-    mbar_init(&bars->gdone, 4);
+    for (int i = 0; i < 3; ++i) mbar_init(&bars->ufull[i], 1);
     mbar_init(&bars->sready, 4);
     mbar_init(&bars->slofree, 1);
     mbar_init(&bars->drain, 1);
@@ -352,26 +385,31 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       cp_async_wait<0>();
       __syncwarp();
 
-      // selections of this sub-chunk and of the next one, one lane per token
-      int s_lane = 0, sn_lane = 0;
-      if (!a.logits) {
-        if (lane < nvalid) s_lane = a.s_in[(b * a.L + t0 + lane) * a.H + h];
-        if (lane < nnext) sn_lane = a.s_in[(b * a.L + t0 + kT + lane) * a.H + h];
-        if (s_lane < 0 || s_lane >= a.K || sn_lane < 0 || sn_lane >= a.K) {
-          flag_error(a.err, kErrSRange);
-          if (s_lane < 0 || s_lane >= a.K) s_lane = 0;
-          if (sn_lane < 0 || sn_lane >= a.K) sn_lane = 0;
+      // selections: lanes 0-15 take this sub-chunk's tokens, lanes 16-31 the next one's
+      int s_lane = 0;
+      {
+        const int tok = lane & 15;
+        const bool nx = lane >= 16;
+        if (tok < (nx ? nnext : nvalid)) {
+          if (a.logits) {
+            s_lane = argmax_row<TL>(in + (nx ? a.in.nlogits : a.in.logits) + tok * a.K * a.logit_size, a.K);
+          } else {
+            s_lane = a.s_in[(b * a.L + t0 + (nx ? kT : 0) + tok) * a.H + h];
+            if (s_lane < 0 || s_lane >= a.K) {
+              flag_error(a.err, kErrSRange);
+              s_lane = 0;
+            }
+          }
+          if (!nx && a.s_out) a.s_out[(b * a.L + t0 + tok) * a.H + h] = s_lane;
         }
-      } else {
-        if (lane < nvalid) s_lane = argmax_row<TL>(in + a.in.logits + lane * a.K * a.logit_size, a.K);
-        if (lane < nnext) sn_lane = argmax_row<TL>(in + a.in.nlogits + lane * a.K * a.logit_size, a.K);
       }
-      if (lane < nvalid && a.s_out) a.s_out[(b * a.L + t0 + lane) * a.H + h] = s_lane;
 
-      // x into the operand stage (2 KB)
+      // x into the operand stage (2 KB); G^T cleared (entries above the diagonal stay 0)
 #pragma unroll
       for (int c = 0; c < 4; ++c)
         reinterpret_cast<uint4 *>(op + kOffX)[lane + 32 * c] = reinterpret_cast<const uint4 *>(in + a.in.x)[lane + 32 * c];
+      reinterpret_cast<uint4 *>(op + kOffGtHi)[lane] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4 *>(op + kOffGtHi)[lane + 32] = make_uint4(0, 0, 0, 0);
 
       const uint8_t *din = in + a.in.d, *Bin = in + a.in.B, *Cin = in + a.in.C;
 
@@ -380,85 +418,92 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       {
         int n0 = j0, n1 = j1;
         for (int tau = 0; tau < nnext; ++tau) {
-          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, sn_lane, tau) * kN;
+          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, 16 + tau) * kN;
           n0 = dk[n0];
           n1 = dk[n1];
         }
         group_positions(n0, n1, ws, lane, posB0, posB1);
       }
       __syncwarp();
-      // ---- this sub-chunk's composite Phi_{T-1} -> the order of S_a, target groups
-      int ia0 = j0, ia1 = j1;
-      float va0 = 1.f, va1 = 1.f;
-      for (int tau = 0; tau < nvalid; ++tau) {
-        const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
-        va0 *= ld_bf16(din, tau * kN + ia0);
-        va1 *= ld_bf16(din, tau * kN + ia1);
-        ia0 = dk[ia0];
-        ia1 = dk[ia1];
+
+      // ---- forward chain: Phi_tau and Ct_tau = Phi_tau^T C_tau (kept in registers
+      //      until the positions in S_a's order are known)
+      int i0 = j0, i1 = j1;
+      float v0 = 1.f, v1 = 1.f;
+      float ct0[kT], ct1[kT];
+#pragma unroll
+      for (int tau = 0; tau < kT; ++tau) {
+        const int s = __shfl_sync(0xffffffffu, s_lane, tau);
+        ct0[tau] = ct1[tau] = 0.f;
+        if (tau < nvalid) {
+          const uint8_t *dk = dict + s * kN;
+          v0 *= ld_bf16(din, tau * kN + i0);
+          v1 *= ld_bf16(din, tau * kN + i1);
+          i0 = dk[i0];
+          i1 = dk[i1];
+          ct0[tau] = v0 * ld_bf16(Cin, tau * kN + i0);
+          ct1[tau] = v1 * ld_bf16(Cin, tau * kN + i1);
+        }
       }
+      // ---- Phi_{T-1} = (i, v): positions of S_a's order and the carry-step records
       int posA0, posA1;
-      group_positions(ia0, ia1, ws, lane, posA0, posA1);
+      group_positions(i0, i1, ws, lane, posA0, posA1);
       {
         const int *cnt = reinterpret_cast<const int *>(ws + kScrCnt);
         const int *offs = reinterpret_cast<const int *>(ws + kScrOffs);
-        // the target's column in the next order: posB of row ia (held by lane ia & 31)
-        const int pb0a = __shfl_sync(0xffffffffu, posB0, ia0 & 31), pb0b = __shfl_sync(0xffffffffu, posB1, ia0 & 31);
-        const int pb1a = __shfl_sync(0xffffffffu, posB0, ia1 & 31), pb1b = __shfl_sync(0xffffffffu, posB1, ia1 & 31);
-        const int f0 = offs[ia0], f1 = offs[ia1];
+        // the target's column in the next order: posB of row i (held by lane i & 31)
+        const int pb0a = __shfl_sync(0xffffffffu, posB0, i0 & 31), pb0b = __shfl_sync(0xffffffffu, posB1, i0 & 31);
+        const int pb1a = __shfl_sync(0xffffffffu, posB0, i1 & 31), pb1b = __shfl_sync(0xffffffffu, posB1, i1 & 31);
+        const int f0 = offs[i0], f1 = offs[i1];
         int *meta = reinterpret_cast<int *>(op + kOffMeta);
-        meta[posA0] = (ia0 < 32 ? pb0a : pb0b) | (posA0 != f0 ? kMetaKeep : 0) |
-                      (posA0 == f0 + cnt[ia0] - 1 ? kMetaEnd : 0);
-        meta[posA1] = (ia1 < 32 ? pb1a : pb1b) | (posA1 != f1 ? kMetaKeep : 0) |
-                      (posA1 == f1 + cnt[ia1] - 1 ? kMetaEnd : 0);
-        reinterpret_cast<float *>(op + kOffNu)[posA0] = va0;
-        reinterpret_cast<float *>(op + kOffNu)[posA1] = va1;
+        meta[posA0] = (i0 < 32 ? pb0a : pb0b) | (posA0 != f0 ? kMetaKeep : 0) |
+                      (posA0 == f0 + cnt[i0] - 1 ? kMetaEnd : 0);
+        meta[posA1] = (i1 < 32 ? pb1a : pb1b) | (posA1 != f1 ? kMetaKeep : 0) |
+                      (posA1 == f1 + cnt[i1] - 1 ? kMetaEnd : 0);
+        reinterpret_cast<float *>(op + kOffNu)[posA0] = v0;
+        reinterpret_cast<float *>(op + kOffNu)[posA1] = v1;
         reinterpret_cast<int *>(op + kOffSrc)[posA0] = j0;
         reinterpret_cast<int *>(op + kOffSrc)[posA1] = j1;
-        reinterpret_cast<int *>(op + kOffPhiIdx)[j0] = ia0;
-        reinterpret_cast<int *>(op + kOffPhiIdx)[j1] = ia1;
-        reinterpret_cast<float *>(op + kOffPhiVal)[j0] = va0;
-        reinterpret_cast<float *>(op + kOffPhiVal)[j1] = va1;
+        reinterpret_cast<int *>(op + kOffPhiIdx)[j0] = i0;
+        reinterpret_cast<int *>(op + kOffPhiIdx)[j1] = i1;
+        reinterpret_cast<float *>(op + kOffPhiVal)[j0] = v0;
+        reinterpret_cast<float *>(op + kOffPhiVal)[j1] = v1;
+      }
+      {
+        const int o0 = kOffCt + off_ct_pos(posA0), o1 = kOffCt + off_ct_pos(posA1);
+#pragma unroll
+        for (int tau = 0; tau < kT; ++tau) {
+          float *c0p = reinterpret_cast<float *>(op + o0 + off_ct_tau(tau));
+          float *c1p = reinterpret_cast<float *>(op + o1 + off_ct_tau(tau));
+          if constexpr (kPrecise) {  // hi as fp32 (read as tf32), lo = the rest
+            const float h0 = tf32_trunc(ct0[tau]), h1 = tf32_trunc(ct1[tau]);
+            c0p[0] = ct0[tau];
+            c1p[0] = ct1[tau];
+            c0p[(kOffCtLo - kOffCt) / 4] = ct0[tau] - h0;
+            c1p[(kOffCtLo - kOffCt) / 4] = ct1[tau] - h1;
+          } else {
+            c0p[0] = tf32_rn(ct0[tau]);
+            c1p[0] = tf32_rn(ct1[tau]);
+          }
+        }
       }
 
-      // ---- three 16-step chains side by side: the prefix Phi_tau (forward), the
-      //      suffix Psi_sigma and the readouts R_sigma (both backward)
-      uint8_t *cthi = op + kOffCtHi, *ctlo = op + kOffCtLo;
-      int i0 = j0, i1 = j1;          // Phi_tau
-      float v0 = 1.f, v1 = 1.f;
+      // ---- backward: the suffix Psi_sigma with Bh_sigma = Psi_sigma B_sigma, and
+      //      the readouts R_sigma[j][tau] = (A_tau...A_{sigma+1})^T C_tau with
+      //      G[tau][sigma] = B_sigma . R_sigma[:, tau]
       int k0 = j0, k1 = j1;          // Psi_sigma
       float m0 = 1.f, m1 = 1.f;
-      float R0[kT], R1[kT];          // R_sigma[j][tau], tau >= sigma
+      float R0[kT], R1[kT];          // R_sigma[j][tau], zero for tau < sigma
 #pragma unroll
       for (int c = 0; c < kT; ++c) R0[c] = R1[c] = 0.f;
 
       for (int k = 0; k < kT; ++k) {
-        // ---- forward step tau = k: Ct_tau = Phi_tau^T C_tau at the source's position in S_a's order
-        {
-          const int tau = k;
-          float c0 = 0.f, c1 = 0.f;
-          if (tau < nvalid) {
-            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
-            v0 *= ld_bf16(din, tau * kN + i0);
-            v1 *= ld_bf16(din, tau * kN + i1);
-            i0 = dk[i0];
-            i1 = dk[i1];
-            c0 = v0 * ld_bf16(Cin, tau * kN + i0);
-            c1 = v1 * ld_bf16(Cin, tau * kN + i1);
-          }
-          const float h0 = tf32_trunc(c0), h1 = tf32_trunc(c1);
-          *reinterpret_cast<float *>(cthi + off_ct(tau, posA0)) = h0;
-          *reinterpret_cast<float *>(cthi + off_ct(tau, posA1)) = h1;
-          *reinterpret_cast<float *>(ctlo + off_ct(tau, posA0)) = c0 - h0;
-          *reinterpret_cast<float *>(ctlo + off_ct(tau, posA1)) = c1 - h1;
-        }
         const int sg = kT - 1 - k;
         const bool sv = sg < nvalid;
         const float bs0 = sv ? ld_bf16(Bin, sg * kN + j0) : 0.f;
         const float bs1 = sv ? ld_bf16(Bin, sg * kN + j1) : 0.f;
-        // ---- backward step sigma = sg: Bh_sigma = Psi_sigma B_sigma as an exact
-        //      fixed-point sum (integer adds are order-independent), written at
-        //      the target's position in S_{a+1}'s order
+        // ---- Bh_sigma as an exact fixed-point sum (integer adds are
+        //      order-independent), written at the target's position in S_{a+1}'s order
         {
           const float w0 = m0 * bs0, w1 = m1 * bs1;
           const unsigned mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(w0), fabsf(w1))));
@@ -490,71 +535,74 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
             m1 = (r1 < 32 ? mc : md) * d1;
           }
         }
-        // ---- readout step sigma = sg: R_sg = A_{sg+1}^T R_{sg+1} (tau > sg), R_sg[:, sg] = C_sg,
-        //      G[tau][sg] = sum_j B_sg[j] R_sg[j][tau]
-        {
-          if (sg + 1 < nvalid) {
-            const int s = __shfl_sync(0xffffffffu, s_lane, sg + 1);
-            const uint8_t *dk = dict + s * kN;
-            const int r0 = dk[j0], r1 = dk[j1];
-            const float d0 = ld_bf16(din, (sg + 1) * kN + j0), d1 = ld_bf16(din, (sg + 1) * kN + j1);
+        // ---- R_sg = A_{sg+1}^T R_{sg+1} for tau > sg (groups of four columns that are
+        //      all at or below sg are skipped), then R_sg[:, sg] = C_sg
+        if (sg + 1 < nvalid) {
+          const int s = __shfl_sync(0xffffffffu, s_lane, sg + 1);
+          const uint8_t *dk = dict + s * kN;
+          const int r0 = dk[j0], r1 = dk[j1];
+          const float d0 = ld_bf16(din, (sg + 1) * kN + j0), d1 = ld_bf16(din, (sg + 1) * kN + j1);
 #pragma unroll
-            for (int tau = 0; tau < kT; ++tau) {
-              if (tau > sg) {
+          for (int g4 = 0; g4 < kT / 4; ++g4) {
+            if (4 * g4 + 3 > sg) {
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int tau = 4 * g4 + c;
                 const float a0 = __shfl_sync(0xffffffffu, R0[tau], r0 & 31);
                 const float a1 = __shfl_sync(0xffffffffu, R1[tau], r0 & 31);
                 const float c0 = __shfl_sync(0xffffffffu, R0[tau], r1 & 31);
                 const float c1 = __shfl_sync(0xffffffffu, R1[tau], r1 & 31);
-                R0[tau] = d0 * (r0 < 32 ? a0 : a1);
-                R1[tau] = d1 * (r1 < 32 ? c0 : c1);
+                if (tau > sg) {
+                  R0[tau] = d0 * (r0 < 32 ? a0 : a1);
+                  R1[tau] = d1 * (r1 < 32 ? c0 : c1);
+                }
               }
             }
           }
-          if (sv) {
-            const float c0 = ld_bf16(Cin, sg * kN + j0), c1 = ld_bf16(Cin, sg * kN + j1);
+        }
+        if (sv) {
+          const float c0 = ld_bf16(Cin, sg * kN + j0), c1 = ld_bf16(Cin, sg * kN + j1);
 #pragma unroll
-            for (int tau = 0; tau < kT; ++tau)
-              if (tau == sg) {
-                R0[tau] = c0;
-                R1[tau] = c1;
-              }
+          for (int tau = 0; tau < kT; ++tau)
+            if (tau == sg) {
+              R0[tau] = c0;
+              R1[tau] = c1;
+            }
+        }
+        // ---- G[tau][sg] for tau in [8 * rnd, 8 * rnd + 8): partials (R is zero for
+        //      tau < sg), then a reduce-scatter of 8 values over 32 lanes; rounds
+        //      entirely below sg keep the cleared zeros
+#pragma unroll
+        for (int rnd = 0; rnd < 2; ++rnd) {
+          if (8 * rnd + 7 < sg) continue;
+          float g[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) g[c] = bs0 * R0[8 * rnd + c] + bs1 * R1[8 * rnd + c];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const bool upr = lane & 16;
+            const float send = upr ? g[c] : g[c + 4];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+            g[c] = (upr ? g[c + 4] : g[c]) + recv;
           }
-          // G[tau][sg] for tau in [8 * rnd, 8 * rnd + 8): partials, then a reduce-scatter
-          // of 8 values over 32 lanes (two rounds keep the register count down)
 #pragma unroll
-          for (int rnd = 0; rnd < 2; ++rnd) {
-            float g[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int tau = 8 * rnd + c;
-              g[c] = (tau >= sg) ? bs0 * R0[tau] + bs1 * R1[tau] : 0.f;
-            }
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const bool upr = lane & 16;
-              const float send = upr ? g[c] : g[c + 4];
-              const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-              g[c] = (upr ? g[c + 4] : g[c]) + recv;
-            }
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const bool upr = lane & 8;
-              const float send = upr ? g[c] : g[c + 2];
-              const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
-              g[c] = (upr ? g[c + 2] : g[c]) + recv;
-            }
-            {
-              const bool upr = lane & 4;
-              const float send = upr ? g[0] : g[1];
-              const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
-              g[0] = (upr ? g[1] : g[0]) + recv;
-            }
-            g[0] += __shfl_xor_sync(0xffffffffu, g[0], 2);
-            g[0] += __shfl_xor_sync(0xffffffffu, g[0], 1);
-            if ((lane & 3) == 0) {
-              const int tau = 8 * rnd + ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-              st_bf16_split(op + kOffGtHi, op + kOffGtLo, off_gt(tau, sg), g[0]);
-            }
+          for (int c = 0; c < 2; ++c) {
+            const bool upr = lane & 8;
+            const float send = upr ? g[c] : g[c + 2];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
+            g[c] = (upr ? g[c + 2] : g[c]) + recv;
+          }
+          {
+            const bool upr = lane & 4;
+            const float send = upr ? g[0] : g[1];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
+            g[0] = (upr ? g[1] : g[0]) + recv;
+          }
+          g[0] += __shfl_xor_sync(0xffffffffu, g[0], 2);
+          g[0] += __shfl_xor_sync(0xffffffffu, g[0], 1);
+          if ((lane & 3) == 0) {
+            const int tau = 8 * rnd + ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+            st_bf16_split(op + kOffGtHi, op + kOffGtLo, off_gt(tau, sg), g[0]);
           }
         }
       }
@@ -575,53 +623,55 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     const int p = 16 * q + lane;            // state column owned by this lane
     const uint32_t lanebase = (uint32_t)(32 * q) << 16;
     const bool issuer = (q == 0) && (lane == 0);
-    const uint32_t id_u = idesc_bf16_f32(64, kN, true, false);
+    const uint32_t id_u = idesc_bf16_f32(64, kN, true, true);
     const uint32_t id_g = idesc_bf16_f32(64, kT, true, false);
     const uint32_t id_c = idesc_tf32_f32(64, kT);
-    // U and the intra-sub-chunk part of Y: need the operands and a free state region
+    // U_sub into state region (sub + 1) mod R and the intra-sub-chunk part of
+    // Y_sub. The region held S_{sub+1-R}: callers issue this only after the carry
+    // step of sub-chunk sub+1-R is complete and its readout has been issued
+    // (tensor-core operations of one thread execute in issue order).
     auto issue_u = [&](int sub) -> bool {
       const int st = sub % kNS;
       if (!wait_bar(bars, &bars->full[st], (sub / kNS) & 1, a.err)) return false;
-      if (sub >= 1 && !wait_bar(bars, &bars->gdone, (sub - 1) & 1, a.err)) return false;
       if (sub >= kNY && !wait_bar(bars, &bars->yfree[sub % kNY], ((sub / kNY) - 1) & 1, a.err)) return false;
       tc_fence_after();
       const uint32_t op = smem_u32(op_base + st * kOpStage);
-      const uint32_t dU = tbase + kColState0 + ((sub + 1) & 1) * 64;
+      const uint32_t dU = tbase + col_state((sub + 1) % kRing);
       const uint32_t dY = tbase + kColY + (sub % kNY) * kT;
       const uint64_t ax = smem_desc(op + kOffX, (kP / 8) * 128, 128);
-      mma_bf16(dU, ax, smem_desc(op + kOffBhHi, 128, 256), id_u, 0);
-      mma_bf16(dU, ax, smem_desc(op + kOffBhLo, 128, 256), id_u, 1);
+      mma_bf16(dU, ax, smem_desc(op + kOffBhHi, kBhLbo, kBhSbo), id_u, 0);
+      mma_bf16(dU, ax, smem_desc(op + kOffBhLo, kBhLbo, kBhSbo), id_u, 1);
       mma_bf16(dY, ax, smem_desc(op + kOffGtHi, 128, 256), id_g, 0);
       mma_bf16(dY, ax, smem_desc(op + kOffGtLo, 128, 256), id_g, 1);
-      mma_commit(&bars->ufull);
+      mma_commit(&bars->ufull[(sub + 1) % kRing]);
       return true;
     };
-    // readout of the entering state S_sub: A operand from tensor memory, tf32 x3
+    // readout of the entering state S_sub: A operand from tensor memory (tf32)
     auto issue_y = [&](int sub) -> bool {
       const int st = sub % kNS;
       if (!wait_bar(bars, &bars->sready, sub & 1, a.err)) return false;
       tc_fence_after();
       const uint32_t op = smem_u32(op_base + st * kOpStage);
       const uint32_t dY = tbase + kColY + (sub % kNY) * kT;
-      const uint32_t aS = tbase + kColState0 + (sub & 1) * 64;
-      const uint32_t aL = tbase + kColSlo;
+      const uint32_t aS = tbase + col_state(sub % kRing);
 #pragma unroll
       for (int ks = 0; ks < kN / 8; ++ks) {
-        const uint64_t bhi = smem_desc(op + kOffCtHi + ks * 256, 128, 2048);
-        const uint64_t blo = smem_desc(op + kOffCtLo + ks * 256, 128, 2048);
+        const uint64_t bhi = smem_desc(op + kOffCt + ks * 2 * kCtLbo, kCtLbo, kCtSbo);
         mma_tf32_ts(dY, aS + ks * 8, bhi, id_c, 1);
-        mma_tf32_ts(dY, aS + ks * 8, blo, id_c, 1);
-        mma_tf32_ts(dY, aL + ks * 8, bhi, id_c, 1);
+        if constexpr (kPrecise) {
+          mma_tf32_ts(dY, aS + ks * 8, smem_desc(op + kOffCtLo + ks * 2 * kCtLbo, kCtLbo, kCtSbo), id_c, 1);
+          mma_tf32_ts(dY, tbase + kColSlo + ks * 8, bhi, id_c, 1);
+        }
       }
       mma_commit(&bars->yfull[sub % kNY]);
       mma_commit(&bars->opfree[st]);
-      mma_commit(&bars->slofree);
+      if constexpr (kPrecise) mma_commit(&bars->slofree);
       return true;
     };
     bool ok = true;
-    if (issuer && nsub > 0) ok = issue_u(0);
-    __syncwarp();
-    // S_0 = h0 (or 0) in the source order of sub-chunk 0's composite, and its tf32 low part
+    for (int u = 0; u + 1 < kRing; ++u)
+      if (issuer && ok && nsub > u) ok = issue_u(u);
+    // S_0 = h0 (or 0) in the source order of sub-chunk 0's composite
     if (nsub > 0 && !wait_bar_warp(bars, &bars->full[0], 0, a.err)) ok = false;
     if (__all_sync(0xffffffffu, ok)) {
       const int *src0 = reinterpret_cast<const int *>(op_base + kOffSrc);
@@ -632,10 +682,12 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           const int row = nsub > 0 ? src0[c0 + i] : c0 + i;
           v[i] = (act && a.h0) ? a.h0[((b * a.H + h) * kN + row) * kP + p] : 0.f;
         }
-        tmem_st16(tbase + lanebase + kColState0 + c0, v);
+        tmem_st16(tbase + lanebase + col_state(0) + c0, v);
+        if constexpr (kPrecise) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] -= tf32_trunc(v[i]);
-        tmem_st16(tbase + lanebase + kColSlo + c0, v);
+          for (int i = 0; i < 16; ++i) v[i] -= tf32_trunc(v[i]);
+          tmem_st16(tbase + lanebase + kColSlo + c0, v);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -652,11 +704,11 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       const uint8_t *op = op_base + st * kOpStage;
       const int t0 = sub * kT;
       const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
-      if (!wait_bar_warp(bars, &bars->ufull, sub & 1, a.err)) break;
+      if (!wait_bar_warp(bars, &bars->ufull[(sub + 1) % kRing], (sub / kRing) & 1, a.err)) break;
       if (!wait_bar_warp(bars, &bars->full[st], (sub / kNS) & 1, a.err)) break;
       tc_fence_after();
-      const uint32_t RS = tbase + lanebase + kColState0 + (sub & 1) * 64;
-      const uint32_t RU = tbase + lanebase + kColState0 + ((sub + 1) & 1) * 64;
+      const uint32_t RS = tbase + lanebase + col_state(sub % kRing);
+      const uint32_t RU = tbase + lanebase + col_state((sub + 1) % kRing);
       const int4 *meta4 = reinterpret_cast<const int4 *>(op + kOffMeta);
       const float4 *nu4 = reinterpret_cast<const float4 *>(op + kOffNu);
       // running whole-sequence product (warp 4 keeps it; sub-chunks arrive in order)
@@ -696,30 +748,33 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         }
       }
       tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->gdone);
-      if (issuer && sub + 1 < nsub) ok = issue_u(sub + 1);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      // tf32 low part of S_{a+1} for the next readout, once this readout is done
-      if (!wait_bar_warp(bars, &bars->slofree, sub & 1, a.err)) break;
-      tc_fence_after();
-      for (int c0 = 0; c0 < kN; c0 += 16) {
-        float v[16];
-        tmem_ld16(RU + c0, v);
-        tmem_wait_ld();
+      if constexpr (kPrecise) {
+        // tf32 low part of S_{a+1}, once the readout of S_a is done with the plane
+        if (!wait_bar_warp(bars, &bars->slofree, sub & 1, a.err)) break;
+        tc_fence_after();
+        for (int c0 = 0; c0 < kN; c0 += 16) {
+          float v[16];
+          tmem_ld16(RU + c0, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] -= tf32_trunc(v[i]);
-        tmem_st16(tbase + lanebase + kColSlo + c0, v);
+          for (int i = 0; i < 16; ++i) v[i] -= tf32_trunc(v[i]);
+          tmem_st16(tbase + lanebase + kColSlo + c0, v);
+        }
+        tmem_wait_st();
       }
-      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bars->sready);
         mbar_arrive(&bars->opfree[st]);
       }
-      if (issuer && sub + 1 < nsub) ok = issue_y(sub + 1);
+      // Next MMAs. The input part of Y_{sub+1} (written by issue_u, not
+      // accumulated) must be issued before its readout: with a ring of three it
+      // was issued one step earlier, with a ring of two it needs this carry step.
+      if (issuer && sub + 1 < nsub) {
+        if constexpr (kRing == 2) ok = wait_bar(bars, &bars->sready, (sub + 1) & 1, a.err) && issue_u(sub + 1);
+        if (ok) ok = issue_y(sub + 1);
+      }
       if (!__all_sync(0xffffffffu, ok)) break;
       // output of this sub-chunk
       if (!wait_bar_warp(bars, &bars->yfull[sub % kNY], (sub / kNY) & 1, a.err)) break;
@@ -737,6 +792,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->yfree[sub % kNY]);
+      if constexpr (kRing == 3)
+        if (issuer && sub + 2 < nsub) ok = issue_u(sub + 2);
     }
     const bool clean = !*(volatile int *)&bars->abort;
     if (q == 0 && clean) {
@@ -751,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       }
     }
     if (clean && a.h_final) {
-      const uint32_t RF = tbase + lanebase + kColState0 + (nsub & 1) * 64;
+      const uint32_t RF = tbase + lanebase + col_state(nsub % kRing);
       for (int c0 = 0; c0 < kN; c0 += 16) {
         float v[16];
         tmem_ld16(RF + c0, v);
@@ -821,8 +878,9 @@ cudaError_t launch_fused_scan(const ScanArgs &s, cudaStream_t st) {
   a.in.x = o; o += kT * kP * 2;
   a.in.bytes = (o + 127) & ~127;
   // smem
+  const bool precise = s.out_t != PDSSM_BF16;
   int off = 0;
-  a.off_op = off; off += kNS * kOpStage; off = (off + 1023) & ~1023;
+  a.off_op = off; off += kNS * op_stage_bytes(precise); off = (off + 1023) & ~1023;
   a.off_in = off; off += kNW * a.in.bytes;
   a.off_dict = off; off += (int)((s.K * kN + 127) & ~127);
   a.off_scr = off; off += kNW * kScrBytes;
@@ -831,10 +889,10 @@ cudaError_t launch_fused_scan(const ScanArgs &s, cudaStream_t st) {
 
   cudaError_t e;
   auto kern = (s.logits_t == PDSSM_BF16)
-                  ? (s.out_t == PDSSM_BF16 ? fused_scan_kernel<__nv_bfloat16, __nv_bfloat16>
-                                           : fused_scan_kernel<__nv_bfloat16, float>)
-                  : (s.out_t == PDSSM_BF16 ? fused_scan_kernel<float, __nv_bfloat16>
-                                           : fused_scan_kernel<float, float>);
+                  ? (precise ? fused_scan_kernel<__nv_bfloat16, float, true>
+                             : fused_scan_kernel<__nv_bfloat16, __nv_bfloat16, false>)
+                  : (precise ? fused_scan_kernel<float, float, true>
+                             : fused_scan_kernel<float, __nv_bfloat16, false>);
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, off);
   if (e != cudaSuccess) return e;
   if ((e = trace_before(st, "fused_scan")) != cudaSuccess) return e;
