@@ -64,7 +64,7 @@ constexpr int kN = 64;   // state rows
 constexpr int kP = 64;   // state columns
 constexpr int kT = 16;   // sub-chunk length
 constexpr int kNW = 4;   // prep warps; warp w prepares sub-chunks w, w + 4, ...
-constexpr int kNS = kNW; // operand stages (one per prep warp)
+constexpr int kMaxStages = 6;  // operand stages (sub-chunk a uses stage a mod nst, nst >= kNW)
 constexpr int kNY = 4;   // output accumulator slots
 constexpr int kThreads = 256;  // 4 prep warps + 4 carry warps (warp 4 also issues the MMAs)
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
@@ -129,11 +129,12 @@ struct FParams {
   int32_t *s_out;
   uint32_t *err;
   InLayout in;
+  int nst;  // operand stages
   int off_in, off_op, off_dict, off_scr, off_bar;
 };
 
 struct Bars {
-  uint64_t full[kNS], opfree[kNS], yfull[kNY], yfree[kNY];
+  uint64_t full[kMaxStages], opfree[kMaxStages], yfull[kNY], yfree[kNY];
   uint64_t ufull[3], sready, slofree, drain;
   uint32_t tmem_base;
   int abort;
@@ -332,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
 
   // ---- setup
   if (tid == 0) {
-    for (int i = 0; i < kNS; ++i) {
+    for (int i = 0; i < kMaxStages; ++i) {
       mbar_init(&bars->full[i], 1);
       mbar_init(&bars->opfree[i], 1 + 4);  // MMA commit + one arrival per carry warp
     }
@@ -366,10 +367,9 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
 
   if (warp < kNW) {
     // ================================================================ prep
-    // Warp w prepares sub-chunks w, w + kNW, ... into operand stage w. Lanes own
-    // rows j0 = lane and j1 = lane + 32.
+    // Warp w prepares sub-chunks w, w + kNW, ... (sub-chunk a into operand stage
+    // a mod nst). Lanes own rows j0 = lane and j1 = lane + 32.
     uint8_t *in = in_base + warp * a.in.bytes;
-    uint8_t *op = op_base + warp * kOpStage;
     uint8_t *ws = scr + warp * kScrBytes;
     int *bins = reinterpret_cast<int *>(ws + kScrBins);
     if (warp < nsub) load_inputs<TL>(a, in, b, h, warp, lane);
@@ -377,11 +377,13 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     bins[lane] = 0;
     bins[lane + 32] = 0;
     const int j0 = lane, j1 = lane + 32;
-    for (int sub = warp, use = 0; sub < nsub; sub += kNW, ++use) {
+    for (int sub = warp; sub < nsub; sub += kNW) {
+      const int stg = sub % a.nst;
+      uint8_t *op = op_base + stg * kOpStage;
       const int t0 = sub * kT;
       const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
       const int nnext = (int)(a.L - t0 - kT < kT ? (a.L - t0 - kT > 0 ? a.L - t0 - kT : 0) : kT);
-      if (!wait_bar_warp(bars, &bars->opfree[warp], (use & 1) ^ 1, a.err)) break;
+      if (!wait_bar_warp(bars, &bars->opfree[stg], ((sub / a.nst) & 1) ^ 1, a.err)) break;
       cp_async_wait<0>();
       __syncwarp();
 
@@ -609,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
 
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->full[warp]);
+      if (lane == 0) mbar_arrive(&bars->full[stg]);
       // prefetch this warp's next sub-chunk into its (now free) input stage
       const int nxt = sub + kNW;
       if (nxt < nsub) load_inputs<TL>(a, in, b, h, nxt, lane);
@@ -631,8 +633,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     // step of sub-chunk sub+1-R is complete and its readout has been issued
     // (tensor-core operations of one thread execute in issue order).
     auto issue_u = [&](int sub) -> bool {
-      const int st = sub % kNS;
-      if (!wait_bar(bars, &bars->full[st], (sub / kNS) & 1, a.err)) return false;
+      const int st = sub % a.nst;
+      if (!wait_bar(bars, &bars->full[st], (sub / a.nst) & 1, a.err)) return false;
       if (sub >= kNY && !wait_bar(bars, &bars->yfree[sub % kNY], ((sub / kNY) - 1) & 1, a.err)) return false;
       tc_fence_after();
       const uint32_t op = smem_u32(op_base + st * kOpStage);
@@ -648,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     };
     // readout of the entering state S_sub: A operand from tensor memory (tf32)
     auto issue_y = [&](int sub) -> bool {
-      const int st = sub % kNS;
+      const int st = sub % a.nst;
       if (!wait_bar(bars, &bars->sready, sub & 1, a.err)) return false;
       tc_fence_after();
       const uint32_t op = smem_u32(op_base + st * kOpStage);
@@ -668,9 +670,22 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       if constexpr (kPrecise) mma_commit(&bars->slofree);
       return true;
     };
+    // Input-term MMAs are issued ahead by the issuing thread: blocking only when
+    // the carry step or the readout about to be issued needs them, otherwise
+    // as soon as their operands are ready (checked without waiting).
+    int next_u = 0;
+    auto issue_us = [&](int upto, bool block) -> bool {
+      for (; next_u <= upto && next_u < nsub; ++next_u) {
+        if (!block) {
+          if (!mbar_try_wait(&bars->full[next_u % a.nst], (next_u / a.nst) & 1)) return true;
+          if (next_u >= kNY && !mbar_try_wait(&bars->yfree[next_u % kNY], ((next_u / kNY) - 1) & 1)) return true;
+        }
+        if (!issue_u(next_u)) return false;
+      }
+      return true;
+    };
     bool ok = true;
-    for (int u = 0; u + 1 < kRing; ++u)
-      if (issuer && ok && nsub > u) ok = issue_u(u);
+    if (issuer) ok = issue_us(0, true) && issue_us(kRing - 2, false);
     // S_0 = h0 (or 0) in the source order of sub-chunk 0's composite
     if (nsub > 0 && !wait_bar_warp(bars, &bars->full[0], 0, a.err)) ok = false;
     if (__all_sync(0xffffffffu, ok)) {
@@ -696,16 +711,26 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     }
     if (issuer && ok && nsub > 0) ok = issue_y(0);
     TO *yout = static_cast<TO *>(a.y);
-    int pidx0 = lane, pidx1 = lane + 32;
-    float pval0 = 1.f, pval1 = 1.f;
-    for (int sub = 0; sub < nsub; ++sub) {
-      if (!__all_sync(0xffffffffu, ok)) break;
-      const int st = sub % kNS;
-      const uint8_t *op = op_base + st * kOpStage;
+    // output rows of sub-chunk sub from its accumulator slot (already loaded)
+    auto store_y = [&](int sub, const float *v) {
       const int t0 = sub * kT;
       const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
+      if (act) {
+#pragma unroll
+        for (int tau = 0; tau < kT; ++tau)
+          if (tau < nvalid) store_out(yout + ((b * a.L + t0 + tau) * a.H + h) * kP + p, v[tau]);
+      }
+    };
+    int pidx0 = lane, pidx1 = lane + 32;
+    float pval0 = 1.f, pval1 = 1.f;
+    int done = 0;  // sub-chunks whose carry step completed
+    for (int sub = 0; sub < nsub; ++sub) {
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int st = sub % a.nst;
+      const uint8_t *op = op_base + st * kOpStage;
       if (!wait_bar_warp(bars, &bars->ufull[(sub + 1) % kRing], (sub / kRing) & 1, a.err)) break;
-      if (!wait_bar_warp(bars, &bars->full[st], (sub / kNS) & 1, a.err)) break;
+      if (!wait_bar_warp(bars, &bars->full[st], (sub / a.nst) & 1, a.err)) break;
+      if (sub > 0 && !wait_bar_warp(bars, &bars->yfull[(sub - 1) % kNY], ((sub - 1) / kNY) & 1, a.err)) break;
       tc_fence_after();
       const uint32_t RS = tbase + lanebase + col_state(sub % kRing);
       const uint32_t RU = tbase + lanebase + col_state((sub + 1) % kRing);
@@ -722,7 +747,9 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       }
       // S_{a+1}[i] = U[i] + sum_{j: Phi[j] = i} nu_j S_a[j], in place over U: the
       // sources of a target are adjacent in S_a, so a segmented sum over the
-      // positions yields each target's total at its group's last position
+      // positions yields each target's total at its group's last position. Four
+      // parts of 16 positions; the previous sub-chunk's output rides on the
+      // first part's tensor-memory round trip.
       float run = 0.f;
 #pragma unroll
       for (int part = 0; part < 4; ++part) {
@@ -731,15 +758,28 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
 #pragma unroll
         for (int r4 = 0; r4 < 4; ++r4) {
           const int4 m4 = meta4[4 * part + r4];
-          const float4 n4 = nu4[4 * part + r4];
           mt[4 * r4 + 0] = m4.x; mt[4 * r4 + 1] = m4.y; mt[4 * r4 + 2] = m4.z; mt[4 * r4 + 3] = m4.w;
-          nu[4 * r4 + 0] = n4.x; nu[4 * r4 + 1] = n4.y; nu[4 * r4 + 2] = n4.z; nu[4 * r4 + 3] = n4.w;
         }
         tmem_ld16(RS + 16 * part, v);
 #pragma unroll
         for (int r = 0; r < 16; ++r)
           if (mt[r] & kMetaEnd) tmem_ld1(RU + (mt[r] & 0xff), u[r]);
-        tmem_wait_ld();
+        if (part == 0 && sub > 0) {
+          float yv[16];
+          tmem_ld16(tbase + lanebase + kColY + ((sub - 1) % kNY) * kT, yv);
+          tmem_wait_ld();
+          store_y(sub - 1, yv);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->yfree[(sub - 1) % kNY]);
+        } else {
+          tmem_wait_ld();
+        }
+#pragma unroll
+        for (int r4 = 0; r4 < 4; ++r4) {
+          const float4 n4 = nu4[4 * part + r4];
+          nu[4 * r4 + 0] = n4.x; nu[4 * r4 + 1] = n4.y; nu[4 * r4 + 2] = n4.z; nu[4 * r4 + 3] = n4.w;
+        }
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
           run = (mt[r] & kMetaKeep) ? run : 0.f;
@@ -768,32 +808,22 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         mbar_arrive(&bars->sready);
         mbar_arrive(&bars->opfree[st]);
       }
-      // Next MMAs. The input part of Y_{sub+1} (written by issue_u, not
-      // accumulated) must be issued before its readout: with a ring of three it
-      // was issued one step earlier, with a ring of two it needs this carry step.
+      done = sub + 1;
+      // Next MMAs: the readout of S_{sub+1} once every quarter of it is complete.
+      // The input part of Y_{sub+1} (written, not accumulated) must precede it.
       if (issuer && sub + 1 < nsub) {
-        if constexpr (kRing == 2) ok = wait_bar(bars, &bars->sready, (sub + 1) & 1, a.err) && issue_u(sub + 1);
-        if (ok) ok = issue_y(sub + 1);
+        ok = wait_bar(bars, &bars->sready, (sub + 1) & 1, a.err) && issue_us(sub + 1, true) && issue_y(sub + 1) &&
+             issue_us(sub + kRing - 1, false);
       }
-      if (!__all_sync(0xffffffffu, ok)) break;
-      // output of this sub-chunk
-      if (!wait_bar_warp(bars, &bars->yfull[sub % kNY], (sub / kNY) & 1, a.err)) break;
+    }
+    // output of the last sub-chunk
+    if (__all_sync(0xffffffffu, ok) && done == nsub && nsub > 0 &&
+        wait_bar_warp(bars, &bars->yfull[(nsub - 1) % kNY], ((nsub - 1) / kNY) & 1, a.err)) {
       tc_fence_after();
-      {
-        float v[16];
-        tmem_ld16(tbase + lanebase + kColY + (sub % kNY) * kT, v);
-        tmem_wait_ld();
-        if (act) {
-#pragma unroll
-          for (int tau = 0; tau < kT; ++tau)
-            if (tau < nvalid) store_out(yout + ((b * a.L + t0 + tau) * a.H + h) * kP + p, v[tau]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->yfree[sub % kNY]);
-      if constexpr (kRing == 3)
-        if (issuer && sub + 2 < nsub) ok = issue_u(sub + 2);
+      float v[16];
+      tmem_ld16(tbase + lanebase + kColY + ((nsub - 1) % kNY) * kT, v);
+      tmem_wait_ld();
+      store_y(nsub - 1, v);
     }
     const bool clean = !*(volatile int *)&bars->abort;
     if (q == 0 && clean) {
@@ -878,14 +908,21 @@ cudaError_t launch_fused_scan(const ScanArgs &s, cudaStream_t st) {
   a.in.x = o; o += kT * kP * 2;
   a.in.bytes = (o + 127) & ~127;
   // smem
+  // As many operand stages as fit two CTAs per SM (at least one per prep warp).
   const bool precise = s.out_t != PDSSM_BF16;
+  constexpr int kTwoCtaBytes = 228 * 1024 / 2 - 1024;  // per-CTA share of an SM, less the reserved 1 KB
   int off = 0;
-  a.off_op = off; off += kNS * op_stage_bytes(precise); off = (off + 1023) & ~1023;
-  a.off_in = off; off += kNW * a.in.bytes;
-  a.off_dict = off; off += (int)((s.K * kN + 127) & ~127);
-  a.off_scr = off; off += kNW * kScrBytes;
-  off = (off + 127) & ~127;
-  a.off_bar = off; off += (int)sizeof(Bars);
+  for (a.nst = kMaxStages; a.nst >= kNW; --a.nst) {
+    off = 0;
+    a.off_op = off; off += a.nst * op_stage_bytes(precise); off = (off + 1023) & ~1023;
+    a.off_in = off; off += kNW * a.in.bytes;
+    a.off_dict = off; off += (int)((s.K * kN + 127) & ~127);
+    a.off_scr = off; off += kNW * kScrBytes;
+    off = (off + 127) & ~127;
+    a.off_bar = off; off += (int)sizeof(Bars);
+    if (off <= kTwoCtaBytes) break;
+  }
+  if (a.nst < kNW) a.nst = kNW;  // the last layout computed (nst = kNW) is kept
 
   cudaError_t e;
   auto kern = (s.logits_t == PDSSM_BF16)
