@@ -50,6 +50,7 @@
 // bounded; a timeout sets an error bit, makes every role leave its loop,
 // drains outstanding MMAs and copies, and frees tensor memory.
 #include <algorithm>
+#include <type_traits>
 
 #include "launch.h"
 #include "sm100.cuh"
@@ -102,11 +103,11 @@ constexpr int kMetaKeep = 1 << 8;
 constexpr int kMetaEnd = 1 << 9;
 
 // per-prep-warp scratch (bytes)
-constexpr int kScrBins = 0;                   // int [N] fixed-point accumulators
-constexpr int kScrCnt = 256;                  // int [N] sources per target
-constexpr int kScrCntLo = 512;                // int [N] sources j < 32 per target
-constexpr int kScrOffs = 768;                 // int [N] first position of each target's group
-constexpr int kScrBytes = 1024;
+constexpr int kScrBins = 0;                   // int [2][N] fixed-point accumulators (by sigma parity)
+constexpr int kScrCnt = 512;                  // int [N] sources per target
+constexpr int kScrCntLo = 768;                // int [N] sources j < 32 per target
+constexpr int kScrOffs = 1024;                // int [N] first position of each target's group
+constexpr int kScrBytes = 1280;
 
 // input stage layout: logits [T][K] raw, d/B/C [T][N] bf16, x canonical
 struct InLayout {
@@ -374,8 +375,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     int *bins = reinterpret_cast<int *>(ws + kScrBins);
     if (warp < nsub) load_inputs<TL>(a, in, b, h, warp, lane);
     cp_async_commit();
-    bins[lane] = 0;
-    bins[lane + 32] = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) bins[lane + 32 * c] = 0;
     const int j0 = lane, j1 = lane + 32;
     for (int sub = warp; sub < nsub; sub += kNW) {
       const int stg = sub % a.nst;
@@ -492,91 +493,75 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
 
       // ---- backward: the suffix Psi_sigma with Bh_sigma = Psi_sigma B_sigma, and
       //      the readouts R_sigma[j][tau] = (A_tau...A_{sigma+1})^T C_tau with
-      //      G[tau][sigma] = B_sigma . R_sigma[:, tau]
+      //      G[tau][sigma] = B_sigma . R_sigma[:, tau]. One step per sigma, without
+      //      branches: rows past the end of the sequence were zero-filled, so their
+      //      readout columns stay 0, and Psi treats those steps as the identity.
       int k0 = j0, k1 = j1;          // Psi_sigma
       float m0 = 1.f, m1 = 1.f;
       float R0[kT], R1[kT];          // R_sigma[j][tau], zero for tau < sigma
 #pragma unroll
       for (int c = 0; c < kT; ++c) R0[c] = R1[c] = 0.f;
 
-      for (int k = 0; k < kT; ++k) {
-        const int sg = kT - 1 - k;
+      // lo_c: readout columns [lo, T) can be nonzero (sigma >= lo)
+      auto bwd_step = [&](auto lo_c, int sg) {
+        constexpr int lo = decltype(lo_c)::value;
         const bool sv = sg < nvalid;
-        const float bs0 = sv ? ld_bf16(Bin, sg * kN + j0) : 0.f;
-        const float bs1 = sv ? ld_bf16(Bin, sg * kN + j1) : 0.f;
-        // ---- Bh_sigma as an exact fixed-point sum (integer adds are
-        //      order-independent), written at the target's position in S_{a+1}'s order
+        const float bs0 = ld_bf16(Bin, sg * kN + j0), bs1 = ld_bf16(Bin, sg * kN + j1);
+        // (1) Bh_sigma as an exact fixed-point sum: integer adds are
+        //     order-independent; they are read back at the end of the step
+        int *bn = bins + (sg & 1) * kN;
+        const float w0 = m0 * bs0, w1 = m1 * bs1;
+        const unsigned mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(w0), fabsf(w1))));
+        // |w| < 2^ex; 64 terms of magnitude < 2^24 stay below 2^30
+        const int ex = (int)((mb >> 23) & 0xff) - 126;
+        const int e = mb ? 24 - ex : 0;
+        const float up = exp2i(e), dn = exp2i(-e);
+        atomicAdd(&bn[k0], __float2int_rn(w0 * up));
+        atomicAdd(&bn[k1], __float2int_rn(w1 * up));
+        // (2) Psi_{sg-1} = Psi_sg A_sg: column j <- d[j] * column idx[j] (identity past the end)
         {
-          const float w0 = m0 * bs0, w1 = m1 * bs1;
-          const unsigned mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(w0), fabsf(w1))));
-          // |w| < 2^ex; 64 terms of magnitude < 2^24 stay below 2^30
-          const int ex = (int)((mb >> 23) & 0xff) - 126;
-          const int e = mb ? 24 - ex : 0;
-          const float up = exp2i(e), dn = exp2i(-e);
-          if (sv) {
-            atomicAdd(&bins[k0], __float2int_rn(w0 * up));
-            atomicAdd(&bins[k1], __float2int_rn(w1 * up));
-          }
-          __syncwarp();
-          const float bh0 = (float)bins[j0] * dn, bh1 = (float)bins[j1] * dn;
-          bins[j0] = 0;
-          bins[j1] = 0;
-          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB0, sg), bh0);
-          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB1, sg), bh1);
-          if (sv && sg > 0) {  // Psi_{sg-1} = Psi_sg A_sg: column j <- d[j] * column idx[j]
-            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, sg) * kN;
-            const int r0 = dk[j0], r1 = dk[j1];
-            const int ka = __shfl_sync(0xffffffffu, k0, r0 & 31), kb = __shfl_sync(0xffffffffu, k1, r0 & 31);
-            const float ma = __shfl_sync(0xffffffffu, m0, r0 & 31), mb2 = __shfl_sync(0xffffffffu, m1, r0 & 31);
-            const int kc = __shfl_sync(0xffffffffu, k0, r1 & 31), kd = __shfl_sync(0xffffffffu, k1, r1 & 31);
-            const float mc = __shfl_sync(0xffffffffu, m0, r1 & 31), md = __shfl_sync(0xffffffffu, m1, r1 & 31);
-            const float d0 = ld_bf16(din, sg * kN + j0), d1 = ld_bf16(din, sg * kN + j1);
-            k0 = r0 < 32 ? ka : kb;
-            m0 = (r0 < 32 ? ma : mb2) * d0;
-            k1 = r1 < 32 ? kc : kd;
-            m1 = (r1 < 32 ? mc : md) * d1;
-          }
+          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, sg) * kN;
+          const int r0 = sv ? dk[j0] : j0, r1 = sv ? dk[j1] : j1;
+          const float d0 = sv ? ld_bf16(din, sg * kN + j0) : 1.f, d1 = sv ? ld_bf16(din, sg * kN + j1) : 1.f;
+          const int ka = __shfl_sync(0xffffffffu, k0, r0 & 31), kb = __shfl_sync(0xffffffffu, k1, r0 & 31);
+          const float ma = __shfl_sync(0xffffffffu, m0, r0 & 31), mb2 = __shfl_sync(0xffffffffu, m1, r0 & 31);
+          const int kc = __shfl_sync(0xffffffffu, k0, r1 & 31), kd = __shfl_sync(0xffffffffu, k1, r1 & 31);
+          const float mc = __shfl_sync(0xffffffffu, m0, r1 & 31), md = __shfl_sync(0xffffffffu, m1, r1 & 31);
+          k0 = r0 < 32 ? ka : kb;
+          m0 = (r0 < 32 ? ma : mb2) * d0;
+          k1 = r1 < 32 ? kc : kd;
+          m1 = (r1 < 32 ? mc : md) * d1;
         }
-        // ---- R_sg = A_{sg+1}^T R_{sg+1} for tau > sg (groups of four columns that are
-        //      all at or below sg are skipped), then R_sg[:, sg] = C_sg
-        if (sg + 1 < nvalid) {
-          const int s = __shfl_sync(0xffffffffu, s_lane, sg + 1);
-          const uint8_t *dk = dict + s * kN;
+        // (3) R_sg = A_{sg+1}^T R_{sg+1} on the columns tau > sg
+        {
+          const int sn = sg + 1 < kT ? sg + 1 : sg;
+          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, sn) * kN;
           const int r0 = dk[j0], r1 = dk[j1];
-          const float d0 = ld_bf16(din, (sg + 1) * kN + j0), d1 = ld_bf16(din, (sg + 1) * kN + j1);
+          const float d0 = ld_bf16(din, sn * kN + j0), d1 = ld_bf16(din, sn * kN + j1);
 #pragma unroll
-          for (int g4 = 0; g4 < kT / 4; ++g4) {
-            if (4 * g4 + 3 > sg) {
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const int tau = 4 * g4 + c;
-                const float a0 = __shfl_sync(0xffffffffu, R0[tau], r0 & 31);
-                const float a1 = __shfl_sync(0xffffffffu, R1[tau], r0 & 31);
-                const float c0 = __shfl_sync(0xffffffffu, R0[tau], r1 & 31);
-                const float c1 = __shfl_sync(0xffffffffu, R1[tau], r1 & 31);
-                if (tau > sg) {
-                  R0[tau] = d0 * (r0 < 32 ? a0 : a1);
-                  R1[tau] = d1 * (r1 < 32 ? c0 : c1);
-                }
-              }
-            }
+          for (int tau = lo + 1; tau < kT; ++tau) {
+            const float a0 = __shfl_sync(0xffffffffu, R0[tau], r0 & 31);
+            const float a1 = __shfl_sync(0xffffffffu, R1[tau], r0 & 31);
+            const float c0 = __shfl_sync(0xffffffffu, R0[tau], r1 & 31);
+            const float c1 = __shfl_sync(0xffffffffu, R1[tau], r1 & 31);
+            const float n0 = d0 * (r0 < 32 ? a0 : a1), n1 = d1 * (r1 < 32 ? c0 : c1);
+            R0[tau] = tau > sg ? n0 : R0[tau];
+            R1[tau] = tau > sg ? n1 : R1[tau];
           }
         }
-        if (sv) {
+        // (4) R_sg[:, sg] = C_sg (sg is in [lo, lo + 8))
+        {
           const float c0 = ld_bf16(Cin, sg * kN + j0), c1 = ld_bf16(Cin, sg * kN + j1);
 #pragma unroll
-          for (int tau = 0; tau < kT; ++tau)
-            if (tau == sg) {
-              R0[tau] = c0;
-              R1[tau] = c1;
-            }
+          for (int tau = lo; tau < lo + 8; ++tau) {
+            R0[tau] = tau == sg ? c0 : R0[tau];
+            R1[tau] = tau == sg ? c1 : R1[tau];
+          }
         }
-        // ---- G[tau][sg] for tau in [8 * rnd, 8 * rnd + 8): partials (R is zero for
-        //      tau < sg), then a reduce-scatter of 8 values over 32 lanes; rounds
-        //      entirely below sg keep the cleared zeros
+        // (5) G[tau][sg] for tau in [8 * rnd, 8 * rnd + 8): partials (R is zero for
+        //     tau < sg), then a reduce-scatter of 8 values over 32 lanes
 #pragma unroll
-        for (int rnd = 0; rnd < 2; ++rnd) {
-          if (8 * rnd + 7 < sg) continue;
+        for (int rnd = lo / 8; rnd < 2; ++rnd) {
           float g[8];
 #pragma unroll
           for (int c = 0; c < 8; ++c) g[c] = bs0 * R0[8 * rnd + c] + bs1 * R1[8 * rnd + c];
@@ -607,7 +592,16 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
             st_bf16_split(op + kOffGtHi, op + kOffGtLo, off_gt(tau, sg), g[0]);
           }
         }
-      }
+        // (6) read back Bh_sg (the other parity's accumulators serve the next step)
+        __syncwarp();
+        const float bh0 = (float)bn[j0] * dn, bh1 = (float)bn[j1] * dn;
+        bn[j0] = 0;
+        bn[j1] = 0;
+        st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB0, sg), bh0);
+        st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB1, sg), bh1);
+      };
+      for (int sg = kT - 1; sg >= 8; --sg) bwd_step(std::integral_constant<int, 8>(), sg);
+      for (int sg = 7; sg >= 0; --sg) bwd_step(std::integral_constant<int, 0>(), sg);
 
       fence_proxy_async_smem();
       __syncwarp();
@@ -748,22 +742,21 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       // S_{a+1}[i] = U[i] + sum_{j: Phi[j] = i} nu_j S_a[j], in place over U: the
       // sources of a target are adjacent in S_a, so a segmented sum over the
       // positions yields each target's total at its group's last position. Four
-      // parts of 16 positions; the previous sub-chunk's output rides on the
-      // first part's tensor-memory round trip.
+      // parts of 16 positions, one tensor-memory round trip each (S_a and U at
+      // the group ends); the previous sub-chunk's output rides on the first.
       float run = 0.f;
 #pragma unroll
       for (int part = 0; part < 4; ++part) {
-        float v[16], u[16], nu[16];
-        int mt[16];
+        float v[16], u[16];
+        tmem_ld16(RS + 16 * part, v);
 #pragma unroll
         for (int r4 = 0; r4 < 4; ++r4) {
           const int4 m4 = meta4[4 * part + r4];
-          mt[4 * r4 + 0] = m4.x; mt[4 * r4 + 1] = m4.y; mt[4 * r4 + 2] = m4.z; mt[4 * r4 + 3] = m4.w;
-        }
-        tmem_ld16(RS + 16 * part, v);
+          const int mt[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-        for (int r = 0; r < 16; ++r)
-          if (mt[r] & kMetaEnd) tmem_ld1(RU + (mt[r] & 0xff), u[r]);
+          for (int c = 0; c < 4; ++c)
+            if (mt[c] & kMetaEnd) tmem_ld1(RU + (mt[c] & 0xff), u[4 * r4 + c]);
+        }
         if (part == 0 && sub > 0) {
           float yv[16];
           tmem_ld16(tbase + lanebase + kColY + ((sub - 1) % kNY) * kT, yv);
@@ -777,14 +770,16 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         }
 #pragma unroll
         for (int r4 = 0; r4 < 4; ++r4) {
+          const int4 m4 = meta4[4 * part + r4];
           const float4 n4 = nu4[4 * part + r4];
-          nu[4 * r4 + 0] = n4.x; nu[4 * r4 + 1] = n4.y; nu[4 * r4 + 2] = n4.z; nu[4 * r4 + 3] = n4.w;
-        }
+          const int mt[4] = {m4.x, m4.y, m4.z, m4.w};
+          const float nu[4] = {n4.x, n4.y, n4.z, n4.w};
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          run = (mt[r] & kMetaKeep) ? run : 0.f;
-          run = fmaf(nu[r], v[r], run);
-          if (mt[r] & kMetaEnd) tmem_st1(RU + (mt[r] & 0xff), u[r] + run);
+          for (int c = 0; c < 4; ++c) {
+            run = (mt[c] & kMetaKeep) ? run : 0.f;
+            run = fmaf(nu[c], v[4 * r4 + c], run);
+            if (mt[c] & kMetaEnd) tmem_st1(RU + (mt[c] & 0xff), u[4 * r4 + c] + run);
+          }
         }
       }
       tmem_wait_st();
