@@ -148,7 +148,7 @@ __device__ __forceinline__ uint64_t now_ns() {
 }
 
 // Bounded wait shared by every role: false (and the abort flag set) on timeout.
-__device__ __forceinline__ bool wait_bar(Bars *bars, uint64_t *bar, uint32_t parity, uint32_t *err) {
+__device__ __noinline__ bool wait_bar(Bars *bars, uint64_t *bar, uint32_t parity, uint32_t *err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = now_ns();
   while (true) {
@@ -217,22 +217,26 @@ __device__ __forceinline__ void load_inputs(const FParams &a, uint8_t *st, int64
   const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
   const int nnext = (int)(a.L - t0 - kT < kT ? (a.L - t0 - kT > 0 ? a.L - t0 - kT : 0) : kT);
   const int64_t row0 = (b * a.L + t0) * a.H + h;  // row of token t0 in [Bt][L][H]
-  // d, B, C, x: 16 rows of 128 B each (8 chunks of 16 B), 4 chunks per lane and array
+  // d, B, C, x: 16 rows of 128 B (8 chunks of 16 B); lane takes chunk lane % 8 of
+  // rows lane / 8 + 4c, c = 0..3
+  const int ch = lane & 7, tau0 = lane >> 3;
+  const int64_t e0 = (row0 + (int64_t)tau0 * a.H) * kN + ch * 8;  // element offset of (tau0, ch)
+  const int64_t estep = (int64_t)4 * a.H * kN;                    // 4 rows further
+  const int so = tau0 * 128 + ch * 16;                            // row-major stage offset
+  const int sx = (tau0 & 7) * 16 + ch * 128;                      // x: (tau%8)*16 + (tau/8)*1024 + (p/8)*128
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    const int e = lane + 32 * c;
-    const int tau = e >> 3, ch = e & 7;
-    const int64_t row = row0 + (int64_t)tau * a.H;
-    uint8_t *dd = st + a.in.d + tau * 128 + ch * 16;
-    uint8_t *db = st + a.in.B + tau * 128 + ch * 16;
-    uint8_t *dc = st + a.in.C + tau * 128 + ch * 16;
-    // x into the MN-major canonical layout: (tau%8)*16 + (tau/8)*1024 + (p/8)*128
-    uint8_t *dx = st + a.in.x + (tau & 7) * 16 + (tau >> 3) * 1024 + ch * 128;
+    const int tau = tau0 + 4 * c;
+    const int64_t ge = e0 + c * estep;
+    uint8_t *dd = st + a.in.d + so + c * 512;
+    uint8_t *db = st + a.in.B + so + c * 512;
+    uint8_t *dc = st + a.in.C + so + c * 512;
+    uint8_t *dx = st + a.in.x + sx + ((tau0 + 4 * c) >> 3) * 1024 + ((4 * c) & 7) * 16;
     if (tau < nvalid) {
-      cp_async16(dd, a.d + row * kN + ch * 8);
-      cp_async16(db, a.B + row * kN + ch * 8);
-      cp_async16(dc, a.C + row * kN + ch * 8);
-      cp_async16(dx, a.x + row * kP + ch * 8);
+      cp_async16(dd, a.d + ge);
+      cp_async16(db, a.B + ge);
+      cp_async16(dc, a.C + ge);
+      cp_async16(dx, a.x + ge);  // P == N
     } else {
       const uint4 z = make_uint4(0, 0, 0, 0);
       *reinterpret_cast<uint4 *>(dd) = z;
@@ -244,6 +248,7 @@ __device__ __forceinline__ void load_inputs(const FParams &a, uint8_t *st, int64
   if (a.logits) {
     const int lchunks = a.K * a.logit_size / 16;  // 16-byte chunks per logits row
     const uint8_t *lg = static_cast<const uint8_t *>(a.logits);
+#pragma unroll 1
     for (int e = lane; e < 2 * kT * lchunks; e += 32) {
       const int nx = e >= kT * lchunks;
       const int f = e - nx * kT * lchunks;
@@ -313,6 +318,63 @@ __device__ __forceinline__ void group_positions(int t0, int t1, uint8_t *ws, int
   const unsigned m1 = __match_any_sync(0xffffffffu, t1);
   pos0 = offs[t0] + __popc(m0 & lt);
   pos1 = offs[t1] + cntlo[t1] + __popc(m1 & lt);
+}
+
+// ------------------------------------------------------------- MMA issue
+
+// U_sub into state region (sub + 1) mod R and the intra-sub-chunk part of Y_sub
+// (written, not accumulated). The region held S_{sub+1-R}: callers issue this
+// only after the carry step of sub-chunk sub+1-R is complete and its readout
+// has been issued (tensor-core operations of one thread execute in issue order).
+// One thread; false after a timeout.
+template <bool kPrecise>
+__device__ __noinline__ bool issue_input_mma(Bars *bars, uint32_t op_base, int nst, uint32_t tbase, int sub,
+                                             uint32_t *err) {
+  constexpr int kRing = kPrecise ? 2 : 3;
+  const int st = sub % nst;
+  if (!wait_bar(bars, &bars->full[st], (sub / nst) & 1, err)) return false;
+  if (sub >= kNY && !wait_bar(bars, &bars->yfree[sub % kNY], ((sub / kNY) - 1) & 1, err)) return false;
+  tc_fence_after();
+  const uint32_t op = op_base + st * op_stage_bytes(kPrecise);
+  const uint32_t dU = tbase + col_state((sub + 1) % kRing);
+  const uint32_t dY = tbase + kColY + (sub % kNY) * kT;
+  const uint32_t id_u = idesc_bf16_f32(64, kN, true, true);
+  const uint32_t id_g = idesc_bf16_f32(64, kT, true, false);
+  const uint64_t ax = smem_desc(op + kOffX, (kP / 8) * 128, 128);
+  mma_bf16(dU, ax, smem_desc(op + kOffBhHi, kBhLbo, kBhSbo), id_u, 0);
+  mma_bf16(dU, ax, smem_desc(op + kOffBhLo, kBhLbo, kBhSbo), id_u, 1);
+  mma_bf16(dY, ax, smem_desc(op + kOffGtHi, 128, 256), id_g, 0);
+  mma_bf16(dY, ax, smem_desc(op + kOffGtLo, 128, 256), id_g, 1);
+  mma_commit(&bars->ufull[(sub + 1) % kRing]);
+  return true;
+}
+
+// Readout of the entering state S_sub into Y_sub: A operand from tensor memory
+// (tf32). Releases the operand stage (and the S_lo plane) when done.
+template <bool kPrecise>
+__device__ __noinline__ bool issue_readout_mma(Bars *bars, uint32_t op_base, int nst, uint32_t tbase, int sub,
+                                               uint32_t *err) {
+  constexpr int kRing = kPrecise ? 2 : 3;
+  const int st = sub % nst;
+  if (!wait_bar(bars, &bars->sready, sub & 1, err)) return false;
+  tc_fence_after();
+  const uint32_t op = op_base + st * op_stage_bytes(kPrecise);
+  const uint32_t dY = tbase + kColY + (sub % kNY) * kT;
+  const uint32_t aS = tbase + col_state(sub % kRing);
+  const uint32_t id_c = idesc_tf32_f32(64, kT);
+#pragma unroll 1
+  for (int ks = 0; ks < kN / 8; ++ks) {
+    const uint64_t bhi = smem_desc(op + kOffCt + ks * 2 * kCtLbo, kCtLbo, kCtSbo);
+    mma_tf32_ts(dY, aS + ks * 8, bhi, id_c, 1);
+    if constexpr (kPrecise) {
+      mma_tf32_ts(dY, aS + ks * 8, smem_desc(op + kOffCtLo + ks * 2 * kCtLbo, kCtLbo, kCtSbo), id_c, 1);
+      mma_tf32_ts(dY, tbase + kColSlo + ks * 8, bhi, id_c, 1);
+    }
+  }
+  mma_commit(&bars->yfull[sub % kNY]);
+  mma_commit(&bars->opfree[st]);
+  if constexpr (kPrecise) mma_commit(&bars->slofree);
+  return true;
 }
 
 // ------------------------------------------------------------- the kernel
@@ -429,28 +491,45 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       }
       __syncwarp();
 
-      // ---- forward chain: Phi_tau and Ct_tau = Phi_tau^T C_tau (kept in registers
-      //      until the positions in S_a's order are known)
-      int i0 = j0, i1 = j1;
+      // ---- Phi_{T-1} (indices): the positions of S_a's order
+      int posA0, posA1, i0 = j0, i1 = j1;
+      for (int tau = 0; tau < nvalid; ++tau) {
+        const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
+        i0 = dk[i0];
+        i1 = dk[i1];
+      }
+      group_positions(i0, i1, ws, lane, posA0, posA1);
+      // ---- forward chain: Phi_tau and Ct_tau = Phi_tau^T C_tau at the positions of S_a's order
       float v0 = 1.f, v1 = 1.f;
-      float ct0[kT], ct1[kT];
-#pragma unroll
-      for (int tau = 0; tau < kT; ++tau) {
-        const int s = __shfl_sync(0xffffffffu, s_lane, tau);
-        ct0[tau] = ct1[tau] = 0.f;
-        if (tau < nvalid) {
-          const uint8_t *dk = dict + s * kN;
-          v0 *= ld_bf16(din, tau * kN + i0);
-          v1 *= ld_bf16(din, tau * kN + i1);
-          i0 = dk[i0];
-          i1 = dk[i1];
-          ct0[tau] = v0 * ld_bf16(Cin, tau * kN + i0);
-          ct1[tau] = v1 * ld_bf16(Cin, tau * kN + i1);
+      {
+        const int o0 = kOffCt + off_ct_pos(posA0), o1 = kOffCt + off_ct_pos(posA1);
+        int f0 = j0, f1 = j1;
+#pragma unroll 1
+        for (int tau = 0; tau < kT; ++tau) {
+          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
+          float c0 = 0.f, c1 = 0.f;
+          if (tau < nvalid) {
+            v0 *= ld_bf16(din, tau * kN + f0);
+            v1 *= ld_bf16(din, tau * kN + f1);
+            f0 = dk[f0];
+            f1 = dk[f1];
+            c0 = v0 * ld_bf16(Cin, tau * kN + f0);
+            c1 = v1 * ld_bf16(Cin, tau * kN + f1);
+          }
+          float *c0p = reinterpret_cast<float *>(op + o0 + off_ct_tau(tau));
+          float *c1p = reinterpret_cast<float *>(op + o1 + off_ct_tau(tau));
+          if constexpr (kPrecise) {  // hi as fp32 (read as tf32), lo = the rest
+            c0p[0] = c0;
+            c1p[0] = c1;
+            c0p[(kOffCtLo - kOffCt) / 4] = c0 - tf32_trunc(c0);
+            c1p[(kOffCtLo - kOffCt) / 4] = c1 - tf32_trunc(c1);
+          } else {
+            c0p[0] = tf32_rn(c0);
+            c1p[0] = tf32_rn(c1);
+          }
         }
       }
-      // ---- Phi_{T-1} = (i, v): positions of S_a's order and the carry-step records
-      int posA0, posA1;
-      group_positions(i0, i1, ws, lane, posA0, posA1);
+      // ---- Phi_{T-1} = (i, v): carry-step records
       {
         const int *cnt = reinterpret_cast<const int *>(ws + kScrCnt);
         const int *offs = reinterpret_cast<const int *>(ws + kScrOffs);
@@ -471,24 +550,6 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         reinterpret_cast<int *>(op + kOffPhiIdx)[j1] = i1;
         reinterpret_cast<float *>(op + kOffPhiVal)[j0] = v0;
         reinterpret_cast<float *>(op + kOffPhiVal)[j1] = v1;
-      }
-      {
-        const int o0 = kOffCt + off_ct_pos(posA0), o1 = kOffCt + off_ct_pos(posA1);
-#pragma unroll
-        for (int tau = 0; tau < kT; ++tau) {
-          float *c0p = reinterpret_cast<float *>(op + o0 + off_ct_tau(tau));
-          float *c1p = reinterpret_cast<float *>(op + o1 + off_ct_tau(tau));
-          if constexpr (kPrecise) {  // hi as fp32 (read as tf32), lo = the rest
-            const float h0 = tf32_trunc(ct0[tau]), h1 = tf32_trunc(ct1[tau]);
-            c0p[0] = ct0[tau];
-            c1p[0] = ct1[tau];
-            c0p[(kOffCtLo - kOffCt) / 4] = ct0[tau] - h0;
-            c1p[(kOffCtLo - kOffCt) / 4] = ct1[tau] - h1;
-          } else {
-            c0p[0] = tf32_rn(ct0[tau]);
-            c1p[0] = tf32_rn(ct1[tau]);
-          }
-        }
       }
 
       // ---- backward: the suffix Psi_sigma with Bh_sigma = Psi_sigma B_sigma, and
@@ -600,7 +661,9 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB0, sg), bh0);
         st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB1, sg), bh1);
       };
+#pragma unroll 1
       for (int sg = kT - 1; sg >= 8; --sg) bwd_step(std::integral_constant<int, 8>(), sg);
+#pragma unroll 1
       for (int sg = 7; sg >= 0; --sg) bwd_step(std::integral_constant<int, 0>(), sg);
 
       fence_proxy_async_smem();
@@ -619,50 +682,11 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     const int p = 16 * q + lane;            // state column owned by this lane
     const uint32_t lanebase = (uint32_t)(32 * q) << 16;
     const bool issuer = (q == 0) && (lane == 0);
-    const uint32_t id_u = idesc_bf16_f32(64, kN, true, true);
-    const uint32_t id_g = idesc_bf16_f32(64, kT, true, false);
-    const uint32_t id_c = idesc_tf32_f32(64, kT);
-    // U_sub into state region (sub + 1) mod R and the intra-sub-chunk part of
-    // Y_sub. The region held S_{sub+1-R}: callers issue this only after the carry
-    // step of sub-chunk sub+1-R is complete and its readout has been issued
-    // (tensor-core operations of one thread execute in issue order).
     auto issue_u = [&](int sub) -> bool {
-      const int st = sub % a.nst;
-      if (!wait_bar(bars, &bars->full[st], (sub / a.nst) & 1, a.err)) return false;
-      if (sub >= kNY && !wait_bar(bars, &bars->yfree[sub % kNY], ((sub / kNY) - 1) & 1, a.err)) return false;
-      tc_fence_after();
-      const uint32_t op = smem_u32(op_base + st * kOpStage);
-      const uint32_t dU = tbase + col_state((sub + 1) % kRing);
-      const uint32_t dY = tbase + kColY + (sub % kNY) * kT;
-      const uint64_t ax = smem_desc(op + kOffX, (kP / 8) * 128, 128);
-      mma_bf16(dU, ax, smem_desc(op + kOffBhHi, kBhLbo, kBhSbo), id_u, 0);
-      mma_bf16(dU, ax, smem_desc(op + kOffBhLo, kBhLbo, kBhSbo), id_u, 1);
-      mma_bf16(dY, ax, smem_desc(op + kOffGtHi, 128, 256), id_g, 0);
-      mma_bf16(dY, ax, smem_desc(op + kOffGtLo, 128, 256), id_g, 1);
-      mma_commit(&bars->ufull[(sub + 1) % kRing]);
-      return true;
+      return issue_input_mma<kPrecise>(bars, smem_u32(op_base), a.nst, tbase, sub, a.err);
     };
-    // readout of the entering state S_sub: A operand from tensor memory (tf32)
     auto issue_y = [&](int sub) -> bool {
-      const int st = sub % a.nst;
-      if (!wait_bar(bars, &bars->sready, sub & 1, a.err)) return false;
-      tc_fence_after();
-      const uint32_t op = smem_u32(op_base + st * kOpStage);
-      const uint32_t dY = tbase + kColY + (sub % kNY) * kT;
-      const uint32_t aS = tbase + col_state(sub % kRing);
-#pragma unroll
-      for (int ks = 0; ks < kN / 8; ++ks) {
-        const uint64_t bhi = smem_desc(op + kOffCt + ks * 2 * kCtLbo, kCtLbo, kCtSbo);
-        mma_tf32_ts(dY, aS + ks * 8, bhi, id_c, 1);
-        if constexpr (kPrecise) {
-          mma_tf32_ts(dY, aS + ks * 8, smem_desc(op + kOffCtLo + ks * 2 * kCtLbo, kCtLbo, kCtSbo), id_c, 1);
-          mma_tf32_ts(dY, tbase + kColSlo + ks * 8, bhi, id_c, 1);
-        }
-      }
-      mma_commit(&bars->yfull[sub % kNY]);
-      mma_commit(&bars->opfree[st]);
-      if constexpr (kPrecise) mma_commit(&bars->slofree);
-      return true;
+      return issue_readout_mma<kPrecise>(bars, smem_u32(op_base), a.nst, tbase, sub, a.err);
     };
     // Input-term MMAs are issued ahead by the issuing thread: blocking only when
     // the carry step or the readout about to be issued needs them, otherwise
@@ -745,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       // parts of 16 positions, one tensor-memory round trip each (S_a and U at
       // the group ends); the previous sub-chunk's output rides on the first.
       float run = 0.f;
-#pragma unroll
+#pragma unroll 1
       for (int part = 0; part < 4; ++part) {
         float v[16], u[16];
         tmem_ld16(RS + 16 * part, v);
