@@ -94,13 +94,16 @@ constexpr int kOffNu = kOffMeta + 256;           // float [N] by position: Phi_{
 constexpr int kOffPhiIdx = kOffNu + 256;         // int [N] by source row: Phi_{T-1} index
 constexpr int kOffPhiVal = kOffPhiIdx + 256;     // float [N] by source row: Phi_{T-1} value
 constexpr int kOffSrc = kOffPhiVal + 256;        // int [N] by position: source row
-constexpr int kOffCtLo = kOffSrc + 256;          // low part of Ct (fp32 output only), as kOffCt
+constexpr int kOffGDst = kOffSrc + 256;          // uint8 [N] by group ordinal: target's column in the next order
+constexpr int kOffHdr = kOffGDst + 64;           // int [4]: number of groups, the group crossing position 32 (or -1)
+constexpr int kOffCtLo = kOffHdr + 16;           // low part of Ct (fp32 output only), as kOffCt
 __host__ __device__ constexpr int op_stage_bytes(bool precise) { return kOffCtLo + (precise ? 2 * kCtSbo : 0); }
 
-// carry-step record of a position: the target's column in the next order, and
-// whether the position continues a target group (else it starts one) and ends it
+// carry-step record of a position: whether it continues a target group (else
+// it starts one), whether it ends it, and the group's ordinal
 constexpr int kMetaKeep = 1 << 8;
 constexpr int kMetaEnd = 1 << 9;
+constexpr int kMetaOrdShift = 10;
 
 // per-prep-warp scratch (bytes)
 constexpr int kScrBins = 0;                   // int [2][N] fixed-point accumulators (by sigma parity)
@@ -320,63 +323,6 @@ __device__ __forceinline__ void group_positions(int t0, int t1, uint8_t *ws, int
   pos1 = offs[t1] + cntlo[t1] + __popc(m1 & lt);
 }
 
-// ------------------------------------------------------------- MMA issue
-
-// U_sub into state region (sub + 1) mod R and the intra-sub-chunk part of Y_sub
-// (written, not accumulated). The region held S_{sub+1-R}: callers issue this
-// only after the carry step of sub-chunk sub+1-R is complete and its readout
-// has been issued (tensor-core operations of one thread execute in issue order).
-// One thread; false after a timeout.
-template <bool kPrecise>
-__device__ __noinline__ bool issue_input_mma(Bars *bars, uint32_t op_base, int nst, uint32_t tbase, int sub,
-                                             uint32_t *err) {
-  constexpr int kRing = kPrecise ? 2 : 3;
-  const int st = sub % nst;
-  if (!wait_bar(bars, &bars->full[st], (sub / nst) & 1, err)) return false;
-  if (sub >= kNY && !wait_bar(bars, &bars->yfree[sub % kNY], ((sub / kNY) - 1) & 1, err)) return false;
-  tc_fence_after();
-  const uint32_t op = op_base + st * op_stage_bytes(kPrecise);
-  const uint32_t dU = tbase + col_state((sub + 1) % kRing);
-  const uint32_t dY = tbase + kColY + (sub % kNY) * kT;
-  const uint32_t id_u = idesc_bf16_f32(64, kN, true, true);
-  const uint32_t id_g = idesc_bf16_f32(64, kT, true, false);
-  const uint64_t ax = smem_desc(op + kOffX, (kP / 8) * 128, 128);
-  mma_bf16(dU, ax, smem_desc(op + kOffBhHi, kBhLbo, kBhSbo), id_u, 0);
-  mma_bf16(dU, ax, smem_desc(op + kOffBhLo, kBhLbo, kBhSbo), id_u, 1);
-  mma_bf16(dY, ax, smem_desc(op + kOffGtHi, 128, 256), id_g, 0);
-  mma_bf16(dY, ax, smem_desc(op + kOffGtLo, 128, 256), id_g, 1);
-  mma_commit(&bars->ufull[(sub + 1) % kRing]);
-  return true;
-}
-
-// Readout of the entering state S_sub into Y_sub: A operand from tensor memory
-// (tf32). Releases the operand stage (and the S_lo plane) when done.
-template <bool kPrecise>
-__device__ __noinline__ bool issue_readout_mma(Bars *bars, uint32_t op_base, int nst, uint32_t tbase, int sub,
-                                               uint32_t *err) {
-  constexpr int kRing = kPrecise ? 2 : 3;
-  const int st = sub % nst;
-  if (!wait_bar(bars, &bars->sready, sub & 1, err)) return false;
-  tc_fence_after();
-  const uint32_t op = op_base + st * op_stage_bytes(kPrecise);
-  const uint32_t dY = tbase + kColY + (sub % kNY) * kT;
-  const uint32_t aS = tbase + col_state(sub % kRing);
-  const uint32_t id_c = idesc_tf32_f32(64, kT);
-#pragma unroll 1
-  for (int ks = 0; ks < kN / 8; ++ks) {
-    const uint64_t bhi = smem_desc(op + kOffCt + ks * 2 * kCtLbo, kCtLbo, kCtSbo);
-    mma_tf32_ts(dY, aS + ks * 8, bhi, id_c, 1);
-    if constexpr (kPrecise) {
-      mma_tf32_ts(dY, aS + ks * 8, smem_desc(op + kOffCtLo + ks * 2 * kCtLbo, kCtLbo, kCtSbo), id_c, 1);
-      mma_tf32_ts(dY, tbase + kColSlo + ks * 8, bhi, id_c, 1);
-    }
-  }
-  mma_commit(&bars->yfull[sub % kNY]);
-  mma_commit(&bars->opfree[st]);
-  if constexpr (kPrecise) mma_commit(&bars->slofree);
-  return true;
-}
-
 // ------------------------------------------------------------- the kernel
 
 template <typename TL, typename TO, bool kPrecise>
@@ -533,15 +479,35 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       {
         const int *cnt = reinterpret_cast<const int *>(ws + kScrCnt);
         const int *offs = reinterpret_cast<const int *>(ws + kScrOffs);
+        // ordinal of each nonempty target group (targets ascending): target t's is
+        // the exclusive count of nonempty targets below t
+        const int na = cnt[2 * lane] > 0, nb = cnt[2 * lane + 1] > 0;
+        int incl = na + nb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += n;
+        }
+        const int gex = incl - na - nb;
+        const int n_img = __shfl_sync(0xffffffffu, incl, 31);
+        const int g0 = __shfl_sync(0xffffffffu, gex, i0 >> 1), h0 = __shfl_sync(0xffffffffu, na, i0 >> 1);
+        const int g1 = __shfl_sync(0xffffffffu, gex, i1 >> 1), h1 = __shfl_sync(0xffffffffu, na, i1 >> 1);
+        const int e0 = g0 + ((i0 & 1) ? h0 : 0), e1 = g1 + ((i1 & 1) ? h1 : 0);
         // the target's column in the next order: posB of row i (held by lane i & 31)
         const int pb0a = __shfl_sync(0xffffffffu, posB0, i0 & 31), pb0b = __shfl_sync(0xffffffffu, posB1, i0 & 31);
         const int pb1a = __shfl_sync(0xffffffffu, posB0, i1 & 31), pb1b = __shfl_sync(0xffffffffu, posB1, i1 & 31);
         const int f0 = offs[i0], f1 = offs[i1];
+        const bool keep0 = posA0 != f0, keep1 = posA1 != f1;
+        const bool end0 = posA0 == f0 + cnt[i0] - 1, end1 = posA1 == f1 + cnt[i1] - 1;
         int *meta = reinterpret_cast<int *>(op + kOffMeta);
-        meta[posA0] = (i0 < 32 ? pb0a : pb0b) | (posA0 != f0 ? kMetaKeep : 0) |
-                      (posA0 == f0 + cnt[i0] - 1 ? kMetaEnd : 0);
-        meta[posA1] = (i1 < 32 ? pb1a : pb1b) | (posA1 != f1 ? kMetaKeep : 0) |
-                      (posA1 == f1 + cnt[i1] - 1 ? kMetaEnd : 0);
+        meta[posA0] = (keep0 ? kMetaKeep : 0) | (end0 ? kMetaEnd : 0) | (e0 << kMetaOrdShift);
+        meta[posA1] = (keep1 ? kMetaKeep : 0) | (end1 ? kMetaEnd : 0) | (e1 << kMetaOrdShift);
+        if (end0) op[kOffGDst + e0] = (uint8_t)(i0 < 32 ? pb0a : pb0b);
+        if (end1) op[kOffGDst + e1] = (uint8_t)(i1 < 32 ? pb1a : pb1b);
+        int *hdr = reinterpret_cast<int *>(op + kOffHdr);
+        if (lane == 0) hdr[0] = n_img;
+        if (posA0 == 32) hdr[1] = keep0 ? e0 : -1;
+        if (posA1 == 32) hdr[1] = keep1 ? e1 : -1;
         reinterpret_cast<float *>(op + kOffNu)[posA0] = v0;
         reinterpret_cast<float *>(op + kOffNu)[posA1] = v1;
         reinterpret_cast<int *>(op + kOffSrc)[posA0] = j0;
@@ -682,24 +648,73 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     const int p = 16 * q + lane;            // state column owned by this lane
     const uint32_t lanebase = (uint32_t)(32 * q) << 16;
     const bool issuer = (q == 0) && (lane == 0);
-    auto issue_u = [&](int sub) -> bool {
-      return issue_input_mma<kPrecise>(bars, smem_u32(op_base), a.nst, tbase, sub, a.err);
+    // ---- MMA issue (one thread). Descriptors of operand stage 0; another stage
+    //      adds its offset / 16 to the start-address field (no carry out of it).
+    constexpr uint32_t kIdU = idesc_bf16_f32(64, kN, true, true);
+    constexpr uint32_t kIdG = idesc_bf16_f32(64, kT, true, false);
+    constexpr uint32_t kIdC = idesc_tf32_f32(64, kT);
+    const uint32_t ob = smem_u32(op_base);
+    const uint64_t dX = smem_desc(ob + kOffX, (kP / 8) * 128, 128);
+    const uint64_t dBh = smem_desc(ob + kOffBhHi, kBhLbo, kBhSbo), dBl = smem_desc(ob + kOffBhLo, kBhLbo, kBhSbo);
+    const uint64_t dGh = smem_desc(ob + kOffGtHi, 128, 256), dGl = smem_desc(ob + kOffGtLo, 128, 256);
+    const uint64_t dCt = smem_desc(ob + kOffCt, kCtLbo, kCtSbo), dCl = smem_desc(ob + kOffCtLo, kCtLbo, kCtSbo);
+    // U_u into state region (u + 1) mod R and the intra-sub-chunk part of Y_u
+    // (written, not accumulated). The region held S_{u+1-R}: this is issued only
+    // after the carry step of sub-chunk u+1-R is complete and its readout has been
+    // issued (tensor-core operations of one thread execute in issue order).
+    auto issue_u_now = [&](int u) {
+      const uint64_t so = (uint64_t)((u % a.nst) * (kOpStage >> 4));
+      const uint32_t dU = tbase + col_state((u + 1) % kRing), dY = tbase + kColY + (u % kNY) * kT;
+      mma_bf16(dU, dX + so, dBh + so, kIdU, 0);
+      mma_bf16(dU, dX + so, dBl + so, kIdU, 1);
+      mma_bf16(dY, dX + so, dGh + so, kIdG, 0);
+      mma_bf16(dY, dX + so, dGl + so, kIdG, 1);
+      mma_commit(&bars->ufull[(u + 1) % kRing]);
     };
-    auto issue_y = [&](int sub) -> bool {
-      return issue_readout_mma<kPrecise>(bars, smem_u32(op_base), a.nst, tbase, sub, a.err);
+    // readout of the entering state S_s: A operand from tensor memory (tf32)
+    auto issue_y_now = [&](int s) {
+      const int st = s % a.nst;
+      const uint64_t so = (uint64_t)(st * (kOpStage >> 4));
+      const uint32_t dY = tbase + kColY + (s % kNY) * kT, aS = tbase + col_state(s % kRing);
+#pragma unroll
+      for (int ks = 0; ks < kN / 8; ++ks) {
+        const uint64_t kso = so + (uint64_t)((ks * 2 * kCtLbo) >> 4);
+        mma_tf32_ts(dY, aS + ks * 8, dCt + kso, kIdC, 1);
+        if constexpr (kPrecise) {
+          mma_tf32_ts(dY, aS + ks * 8, dCl + kso, kIdC, 1);
+          mma_tf32_ts(dY, tbase + kColSlo + ks * 8, dCt + kso, kIdC, 1);
+        }
+      }
+      mma_commit(&bars->yfull[s % kNY]);
+      mma_commit(&bars->opfree[st]);
+      if constexpr (kPrecise) mma_commit(&bars->slofree);
     };
-    // Input-term MMAs are issued ahead by the issuing thread: blocking only when
-    // the carry step or the readout about to be issued needs them, otherwise
-    // as soon as their operands are ready (checked without waiting).
+    // issue U groups up to `upto`: waiting for their operands and output slot when
+    // `block`, else only those already ready
     int next_u = 0;
     auto issue_us = [&](int upto, bool block) -> bool {
       for (; next_u <= upto && next_u < nsub; ++next_u) {
+        const int st = next_u % a.nst;
+        uint64_t *fb = &bars->full[st];
+        const uint32_t fp = (next_u / a.nst) & 1;
+        const bool needy = next_u >= kNY;
+        uint64_t *yb = &bars->yfree[next_u % kNY];
+        const uint32_t yp = ((next_u / kNY) - 1) & 1;
         if (!block) {
-          if (!mbar_try_wait(&bars->full[next_u % a.nst], (next_u / a.nst) & 1)) return true;
-          if (next_u >= kNY && !mbar_try_wait(&bars->yfree[next_u % kNY], ((next_u / kNY) - 1) & 1)) return true;
+          if (!mbar_test_wait(fb, fp) || (needy && !mbar_test_wait(yb, yp))) return true;
+        } else {
+          if (!mbar_test_wait(fb, fp) && !wait_bar(bars, fb, fp, a.err)) return false;
+          if (needy && !mbar_test_wait(yb, yp) && !wait_bar(bars, yb, yp, a.err)) return false;
         }
-        if (!issue_u(next_u)) return false;
+        tc_fence_after();
+        issue_u_now(next_u);
       }
+      return true;
+    };
+    auto issue_y = [&](int s) -> bool {
+      if (!mbar_test_wait(&bars->sready, s & 1) && !wait_bar(bars, &bars->sready, s & 1, a.err)) return false;
+      tc_fence_after();
+      issue_y_now(s);
       return true;
     };
     bool ok = true;
@@ -763,47 +778,74 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         pidx0 = pi[pidx0];
         pidx1 = pi[pidx1];
       }
-      // S_{a+1}[i] = U[i] + sum_{j: Phi[j] = i} nu_j S_a[j], in place over U: the
+      // S_{a+1}[i] = U[i] + sum_{j: Phi[j] = i} nu_j S_a[j], in place over U. The
       // sources of a target are adjacent in S_a, so a segmented sum over the
-      // positions yields each target's total at its group's last position. Four
-      // parts of 16 positions, one tensor-memory round trip each (S_a and U at
-      // the group ends); the previous sub-chunk's output rides on the first.
-      float run = 0.f;
-#pragma unroll 1
-      for (int part = 0; part < 4; ++part) {
-        float v[16], u[16];
-        tmem_ld16(RS + 16 * part, v);
+      // positions yields each target's total at its group's last position. All 32
+      // threads work: thread (hh, pl) holds state column 16 q + pl at positions
+      // [32 hh, 32 hh + 32). The previous sub-chunk's output rides on the same
+      // tensor-memory round trip.
+      {
+        const int hh = lane >> 4, pl = lane & 15;
+        float v[32];
+        tmem_ld_x2_32<32>(RS, v);
+        float yv[8];
+        if (sub > 0) tmem_ld_x2_8<8>(tbase + lanebase + kColY + ((sub - 1) % kNY) * kT, yv);
+        tmem_wait_ld();
+        if (sub > 0) {
+          const int tp = (sub - 1) * kT;
+          const int nv = (int)(a.L - tp < kT ? a.L - tp : kT);
 #pragma unroll
-        for (int r4 = 0; r4 < 4; ++r4) {
-          const int4 m4 = meta4[4 * part + r4];
-          const int mt[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            if (mt[c] & kMetaEnd) tmem_ld1(RU + (mt[c] & 0xff), u[4 * r4 + c]);
-        }
-        if (part == 0 && sub > 0) {
-          float yv[16];
-          tmem_ld16(tbase + lanebase + kColY + ((sub - 1) % kNY) * kT, yv);
-          tmem_wait_ld();
-          store_y(sub - 1, yv);
+          for (int i = 0; i < 8; ++i)
+            if (8 * hh + i < nv) store_out(yout + ((b * a.L + tp + 8 * hh + i) * a.H + h) * kP + 16 * q + pl, yv[i]);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->yfree[(sub - 1) % kNY]);
-        } else {
-          tmem_wait_ld();
         }
+        const int *hdr = reinterpret_cast<const int *>(op + kOffHdr);
+        const int n_img = hdr[0], ecross = hdr[1];
+        // group totals go through this warp's 1 KB of the stage's Bh area (its MMA
+        // completed before ufull was signalled)
+        float *cs = reinterpret_cast<float *>(const_cast<uint8_t *>(op) + kOffBhHi) + q * 256;
+        for (int base = 0; base < n_img; base += 16) {
+          float run = 0.f;
 #pragma unroll
-        for (int r4 = 0; r4 < 4; ++r4) {
-          const int4 m4 = meta4[4 * part + r4];
-          const float4 n4 = nu4[4 * part + r4];
-          const int mt[4] = {m4.x, m4.y, m4.z, m4.w};
-          const float nu[4] = {n4.x, n4.y, n4.z, n4.w};
+          for (int r4 = 0; r4 < 8; ++r4) {
+            const int4 m4 = meta4[8 * hh + r4];
+            const float4 n4 = nu4[8 * hh + r4];
+            const int mt[4] = {m4.x, m4.y, m4.z, m4.w};
+            const float nu[4] = {n4.x, n4.y, n4.z, n4.w};
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            run = (mt[c] & kMetaKeep) ? run : 0.f;
-            run = fmaf(nu[c], v[4 * r4 + c], run);
-            if (mt[c] & kMetaEnd) tmem_st1(RU + (mt[c] & 0xff), u[4 * r4 + c] + run);
+            for (int c = 0; c < 4; ++c) {
+              run = (mt[c] & kMetaKeep) ? run : 0.f;
+              run = fmaf(nu[c], v[4 * r4 + c], run);
+              const unsigned e = (unsigned)((mt[c] >> kMetaOrdShift) - base);
+              if ((mt[c] & kMetaEnd) && e < 16u) cs[e * 16 + pl] = run;
+            }
           }
+          // the group that crosses positions 31 | 32 gets the lower half's part
+          const float tail = __shfl_sync(0xffffffffu, run, pl);
+          const unsigned ec = (unsigned)(ecross - base);
+          if (hh == 1 && ecross >= 0 && ec < 16u) cs[ec * 16 + pl] += tail;
+          __syncwarp();
+          // U at the group ends += group totals (the second eight only when needed)
+          const bool more = base + 8 < n_img;
+          float u[16];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) tmem_ld1_if(RU + op[kOffGDst + base + e], u[e], base + e < n_img);
+          if (more) {
+#pragma unroll
+            for (int e = 8; e < 16; ++e) tmem_ld1_if(RU + op[kOffGDst + base + e], u[e], base + e < n_img);
+          }
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            tmem_st1_if(RU + op[kOffGDst + base + e], u[e] + cs[e * 16 + pl], base + e < n_img);
+          if (more) {
+#pragma unroll
+            for (int e = 8; e < 16; ++e)
+              tmem_st1_if(RU + op[kOffGDst + base + e], u[e] + cs[e * 16 + pl], base + e < n_img);
+          }
+          __syncwarp();
         }
       }
       tmem_wait_st();
@@ -811,14 +853,12 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         // tf32 low part of S_{a+1}, once the readout of S_a is done with the plane
         if (!wait_bar_warp(bars, &bars->slofree, sub & 1, a.err)) break;
         tc_fence_after();
-        for (int c0 = 0; c0 < kN; c0 += 16) {
-          float v[16];
-          tmem_ld16(RU + c0, v);
-          tmem_wait_ld();
+        float v[32];
+        tmem_ld_x2_32<32>(RU, v);
+        tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] -= tf32_trunc(v[i]);
-          tmem_st16(tbase + lanebase + kColSlo + c0, v);
-        }
+        for (int i = 0; i < 32; ++i) v[i] -= tf32_trunc(v[i]);
+        tmem_st_x2_32<32>(tbase + lanebase + kColSlo, v);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -831,8 +871,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       // Next MMAs: the readout of S_{sub+1} once every quarter of it is complete.
       // The input part of Y_{sub+1} (written, not accumulated) must precede it.
       if (issuer && sub + 1 < nsub) {
-        ok = wait_bar(bars, &bars->sready, (sub + 1) & 1, a.err) && issue_us(sub + 1, true) && issue_y(sub + 1) &&
-             issue_us(sub + kRing - 1, false);
+        ok = (mbar_test_wait(&bars->sready, (sub + 1) & 1) || wait_bar(bars, &bars->sready, (sub + 1) & 1, a.err)) &&
+             issue_us(sub + 1, true) && issue_y(sub + 1) && issue_us(sub + kRing - 1, false);
       }
     }
     // output of the last sub-chunk
