@@ -157,6 +157,39 @@ def load_peaks():
         return dict(FALLBACK_PEAKS, source="fallback")
 
 
+# ------------------------------------------------------------ recorded traffic
+
+# Kernel sources whose hash a profile summary records; the DRAM traffic it
+# reports is valid only for exactly these sources.
+KERNEL_SOURCES = {
+    "fused_scan": ["structured_sparse_selective_b200/csrc/scan_fused.cu",
+                   "structured_sparse_selective_b200/csrc/sm100.cuh"],
+}
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """dram bytes (read + write) per launch from profiles/<kernel>_<workload>.md, or None
+    when there is no summary or the kernel's sources changed since it was captured."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    srcs = KERNEL_SOURCES.get(kernel)
+    if not srcs or not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            k, _, v = line.strip().partition(":")
+            if k in ("traffic_bytes_per_launch", "kernel_sources_sha256"):
+                fields[k] = v.strip()
+    h = hashlib.sha256()
+    for src in srcs:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    if fields.get("kernel_sources_sha256") != h.hexdigest() or "traffic_bytes_per_launch" not in fields:
+        return None
+    return int(fields["traffic_bytes_per_launch"])
+
+
 # ------------------------------------------------------------ workload
 
 def workload_config(sp: workloads.Spec, chunk: int, world: int):
@@ -278,12 +311,13 @@ def run_ours(args, rank, world, local):
         "select": units * (with_logits + 4),
     }.get(dominant)
     peaks = load_peaks()
+    traffic = recorded_traffic(dominant, args.workload)
     roofline = None
     if alg_bytes is not None:
         achieved = alg_bytes / (dom_ms / 1e3) / 1e9
         roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1),
                     "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
-                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                     "algorithmic_bytes_per_launch": int(alg_bytes), "launch_ms": round(dom_ms, 4)}
 
     # ---- end to end through the public API with host buffers

@@ -1,0 +1,44 @@
+"""Host-side logic of bench.py that needs no GPU: the recorded DRAM traffic is reported
+only while the kernel sources still hash to the value the profile summary recorded."""
+import hashlib
+import os
+
+import bench
+
+
+def _setup(tmp_path, monkeypatch, recorded_hash=None):
+    src = tmp_path / "k.cu"
+    src.write_text("__global__ void k() {}\n")
+    (tmp_path / "profiles").mkdir()
+    h = recorded_hash or hashlib.sha256(src.read_bytes()).hexdigest()
+    (tmp_path / "profiles" / "kern_wl.md").write_text(
+        "# summary\n\n    traffic_bytes_per_launch: 12345\n    kernel_sources_sha256: %s\n" % h)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setitem(bench.KERNEL_SOURCES, "kern", ["k.cu"])
+    return src
+
+
+def test_traffic_reported_while_sources_match(tmp_path, monkeypatch):
+    _setup(tmp_path, monkeypatch)
+    assert bench.recorded_traffic("kern", "wl") == 12345
+
+
+def test_traffic_dropped_once_the_kernel_changes(tmp_path, monkeypatch):
+    src = _setup(tmp_path, monkeypatch)
+    src.write_text("__global__ void k() { /* changed */ }\n")
+    assert bench.recorded_traffic("kern", "wl") is None
+
+
+def test_traffic_absent_without_summary_or_known_sources(tmp_path, monkeypatch):
+    _setup(tmp_path, monkeypatch)
+    assert bench.recorded_traffic("kern", "other") is None
+    assert bench.recorded_traffic("unknown", "wl") is None
+
+
+def test_committed_summary_names_known_sources():
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles", "fused_scan_lm.md")
+    with open(path) as f:
+        text = f.read()
+    assert "traffic_bytes_per_launch:" in text and "kernel_sources_sha256:" in text
+    for s in bench.KERNEL_SOURCES["fused_scan"]:
+        assert os.path.exists(os.path.join(os.path.dirname(path), "..", s))
