@@ -64,10 +64,12 @@ namespace {
 constexpr int kN = 64;   // state rows
 constexpr int kP = 64;   // state columns
 constexpr int kT = 16;   // sub-chunk length
-constexpr int kNW = 4;   // prep warps; warp w prepares sub-chunks w, w + 4, ...
+constexpr int kNW = 4;   // prep warp pairs; pair w prepares sub-chunks w, w + 4, ...
+constexpr int kPrepWarps = 2 * kNW;
+constexpr int kCarryWarp0 = kPrepWarps;  // warps 8-11 carry the state (one per tensor-memory quarter)
 constexpr int kMaxStages = 6;  // operand stages (sub-chunk a uses stage a mod nst, nst >= kNW)
 constexpr int kNY = 4;   // output accumulator slots
-constexpr int kThreads = 256;  // 4 prep warps + 4 carry warps (warp 4 also issues the MMAs)
+constexpr int kThreads = 32 * (kPrepWarps + 4);  // 8 prep warps + 4 carry warps (warp 8 also issues the MMAs)
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
 
 // tensor-memory columns: 64-column state regions (a ring of 3, or 2 plus S_lo
@@ -323,6 +325,21 @@ __device__ __forceinline__ void group_positions(int t0, int t1, uint8_t *ws, int
   pos1 = offs[t1] + cntlo[t1] + __popc(m1 & lt);
 }
 
+// Named barrier over the two warps of a prep pair; the _and form also returns
+// whether the predicate held in every thread of both warps.
+__device__ __forceinline__ void pair_sync(uint32_t id) {
+  asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ bool pair_and(uint32_t id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.b32 p, %1, 0;\n bar.red.and.pred q, %2, 64, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
 // ------------------------------------------------------------- the kernel
 
 template <typename TL, typename TO, bool kPrecise>
@@ -343,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
   // ---- setup
   if (tid == 0) {
     for (int i = 0; i < kMaxStages; ++i) {
-      mbar_init(&bars->full[i], 1);
+      mbar_init(&bars->full[i], 2);  // both warps of the prep pair
       mbar_init(&bars->opfree[i], 1 + 4);  // MMA commit + one arrival per carry warp
     }
     for (int i = 0; i < kNY; ++i) {
@@ -365,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     }
     dict[e] = (uint8_t)v;
   }
-  if (warp == kNW) {
+  if (warp == kCarryWarp0) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -374,27 +391,34 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
   tc_fence_after();
   const uint32_t tbase = bars->tmem_base;
 
-  if (warp < kNW) {
+  if (warp < kPrepWarps) {
     // ================================================================ prep
-    // Warp w prepares sub-chunks w, w + kNW, ... (sub-chunk a into operand stage
-    // a mod nst). Lanes own rows j0 = lane and j1 = lane + 32.
-    uint8_t *in = in_base + warp * a.in.bytes;
-    uint8_t *ws = scr + warp * kScrBytes;
+    // Warp pair w prepares sub-chunks w, w + kNW, ... (sub-chunk a into operand
+    // stage a mod nst). Role 0 loads the inputs and builds the composites, the
+    // forward chain (Ct), the carry records and the suffix scatter (Bh); role 1
+    // the backward readouts and G. Lanes own rows j0 = lane and j1 = lane + 32.
+    const int pair = warp >> 1, role = warp & 1;
+    const uint32_t pbar = 1 + pair;
+    uint8_t *in = in_base + pair * a.in.bytes;
+    uint8_t *ws = scr + pair * kScrBytes;
     int *bins = reinterpret_cast<int *>(ws + kScrBins);
-    if (warp < nsub) load_inputs<TL>(a, in, b, h, warp, lane);
-    cp_async_commit();
+    if (role == 0) {
+      if (pair < nsub) load_inputs<TL>(a, in, b, h, pair, lane);
+      cp_async_commit();
 #pragma unroll
-    for (int c = 0; c < 4; ++c) bins[lane + 32 * c] = 0;
+      for (int c = 0; c < 4; ++c) bins[lane + 32 * c] = 0;
+    }
     const int j0 = lane, j1 = lane + 32;
-    for (int sub = warp; sub < nsub; sub += kNW) {
+    for (int sub = pair; sub < nsub; sub += kNW) {
       const int stg = sub % a.nst;
       uint8_t *op = op_base + stg * kOpStage;
       const int t0 = sub * kT;
       const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
       const int nnext = (int)(a.L - t0 - kT < kT ? (a.L - t0 - kT > 0 ? a.L - t0 - kT : 0) : kT);
-      if (!wait_bar_warp(bars, &bars->opfree[stg], ((sub / a.nst) & 1) ^ 1, a.err)) break;
-      cp_async_wait<0>();
-      __syncwarp();
+      bool ok = wait_bar_warp(bars, &bars->opfree[stg], ((sub / a.nst) & 1) ^ 1, a.err);
+      if (role == 0) cp_async_wait<0>();
+      // one decision for the pair; the barrier also publishes the loaded inputs
+      if (!pair_and(pbar, ok)) break;
 
       // selections: lanes 0-15 take this sub-chunk's tokens, lanes 16-31 the next one's
       int s_lane = 0;
@@ -411,236 +435,245 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
               s_lane = 0;
             }
           }
-          if (!nx && a.s_out) a.s_out[(b * a.L + t0 + tok) * a.H + h] = s_lane;
+          if (role == 0 && !nx && a.s_out) a.s_out[(b * a.L + t0 + tok) * a.H + h] = s_lane;
         }
       }
 
-      // x into the operand stage (2 KB); G^T cleared (entries above the diagonal stay 0)
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        reinterpret_cast<uint4 *>(op + kOffX)[lane + 32 * c] = reinterpret_cast<const uint4 *>(in + a.in.x)[lane + 32 * c];
-      reinterpret_cast<uint4 *>(op + kOffGtHi)[lane] = make_uint4(0, 0, 0, 0);
-      reinterpret_cast<uint4 *>(op + kOffGtHi)[lane + 32] = make_uint4(0, 0, 0, 0);
 
       const uint8_t *din = in + a.in.d, *Bin = in + a.in.B, *Cin = in + a.in.C;
-
-      // ---- the next sub-chunk's composite (indices only) -> the order of S_{a+1}
-      int posB0, posB1;
-      {
-        int n0 = j0, n1 = j1;
-        for (int tau = 0; tau < nnext; ++tau) {
-          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, 16 + tau) * kN;
-          n0 = dk[n0];
-          n1 = dk[n1];
-        }
-        group_positions(n0, n1, ws, lane, posB0, posB1);
-      }
-      __syncwarp();
-
-      // ---- Phi_{T-1} (indices): the positions of S_a's order
-      int posA0, posA1, i0 = j0, i1 = j1;
-      for (int tau = 0; tau < nvalid; ++tau) {
-        const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
-        i0 = dk[i0];
-        i1 = dk[i1];
-      }
-      group_positions(i0, i1, ws, lane, posA0, posA1);
-      // ---- forward chain: Phi_tau and Ct_tau = Phi_tau^T C_tau at the positions of S_a's order
-      float v0 = 1.f, v1 = 1.f;
-      {
-        const int o0 = kOffCt + off_ct_pos(posA0), o1 = kOffCt + off_ct_pos(posA1);
-        int f0 = j0, f1 = j1;
-#pragma unroll 1
-        for (int tau = 0; tau < kT; ++tau) {
-          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
-          float c0 = 0.f, c1 = 0.f;
-          if (tau < nvalid) {
-            v0 *= ld_bf16(din, tau * kN + f0);
-            v1 *= ld_bf16(din, tau * kN + f1);
-            f0 = dk[f0];
-            f1 = dk[f1];
-            c0 = v0 * ld_bf16(Cin, tau * kN + f0);
-            c1 = v1 * ld_bf16(Cin, tau * kN + f1);
-          }
-          float *c0p = reinterpret_cast<float *>(op + o0 + off_ct_tau(tau));
-          float *c1p = reinterpret_cast<float *>(op + o1 + off_ct_tau(tau));
-          if constexpr (kPrecise) {  // hi as fp32 (read as tf32), lo = the rest
-            c0p[0] = c0;
-            c1p[0] = c1;
-            c0p[(kOffCtLo - kOffCt) / 4] = c0 - tf32_trunc(c0);
-            c1p[(kOffCtLo - kOffCt) / 4] = c1 - tf32_trunc(c1);
-          } else {
-            c0p[0] = tf32_rn(c0);
-            c1p[0] = tf32_rn(c1);
-          }
-        }
-      }
-      // ---- Phi_{T-1} = (i, v): carry-step records
-      {
-        const int *cnt = reinterpret_cast<const int *>(ws + kScrCnt);
-        const int *offs = reinterpret_cast<const int *>(ws + kScrOffs);
-        // ordinal of each nonempty target group (targets ascending): target t's is
-        // the exclusive count of nonempty targets below t
-        const int na = cnt[2 * lane] > 0, nb = cnt[2 * lane + 1] > 0;
-        int incl = na + nb;
+      if (role == 0) {
+        // x into the operand stage (2 KB)
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int n = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += n;
-        }
-        const int gex = incl - na - nb;
-        const int n_img = __shfl_sync(0xffffffffu, incl, 31);
-        const int g0 = __shfl_sync(0xffffffffu, gex, i0 >> 1), h0 = __shfl_sync(0xffffffffu, na, i0 >> 1);
-        const int g1 = __shfl_sync(0xffffffffu, gex, i1 >> 1), h1 = __shfl_sync(0xffffffffu, na, i1 >> 1);
-        const int e0 = g0 + ((i0 & 1) ? h0 : 0), e1 = g1 + ((i1 & 1) ? h1 : 0);
-        // the target's column in the next order: posB of row i (held by lane i & 31)
-        const int pb0a = __shfl_sync(0xffffffffu, posB0, i0 & 31), pb0b = __shfl_sync(0xffffffffu, posB1, i0 & 31);
-        const int pb1a = __shfl_sync(0xffffffffu, posB0, i1 & 31), pb1b = __shfl_sync(0xffffffffu, posB1, i1 & 31);
-        const int f0 = offs[i0], f1 = offs[i1];
-        const bool keep0 = posA0 != f0, keep1 = posA1 != f1;
-        const bool end0 = posA0 == f0 + cnt[i0] - 1, end1 = posA1 == f1 + cnt[i1] - 1;
-        int *meta = reinterpret_cast<int *>(op + kOffMeta);
-        meta[posA0] = (keep0 ? kMetaKeep : 0) | (end0 ? kMetaEnd : 0) | (e0 << kMetaOrdShift);
-        meta[posA1] = (keep1 ? kMetaKeep : 0) | (end1 ? kMetaEnd : 0) | (e1 << kMetaOrdShift);
-        if (end0) op[kOffGDst + e0] = (uint8_t)(i0 < 32 ? pb0a : pb0b);
-        if (end1) op[kOffGDst + e1] = (uint8_t)(i1 < 32 ? pb1a : pb1b);
-        int *hdr = reinterpret_cast<int *>(op + kOffHdr);
-        if (lane == 0) hdr[0] = n_img;
-        if (posA0 == 32) hdr[1] = keep0 ? e0 : -1;
-        if (posA1 == 32) hdr[1] = keep1 ? e1 : -1;
-        reinterpret_cast<float *>(op + kOffNu)[posA0] = v0;
-        reinterpret_cast<float *>(op + kOffNu)[posA1] = v1;
-        reinterpret_cast<int *>(op + kOffSrc)[posA0] = j0;
-        reinterpret_cast<int *>(op + kOffSrc)[posA1] = j1;
-        reinterpret_cast<int *>(op + kOffPhiIdx)[j0] = i0;
-        reinterpret_cast<int *>(op + kOffPhiIdx)[j1] = i1;
-        reinterpret_cast<float *>(op + kOffPhiVal)[j0] = v0;
-        reinterpret_cast<float *>(op + kOffPhiVal)[j1] = v1;
-      }
+        for (int c = 0; c < 4; ++c)
+          reinterpret_cast<uint4 *>(op + kOffX)[lane + 32 * c] = reinterpret_cast<const uint4 *>(in + a.in.x)[lane + 32 * c];
 
-      // ---- backward: the suffix Psi_sigma with Bh_sigma = Psi_sigma B_sigma, and
-      //      the readouts R_sigma[j][tau] = (A_tau...A_{sigma+1})^T C_tau with
-      //      G[tau][sigma] = B_sigma . R_sigma[:, tau]. One step per sigma, without
-      //      branches: rows past the end of the sequence were zero-filled, so their
-      //      readout columns stay 0, and Psi treats those steps as the identity.
-      int k0 = j0, k1 = j1;          // Psi_sigma
-      float m0 = 1.f, m1 = 1.f;
-      float R0[kT], R1[kT];          // R_sigma[j][tau], zero for tau < sigma
-#pragma unroll
-      for (int c = 0; c < kT; ++c) R0[c] = R1[c] = 0.f;
-
-      // lo_c: readout columns [lo, T) can be nonzero (sigma >= lo)
-      auto bwd_step = [&](auto lo_c, int sg) {
-        constexpr int lo = decltype(lo_c)::value;
-        const bool sv = sg < nvalid;
-        const float bs0 = ld_bf16(Bin, sg * kN + j0), bs1 = ld_bf16(Bin, sg * kN + j1);
-        // (1) Bh_sigma as an exact fixed-point sum: integer adds are
-        //     order-independent; they are read back at the end of the step
-        int *bn = bins + (sg & 1) * kN;
-        const float w0 = m0 * bs0, w1 = m1 * bs1;
-        const unsigned mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(w0), fabsf(w1))));
-        // |w| < 2^ex; 64 terms of magnitude < 2^24 stay below 2^30
-        const int ex = (int)((mb >> 23) & 0xff) - 126;
-        const int e = mb ? 24 - ex : 0;
-        const float up = exp2i(e), dn = exp2i(-e);
-        atomicAdd(&bn[k0], __float2int_rn(w0 * up));
-        atomicAdd(&bn[k1], __float2int_rn(w1 * up));
-        // (2) Psi_{sg-1} = Psi_sg A_sg: column j <- d[j] * column idx[j] (identity past the end)
+        // ---- the next sub-chunk's composite (indices only) -> the order of S_{a+1}
+        int posB0, posB1;
         {
-          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, sg) * kN;
-          const int r0 = sv ? dk[j0] : j0, r1 = sv ? dk[j1] : j1;
-          const float d0 = sv ? ld_bf16(din, sg * kN + j0) : 1.f, d1 = sv ? ld_bf16(din, sg * kN + j1) : 1.f;
-          const int ka = __shfl_sync(0xffffffffu, k0, r0 & 31), kb = __shfl_sync(0xffffffffu, k1, r0 & 31);
-          const float ma = __shfl_sync(0xffffffffu, m0, r0 & 31), mb2 = __shfl_sync(0xffffffffu, m1, r0 & 31);
-          const int kc = __shfl_sync(0xffffffffu, k0, r1 & 31), kd = __shfl_sync(0xffffffffu, k1, r1 & 31);
-          const float mc = __shfl_sync(0xffffffffu, m0, r1 & 31), md = __shfl_sync(0xffffffffu, m1, r1 & 31);
-          k0 = r0 < 32 ? ka : kb;
-          m0 = (r0 < 32 ? ma : mb2) * d0;
-          k1 = r1 < 32 ? kc : kd;
-          m1 = (r1 < 32 ? mc : md) * d1;
+          int n0 = j0, n1 = j1;
+          for (int tau = 0; tau < nnext; ++tau) {
+            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, 16 + tau) * kN;
+            n0 = dk[n0];
+            n1 = dk[n1];
+          }
+          group_positions(n0, n1, ws, lane, posB0, posB1);
         }
-        // (3) R_sg = A_{sg+1}^T R_{sg+1} on the columns tau > sg
-        {
-          const int sn = sg + 1 < kT ? sg + 1 : sg;
-          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, sn) * kN;
-          const int r0 = dk[j0], r1 = dk[j1];
-          const float d0 = ld_bf16(din, sn * kN + j0), d1 = ld_bf16(din, sn * kN + j1);
-#pragma unroll
-          for (int tau = lo + 1; tau < kT; ++tau) {
-            const float a0 = __shfl_sync(0xffffffffu, R0[tau], r0 & 31);
-            const float a1 = __shfl_sync(0xffffffffu, R1[tau], r0 & 31);
-            const float c0 = __shfl_sync(0xffffffffu, R0[tau], r1 & 31);
-            const float c1 = __shfl_sync(0xffffffffu, R1[tau], r1 & 31);
-            const float n0 = d0 * (r0 < 32 ? a0 : a1), n1 = d1 * (r1 < 32 ? c0 : c1);
-            R0[tau] = tau > sg ? n0 : R0[tau];
-            R1[tau] = tau > sg ? n1 : R1[tau];
-          }
-        }
-        // (4) R_sg[:, sg] = C_sg (sg is in [lo, lo + 8))
-        {
-          const float c0 = ld_bf16(Cin, sg * kN + j0), c1 = ld_bf16(Cin, sg * kN + j1);
-#pragma unroll
-          for (int tau = lo; tau < lo + 8; ++tau) {
-            R0[tau] = tau == sg ? c0 : R0[tau];
-            R1[tau] = tau == sg ? c1 : R1[tau];
-          }
-        }
-        // (5) G[tau][sg] for tau in [8 * rnd, 8 * rnd + 8): partials (R is zero for
-        //     tau < sg), then a reduce-scatter of 8 values over 32 lanes
-#pragma unroll
-        for (int rnd = lo / 8; rnd < 2; ++rnd) {
-          float g[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) g[c] = bs0 * R0[8 * rnd + c] + bs1 * R1[8 * rnd + c];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const bool upr = lane & 16;
-            const float send = upr ? g[c] : g[c + 4];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-            g[c] = (upr ? g[c + 4] : g[c]) + recv;
-          }
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const bool upr = lane & 8;
-            const float send = upr ? g[c] : g[c + 2];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
-            g[c] = (upr ? g[c + 2] : g[c]) + recv;
-          }
-          {
-            const bool upr = lane & 4;
-            const float send = upr ? g[0] : g[1];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
-            g[0] = (upr ? g[1] : g[0]) + recv;
-          }
-          g[0] += __shfl_xor_sync(0xffffffffu, g[0], 2);
-          g[0] += __shfl_xor_sync(0xffffffffu, g[0], 1);
-          if ((lane & 3) == 0) {
-            const int tau = 8 * rnd + ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-            st_bf16_split(op + kOffGtHi, op + kOffGtLo, off_gt(tau, sg), g[0]);
-          }
-        }
-        // (6) read back Bh_sg (the other parity's accumulators serve the next step)
         __syncwarp();
-        const float bh0 = (float)bn[j0] * dn, bh1 = (float)bn[j1] * dn;
-        bn[j0] = 0;
-        bn[j1] = 0;
-        st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB0, sg), bh0);
-        st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB1, sg), bh1);
-      };
+
+        // ---- Phi_{T-1} (indices): the positions of S_a's order
+        int posA0, posA1, i0 = j0, i1 = j1;
+        for (int tau = 0; tau < nvalid; ++tau) {
+          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
+          i0 = dk[i0];
+          i1 = dk[i1];
+        }
+        group_positions(i0, i1, ws, lane, posA0, posA1);
+        // ---- forward chain: Phi_tau and Ct_tau = Phi_tau^T C_tau at the positions of S_a's order
+        float v0 = 1.f, v1 = 1.f;
+        {
+          const int o0 = kOffCt + off_ct_pos(posA0), o1 = kOffCt + off_ct_pos(posA1);
+          int f0 = j0, f1 = j1;
 #pragma unroll 1
-      for (int sg = kT - 1; sg >= 8; --sg) bwd_step(std::integral_constant<int, 8>(), sg);
+          for (int tau = 0; tau < kT; ++tau) {
+            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
+            float c0 = 0.f, c1 = 0.f;
+            if (tau < nvalid) {
+              v0 *= ld_bf16(din, tau * kN + f0);
+              v1 *= ld_bf16(din, tau * kN + f1);
+              f0 = dk[f0];
+              f1 = dk[f1];
+              c0 = v0 * ld_bf16(Cin, tau * kN + f0);
+              c1 = v1 * ld_bf16(Cin, tau * kN + f1);
+            }
+            float *c0p = reinterpret_cast<float *>(op + o0 + off_ct_tau(tau));
+            float *c1p = reinterpret_cast<float *>(op + o1 + off_ct_tau(tau));
+            if constexpr (kPrecise) {  // hi as fp32 (read as tf32), lo = the rest
+              c0p[0] = c0;
+              c1p[0] = c1;
+              c0p[(kOffCtLo - kOffCt) / 4] = c0 - tf32_trunc(c0);
+              c1p[(kOffCtLo - kOffCt) / 4] = c1 - tf32_trunc(c1);
+            } else {
+              c0p[0] = tf32_rn(c0);
+              c1p[0] = tf32_rn(c1);
+            }
+          }
+        }
+        // ---- Phi_{T-1} = (i, v): carry-step records
+        {
+          const int *cnt = reinterpret_cast<const int *>(ws + kScrCnt);
+          const int *offs = reinterpret_cast<const int *>(ws + kScrOffs);
+          // ordinal of each nonempty target group (targets ascending): target t's is
+          // the exclusive count of nonempty targets below t
+          const int na = cnt[2 * lane] > 0, nb = cnt[2 * lane + 1] > 0;
+          int incl = na + nb;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+          }
+          const int gex = incl - na - nb;
+          const int n_img = __shfl_sync(0xffffffffu, incl, 31);
+          const int g0 = __shfl_sync(0xffffffffu, gex, i0 >> 1), h0 = __shfl_sync(0xffffffffu, na, i0 >> 1);
+          const int g1 = __shfl_sync(0xffffffffu, gex, i1 >> 1), h1 = __shfl_sync(0xffffffffu, na, i1 >> 1);
+          const int e0 = g0 + ((i0 & 1) ? h0 : 0), e1 = g1 + ((i1 & 1) ? h1 : 0);
+          // the target's column in the next order: posB of row i (held by lane i & 31)
+          const int pb0a = __shfl_sync(0xffffffffu, posB0, i0 & 31), pb0b = __shfl_sync(0xffffffffu, posB1, i0 & 31);
+          const int pb1a = __shfl_sync(0xffffffffu, posB0, i1 & 31), pb1b = __shfl_sync(0xffffffffu, posB1, i1 & 31);
+          const int f0 = offs[i0], f1 = offs[i1];
+          const bool keep0 = posA0 != f0, keep1 = posA1 != f1;
+          const bool end0 = posA0 == f0 + cnt[i0] - 1, end1 = posA1 == f1 + cnt[i1] - 1;
+          int *meta = reinterpret_cast<int *>(op + kOffMeta);
+          meta[posA0] = (keep0 ? kMetaKeep : 0) | (end0 ? kMetaEnd : 0) | (e0 << kMetaOrdShift);
+          meta[posA1] = (keep1 ? kMetaKeep : 0) | (end1 ? kMetaEnd : 0) | (e1 << kMetaOrdShift);
+          if (end0) op[kOffGDst + e0] = (uint8_t)(i0 < 32 ? pb0a : pb0b);
+          if (end1) op[kOffGDst + e1] = (uint8_t)(i1 < 32 ? pb1a : pb1b);
+          int *hdr = reinterpret_cast<int *>(op + kOffHdr);
+          if (lane == 0) hdr[0] = n_img;
+          if (posA0 == 32) hdr[1] = keep0 ? e0 : -1;
+          if (posA1 == 32) hdr[1] = keep1 ? e1 : -1;
+          reinterpret_cast<float *>(op + kOffNu)[posA0] = v0;
+          reinterpret_cast<float *>(op + kOffNu)[posA1] = v1;
+          reinterpret_cast<int *>(op + kOffSrc)[posA0] = j0;
+          reinterpret_cast<int *>(op + kOffSrc)[posA1] = j1;
+          reinterpret_cast<int *>(op + kOffPhiIdx)[j0] = i0;
+          reinterpret_cast<int *>(op + kOffPhiIdx)[j1] = i1;
+          reinterpret_cast<float *>(op + kOffPhiVal)[j0] = v0;
+          reinterpret_cast<float *>(op + kOffPhiVal)[j1] = v1;
+        }
+
+
+        // ---- backward: the suffix Psi_sigma and Bh_sigma = Psi_sigma B_sigma as an
+        //      exact fixed-point sum (integer adds are order-independent), written at
+        //      the target's position in S_{a+1}'s order. Steps past the end of the
+        //      sequence are the identity; their B rows were zero-filled.
+        int k0 = j0, k1 = j1;          // Psi_sigma
+        float m0 = 1.f, m1 = 1.f;
 #pragma unroll 1
-      for (int sg = 7; sg >= 0; --sg) bwd_step(std::integral_constant<int, 0>(), sg);
+        for (int sg = kT - 1; sg >= 0; --sg) {
+          const bool sv = sg < nvalid;
+          const float bs0 = ld_bf16(Bin, sg * kN + j0), bs1 = ld_bf16(Bin, sg * kN + j1);
+          int *bn = bins + (sg & 1) * kN;  // the other parity's accumulators serve the next step
+          const float w0 = m0 * bs0, w1 = m1 * bs1;
+          const unsigned mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(w0), fabsf(w1))));
+          // |w| < 2^ex; 64 terms of magnitude < 2^24 stay below 2^30
+          const int ex = (int)((mb >> 23) & 0xff) - 126;
+          const int e = mb ? 24 - ex : 0;
+          const float up = exp2i(e), dn = exp2i(-e);
+          atomicAdd(&bn[k0], __float2int_rn(w0 * up));
+          atomicAdd(&bn[k1], __float2int_rn(w1 * up));
+          // Psi_{sg-1} = Psi_sg A_sg: column j <- d[j] * column idx[j]
+          {
+            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, sg) * kN;
+            const int r0 = sv ? dk[j0] : j0, r1 = sv ? dk[j1] : j1;
+            const float d0 = sv ? ld_bf16(din, sg * kN + j0) : 1.f, d1 = sv ? ld_bf16(din, sg * kN + j1) : 1.f;
+            const int ka = __shfl_sync(0xffffffffu, k0, r0 & 31), kb = __shfl_sync(0xffffffffu, k1, r0 & 31);
+            const float ma = __shfl_sync(0xffffffffu, m0, r0 & 31), mb2 = __shfl_sync(0xffffffffu, m1, r0 & 31);
+            const int kc = __shfl_sync(0xffffffffu, k0, r1 & 31), kd = __shfl_sync(0xffffffffu, k1, r1 & 31);
+            const float mc = __shfl_sync(0xffffffffu, m0, r1 & 31), md = __shfl_sync(0xffffffffu, m1, r1 & 31);
+            k0 = r0 < 32 ? ka : kb;
+            m0 = (r0 < 32 ? ma : mb2) * d0;
+            k1 = r1 < 32 ? kc : kd;
+            m1 = (r1 < 32 ? mc : md) * d1;
+          }
+          __syncwarp();
+          const float bh0 = (float)bn[j0] * dn, bh1 = (float)bn[j1] * dn;
+          bn[j0] = 0;
+          bn[j1] = 0;
+          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB0, sg), bh0);
+          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB1, sg), bh1);
+        }
+      } else {
+        // ---- backward readouts R_sigma[j][tau] = (A_tau...A_{sigma+1})^T C_tau and
+        //      G[tau][sigma] = B_sigma . R_sigma[:, tau]. Columns tau < sigma are zero
+        //      and stay zero under the gathers; rows past the end of the sequence
+        //      were zero-filled, so their columns stay zero too.
+        reinterpret_cast<uint4 *>(op + kOffGtHi)[lane] = make_uint4(0, 0, 0, 0);  // G^T above the diagonal
+        reinterpret_cast<uint4 *>(op + kOffGtHi)[lane + 32] = make_uint4(0, 0, 0, 0);
+        float R0[kT], R1[kT];
+#pragma unroll
+        for (int c = 0; c < kT; ++c) R0[c] = R1[c] = 0.f;
+        // lo_c: readout columns [lo, T) can be nonzero (sigma >= lo)
+        auto readout_step = [&](auto lo_c, int sg) {
+          constexpr int lo = decltype(lo_c)::value;
+          const float bs0 = ld_bf16(Bin, sg * kN + j0), bs1 = ld_bf16(Bin, sg * kN + j1);
+          // R_sg = A_{sg+1}^T R_{sg+1} on the columns tau > sg
+          {
+            const int sn = sg + 1 < kT ? sg + 1 : sg;
+            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, sn) * kN;
+            const int r0 = dk[j0], r1 = dk[j1];
+            const float d0 = ld_bf16(din, sn * kN + j0), d1 = ld_bf16(din, sn * kN + j1);
+#pragma unroll
+            for (int tau = lo + 1; tau < kT; ++tau) {
+              const float a0 = __shfl_sync(0xffffffffu, R0[tau], r0 & 31);
+              const float a1 = __shfl_sync(0xffffffffu, R1[tau], r0 & 31);
+              const float c0 = __shfl_sync(0xffffffffu, R0[tau], r1 & 31);
+              const float c1 = __shfl_sync(0xffffffffu, R1[tau], r1 & 31);
+              R0[tau] = d0 * (r0 < 32 ? a0 : a1);
+              R1[tau] = d1 * (r1 < 32 ? c0 : c1);
+            }
+          }
+          // R_sg[:, sg] = C_sg (sg is in [lo, lo + 8))
+          {
+            const float c0 = ld_bf16(Cin, sg * kN + j0), c1 = ld_bf16(Cin, sg * kN + j1);
+#pragma unroll
+            for (int tau = lo; tau < lo + 8; ++tau) {
+              R0[tau] = tau == sg ? c0 : R0[tau];
+              R1[tau] = tau == sg ? c1 : R1[tau];
+            }
+          }
+          // G[tau][sg] for tau in [8 * rnd, 8 * rnd + 8): partials, then a
+          // reduce-scatter of 8 values over 32 lanes
+#pragma unroll
+          for (int rnd = lo / 8; rnd < 2; ++rnd) {
+            float g[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) g[c] = bs0 * R0[8 * rnd + c] + bs1 * R1[8 * rnd + c];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const bool upr = lane & 16;
+              const float send = upr ? g[c] : g[c + 4];
+              const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+              g[c] = (upr ? g[c + 4] : g[c]) + recv;
+            }
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const bool upr = lane & 8;
+              const float send = upr ? g[c] : g[c + 2];
+              const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
+              g[c] = (upr ? g[c + 2] : g[c]) + recv;
+            }
+            {
+              const bool upr = lane & 4;
+              const float send = upr ? g[0] : g[1];
+              const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
+              g[0] = (upr ? g[1] : g[0]) + recv;
+            }
+            g[0] += __shfl_xor_sync(0xffffffffu, g[0], 2);
+            g[0] += __shfl_xor_sync(0xffffffffu, g[0], 1);
+            if ((lane & 3) == 0) {
+              const int tau = 8 * rnd + ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+              st_bf16_split(op + kOffGtHi, op + kOffGtLo, off_gt(tau, sg), g[0]);
+            }
+          }
+        };
+#pragma unroll 1
+        for (int sg = kT - 1; sg >= 8; --sg) readout_step(std::integral_constant<int, 8>(), sg);
+#pragma unroll 1
+        for (int sg = 7; sg >= 0; --sg) readout_step(std::integral_constant<int, 0>(), sg);
+      }
 
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->full[stg]);
-      // prefetch this warp's next sub-chunk into its (now free) input stage
-      const int nxt = sub + kNW;
-      if (nxt < nsub) load_inputs<TL>(a, in, b, h, nxt, lane);
-      cp_async_commit();
+      // both warps are done with the input stage: prefetch the pair's next sub-chunk
+      pair_sync(pbar);
+      if (role == 0) {
+        const int nxt = sub + kNW;
+        if (nxt < nsub) load_inputs<TL>(a, in, b, h, nxt, lane);
+        cp_async_commit();
+      }
     }
-    cp_async_wait<0>();
+    if (role == 0) cp_async_wait<0>();
   } else {
     // ============================================ carry state, output, and the MMA issue (warp 4, lane 0)
     const int q = warp & 3;                 // tensor-memory quarter
@@ -648,37 +681,34 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     const int p = 16 * q + lane;            // state column owned by this lane
     const uint32_t lanebase = (uint32_t)(32 * q) << 16;
     const bool issuer = (q == 0) && (lane == 0);
-    // ---- MMA issue (one thread). Descriptors of operand stage 0; another stage
-    //      adds its offset / 16 to the start-address field (no carry out of it).
+    // ---- MMA issue (one thread)
     constexpr uint32_t kIdU = idesc_bf16_f32(64, kN, true, true);
     constexpr uint32_t kIdG = idesc_bf16_f32(64, kT, true, false);
     constexpr uint32_t kIdC = idesc_tf32_f32(64, kT);
     const uint32_t ob = smem_u32(op_base);
-    const uint64_t dX = smem_desc(ob + kOffX, (kP / 8) * 128, 128);
-    const uint64_t dBh = smem_desc(ob + kOffBhHi, kBhLbo, kBhSbo), dBl = smem_desc(ob + kOffBhLo, kBhLbo, kBhSbo);
-    const uint64_t dGh = smem_desc(ob + kOffGtHi, 128, 256), dGl = smem_desc(ob + kOffGtLo, 128, 256);
-    const uint64_t dCt = smem_desc(ob + kOffCt, kCtLbo, kCtSbo), dCl = smem_desc(ob + kOffCtLo, kCtLbo, kCtSbo);
     // U_u into state region (u + 1) mod R and the intra-sub-chunk part of Y_u
     // (written, not accumulated). The region held S_{u+1-R}: this is issued only
     // after the carry step of sub-chunk u+1-R is complete and its readout has been
     // issued (tensor-core operations of one thread execute in issue order).
     auto issue_u_now = [&](int u) {
-      const uint64_t so = (uint64_t)((u % a.nst) * (kOpStage >> 4));
+      const uint32_t o = ob + (u % a.nst) * kOpStage;
       const uint32_t dU = tbase + col_state((u + 1) % kRing), dY = tbase + kColY + (u % kNY) * kT;
-      mma_bf16(dU, dX + so, dBh + so, kIdU, 0);
-      mma_bf16(dU, dX + so, dBl + so, kIdU, 1);
-      mma_bf16(dY, dX + so, dGh + so, kIdG, 0);
-      mma_bf16(dY, dX + so, dGl + so, kIdG, 1);
+      const uint64_t dX = smem_desc(o + kOffX, (kP / 8) * 128, 128);
+      mma_bf16(dU, dX, smem_desc(o + kOffBhHi, kBhLbo, kBhSbo), kIdU, 0);
+      mma_bf16(dU, dX, smem_desc(o + kOffBhLo, kBhLbo, kBhSbo), kIdU, 1);
+      mma_bf16(dY, dX, smem_desc(o + kOffGtHi, 128, 256), kIdG, 0);
+      mma_bf16(dY, dX, smem_desc(o + kOffGtLo, 128, 256), kIdG, 1);
       mma_commit(&bars->ufull[(u + 1) % kRing]);
     };
     // readout of the entering state S_s: A operand from tensor memory (tf32)
     auto issue_y_now = [&](int s) {
       const int st = s % a.nst;
-      const uint64_t so = (uint64_t)(st * (kOpStage >> 4));
+      const uint32_t o = ob + st * kOpStage;
       const uint32_t dY = tbase + kColY + (s % kNY) * kT, aS = tbase + col_state(s % kRing);
+      const uint64_t dCt = smem_desc(o + kOffCt, kCtLbo, kCtSbo), dCl = smem_desc(o + kOffCtLo, kCtLbo, kCtSbo);
 #pragma unroll
       for (int ks = 0; ks < kN / 8; ++ks) {
-        const uint64_t kso = so + (uint64_t)((ks * 2 * kCtLbo) >> 4);
+        const uint64_t kso = (uint64_t)((ks * 2 * kCtLbo) >> 4);  // start-address field step (no carry out)
         mma_tf32_ts(dY, aS + ks * 8, dCt + kso, kIdC, 1);
         if constexpr (kPrecise) {
           mma_tf32_ts(dY, aS + ks * 8, dCl + kso, kIdC, 1);
@@ -827,23 +857,16 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           const unsigned ec = (unsigned)(ecross - base);
           if (hh == 1 && ecross >= 0 && ec < 16u) cs[ec * 16 + pl] += tail;
           __syncwarp();
-          // U at the group ends += group totals (the second eight only when needed)
-          const bool more = base + 8 < n_img;
-          float u[16];
+          // U at the group ends += group totals, eight at a time
+#pragma unroll 1
+          for (int e8 = base; e8 < base + 16 && e8 < n_img; e8 += 8) {
+            float u[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) tmem_ld1_if(RU + op[kOffGDst + base + e], u[e], base + e < n_img);
-          if (more) {
+            for (int e = 0; e < 8; ++e) tmem_ld1_if(RU + op[kOffGDst + e8 + e], u[e], e8 + e < n_img);
+            tmem_wait_ld();
 #pragma unroll
-            for (int e = 8; e < 16; ++e) tmem_ld1_if(RU + op[kOffGDst + base + e], u[e], base + e < n_img);
-          }
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            tmem_st1_if(RU + op[kOffGDst + base + e], u[e] + cs[e * 16 + pl], base + e < n_img);
-          if (more) {
-#pragma unroll
-            for (int e = 8; e < 16; ++e)
-              tmem_st1_if(RU + op[kOffGDst + base + e], u[e] + cs[e * 16 + pl], base + e < n_img);
+            for (int e = 0; e < 8; ++e)
+              tmem_st1_if(RU + op[kOffGDst + e8 + e], u[e] + cs[(e8 - base + e) * 16 + pl], e8 + e < n_img);
           }
           __syncwarp();
         }
@@ -918,7 +941,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kNW) {
+  if (warp == kCarryWarp0) {
     tc_fence_after();
     tmem_dealloc(tbase, kTmemCols);
   }
