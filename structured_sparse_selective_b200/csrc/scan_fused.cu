@@ -67,9 +67,10 @@ constexpr int kT = 16;   // sub-chunk length
 constexpr int kNW = 4;   // prep warp pairs; pair w prepares sub-chunks w, w + 4, ...
 constexpr int kPrepWarps = 2 * kNW;
 constexpr int kCarryWarp0 = kPrepWarps;  // warps 8-11 carry the state (one per tensor-memory quarter)
+constexpr int kIssuerWarp = kCarryWarp0 + 4;  // warp 12: one thread issues the MMAs
 constexpr int kMaxStages = 6;  // operand stages (sub-chunk a uses stage a mod nst, nst >= kNW)
 constexpr int kNY = 4;   // output accumulator slots
-constexpr int kThreads = 32 * (kPrepWarps + 4);  // 8 prep warps + 4 carry warps (warp 8 also issues the MMAs)
+constexpr int kThreads = 32 * (kPrepWarps + 5);  // 8 prep warps, 4 carry warps, 1 MMA-issuing warp
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
 
 // tensor-memory columns: 64-column state regions (a ring of 3, or 2 plus S_lo
@@ -157,7 +158,7 @@ __device__ __noinline__ bool wait_bar(Bars *bars, uint64_t *bar, uint32_t parity
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = now_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
     if (*(volatile int *)&bars->abort) return false;
     if (now_ns() - t0 > kTimeoutNs) {
       *(volatile int *)&bars->abort = 1;
@@ -674,81 +675,13 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       }
     }
     if (role == 0) cp_async_wait<0>();
-  } else {
-    // ============================================ carry state, output, and the MMA issue (warp 4, lane 0)
+  } else if (warp < kIssuerWarp) {
+    // ============================================ carry state and output (warps 8-11)
     const int q = warp & 3;                 // tensor-memory quarter
     const bool act = lane < 16;
     const int p = 16 * q + lane;            // state column owned by this lane
     const uint32_t lanebase = (uint32_t)(32 * q) << 16;
-    const bool issuer = (q == 0) && (lane == 0);
-    // ---- MMA issue (one thread)
-    constexpr uint32_t kIdU = idesc_bf16_f32(64, kN, true, true);
-    constexpr uint32_t kIdG = idesc_bf16_f32(64, kT, true, false);
-    constexpr uint32_t kIdC = idesc_tf32_f32(64, kT);
-    const uint32_t ob = smem_u32(op_base);
-    // U_u into state region (u + 1) mod R and the intra-sub-chunk part of Y_u
-    // (written, not accumulated). The region held S_{u+1-R}: this is issued only
-    // after the carry step of sub-chunk u+1-R is complete and its readout has been
-    // issued (tensor-core operations of one thread execute in issue order).
-    auto issue_u_now = [&](int u) {
-      const uint32_t o = ob + (u % a.nst) * kOpStage;
-      const uint32_t dU = tbase + col_state((u + 1) % kRing), dY = tbase + kColY + (u % kNY) * kT;
-      const uint64_t dX = smem_desc(o + kOffX, (kP / 8) * 128, 128);
-      mma_bf16(dU, dX, smem_desc(o + kOffBhHi, kBhLbo, kBhSbo), kIdU, 0);
-      mma_bf16(dU, dX, smem_desc(o + kOffBhLo, kBhLbo, kBhSbo), kIdU, 1);
-      mma_bf16(dY, dX, smem_desc(o + kOffGtHi, 128, 256), kIdG, 0);
-      mma_bf16(dY, dX, smem_desc(o + kOffGtLo, 128, 256), kIdG, 1);
-      mma_commit(&bars->ufull[(u + 1) % kRing]);
-    };
-    // readout of the entering state S_s: A operand from tensor memory (tf32)
-    auto issue_y_now = [&](int s) {
-      const int st = s % a.nst;
-      const uint32_t o = ob + st * kOpStage;
-      const uint32_t dY = tbase + kColY + (s % kNY) * kT, aS = tbase + col_state(s % kRing);
-      const uint64_t dCt = smem_desc(o + kOffCt, kCtLbo, kCtSbo), dCl = smem_desc(o + kOffCtLo, kCtLbo, kCtSbo);
-#pragma unroll
-      for (int ks = 0; ks < kN / 8; ++ks) {
-        const uint64_t kso = (uint64_t)((ks * 2 * kCtLbo) >> 4);  // start-address field step (no carry out)
-        mma_tf32_ts(dY, aS + ks * 8, dCt + kso, kIdC, 1);
-        if constexpr (kPrecise) {
-          mma_tf32_ts(dY, aS + ks * 8, dCl + kso, kIdC, 1);
-          mma_tf32_ts(dY, tbase + kColSlo + ks * 8, dCt + kso, kIdC, 1);
-        }
-      }
-      mma_commit(&bars->yfull[s % kNY]);
-      mma_commit(&bars->opfree[st]);
-      if constexpr (kPrecise) mma_commit(&bars->slofree);
-    };
-    // issue U groups up to `upto`: waiting for their operands and output slot when
-    // `block`, else only those already ready
-    int next_u = 0;
-    auto issue_us = [&](int upto, bool block) -> bool {
-      for (; next_u <= upto && next_u < nsub; ++next_u) {
-        const int st = next_u % a.nst;
-        uint64_t *fb = &bars->full[st];
-        const uint32_t fp = (next_u / a.nst) & 1;
-        const bool needy = next_u >= kNY;
-        uint64_t *yb = &bars->yfree[next_u % kNY];
-        const uint32_t yp = ((next_u / kNY) - 1) & 1;
-        if (!block) {
-          if (!mbar_test_wait(fb, fp) || (needy && !mbar_test_wait(yb, yp))) return true;
-        } else {
-          if (!mbar_test_wait(fb, fp) && !wait_bar(bars, fb, fp, a.err)) return false;
-          if (needy && !mbar_test_wait(yb, yp) && !wait_bar(bars, yb, yp, a.err)) return false;
-        }
-        tc_fence_after();
-        issue_u_now(next_u);
-      }
-      return true;
-    };
-    auto issue_y = [&](int s) -> bool {
-      if (!mbar_test_wait(&bars->sready, s & 1) && !wait_bar(bars, &bars->sready, s & 1, a.err)) return false;
-      tc_fence_after();
-      issue_y_now(s);
-      return true;
-    };
     bool ok = true;
-    if (issuer) ok = issue_us(0, true) && issue_us(kRing - 2, false);
     // S_0 = h0 (or 0) in the source order of sub-chunk 0's composite
     if (nsub > 0 && !wait_bar_warp(bars, &bars->full[0], 0, a.err)) ok = false;
     if (__all_sync(0xffffffffu, ok)) {
@@ -772,7 +705,6 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sready);
     }
-    if (issuer && ok && nsub > 0) ok = issue_y(0);
     TO *yout = static_cast<TO *>(a.y);
     // output rows of sub-chunk sub from its accumulator slot (already loaded)
     auto store_y = [&](int sub, const float *v) {
@@ -891,12 +823,6 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         mbar_arrive(&bars->opfree[st]);
       }
       done = sub + 1;
-      // Next MMAs: the readout of S_{sub+1} once every quarter of it is complete.
-      // The input part of Y_{sub+1} (written, not accumulated) must precede it.
-      if (issuer && sub + 1 < nsub) {
-        ok = (mbar_test_wait(&bars->sready, (sub + 1) & 1) || wait_bar(bars, &bars->sready, (sub + 1) & 1, a.err)) &&
-             issue_us(sub + 1, true) && issue_y(sub + 1) && issue_us(sub + kRing - 1, false);
-      }
     }
     // output of the last sub-chunk
     if (__all_sync(0xffffffffu, ok) && done == nsub && nsub > 0 &&
@@ -929,14 +855,91 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           for (int i = 0; i < 16; ++i) a.h_final[((b * a.H + h) * kN + c0 + i) * kP + p] = v[i];
       }
     }
-    if (issuer) {
-      // every MMA issued so far has completed once this arrives
-      mma_commit(&bars->drain);
-      const uint64_t t0 = now_ns();
-      while (!mbar_try_wait(&bars->drain, 0) && now_ns() - t0 < kTimeoutNs) {
-      }
-    }
     __syncwarp();
+
+  } else if (lane == 0) {
+    // ============================================ MMA issue (warp 12, one thread)
+    // ---- MMA issue (one thread)
+    constexpr uint32_t kIdU = idesc_bf16_f32(64, kN, true, true);
+    constexpr uint32_t kIdG = idesc_bf16_f32(64, kT, true, false);
+    constexpr uint32_t kIdC = idesc_tf32_f32(64, kT);
+    const uint32_t ob = smem_u32(op_base);
+    // U_u into state region (u + 1) mod R and the intra-sub-chunk part of Y_u
+    // (written, not accumulated). The region held S_{u+1-R}: this is issued only
+    // after the carry step of sub-chunk u+1-R is complete and its readout has been
+    // issued (tensor-core operations of one thread execute in issue order).
+    auto issue_u_now = [&](int u) {
+      const uint32_t o = ob + (u % a.nst) * kOpStage;
+      const uint32_t dU = tbase + col_state((u + 1) % kRing), dY = tbase + kColY + (u % kNY) * kT;
+      const uint64_t dX = smem_desc(o + kOffX, (kP / 8) * 128, 128);
+      mma_bf16(dU, dX, smem_desc(o + kOffBhHi, kBhLbo, kBhSbo), kIdU, 0);
+      mma_bf16(dU, dX, smem_desc(o + kOffBhLo, kBhLbo, kBhSbo), kIdU, 1);
+      mma_bf16(dY, dX, smem_desc(o + kOffGtHi, 128, 256), kIdG, 0);
+      mma_bf16(dY, dX, smem_desc(o + kOffGtLo, 128, 256), kIdG, 1);
+      mma_commit(&bars->ufull[(u + 1) % kRing]);
+    };
+    // readout of the entering state S_s: A operand from tensor memory (tf32)
+    auto issue_y_now = [&](int s) {
+      const int st = s % a.nst;
+      const uint32_t o = ob + st * kOpStage;
+      const uint32_t dY = tbase + kColY + (s % kNY) * kT, aS = tbase + col_state(s % kRing);
+      const uint64_t dCt = smem_desc(o + kOffCt, kCtLbo, kCtSbo), dCl = smem_desc(o + kOffCtLo, kCtLbo, kCtSbo);
+#pragma unroll
+      for (int ks = 0; ks < kN / 8; ++ks) {
+        const uint64_t kso = (uint64_t)((ks * 2 * kCtLbo) >> 4);  // start-address field step (no carry out)
+        mma_tf32_ts(dY, aS + ks * 8, dCt + kso, kIdC, 1);
+        if constexpr (kPrecise) {
+          mma_tf32_ts(dY, aS + ks * 8, dCl + kso, kIdC, 1);
+          mma_tf32_ts(dY, tbase + kColSlo + ks * 8, dCt + kso, kIdC, 1);
+        }
+      }
+      mma_commit(&bars->yfull[s % kNY]);
+      mma_commit(&bars->opfree[st]);
+      if constexpr (kPrecise) mma_commit(&bars->slofree);
+    };
+    // issue U groups up to `upto`: waiting for their operands and output slot when
+    // `block`, else only those already ready
+    int next_u = 0;
+    auto issue_us = [&](int upto, bool block) -> bool {
+      for (; next_u <= upto && next_u < nsub; ++next_u) {
+        const int st = next_u % a.nst;
+        uint64_t *fb = &bars->full[st];
+        const uint32_t fp = (next_u / a.nst) & 1;
+        const bool needy = next_u >= kNY;
+        uint64_t *yb = &bars->yfree[next_u % kNY];
+        const uint32_t yp = ((next_u / kNY) - 1) & 1;
+        if (!block) {
+          if (!mbar_test_wait(fb, fp) || (needy && !mbar_test_wait(yb, yp))) return true;
+        } else {
+          if (!mbar_test_wait(fb, fp) && !wait_bar(bars, fb, fp, a.err)) return false;
+          if (needy && !mbar_test_wait(yb, yp) && !wait_bar(bars, yb, yp, a.err)) return false;
+        }
+        tc_fence_after();
+        issue_u_now(next_u);
+      }
+      return true;
+    };
+    auto issue_y = [&](int s) -> bool {
+      if (!mbar_test_wait(&bars->sready, s & 1) && !wait_bar(bars, &bars->sready, s & 1, a.err)) return false;
+      tc_fence_after();
+      issue_y_now(s);
+      return true;
+    };
+    // U_0 (and U_1 when ready), the readout of S_0 once the carry warps wrote it,
+    // then per sub-chunk: the readout of S_{s+1} once every quarter of it is
+    // complete (after the input part of Y_{s+1}, which is written, not
+    // accumulated) and the input terms as far ahead as the ring allows.
+    bool ok = issue_us(0, true) && issue_us(kRing - 2, false) && (nsub == 0 || issue_y(0));
+    for (int s = 0; ok && s + 1 < nsub; ++s) {
+      if constexpr (kRing == 2)  // U_{s+1} overwrites S_s: the carry step of s must be complete
+        ok = mbar_test_wait(&bars->sready, (s + 1) & 1) || wait_bar(bars, &bars->sready, (s + 1) & 1, a.err);
+      ok = ok && issue_us(s + 1, true) && issue_y(s + 1) && issue_us(s + kRing - 1, false);
+    }
+    // every MMA issued so far has completed once this arrives
+    mma_commit(&bars->drain);
+    const uint64_t t0 = now_ns();
+    while (!mbar_try_wait(&bars->drain, 0) && now_ns() - t0 < kTimeoutNs) {
+    }
   }
 
   tc_fence_before();
