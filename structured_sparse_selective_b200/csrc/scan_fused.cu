@@ -756,9 +756,11 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         if (sub > 0) {
           const int tp = (sub - 1) * kT;
           const int nv = (int)(a.L - tp < kT ? a.L - tp : kT);
+          TO *yrow = yout + ((b * a.L + tp + 8 * hh) * a.H + h) * kP + 16 * q + pl;
+          const int64_t ystep = a.H * kP;
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            if (8 * hh + i < nv) store_out(yout + ((b * a.L + tp + 8 * hh + i) * a.H + h) * kP + 16 * q + pl, yv[i]);
+            if (8 * hh + i < nv) store_out(yrow + i * ystep, yv[i]);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->yfree[(sub - 1) % kNY]);
