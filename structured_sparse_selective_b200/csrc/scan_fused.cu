@@ -341,6 +341,51 @@ __device__ __forceinline__ bool pair_and(uint32_t id, bool v) {
   return r != 0;
 }
 
+// ------------------------------------------------------------- MMA issue
+
+// U_u into state region (u + 1) mod R and the intra-sub-chunk part of Y_u
+// (written, not accumulated). The region held S_{u+1-R}: this is issued only
+// after the carry step of sub-chunk u+1-R is complete and its readout has been
+// issued (tensor-core operations of one thread execute in issue order).
+template <bool kPrecise>
+__device__ __noinline__ void mma_issue_input(Bars *bars, uint32_t ob, int nst, uint32_t tbase, int u) {
+  constexpr int kRing = kPrecise ? 2 : 3;
+  constexpr uint32_t kIdU = idesc_bf16_f32(64, kN, true, true);
+  constexpr uint32_t kIdG = idesc_bf16_f32(64, kT, true, false);
+  const uint32_t o = ob + (u % nst) * op_stage_bytes(kPrecise);
+  const uint32_t dU = tbase + col_state((u + 1) % kRing), dY = tbase + kColY + (u % kNY) * kT;
+  const uint64_t dX = smem_desc(o + kOffX, (kP / 8) * 128, 128);
+  mma_bf16(dU, dX, smem_desc(o + kOffBhHi, kBhLbo, kBhSbo), kIdU, 0);
+  mma_bf16(dU, dX, smem_desc(o + kOffBhLo, kBhLbo, kBhSbo), kIdU, 1);
+  mma_bf16(dY, dX, smem_desc(o + kOffGtHi, 128, 256), kIdG, 0);
+  mma_bf16(dY, dX, smem_desc(o + kOffGtLo, 128, 256), kIdG, 1);
+  mma_commit(&bars->ufull[(u + 1) % kRing]);
+}
+
+// Readout of the entering state S_s into Y_s: A operand from tensor memory (tf32).
+// Releases the operand stage (and the S_lo plane) once done.
+template <bool kPrecise>
+__device__ __noinline__ void mma_issue_readout(Bars *bars, uint32_t ob, int nst, uint32_t tbase, int s) {
+  constexpr int kRing = kPrecise ? 2 : 3;
+  constexpr uint32_t kIdC = idesc_tf32_f32(64, kT);
+  const int st = s % nst;
+  const uint32_t o = ob + st * op_stage_bytes(kPrecise);
+  const uint32_t dY = tbase + kColY + (s % kNY) * kT, aS = tbase + col_state(s % kRing);
+  const uint64_t dCt = smem_desc(o + kOffCt, kCtLbo, kCtSbo), dCl = smem_desc(o + kOffCtLo, kCtLbo, kCtSbo);
+#pragma unroll
+  for (int ks = 0; ks < kN / 8; ++ks) {
+    const uint64_t kso = (uint64_t)((ks * 2 * kCtLbo) >> 4);  // start-address field step (no carry out)
+    mma_tf32_ts(dY, aS + ks * 8, dCt + kso, kIdC, 1);
+    if constexpr (kPrecise) {
+      mma_tf32_ts(dY, aS + ks * 8, dCl + kso, kIdC, 1);
+      mma_tf32_ts(dY, tbase + kColSlo + ks * 8, dCt + kso, kIdC, 1);
+    }
+  }
+  mma_commit(&bars->yfull[s % kNY]);
+  mma_commit(&bars->opfree[st]);
+  if constexpr (kPrecise) mma_commit(&bars->slofree);
+}
+
 // ------------------------------------------------------------- the kernel
 
 template <typename TL, typename TO, bool kPrecise>
@@ -861,44 +906,9 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
 
   } else if (lane == 0) {
     // ============================================ MMA issue (warp 12, one thread)
-    // ---- MMA issue (one thread)
-    constexpr uint32_t kIdU = idesc_bf16_f32(64, kN, true, true);
-    constexpr uint32_t kIdG = idesc_bf16_f32(64, kT, true, false);
-    constexpr uint32_t kIdC = idesc_tf32_f32(64, kT);
     const uint32_t ob = smem_u32(op_base);
-    // U_u into state region (u + 1) mod R and the intra-sub-chunk part of Y_u
-    // (written, not accumulated). The region held S_{u+1-R}: this is issued only
-    // after the carry step of sub-chunk u+1-R is complete and its readout has been
-    // issued (tensor-core operations of one thread execute in issue order).
-    auto issue_u_now = [&](int u) {
-      const uint32_t o = ob + (u % a.nst) * kOpStage;
-      const uint32_t dU = tbase + col_state((u + 1) % kRing), dY = tbase + kColY + (u % kNY) * kT;
-      const uint64_t dX = smem_desc(o + kOffX, (kP / 8) * 128, 128);
-      mma_bf16(dU, dX, smem_desc(o + kOffBhHi, kBhLbo, kBhSbo), kIdU, 0);
-      mma_bf16(dU, dX, smem_desc(o + kOffBhLo, kBhLbo, kBhSbo), kIdU, 1);
-      mma_bf16(dY, dX, smem_desc(o + kOffGtHi, 128, 256), kIdG, 0);
-      mma_bf16(dY, dX, smem_desc(o + kOffGtLo, 128, 256), kIdG, 1);
-      mma_commit(&bars->ufull[(u + 1) % kRing]);
-    };
-    // readout of the entering state S_s: A operand from tensor memory (tf32)
-    auto issue_y_now = [&](int s) {
-      const int st = s % a.nst;
-      const uint32_t o = ob + st * kOpStage;
-      const uint32_t dY = tbase + kColY + (s % kNY) * kT, aS = tbase + col_state(s % kRing);
-      const uint64_t dCt = smem_desc(o + kOffCt, kCtLbo, kCtSbo), dCl = smem_desc(o + kOffCtLo, kCtLbo, kCtSbo);
-#pragma unroll
-      for (int ks = 0; ks < kN / 8; ++ks) {
-        const uint64_t kso = (uint64_t)((ks * 2 * kCtLbo) >> 4);  // start-address field step (no carry out)
-        mma_tf32_ts(dY, aS + ks * 8, dCt + kso, kIdC, 1);
-        if constexpr (kPrecise) {
-          mma_tf32_ts(dY, aS + ks * 8, dCl + kso, kIdC, 1);
-          mma_tf32_ts(dY, tbase + kColSlo + ks * 8, dCt + kso, kIdC, 1);
-        }
-      }
-      mma_commit(&bars->yfull[s % kNY]);
-      mma_commit(&bars->opfree[st]);
-      if constexpr (kPrecise) mma_commit(&bars->slofree);
-    };
+    auto issue_u_now = [&](int u) { mma_issue_input<kPrecise>(bars, ob, a.nst, tbase, u); };
+    auto issue_y_now = [&](int s_) { mma_issue_readout<kPrecise>(bars, ob, a.nst, tbase, s_); };
     // issue U groups up to `upto`: waiting for their operands and output slot when
     // `block`, else only those already ready
     int next_u = 0;
@@ -928,14 +938,16 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       return true;
     };
     // U_0 (and U_1 when ready), the readout of S_0 once the carry warps wrote it,
-    // then per sub-chunk: the readout of S_{s+1} once every quarter of it is
-    // complete (after the input part of Y_{s+1}, which is written, not
-    // accumulated) and the input terms as far ahead as the ring allows.
+    // then per sub-chunk s, once S_{s+1} is complete: U_{s+1} (its output part
+    // must precede the readout of S_{s+1}: it is written, not accumulated), the
+    // input term furthest ahead that the ring allows if its operands are ready
+    // (the next carry steps wait for it), the readout of S_{s+1}, and that input
+    // term after all.
     bool ok = issue_us(0, true) && issue_us(kRing - 2, false) && (nsub == 0 || issue_y(0));
     for (int s = 0; ok && s + 1 < nsub; ++s) {
-      if constexpr (kRing == 2)  // U_{s+1} overwrites S_s: the carry step of s must be complete
-        ok = mbar_test_wait(&bars->sready, (s + 1) & 1) || wait_bar(bars, &bars->sready, (s + 1) & 1, a.err);
-      ok = ok && issue_us(s + 1, true) && issue_y(s + 1) && issue_us(s + kRing - 1, false);
+      ok = mbar_test_wait(&bars->sready, (s + 1) & 1) || wait_bar(bars, &bars->sready, (s + 1) & 1, a.err);
+      ok = ok && issue_us(s + 1, true) && issue_us(s + kRing - 1, false) && issue_y(s + 1) &&
+           issue_us(s + kRing - 1, true);
     }
     // every MMA issued so far has completed once this arrives
     mma_commit(&bars->drain);
