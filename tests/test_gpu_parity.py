@@ -286,3 +286,35 @@ def test_fused_path_logit_and_output_dtypes(cuda_device, ldt, odt):
     out = pd.forward(g["logits"], g["idx"], g["d"], g["B"], g["C"], g["x"], out_dtype=odt, want_s=True)
     torch.cuda.synchronize()
     compare_full(inp, out)
+
+
+# ------------------------------------------- recurrent decode: one token per call
+
+@pytest.mark.parametrize("recipe,kw", [("lm", dict(batch=2, seqlen=40, heads=2)),
+                                       ("tiny", dict(batch=1, seqlen=33, heads=2))])
+def test_token_by_token_decode_matches_the_whole_sequence(cuda_device, recipe, kw):
+    """Decoding one step at a time (L = 1, the state carried through h0 -> h_final)
+    gives the outputs and final state of the whole-sequence forward pass, which is the
+    oracle's recurrence read one step at a time."""
+    sp = workloads.spec(recipe, **kw)
+    inp = workloads.generate(sp, seed=16)
+    g = {k: v.to(cuda_device) for k, v in inp.items()}
+    whole = pd.forward(g["logits"], g["idx"], g["d"], g["B"], g["C"], g["x"], out_dtype=torch.float32,
+                       want_s=True)
+    h = torch.zeros(sp.batch, sp.heads, sp.N, sp.P, dtype=torch.float32, device=cuda_device)
+    ys, ss = [], []
+    for t in range(sp.seqlen):
+        step = {k: g[k][:, t:t + 1].contiguous() for k in ("logits", "d", "B", "C", "x")}
+        o = pd.forward(step["logits"], g["idx"], step["d"], step["B"], step["C"], step["x"], h0=h,
+                       out_dtype=torch.float32, want_s=True)
+        ys.append(o["y"])
+        ss.append(o["s"])
+        h = o["h_final"]
+    torch.cuda.synchronize(cuda_device)
+    y = torch.cat(ys, dim=1)
+    assert torch.equal(torch.cat(ss, dim=1), whole["s"])
+    scale = whole["y"].abs().amax().item()
+    assert (y - whole["y"]).abs().amax().item() <= 1e-4 * scale
+    hs = whole["h_final"].abs().amax().item()
+    assert (h - whole["h_final"]).abs().amax().item() <= 1e-4 * hs
+    compare_full(inp, {"y": y.cpu(), "h_final": h.cpu()})
