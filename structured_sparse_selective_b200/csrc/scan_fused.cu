@@ -295,7 +295,7 @@ __device__ __forceinline__ int argmax_row(const uint8_t *row, int K) {
 // Positions of the 64 sources j0 = lane, j1 = lane + 32 of an index map when the
 // sources are grouped by target row (targets ascending, sources ascending in a
 // group). Leaves per-target counts and first positions in the warp's scratch.
-__device__ __forceinline__ void group_positions(int t0, int t1, uint8_t *ws, int lane, int &pos0, int &pos1) {
+__device__ __noinline__ int2 group_positions(int t0, int t1, uint8_t *ws, int lane) {
   int *cnt = reinterpret_cast<int *>(ws + kScrCnt);
   int *cntlo = reinterpret_cast<int *>(ws + kScrCntLo);
   int *offs = reinterpret_cast<int *>(ws + kScrOffs);
@@ -322,8 +322,7 @@ __device__ __forceinline__ void group_positions(int t0, int t1, uint8_t *ws, int
   const unsigned lt = (1u << lane) - 1u;
   const unsigned m0 = __match_any_sync(0xffffffffu, t0);
   const unsigned m1 = __match_any_sync(0xffffffffu, t1);
-  pos0 = offs[t0] + __popc(m0 & lt);
-  pos1 = offs[t1] + cntlo[t1] + __popc(m1 & lt);
+  return make_int2(offs[t0] + __popc(m0 & lt), offs[t1] + cntlo[t1] + __popc(m1 & lt));
 }
 
 // Named barrier over the two warps of a prep pair; the _and form also returns
@@ -449,8 +448,6 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     uint8_t *ws = scr + pair * kScrBytes;
     int *bins = reinterpret_cast<int *>(ws + kScrBins);
     if (role == 0) {
-      if (pair < nsub) load_inputs<TL>(a, in, b, h, pair, lane);
-      cp_async_commit();
 #pragma unroll
       for (int c = 0; c < 4; ++c) bins[lane + 32 * c] = 0;
     }
@@ -461,6 +458,11 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       const int t0 = sub * kT;
       const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
       const int nnext = (int)(a.L - t0 - kT < kT ? (a.L - t0 - kT > 0 ? a.L - t0 - kT : 0) : kT);
+      // the inputs load while the stage is being released
+      if (role == 0) {
+        load_inputs<TL>(a, in, b, h, sub, lane);
+        cp_async_commit();
+      }
       bool ok = wait_bar_warp(bars, &bars->opfree[stg], ((sub / a.nst) & 1) ^ 1, a.err);
       if (role == 0) cp_async_wait<0>();
       // one decision for the pair; the barrier also publishes the loaded inputs
@@ -502,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
             n0 = dk[n0];
             n1 = dk[n1];
           }
-          group_positions(n0, n1, ws, lane, posB0, posB1);
+          { const int2 pp = group_positions(n0, n1, ws, lane); posB0 = pp.x; posB1 = pp.y; }
         }
         __syncwarp();
 
@@ -513,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           i0 = dk[i0];
           i1 = dk[i1];
         }
-        group_positions(i0, i1, ws, lane, posA0, posA1);
+        { const int2 pp = group_positions(i0, i1, ws, lane); posA0 = pp.x; posA1 = pp.y; }
         // ---- forward chain: Phi_tau and Ct_tau = Phi_tau^T C_tau at the positions of S_a's order
         float v0 = 1.f, v1 = 1.f;
         {
@@ -711,15 +713,9 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->full[stg]);
-      // both warps are done with the input stage: prefetch the pair's next sub-chunk
+      // both warps are done with the input stage before the next load overwrites it
       pair_sync(pbar);
-      if (role == 0) {
-        const int nxt = sub + kNW;
-        if (nxt < nsub) load_inputs<TL>(a, in, b, h, nxt, lane);
-        cp_async_commit();
-      }
     }
-    if (role == 0) cp_async_wait<0>();
   } else if (warp < kIssuerWarp) {
     // ============================================ carry state and output (warps 8-11)
     const int q = warp & 3;                 // tensor-memory quarter
