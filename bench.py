@@ -281,6 +281,10 @@ def run_ours(args, rank, world, local):
             ends[i].record(stream)
         torch.cuda.synchronize(device)
     barrier(world, device)
+    # a bounded wait that gave up, or a range error, voids the measurement
+    check = pd.pdssm_read_device_check(ws)
+    if check:
+        raise RuntimeError(f"device check status {check} after the timed steps")
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms_local = sum(step_ms) / len(step_ms)
     ms = max_over_ranks(ms_local, world, device)
@@ -350,6 +354,9 @@ def run_ours(args, rank, world, local):
     e_e.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / args.steps, world, device)
+    check = pd.pdssm_read_device_check(ws)
+    if check:
+        raise RuntimeError(f"device check status {check} after the end-to-end steps")
 
     result = None
     if rank == 0:

@@ -142,7 +142,10 @@ struct FParams {
 
 struct Bars {
   uint64_t full[kMaxStages], opfree[kMaxStages], yfull[kNY], yfree[kNY];
-  uint64_t ufull[3], sready, slofree, drain;
+  // sready[k % 4]: S_k complete (all four carry warps). A ring: the carry warps
+  // can complete the next state before the issuing thread has observed this one,
+  // and two completions of one barrier ahead of its waiter alias in the parity test.
+  uint64_t ufull[3], sready[4], slofree, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -413,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       mbar_init(&bars->yfree[i], 4);
     }
     for (int i = 0; i < 3; ++i) mbar_init(&bars->ufull[i], 1);
-    mbar_init(&bars->sready, 4);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars->sready[i], 4);
     mbar_init(&bars->slofree, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -744,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->sready);
+      if (lane == 0) mbar_arrive(&bars->sready[0]);
     }
     TO *yout = static_cast<TO *>(a.y);
     // output rows of sub-chunk sub from its accumulator slot (already loaded)
@@ -862,7 +865,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&bars->sready);
+        mbar_arrive(&bars->sready[(sub + 1) & 3]);
         mbar_arrive(&bars->opfree[st]);
       }
       done = sub + 1;
@@ -928,7 +931,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       return true;
     };
     auto issue_y = [&](int s) -> bool {
-      if (!mbar_test_wait(&bars->sready, s & 1) && !wait_bar(bars, &bars->sready, s & 1, a.err)) return false;
+      uint64_t *sb = &bars->sready[s & 3];
+      if (!mbar_test_wait(sb, (s >> 2) & 1) && !wait_bar(bars, sb, (s >> 2) & 1, a.err)) return false;
       tc_fence_after();
       issue_y_now(s);
       return true;
@@ -941,7 +945,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     // term after all.
     bool ok = issue_us(0, true) && issue_us(kRing - 2, false) && (nsub == 0 || issue_y(0));
     for (int s = 0; ok && s + 1 < nsub; ++s) {
-      ok = mbar_test_wait(&bars->sready, (s + 1) & 1) || wait_bar(bars, &bars->sready, (s + 1) & 1, a.err);
+      uint64_t *sb = &bars->sready[(s + 1) & 3];
+      ok = mbar_test_wait(sb, ((s + 1) >> 2) & 1) || wait_bar(bars, sb, ((s + 1) >> 2) & 1, a.err);
       ok = ok && issue_us(s + 1, true) && issue_us(s + kRing - 1, false) && issue_y(s + 1) &&
            issue_us(s + kRing - 1, true);
     }

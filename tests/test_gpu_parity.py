@@ -318,3 +318,17 @@ def test_token_by_token_decode_matches_the_whole_sequence(cuda_device, recipe, k
     hs = whole["h_final"].abs().amax().item()
     assert (h - whole["h_final"]).abs().amax().item() <= 1e-4 * hs
     compare_full(inp, {"y": y.cpu(), "h_final": h.cpu()})
+
+
+def test_fused_path_reports_no_device_error_across_repeated_launches(cuda_device):
+    """The fused kernel's bounded waits never give up on the LM workload: the device
+    check word stays clear over repeated full-size launches (a stall that the bounded
+    waits caught would set its timeout bit)."""
+    sp = workloads.spec("lm")
+    inp = workloads.generate(sp, seed=17, device=cuda_device)
+    pb = pd.make_problem(inp["logits"], inp["d"], inp["B"], inp["x"])
+    ws = pd.alloc_workspace(pb, cuda_device)
+    for _ in range(8):
+        out = pd.forward(inp["logits"], inp["idx"], inp["d"], inp["B"], inp["C"], inp["x"], workspace=ws)
+        assert pd.pdssm_read_device_check(ws) == 0  # PDSSM_OK
+    assert torch.isfinite(out["y"].float()).all()
