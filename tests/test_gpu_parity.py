@@ -332,3 +332,21 @@ def test_fused_path_reports_no_device_error_across_repeated_launches(cuda_device
         out = pd.forward(inp["logits"], inp["idx"], inp["d"], inp["B"], inp["C"], inp["x"], workspace=ws)
         assert pd.pdssm_read_device_check(ws) == 0  # PDSSM_OK
     assert torch.isfinite(out["y"].float()).all()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("chunk", [0, 1, 3])
+@pytest.mark.parametrize("via_scan", [False, True])
+def test_hand_worked_automaton_runs(cuda_device, chunk, via_scan):
+    """The C-ABI reproduces the hand-worked automaton runs of tests/golden exactly
+    (Proposition 1 of the Flash PD-SSM summary page): selections, every output,
+    the final state and the composed product."""
+    from tests import golden
+    for name in golden.names():
+        inp, exp = golden.load(name)
+        out = run_gpu(inp, cuda_device, chunk=chunk, via_scan=via_scan)
+        assert out["s"][0, :, 0].tolist() == exp["s"], name
+        assert out["y"][0, :, 0, 0].tolist() == exp["y"], name
+        assert out["h_final"][0, 0, :, 0].tolist() == exp["h_final"], name
+        assert out["prod_idx"][0, 0].tolist() == exp["prod_idx"], name
+        assert out["prod_val"][0, 0].tolist() == exp["prod_val"], name
