@@ -34,9 +34,16 @@ struct Plan {
 };
 
 int64_t default_chunk(const pdssm_problem *pb) {
-  // Long enough that chunk-end states stay O(L*N) (T >= P), short enough
-  // that every SM gets several (batch, head, chunk) blocks.
-  return std::max<int64_t>(64, pb->P);
+  // Long enough that chunk-end states stay O(L*N) (T >= P) and the sequential
+  // carry scan over chunks stays short; short enough that the chunk-parallel
+  // phases still fill the GPU: about 1024 threads on each of the 148 SMs, in
+  // blocks of 32 columns x the kernels' row groups (1, 2 or 8 by N).
+  const int64_t col_blocks = (pb->P + 31) / 32;
+  const int64_t row_groups = pb->N <= 16 ? 1 : (pb->N <= 32 ? 2 : 8);
+  const int64_t want = 148 * 1024 / (32 * row_groups);
+  int64_t T = 256;
+  while (T > 64 && pb->batch * pb->heads * col_blocks * ((pb->seqlen + T - 1) / T) < want) T /= 2;
+  return std::max<int64_t>(T, pb->P);
 }
 
 pdssm_status make_plan(const pdssm_problem *pb, Plan *pl) {

@@ -9,13 +9,16 @@
 // one-hot-column transitions (the associative-operator framing of the Prefix
 // Scannable Models abstract): (idx, val) o (idx', val') = (idx[idx'], val[idx']*val').
 //
-// Thread p of a block owns column p of the N x P state, so the row gather
-// H'[i][p] = sum_{j in pre(i)} d[j] H[j][p] + B[i] x[p] needs no exchange
-// between threads, and y_t[p] = sum_i C[i] H'[i][p] is a per-thread sum.
-// The state lives in shared memory because the gather index is dynamic.
-// Per-step vectors (d, B, C, x and the selected entry's preimage lists) are
-// staged in shared memory by all threads. The chunk's own pair (idx, val) is
-// kept by the thread that owns column j of it.
+// A block owns up to 32 columns of one (batch, head) state and all N rows, in
+// shared memory (the gather index is dynamic). Its threads are RG row groups of
+// 32 columns (RG = 1, 2 or 8, so that a thread has at most 16 rows): thread
+// (g, p) updates rows i = g, g + RG, ... of column p, so a warp always reads one
+// state row across 32 consecutive columns (no bank conflicts) and the CSR work
+// of a step is spread over the row groups. New rows are held in registers until
+// every thread has read the old state, so one state buffer suffices. Per-step
+// vectors (d, B, C, x and the selected entry's preimage lists) are fetched into
+// registers one step ahead and staged in shared memory; a column's output is
+// the sum of the row groups' parts.
 #include <algorithm>
 
 #include "launch.h"
@@ -24,11 +27,12 @@ namespace pdssm {
 
 namespace {
 
-constexpr int kMaxPairsPerThread = PDSSM_MAX_N / 32;
+constexpr int kPB = 32;       // columns per block (one warp per row group)
+constexpr int kMaxRows = 16;  // rows per thread at most
 
 struct KParams {
   int64_t L, H, N, P, K, T, nC;
-  int64_t PB, nPB;  // columns per block and column blocks (columns are independent)
+  int64_t nPB;  // column blocks (columns are independent)
   const int32_t *s;
   const int32_t *idx;  // sanitised [K][N]
   const int32_t *off;  // [K][N+1]
@@ -49,35 +53,34 @@ __device__ __forceinline__ int load_s(const KParams &a, int64_t row) {
 }
 
 // ------------------------------------------------------------------ phase A
-template <bool CPLX, typename TD, typename TIn>
-__global__ void __launch_bounds__(128) phase_a_kernel(KParams a) {
+// Within chunk c, from a zero state: H_t[i] = B_t[i] x_t + sum_{j in pre(i)} d_t[j] H_{t-1}[j],
+// y_loc_t = H_t^T C_t; the chunk's pair is the composition of its steps' pairs.
+template <typename T>
+struct StepVec {  // one thread's share of a step's vectors (entry j = tid)
+  T d;
+  float B, C, x;
+  int src, off, st;
+};
+
+template <int RG, bool CPLX, typename TD, typename TIn>
+__global__ void __launch_bounds__(RG * kPB) phase_a_kernel(KParams a) {
   using Nm = Num<CPLX>;
   using T = typename Nm::T;
+  constexpr int NT = RG * kPB;
   extern __shared__ __align__(16) unsigned char smem[];
-  const int N = (int)a.N, NT = blockDim.x, tid = threadIdx.x;
+  const int N = (int)a.N, tid = threadIdx.x, pl = tid % kPB, g = tid / kPB;
   const int64_t c = blockIdx.x / a.nPB, pb = blockIdx.x % a.nPB, h = blockIdx.y, b = blockIdx.z;
-  const int p0 = (int)(pb * a.PB), P = (int)min(a.PB, a.P - p0), PG = (int)a.P;
+  const int p0 = (int)(pb * kPB), P = (int)min((int64_t)kPB, a.P - p0), PG = (int)a.P;
   const int64_t t0 = c * a.T, t1 = min(t0 + a.T, a.L);
 
-  T *Hc = reinterpret_cast<T *>(smem);
-  T *Hn = Hc + N * P;
-  T *dsh = Hn + N * P;
+  T *Hs = reinterpret_cast<T *>(smem);  // [N][kPB]
+  T *ysh = Hs + N * kPB;                // [RG][kPB]
+  T *dsh = ysh + RG * kPB;              // [N]
   float *Bsh = reinterpret_cast<float *>(dsh + N);
   float *Csh = Bsh + N;
-  float *xsh = Csh + N;
-  int *offsh = reinterpret_cast<int *>(xsh + P);
+  float *xsh = Csh + N;                 // [kPB]
+  int *offsh = reinterpret_cast<int *>(xsh + kPB);
   int *srcsh = offsh + N + 1;
-
-  for (int p = tid; p < P; p += NT)
-    for (int i = 0; i < N; ++i) Hc[i * P + p] = Nm::zero();
-
-  int pidx[kMaxPairsPerThread];
-  T pval[kMaxPairsPerThread];
-#pragma unroll
-  for (int m = 0; m < kMaxPairsPerThread; ++m) {
-    pidx[m] = tid + m * NT;
-    pval[m] = Nm::one();
-  }
 
   const TD *dg = static_cast<const TD *>(a.d);
   const TIn *Bg = static_cast<const TIn *>(a.B);
@@ -85,210 +88,305 @@ __global__ void __launch_bounds__(128) phase_a_kernel(KParams a) {
   const TIn *xg = static_cast<const TIn *>(a.x);
   T *yl = static_cast<T *>(a.y_loc);
 
-  for (int64_t t = t0; t < t1; ++t) {
+  for (int e = tid; e < N * kPB; e += NT) Hs[e] = Nm::zero();
+  int pidx = tid;  // chunk pair entry tid (tid < N)
+  T pval = Nm::one();
+
+  // NT >= 2N: thread tid fetches entry tid of each vector (and off[N], x[tid])
+  auto fetch = [&](int64_t t) {
+    StepVec<T> v;
     const int64_t row = (b * a.L + t) * a.H + h;
-    const int st = load_s(a, row);
-    __syncthreads();  // the previous step is done with the staged vectors
-    for (int j = tid; j < N; j += NT) {
-      dsh[j] = LoadD<CPLX, TD>::ld(dg + row * N + j);
-      Bsh[j] = ldf(Bg + row * N + j);
-      Csh[j] = ldf(Cg + row * N + j);
-      srcsh[j] = a.src[(int64_t)st * N + j];
+    v.st = load_s(a, row);
+    if (tid < N) {
+      v.d = LoadD<CPLX, TD>::ld(dg + row * N + tid);
+      v.B = ldf(Bg + row * N + tid);
+      v.C = ldf(Cg + row * N + tid);
+      v.src = a.src[(int64_t)v.st * N + tid];
     }
-    for (int j = tid; j <= N; j += NT) offsh[j] = a.off[(int64_t)st * (N + 1) + j];
-    for (int p = tid; p < P; p += NT) xsh[p] = ldf(xg + row * PG + p0 + p);
-    __syncthreads();
-
-    // chunk pair <- (idx_s, d_t) o pair
+    if (tid <= N) v.off = a.off[(int64_t)v.st * (N + 1) + tid];
+    if (tid < kPB) v.x = tid < P ? ldf(xg + row * PG + p0 + tid) : 0.f;
+    return v;
+  };
+  auto commit = [&](const StepVec<T> &v) {
+    if (tid < N) {
+      dsh[tid] = v.d;
+      Bsh[tid] = v.B;
+      Csh[tid] = v.C;
+      srcsh[tid] = v.src;
+    }
+    if (tid <= N) offsh[tid] = v.off;
+    if (tid < kPB) xsh[tid] = v.x;
+  };
+  // output of step t from the row groups' parts
+  auto finish_y = [&](int64_t t) {
+    if (g == 0 && pl < P) {
+      T acc = ysh[pl];
 #pragma unroll
-    for (int m = 0; m < kMaxPairsPerThread; ++m) {
-      if (tid + m * NT < N) {
-        const int r = pidx[m];
-        pval[m] = Nm::mul(dsh[r], pval[m]);
-        pidx[m] = a.idx[(int64_t)st * N + r];
-      }
+      for (int q = 1; q < RG; ++q) acc = Nm::add(acc, ysh[q * kPB + pl]);
+      yl[((b * a.L + t) * a.H + h) * PG + p0 + pl] = acc;
     }
+  };
 
-    for (int p = tid; p < P; p += NT) {
-      const float xp = xsh[p];
-      T yacc = Nm::zero();
-      for (int i = 0; i < N; ++i) {
-        T acc = Nm::from_real(Bsh[i] * xp);
-        const int r1 = offsh[i + 1];
-        for (int r = offsh[i]; r < r1; ++r) {
-          const int j = srcsh[r];
-          acc = Nm::fma(dsh[j], Hc[j * P + p], acc);
-        }
-        Hn[i * P + p] = acc;
-        yacc = Nm::fma_r(Csh[i], acc, yacc);
-      }
-      yl[row * PG + p0 + p] = yacc;
+  StepVec<T> cur = fetch(t0);  // t0 < t1: every chunk holds a token
+  commit(cur);
+  int st = cur.st;
+  for (int64_t t = t0; t < t1; ++t) {
+    StepVec<T> nxt;
+    if (t + 1 < t1) nxt = fetch(t + 1);  // in flight during this step
+    __syncthreads();  // step t's vectors, the state and the parts of step t - 1 are visible
+    if (t > t0) finish_y(t - 1);
+    if (tid < N) {  // chunk pair <- (idx_s, d_t) o pair
+      pval = Nm::mul(dsh[pidx], pval);
+      pidx = a.idx[(int64_t)st * N + pidx];
     }
-    T *tmp = Hc;
-    Hc = Hn;
-    Hn = tmp;
+    T nv[kMaxRows];
+    T yp = Nm::zero();
+    const float xp = xsh[pl];
+#pragma unroll
+    for (int m = 0; m < kMaxRows; ++m) {
+      const int i = g + RG * m;
+      if (i < N) {
+        T acc = Nm::from_real(Bsh[i] * xp);
+        // sources in increasing order; the first two outside the loop so that
+        // their loads overlap (most rows have at most two)
+        const int r0 = offsh[i], r1 = offsh[i + 1];
+        if (r0 < r1) {
+          const int ja = srcsh[r0];
+          acc = Nm::fma(dsh[ja], Hs[ja * kPB + pl], acc);
+          if (r0 + 1 < r1) {
+            const int jb = srcsh[r0 + 1];
+            acc = Nm::fma(dsh[jb], Hs[jb * kPB + pl], acc);
+            for (int r = r0 + 2; r < r1; ++r) {
+              const int j = srcsh[r];
+              acc = Nm::fma(dsh[j], Hs[j * kPB + pl], acc);
+            }
+          }
+        }
+        nv[m] = acc;
+        yp = Nm::fma_r(Csh[i], acc, yp);
+      }
+    }
+    __syncthreads();  // every read of the old state and of the staged vectors is done
+#pragma unroll
+    for (int m = 0; m < kMaxRows; ++m) {
+      const int i = g + RG * m;
+      if (i < N) Hs[i * kPB + pl] = nv[m];
+    }
+    ysh[g * kPB + pl] = yp;
+    if (t + 1 < t1) {
+      commit(nxt);
+      st = nxt.st;
+    }
   }
+  __syncthreads();
+  finish_y(t1 - 1);
 
   // chunk-end local state and chunk pair
   const int64_t slot = (b * a.H + h) * a.nC + c;
   T *cs = static_cast<T *>(a.chunk_state) + slot * N * PG;
-  for (int p = tid; p < P; p += NT)
-    for (int i = 0; i < N; ++i) cs[i * PG + p0 + p] = Hc[i * P + p];
-  if (pb != 0) return;  // every column block computes the pair; one writes it
-  T *cv = static_cast<T *>(a.chunk_val) + slot * N;
-  int32_t *ci = a.chunk_idx + slot * N;
-#pragma unroll
-  for (int m = 0; m < kMaxPairsPerThread; ++m) {
-    const int j = tid + m * NT;
-    if (j < N) {
-      ci[j] = pidx[m];
-      cv[j] = pval[m];
-    }
-  }
+  if (pl < P)
+    for (int i = g; i < N; i += RG) cs[i * PG + p0 + pl] = Hs[i * kPB + pl];
+  if (pb != 0 || tid >= N) return;  // every column block computes the pair; one writes it
+  a.chunk_idx[slot * N + tid] = pidx;
+  static_cast<T *>(a.chunk_val)[slot * N + tid] = pval;
 }
 
 // ------------------------------------------------------------------ phase B
-// carry_c = apply(pair_c, carry_{c-1}) + local_c, carry_{-1} = h0 (or 0);
-// apply((idx, val), H)[idx[j]] += val[j] * H[j]. The carries overwrite the
-// local states in place; h_final is the last carry and (prod_idx, prod_val)
-// the composition of all chunk pairs.
-template <bool CPLX>
-__global__ void __launch_bounds__(128) phase_b_kernel(KParams a) {
+// carry_c = apply(pair_c, carry_{c-1}) + local_c, carry_{-1} = h0 (or 0), with
+// apply((idx, val), H)[i] = sum_{j: idx[j] = i} val[j] H[j], sources in increasing
+// j. The carries overwrite the local states in place; h_final is the last carry
+// and (prod_idx, prod_val) the composition of all chunk pairs.
+template <int RG, bool CPLX>
+__global__ void __launch_bounds__(RG * kPB) phase_b_kernel(KParams a) {
   using Nm = Num<CPLX>;
   using T = typename Nm::T;
+  constexpr int NT = RG * kPB;
   extern __shared__ __align__(16) unsigned char smem[];
-  const int N = (int)a.N, NT = blockDim.x, tid = threadIdx.x;
+  const int N = (int)a.N, tid = threadIdx.x, pl = tid % kPB, g = tid / kPB;
   const int64_t h = blockIdx.x / a.nPB, pb = blockIdx.x % a.nPB, b = blockIdx.y;
-  const int p0 = (int)(pb * a.PB), P = (int)min(a.PB, a.P - p0), PG = (int)a.P;
-  T *Hc = reinterpret_cast<T *>(smem);
-  T *Hn = Hc + N * P;
-  T *pv = Hn + N * P;
+  const int p0 = (int)(pb * kPB), P = (int)min((int64_t)kPB, a.P - p0), PG = (int)a.P;
+  const bool col = pl < P;
+  T *Hs = reinterpret_cast<T *>(smem);  // [N][kPB]
+  T *pv = Hs + N * kPB;                 // [N]
   int *pi = reinterpret_cast<int *>(pv + N);
+  int *off = pi + N;                    // [N+1] preimage lists of the chunk pair's index map
+  int *src = off + N + 1;               // [N]
 
   const T *h0 = static_cast<const T *>(a.h0);
-  for (int p = tid; p < P; p += NT)
-    for (int i = 0; i < N; ++i)
-      Hc[i * P + p] = h0 ? h0[((b * a.H + h) * N + i) * PG + p0 + p] : Nm::zero();
-
-  int tidx[kMaxPairsPerThread];
-  T tval[kMaxPairsPerThread];
-#pragma unroll
-  for (int m = 0; m < kMaxPairsPerThread; ++m) {
-    tidx[m] = tid + m * NT;
-    tval[m] = Nm::one();
+  for (int i = g; i < N; i += RG)
+    Hs[i * kPB + pl] = (h0 && col) ? h0[((b * a.H + h) * N + i) * PG + p0 + pl] : Nm::zero();
+  int tidx = tid;  // whole-sequence product entry tid (tid < N)
+  T tval = Nm::one();
+  const int64_t slot0 = (b * a.H + h) * a.nC;
+  int pi_n = 0;  // the next chunk's pair entry tid, fetched one chunk ahead
+  T pv_n = Nm::zero();
+  if (tid < N && a.nC > 0) {
+    pi_n = a.chunk_idx[slot0 * N + tid];
+    pv_n = static_cast<const T *>(a.chunk_val)[slot0 * N + tid];
   }
 
   for (int64_t c = 0; c < a.nC; ++c) {
-    const int64_t slot = (b * a.H + h) * a.nC + c;
-    __syncthreads();
-    for (int j = tid; j < N; j += NT) {
-      pi[j] = a.chunk_idx[slot * N + j];
-      pv[j] = static_cast<const T *>(a.chunk_val)[slot * N + j];
+    T *cs = static_cast<T *>(a.chunk_state) + (slot0 + c) * N * PG + p0;
+    T nv[kMaxRows];  // the local state's rows, loaded while the lists are built
+#pragma unroll
+    for (int m = 0; m < kMaxRows; ++m) {
+      const int i = g + RG * m;
+      if (i < N) nv[m] = col ? cs[i * PG + pl] : Nm::zero();
+    }
+    __syncthreads();  // the previous chunk's lists are no longer read
+    if (tid < N) {
+      pi[tid] = pi_n;
+      pv[tid] = pv_n;
+      if (c + 1 < a.nC) {
+        pi_n = a.chunk_idx[(slot0 + c + 1) * N + tid];
+        pv_n = static_cast<const T *>(a.chunk_val)[(slot0 + c + 1) * N + tid];
+      }
     }
     __syncthreads();
-    T *cs = static_cast<T *>(a.chunk_state) + slot * N * PG + p0;
-    for (int p = tid; p < P; p += NT) {
-      for (int i = 0; i < N; ++i) Hn[i * P + p] = cs[i * PG + p];
+    // stable counting sort of the sources by target: off[i] = #{j : pi[j] < i},
+    // source tid goes to off[pi[tid]] + #{j < tid : pi[j] = pi[tid]}
+    int mine = 0, rank = 0;
+    if (tid < N) {
+      mine = pi[tid];
+      int below = 0;
       for (int j = 0; j < N; ++j) {
-        T &dst = Hn[pi[j] * P + p];
-        dst = Nm::fma(pv[j], Hc[j * P + p], dst);
+        const int pj = pi[j];
+        below += pj < tid;
+        rank += (j < tid) & (pj == mine);
       }
-      for (int i = 0; i < N; ++i) cs[i * PG + p] = Hn[i * P + p];
+      off[tid] = below;
+      if (tid == 0) off[N] = N;
+      tval = Nm::mul(pv[tidx], tval);  // product <- pair_c o product
+      tidx = pi[tidx];
     }
+    __syncthreads();
+    if (tid < N) src[off[mine] + rank] = tid;
+    __syncthreads();
 #pragma unroll
-    for (int m = 0; m < kMaxPairsPerThread; ++m) {
-      if (tid + m * NT < N) {
-        const int r = tidx[m];
-        tval[m] = Nm::mul(pv[r], tval[m]);
-        tidx[m] = pi[r];
+    for (int m = 0; m < kMaxRows; ++m) {
+      const int i = g + RG * m;
+      if (i < N) {
+        T acc = nv[m];
+        const int r0 = off[i], r1 = off[i + 1];
+        if (r0 < r1) {
+          const int ja = src[r0];
+          acc = Nm::fma(pv[ja], Hs[ja * kPB + pl], acc);
+          if (r0 + 1 < r1) {
+            const int jb = src[r0 + 1];
+            acc = Nm::fma(pv[jb], Hs[jb * kPB + pl], acc);
+            for (int r = r0 + 2; r < r1; ++r) {
+              const int j = src[r];
+              acc = Nm::fma(pv[j], Hs[j * kPB + pl], acc);
+            }
+          }
+        }
+        nv[m] = acc;
       }
     }
-    T *tmp = Hc;
-    Hc = Hn;
-    Hn = tmp;
+    __syncthreads();  // every read of the previous carry is done
+#pragma unroll
+    for (int m = 0; m < kMaxRows; ++m) {
+      const int i = g + RG * m;
+      if (i < N) {
+        Hs[i * kPB + pl] = nv[m];
+        if (col) cs[i * PG + pl] = nv[m];
+      }
+    }
   }
+  __syncthreads();
 
-  if (a.h_final) {
+  if (a.h_final && col) {
     T *hf = static_cast<T *>(a.h_final) + (b * a.H + h) * N * PG + p0;
-    for (int p = tid; p < P; p += NT)
-      for (int i = 0; i < N; ++i) hf[i * PG + p] = Hc[i * P + p];
+    for (int i = g; i < N; i += RG) hf[i * PG + pl] = Hs[i * kPB + pl];
   }
-  if (pb != 0) return;
-#pragma unroll
-  for (int m = 0; m < kMaxPairsPerThread; ++m) {
-    const int j = tid + m * NT;
-    if (j < N) {
-      if (a.prod_idx) a.prod_idx[(b * a.H + h) * N + j] = tidx[m];
-      if (a.prod_val) static_cast<T *>(a.prod_val)[(b * a.H + h) * N + j] = tval[m];
-    }
-  }
+  (void)NT;
+  if (pb != 0 || tid >= N) return;
+  if (a.prod_idx) a.prod_idx[(b * a.H + h) * N + tid] = tidx;
+  if (a.prod_val) static_cast<T *>(a.prod_val)[(b * a.H + h) * N + tid] = tval;
 }
 
 // ------------------------------------------------------------------ phase C
 // y_t = y_loc_t + carry_in^T Ctil_t, Ctil_t[j] = val_t[j] * C_t[idx_t[j]], where
 // (idx_t, val_t) is the pair of the chunk's prefix up to and including t.
-template <bool CPLX, typename TD, typename TIn, typename TOut>
-__global__ void __launch_bounds__(128) phase_c_kernel(KParams a) {
+template <int RG, bool CPLX, typename TD, typename TIn, typename TOut>
+__global__ void __launch_bounds__(RG * kPB) phase_c_kernel(KParams a) {
   using Nm = Num<CPLX>;
   using T = typename Nm::T;
   extern __shared__ __align__(16) unsigned char smem[];
-  const int N = (int)a.N, NT = blockDim.x, tid = threadIdx.x;
+  const int N = (int)a.N, tid = threadIdx.x, pl = tid % kPB, g = tid / kPB;
   const int64_t c = blockIdx.x / a.nPB, pb = blockIdx.x % a.nPB, h = blockIdx.y, b = blockIdx.z;
-  const int p0 = (int)(pb * a.PB), P = (int)min(a.PB, a.P - p0), PG = (int)a.P;
+  const int p0 = (int)(pb * kPB), P = (int)min((int64_t)kPB, a.P - p0), PG = (int)a.P;
+  const bool col = pl < P;
   const int64_t t0 = c * a.T, t1 = min(t0 + a.T, a.L);
-  T *Hin = reinterpret_cast<T *>(smem);
-  T *ct = Hin + N * P;
-  T *dsh = ct + N;
-  float *Csh = reinterpret_cast<float *>(dsh + N);
+  T *Hin = reinterpret_cast<T *>(smem);  // [N][kPB]
+  T *ysh = Hin + N * kPB;                // [RG][kPB]
+  T *ct = ysh + RG * kPB;                // [N]
 
-  const bool carry = (c > 0) || (a.h0 != nullptr);
-  if (carry) {
-    const T *src = c > 0 ? static_cast<const T *>(a.chunk_state) + ((b * a.H + h) * a.nC + c - 1) * N * PG
-                         : static_cast<const T *>(a.h0) + (b * a.H + h) * N * PG;
-    for (int p = tid; p < P; p += NT)
-      for (int i = 0; i < N; ++i) Hin[i * P + p] = src[i * PG + p0 + p];
-  }
-  int pidx[kMaxPairsPerThread];
-  T pval[kMaxPairsPerThread];
-#pragma unroll
-  for (int m = 0; m < kMaxPairsPerThread; ++m) {
-    pidx[m] = tid + m * NT;
-    pval[m] = Nm::one();
-  }
   const TD *dg = static_cast<const TD *>(a.d);
   const TIn *Cg = static_cast<const TIn *>(a.C);
   const T *yl = static_cast<const T *>(a.y_loc);
   TOut *yo = static_cast<TOut *>(a.y);
+  auto yoff = [&](int64_t t) { return ((b * a.L + t) * a.H + h) * PG + p0 + pl; };
 
-  for (int64_t t = t0; t < t1; ++t) {
-    const int64_t row = (b * a.L + t) * a.H + h;
-    if (carry) {
-      const int st = load_s(a, row);
-      __syncthreads();
-      for (int j = tid; j < N; j += NT) {
-        dsh[j] = LoadD<CPLX, TD>::ld(dg + row * N + j);
-        Csh[j] = ldf(Cg + row * N + j);
-      }
-      __syncthreads();
-#pragma unroll
-      for (int m = 0; m < kMaxPairsPerThread; ++m) {
-        const int j = tid + m * NT;
-        if (j < N) {
-          const int r = pidx[m];
-          pval[m] = Nm::mul(dsh[r], pval[m]);
-          pidx[m] = a.idx[(int64_t)st * N + r];
-          ct[j] = Nm::mul(pval[m], Nm::from_real(Csh[pidx[m]]));
-        }
-      }
-      __syncthreads();
-    }
-    for (int p = tid; p < P; p += NT) {
-      T acc = yl[row * PG + p0 + p];
-      if (carry)
-        for (int j = 0; j < N; ++j) acc = Nm::fma(ct[j], Hin[j * P + p], acc);
-      st_out(yo + row * PG + p0 + p, acc);
-    }
+  const bool carry = (c > 0) || (a.h0 != nullptr);
+  if (!carry) {
+    if (g == 0 && col)
+      for (int64_t t = t0; t < t1; ++t) st_out(yo + yoff(t), yl[yoff(t)]);
+    return;
   }
+  const T *hin = c > 0 ? static_cast<const T *>(a.chunk_state) + ((b * a.H + h) * a.nC + c - 1) * N * PG
+                       : static_cast<const T *>(a.h0) + (b * a.H + h) * N * PG;
+  for (int i = g; i < N; i += RG) Hin[i * kPB + pl] = col ? hin[i * PG + p0 + pl] : Nm::zero();
+  int pidx = tid;  // prefix pair entry tid (tid < N)
+  T pval = Nm::one();
+  // the prefix pair needs d_t[pidx] and C_t[idx_t[pidx]]: entries of the step's
+  // vectors that another thread may own, so the vectors go through shared memory
+  T *dsh = ct + N;                                  // [N]
+  float *Csh = reinterpret_cast<float *>(dsh + N);  // [N]
+  T dn = Nm::zero();
+  float cn = 0.f;
+  int sn = 0;
+  auto fetch = [&](int64_t t) {
+    const int64_t row = (b * a.L + t) * a.H + h;
+    if (tid < N) {
+      dn = LoadD<CPLX, TD>::ld(dg + row * N + tid);
+      cn = ldf(Cg + row * N + tid);
+      sn = load_s(a, row);
+    }
+  };
+  T ylv = Nm::zero();  // y_loc of the step being finished, fetched a step ahead
+  auto finish_y = [&](int64_t t) {
+    if (g == 0 && col) {
+      T acc = ylv;
+#pragma unroll
+      for (int q = 0; q < RG; ++q) acc = Nm::add(acc, ysh[q * kPB + pl]);
+      st_out(yo + yoff(t), acc);
+    }
+  };
+
+  fetch(t0);
+  for (int64_t t = t0; t < t1; ++t) {
+    if (tid < N) {
+      dsh[tid] = dn;
+      Csh[tid] = cn;
+    }
+    const int st = sn;
+    if (t + 1 < t1) fetch(t + 1);
+    __syncthreads();  // step t's vectors and the parts of step t - 1 are visible
+    if (t > t0) finish_y(t - 1);
+    if (g == 0 && col) ylv = yl[yoff(t)];
+    if (tid < N) {
+      pval = Nm::mul(dsh[pidx], pval);
+      pidx = a.idx[(int64_t)st * N + pidx];
+      ct[tid] = Nm::mul(pval, Nm::from_real(Csh[pidx]));
+    }
+    __syncthreads();  // Ctil_t is complete; the parts of step t - 1 were read
+    T yp = Nm::zero();
+    for (int i = g; i < N; i += RG) yp = Nm::fma(ct[i], Hin[i * kPB + pl], yp);
+    ysh[g * kPB + pl] = yp;
+  }
+  __syncthreads();
+  finish_y(t1 - 1);
 }
 
 // ------------------------------------------------------------ empty L == 0
@@ -309,7 +407,7 @@ __global__ void empty_outputs_kernel(KParams a, int64_t slices) {
 KParams make_params(const ScanArgs &s) {
   KParams k;
   k.L = s.L; k.H = s.H; k.N = s.N; k.P = s.P; k.K = s.K; k.T = s.T; k.nC = s.nC;
-  k.PB = s.P; k.nPB = 1;
+  k.nPB = (s.P + kPB - 1) / kPB;
   k.s = s.s; k.idx = s.ws.idx; k.off = s.ws.csr_off; k.src = s.ws.csr_src;
   k.d = s.d; k.B = s.B; k.C = s.C; k.x = s.x; k.h0 = s.h0;
   k.y_loc = s.ws.y_loc; k.chunk_state = s.ws.chunk_state; k.chunk_val = s.ws.chunk_val;
@@ -319,8 +417,8 @@ KParams make_params(const ScanArgs &s) {
 }
 
 template <typename Kern>
-cudaError_t launch_dyn(Kern kern, const char *name, dim3 grid, int threads, size_t smem,
-                       cudaStream_t st, const KParams &k) {
+cudaError_t launch_dyn(Kern kern, const char *name, dim3 grid, int threads, size_t smem, cudaStream_t st,
+                       const KParams &k) {
   cudaError_t e;
   if (smem > 48 * 1024) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -332,27 +430,32 @@ cudaError_t launch_dyn(Kern kern, const char *name, dim3 grid, int threads, size
   return trace_after(st);
 }
 
+template <int RG, bool CPLX, typename TD, typename TIn, typename TOut>
+cudaError_t run_chunked_rg(const ScanArgs &s, cudaStream_t st) {
+  using T = typename Num<CPLX>::T;
+  const KParams k = make_params(s);
+  const size_t ts = sizeof(T), N = (size_t)s.N;
+  const size_t smem_a = N * kPB * ts + RG * kPB * ts + N * ts + 2 * N * 4 + kPB * 4 + (2 * N + 1) * 4;
+  const size_t smem_b = N * kPB * ts + N * ts + N * 4 + (2 * N + 1) * 4;
+  const size_t smem_c = N * kPB * ts + RG * kPB * ts + 2 * N * ts + N * 4;
+  const dim3 grid_chunks((unsigned)(s.nC * k.nPB), (unsigned)s.H, (unsigned)s.Bt);
+  cudaError_t e = launch_dyn(phase_a_kernel<RG, CPLX, TD, TIn>, "chunked_phase_a", grid_chunks, RG * kPB, smem_a,
+                             st, k);
+  if (e != cudaSuccess) return e;
+  e = launch_dyn(phase_b_kernel<RG, CPLX>, "chunked_phase_b", dim3((unsigned)(s.H * k.nPB), (unsigned)s.Bt),
+                 RG * kPB, smem_b, st, k);
+  if (e != cudaSuccess) return e;
+  return launch_dyn(phase_c_kernel<RG, CPLX, TD, TIn, TOut>, "chunked_phase_c", grid_chunks, RG * kPB, smem_c, st,
+                    k);
+}
+
+// Row groups: a thread updates at most kMaxRows rows, and the block's threads
+// (32 per row group) are at least twice N.
 template <bool CPLX, typename TD, typename TIn, typename TOut>
 cudaError_t run_chunked(const ScanArgs &s, cudaStream_t st) {
-  using T = typename Num<CPLX>::T;
-  KParams k = make_params(s);
-  const size_t ts = sizeof(T);
-  auto smem_a = [&](int64_t pb) { return 2 * s.N * pb * ts + s.N * ts + (2 * s.N + pb) * 4 + (2 * s.N + 1) * 4; };
-  // columns are independent: split them over blocks until the state fits
-  int64_t PB = s.P;
-  while (smem_a(PB) > 200 * 1024) PB = (PB + 1) / 2;
-  k.PB = PB;
-  k.nPB = (s.P + PB - 1) / PB;
-  const int threads = (int)std::min<int64_t>(128, std::max<int64_t>(32, (PB + 31) / 32 * 32));
-  const size_t smem_b = 2 * s.N * PB * ts + s.N * ts + s.N * 4;
-  const size_t smem_c = s.N * PB * ts + 2 * s.N * ts + s.N * 4;
-  const dim3 grid_chunks((unsigned)(s.nC * k.nPB), (unsigned)s.H, (unsigned)s.Bt);
-  cudaError_t e = launch_dyn(phase_a_kernel<CPLX, TD, TIn>, "chunked_phase_a", grid_chunks, threads, smem_a(PB), st, k);
-  if (e != cudaSuccess) return e;
-  e = launch_dyn(phase_b_kernel<CPLX>, "chunked_phase_b", dim3((unsigned)(s.H * k.nPB), (unsigned)s.Bt), threads, smem_b,
-                 st, k);
-  if (e != cudaSuccess) return e;
-  return launch_dyn(phase_c_kernel<CPLX, TD, TIn, TOut>, "chunked_phase_c", grid_chunks, threads, smem_c, st, k);
+  if (s.N <= 16) return run_chunked_rg<1, CPLX, TD, TIn, TOut>(s, st);
+  if (s.N <= 32) return run_chunked_rg<2, CPLX, TD, TIn, TOut>(s, st);
+  return run_chunked_rg<8, CPLX, TD, TIn, TOut>(s, st);
 }
 
 }  // namespace

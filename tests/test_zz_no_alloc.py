@@ -58,7 +58,7 @@ def test_noalloc_matches_forward_on_consecutive_calls(cuda_device, recipe, kw):
 
 def test_noalloc_rejects_problems_beyond_its_workspace(cuda_device):
     # real, full-size buffers: nothing here can make a kernel touch memory it does not own
-    sp = workloads.spec("lm", batch=4, seqlen=2048, heads=8)
+    sp = workloads.spec("lm", batch=8, seqlen=2048, heads=8)
     g = torch.Generator(device=cuda_device).manual_seed(0)
     inp = {
         "logits": torch.randn(sp.batch, sp.seqlen, sp.heads, sp.K, device=cuda_device, generator=g).to(torch.bfloat16),
