@@ -164,6 +164,8 @@ def load_peaks():
 KERNEL_SOURCES = {
     "fused_scan": ["structured_sparse_selective_b200/csrc/scan_fused.cu",
                    "structured_sparse_selective_b200/csrc/sm100.cuh"],
+    "chunked_phase_a": ["structured_sparse_selective_b200/csrc/scan_chunked.cu",
+                        "structured_sparse_selective_b200/csrc/common.cuh"],
 }
 
 

@@ -3,6 +3,8 @@ only while the kernel sources still hash to the value the profile summary record
 import hashlib
 import os
 
+import pytest
+
 import bench
 
 
@@ -35,10 +37,12 @@ def test_traffic_absent_without_summary_or_known_sources(tmp_path, monkeypatch):
     assert bench.recorded_traffic("unknown", "wl") is None
 
 
-def test_committed_summary_names_known_sources():
-    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles", "fused_scan_lm.md")
+@pytest.mark.parametrize("kernel,workload", [("fused_scan", "lm"), ("chunked_phase_a", "long")])
+def test_committed_summary_names_known_sources(kernel, workload):
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles",
+                        f"{kernel}_{workload}.md")
     with open(path) as f:
         text = f.read()
     assert "traffic_bytes_per_launch:" in text and "kernel_sources_sha256:" in text
-    for s in bench.KERNEL_SOURCES["fused_scan"]:
+    for s in bench.KERNEL_SOURCES[kernel]:
         assert os.path.exists(os.path.join(os.path.dirname(path), "..", s))
