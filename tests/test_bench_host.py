@@ -46,3 +46,35 @@ def test_committed_summary_names_known_sources(kernel, workload):
     assert "traffic_bytes_per_launch:" in text and "kernel_sources_sha256:" in text
     for s in bench.KERNEL_SOURCES[kernel]:
         assert os.path.exists(os.path.join(os.path.dirname(path), "..", s))
+
+
+def test_reference_arm_prints_one_contract_line():
+    """``bench.py --impl reference`` (the oracle on the host cores) prints exactly one
+    JSON line with the contract's keys, its e2e and cpu_baseline describing itself."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--steps", "2", "--warmup", "3"], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    res = json.loads(lines[0])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in res, k
+    assert res["impl"] == "reference" and res["steps"] == 2 and res["warmup"] == 3
+    assert res["value"] > 0 and res["e2e"]["value"] == res["value"]
+    assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["e2e"]["d2h_bytes_per_step"] == 0
+    assert res["cpu_baseline"]["kind"] == "oracle" and res["cpu_baseline"]["cores"] >= 1
+    assert res["config"]["workload"].startswith("tiny")
+
+
+def test_bench_rejects_short_warmup():
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--warmup", "2"],
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "at least 3" in r.stderr
