@@ -177,3 +177,21 @@ def test_binding_refuses_cpu_tensors():
     t = torch.zeros(4)
     with pytest.raises(ValueError):
         pd._ptr(t)
+
+
+def test_default_chunk_keeps_the_workspace_below_the_fixed_chunk_one():
+    """The default chunk length (chunk = 0) is never shorter than 64 nor than P, so the
+    default workspace never exceeds the one of chunk = max(64, P); on long sequences with
+    many (batch, head) slices it picks longer chunks and the workspace shrinks."""
+    def ws(**kw):
+        rc, n = _ws(_pb(**kw))
+        assert rc == OK
+        return n
+    for kw in (dict(batch=4, heads=8, seqlen=18000, N=32, P=32, K=8),
+               dict(batch=16, heads=64, seqlen=8192, N=128, P=64, K=64),
+               dict(batch=1, heads=1, seqlen=256, N=8, P=4, K=4),
+               dict(batch=8, heads=32, seqlen=2048, N=64, P=128, K=16)):
+        fixed = ws(chunk=max(64, kw["P"]), **kw)
+        assert ws(chunk=0, **kw) <= fixed, kw
+    many = dict(batch=16, heads=64, seqlen=8192, N=128, P=64, K=64)
+    assert ws(chunk=0, **many) < ws(chunk=64, **many)
