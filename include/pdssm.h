@@ -190,9 +190,44 @@ pdssm_status pdssm_forward_noalloc(const pdssm_problem *pb, const void *logits, 
                                    void *prod_val, int32_t *s_out, pdssm_stream_t stream);
 
 /*
- * Synchronises `stream` and reads the error word that the last pdssm_scan_fwd
- * or pdssm_forward call on `workspace` left: PDSSM_OK, PDSSM_ERR_DEVICE_CHECK
- * (an idx or s value was out of range) or PDSSM_ERR_TIMEOUT.
+ * Backward pass (real state): workspace bytes for pdssm_scan_bwd. Checkpoints
+ * of the state every 16 steps plus a 16-step scratch per (batch, head) slice:
+ * 4 * N * P * batch * heads * (ceil(L / 16) + 16) bytes, plus the dictionary's
+ * preimage lists. PDSSM_ERR_UNSUPPORTED for a complex state.
+ */
+pdssm_status pdssm_bwd_workspace_size(const pdssm_problem *pb, size_t *bytes);
+
+/*
+ * Backward pass of the scan (Flash PD-SSM page, Technical Summary,
+ * Methodology 2 "Gradient Propagation": hard argmax forward, tempered softmax
+ * backward through a straight-through estimator). Gradients of
+ *   Loss = sum_t <dy_t, y_t> + <dh_final, H_{L-1}>
+ * where y, H are the forward pass of pdssm_scan_fwd on the same arguments:
+ *   dd, dB, dC  float [batch][seqlen][heads][N]: exact derivatives;
+ *   dx          float [batch][seqlen][heads][P]: exact derivative;
+ *   dh0         float [batch][heads][N][P] or NULL: derivative in h0;
+ *   dlogits     float [batch][seqlen][heads][K] or NULL (then `logits` is NULL
+ *               too): with pit = softmax(logits_t / tau) and
+ *               dpi_t[k] = sum_j (Lam_t H_{t-1}^T)[idx[k][j]][j] d_t[j]
+ *               (Lam_t = dLoss/dH_t), dlogits_t = pit * (dpi_t - <pit, dpi_t>) / tau.
+ * Inputs: s (device int32 [batch][seqlen][heads], the forward's selections),
+ * idx, d, B, C, x, h0 as for pdssm_scan_fwd (h0 float or NULL); dy in the
+ * problem's out_t ([batch][seqlen][heads][P]); dh_final float
+ * [batch][heads][N][P] or NULL (zero); logits in logits_t; tau > 0.
+ * Real state only (state_t = PDSSM_F32); every gradient is float.
+ * Errors as pdssm_scan_fwd; the workspace is pdssm_bwd_workspace_size bytes.
+ */
+pdssm_status pdssm_scan_bwd(const pdssm_problem *pb, const void *logits, const int32_t *s,
+                            const int32_t *idx, const void *d, const void *B, const void *C,
+                            const void *x, const float *h0, const void *dy, const float *dh_final,
+                            float tau, float *dlogits, float *dd, float *dB, float *dC, float *dx,
+                            float *dh0, void *workspace, size_t workspace_bytes,
+                            pdssm_stream_t stream);
+
+/*
+ * Synchronises `stream` and reads the error word that the last pdssm_scan_fwd,
+ * pdssm_forward or pdssm_scan_bwd call on `workspace` left: PDSSM_OK,
+ * PDSSM_ERR_DEVICE_CHECK (an idx or s value was out of range) or PDSSM_ERR_TIMEOUT.
  */
 pdssm_status pdssm_read_device_check(const void *workspace, pdssm_stream_t stream);
 

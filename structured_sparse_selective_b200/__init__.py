@@ -12,9 +12,13 @@ The functions keep the C names:
     pdssm_scan_fwd(problem, s, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val, workspace, stream=None)
     pdssm_forward(problem, logits, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val, s_out, workspace, stream=None)
     pdssm_read_device_check(workspace, stream=None)
+    pdssm_bwd_workspace_size(problem) -> int
+    pdssm_scan_bwd(problem, logits, s, idx, d, B, C, x, h0, dy, dh_final, tau, dlogits, dd, dB, dC, dx, dh0,
+                   workspace, stream=None)
 
 ``forward(...)`` is a convenience wrapper that allocates the outputs and the
-workspace with torch and calls ``pdssm_forward``.
+workspace with torch and calls ``pdssm_forward``; ``backward(...)`` does the
+same for ``pdssm_scan_bwd``.
 """
 from __future__ import annotations
 
@@ -28,7 +32,8 @@ __all__ = [
     "PdssmError", "Problem", "F32", "BF16", "C64", "FLAG_DEVICE_CHECK", "FLAG_REFERENCE_PATH",
     "library_path", "make_problem", "pdssm_workspace_size", "pdssm_select", "pdssm_scan_fwd",
     "pdssm_forward", "pdssm_read_device_check", "pdssm_status_string", "forward", "EXPORTED_SYMBOLS",
-    "KernelTrace", "alloc_workspace", "pdssm_forward_noalloc",
+    "KernelTrace", "alloc_workspace", "pdssm_forward_noalloc", "pdssm_bwd_workspace_size", "pdssm_scan_bwd",
+    "backward",
 ]
 
 F32, BF16, C64 = 0, 1, 2
@@ -39,7 +44,8 @@ MAX_N, MAX_P, MAX_K = 128, 128, 64
 EXPORTED_SYMBOLS = (
     "pdssm_status_string", "pdssm_version", "pdssm_workspace_size", "pdssm_select",
     "pdssm_scan_fwd", "pdssm_forward", "pdssm_read_device_check", "pdssm_trace_begin",
-    "pdssm_trace_end", "pdssm_trace_kernel_name", "pdssm_forward_noalloc",
+    "pdssm_trace_end", "pdssm_trace_kernel_name", "pdssm_forward_noalloc", "pdssm_bwd_workspace_size",
+    "pdssm_scan_bwd",
 )
 
 _DIR = os.path.dirname(os.path.abspath(__file__))
@@ -88,6 +94,11 @@ def _load() -> ctypes.CDLL:
     lib.pdssm_forward.restype = ctypes.c_int
     lib.pdssm_forward_noalloc.argtypes = [pb, vp, i32p, vp, vp, vp, vp, vp, vp, vp, i32p, vp, i32p, vp]
     lib.pdssm_forward_noalloc.restype = ctypes.c_int
+    lib.pdssm_bwd_workspace_size.argtypes = [pb, ctypes.POINTER(sz)]
+    lib.pdssm_bwd_workspace_size.restype = ctypes.c_int
+    lib.pdssm_scan_bwd.argtypes = [pb, vp, i32p, i32p, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float,
+                                   vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.pdssm_scan_bwd.restype = ctypes.c_int
     lib.pdssm_read_device_check.argtypes = [vp, vp]
     lib.pdssm_read_device_check.restype = ctypes.c_int
     lib.pdssm_trace_begin.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
@@ -197,6 +208,23 @@ def pdssm_forward_noalloc(pb: Problem, logits, idx, d, B, C, x, h0, y, h_final, 
         _ptr(prod_val, dev), _ptr(s_out, dev), _stream(stream, dev)), "pdssm_forward_noalloc")
 
 
+def pdssm_bwd_workspace_size(pb: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.pdssm_bwd_workspace_size(ctypes.byref(pb), ctypes.byref(n)), "pdssm_bwd_workspace_size")
+    return int(n.value)
+
+
+def pdssm_scan_bwd(pb: Problem, logits, s, idx, d, B, C, x, h0, dy, dh_final, tau: float, dlogits, dd, dB, dC,
+                   dx, dh0, workspace, stream=None) -> None:
+    dev = idx.device
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pdssm_scan_bwd(
+        ctypes.byref(pb), _ptr(logits, dev), _ptr(s, dev), _ptr(idx, dev), _ptr(d, dev), _ptr(B, dev),
+        _ptr(C, dev), _ptr(x, dev), _ptr(h0, dev), _ptr(dy, dev), _ptr(dh_final, dev), float(tau),
+        _ptr(dlogits, dev), _ptr(dd, dev), _ptr(dB, dev), _ptr(dC, dev), _ptr(dx, dev), _ptr(dh0, dev),
+        _ptr(workspace, dev), ws_bytes, _stream(stream, dev)), "pdssm_scan_bwd")
+
+
 def pdssm_read_device_check(workspace: torch.Tensor, stream=None) -> int:
     """Status left in the workspace's error word by the last scan (synchronises)."""
     return int(_lib.pdssm_read_device_check(_ptr(workspace), _stream(stream, workspace.device)))
@@ -258,4 +286,29 @@ def forward(logits: torch.Tensor, idx: torch.Tensor, d: torch.Tensor, B: torch.T
     ws = workspace if workspace is not None else alloc_workspace(pb, dev)
     pdssm_forward(pb, logits, idx, d, B, C, x, h0, out["y"], out["h_final"], out.get("prod_idx"),
                   out.get("prod_val"), out.get("s"), ws, stream)
+    return out
+
+
+def backward(logits: Optional[torch.Tensor], s: torch.Tensor, idx: torch.Tensor, d: torch.Tensor,
+             B: torch.Tensor, C: torch.Tensor, x: torch.Tensor, dy: torch.Tensor,
+             h0: Optional[torch.Tensor] = None, dh_final: Optional[torch.Tensor] = None, tau: float = 1.0,
+             want_dh0: bool = True, workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
+    """Allocates the gradients (float32) and runs ``pdssm_scan_bwd``; ``s`` are the forward's
+    selections, ``dy`` has the forward output's dtype. No logits -> no ``dlogits``."""
+    K = logits.shape[-1] if logits is not None else int(idx.shape[0])
+    pb = make_problem(logits, d, B, x, out_dtype=dy.dtype, K=K)
+    dev = B.device
+    Bt, L, H, N = B.shape
+    P = x.shape[-1]
+    f = dict(dtype=torch.float32, device=dev)
+    out = {"dd": torch.empty(Bt, L, H, N, **f), "dB": torch.empty(Bt, L, H, N, **f),
+           "dC": torch.empty(Bt, L, H, N, **f), "dx": torch.empty(Bt, L, H, P, **f)}
+    if logits is not None:
+        out["dlogits"] = torch.empty(Bt, L, H, K, **f)
+    if want_dh0:
+        out["dh0"] = torch.empty(Bt, H, N, P, **f)
+    ws = workspace if workspace is not None else torch.empty(max(1, pdssm_bwd_workspace_size(pb)),
+                                                              dtype=torch.uint8, device=dev)
+    pdssm_scan_bwd(pb, logits, s, idx, d, B, C, x, h0, dy, dh_final, tau, out.get("dlogits"), out["dd"], out["dB"],
+                   out["dC"], out["dx"], out.get("dh0"), ws, stream)
     return out

@@ -187,6 +187,37 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &p, const int32_t *s,
   return finish(pb, w, stream);
 }
 
+// Workspace of the backward pass: error word, dictionary preimage lists,
+// checkpoints [Bt][H][nCk][N][P] and the per-slice scratch [Bt][H][16][N][P].
+struct BwdPlan {
+  int64_t Bt, L, H, N, P, K, rows, nCk;
+  size_t o_err, o_idx, o_off, o_src, o_ckpt, o_scr, total;
+};
+
+pdssm_status make_bwd_plan(const pdssm_problem *pb, BwdPlan *bp) {
+  Plan p;
+  pdssm_status st = make_plan(pb, &p);
+  if (st != PDSSM_OK) return st;
+  if (p.cplx) return PDSSM_ERR_UNSUPPORTED;
+  BwdPlan q;
+  q.Bt = p.Bt; q.L = p.L; q.H = p.H; q.N = p.N; q.P = p.P; q.K = p.K; q.rows = p.rows;
+  q.nCk = scan_bwd_checkpoints(p.L);
+  int64_t slices = p.Bt * p.H, per_slice, tot;
+  if (!mul_ok(p.N * p.P, q.nCk + scan_bwd_scratch_steps(), &per_slice) || !mul_ok(slices, per_slice, &tot) ||
+      !mul_ok(tot, 4, &tot))
+    return PDSSM_ERR_UNSUPPORTED;
+  size_t o = 0;
+  q.o_err = o; o = align256(o + 4);
+  q.o_idx = o; o = align256(o + (size_t)(p.K * p.N) * 4);
+  q.o_off = o; o = align256(o + (size_t)(p.K * (p.N + 1)) * 4);
+  q.o_src = o; o = align256(o + (size_t)(p.K * p.N) * 4);
+  q.o_ckpt = o; o = align256(o + (size_t)(slices * q.nCk * p.N * p.P) * 4);
+  q.o_scr = o; o = align256(o + (size_t)(slices * scan_bwd_scratch_steps() * p.N * p.P) * 4);
+  q.total = o;
+  *bp = q;
+  return PDSSM_OK;
+}
+
 constexpr int kMaxTraced = 64;
 struct TraceState {
   void *const *events = nullptr;
@@ -317,6 +348,74 @@ pdssm_status pdssm_forward(const pdssm_problem *pb, const void *logits, const in
   if ((st = bind_device(cs)) != PDSSM_OK) return st;
   return run_scan(pb, p, nullptr, logits, s_out, idx, d, B, C, x, h0, y, h_final, prod_idx,
                   prod_val, workspace, cs);
+}
+
+pdssm_status pdssm_bwd_workspace_size(const pdssm_problem *pb, size_t *bytes) {
+  if (!bytes) return PDSSM_ERR_INVALID_ARG;
+  BwdPlan q;
+  pdssm_status st = make_bwd_plan(pb, &q);
+  if (st != PDSSM_OK) return st;
+  *bytes = q.total;
+  return PDSSM_OK;
+}
+
+pdssm_status pdssm_scan_bwd(const pdssm_problem *pb, const void *logits, const int32_t *s,
+                            const int32_t *idx, const void *d, const void *B, const void *C,
+                            const void *x, const float *h0, const void *dy, const float *dh_final,
+                            float tau, float *dlogits, float *dd, float *dB, float *dC, float *dx,
+                            float *dh0, void *workspace, size_t workspace_bytes,
+                            pdssm_stream_t stream) {
+  BwdPlan q;
+  pdssm_status st = make_bwd_plan(pb, &q);
+  if (st != PDSSM_OK) return st;
+  if (!idx || !(tau > 0.f) || !(tau < INFINITY)) return PDSSM_ERR_INVALID_ARG;
+  if ((logits == nullptr) != (dlogits == nullptr)) return PDSSM_ERR_INVALID_ARG;
+  if (q.rows > 0 && (!s || !d || !B || !C || !x || !dy || !dd || !dB || !dC || !dx))
+    return PDSSM_ERR_INVALID_ARG;
+  const size_t es_in = dtype_size(pb->in_t), es_d = dtype_size(pb->d_t), es_o = dtype_size(pb->out_t);
+  if (!aligned(idx, 4) || !aligned(s, 4) || !aligned(d, es_d) || !aligned(B, es_in) || !aligned(C, es_in) ||
+      !aligned(x, es_in) || !aligned(dy, es_o) || !aligned(logits, dtype_size(pb->logits_t)) ||
+      !aligned(h0, 4) || !aligned(dh_final, 4) || !aligned(dlogits, 4) || !aligned(dd, 4) ||
+      !aligned(dB, 4) || !aligned(dC, 4) || !aligned(dx, 4) || !aligned(dh0, 4))
+    return PDSSM_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < q.total) return PDSSM_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return PDSSM_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = bind_device(cs)) != PDSSM_OK) return st;
+
+  char *base = static_cast<char *>(workspace);
+  Workspace w{};
+  w.err = reinterpret_cast<uint32_t *>(base + q.o_err);
+  w.idx = reinterpret_cast<int32_t *>(base + q.o_idx);
+  w.csr_off = reinterpret_cast<int32_t *>(base + q.o_off);
+  w.csr_src = reinterpret_cast<int32_t *>(base + q.o_src);
+  if (cudaMemsetAsync(w.err, 0, 4, cs) != cudaSuccess) return PDSSM_ERR_CUDA;
+  const int64_t slices = q.Bt * q.H;
+  if (slices == 0) return finish(pb, w, cs);
+  if (q.L == 0) {  // no steps: the final state is the initial one
+    if (dh0) {
+      const size_t n = (size_t)(slices * q.N * q.P) * 4;
+      cudaError_t e = dh_final ? cudaMemcpyAsync(dh0, dh_final, n, cudaMemcpyDeviceToDevice, cs)
+                               : cudaMemsetAsync(dh0, 0, n, cs);
+      if (e != cudaSuccess) return PDSSM_ERR_CUDA;
+    }
+    return finish(pb, w, cs);
+  }
+  st = cuda_status(launch_prep_dict(idx, (int)q.K, (int)q.N, w, cs));
+  if (st != PDSSM_OK) return st;
+  ScanBwdArgs a;
+  a.Bt = q.Bt; a.L = q.L; a.H = q.H; a.N = q.N; a.P = q.P; a.K = q.K;
+  a.d_t = pb->d_t; a.in_t = pb->in_t; a.out_t = pb->out_t; a.logits_t = pb->logits_t;
+  a.tau = tau;
+  a.s = s; a.logits = logits; a.d = d; a.B = B; a.C = C; a.x = x; a.dy = dy;
+  a.h0 = h0; a.dh_final = dh_final;
+  a.ckpt = reinterpret_cast<float *>(base + q.o_ckpt);
+  a.scratch = reinterpret_cast<float *>(base + q.o_scr);
+  a.dlogits = dlogits; a.dd = dd; a.dB = dB; a.dC = dC; a.dx = dx; a.dh0 = dh0;
+  a.ws = w;
+  st = cuda_status(launch_scan_bwd(a, cs));
+  if (st != PDSSM_OK) return st;
+  return finish(pb, w, cs);
 }
 
 pdssm_status pdssm_read_device_check(const void *workspace, pdssm_stream_t stream) {

@@ -41,4 +41,23 @@ cudaError_t launch_fused_scan(const ScanArgs &a, cudaStream_t st);
 // Outputs of an empty sequence (L == 0): h_final = h0 (or 0), prod = identity.
 cudaError_t launch_empty_outputs(const ScanArgs &a, cudaStream_t st);
 
+// Everything a backward launch needs (real state); validated by the C-ABI layer.
+struct ScanBwdArgs {
+  int64_t Bt, L, H, N, P, K;
+  int d_t, in_t, out_t, logits_t;
+  float tau;
+  const int32_t *s;
+  const void *logits, *d, *B, *C, *x, *dy;
+  const float *h0, *dh_final;
+  float *ckpt, *scratch;
+  float *dlogits, *dd, *dB, *dC, *dx, *dh0;
+  Workspace ws;  // err, idx, csr_off, csr_src
+};
+// Shared memory of one backward block, checkpoints of a sequence, and the steps
+// between checkpoints (the per-sequence scratch holds that many states).
+size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t K);
+int64_t scan_bwd_checkpoints(int64_t L);
+int64_t scan_bwd_scratch_steps();
+cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t st);
+
 }  // namespace pdssm

@@ -1,0 +1,284 @@
+// Backward pass of the PD scan (real state): gradients of the loss
+//   sum_t <dy_t, y_t> + <dh_final, H_{L-1}>
+// with respect to d, B, C, x, h0 and, through the straight-through estimator
+// with a tempered softmax, the selection logits.
+//
+// Flash PD-SSM page, Technical Summary, Methodology 2 ("Gradient Propagation"):
+// the forward pass uses the hard argmax; the backward pass approximates the
+// selection by a tempered softmax. The step's transition is read as the mixture
+// A_t = sum_k pi_k P_k diag(d_t), one-hot at s_t in the forward pass; the gradient
+// in the weights, dpi_t[k] = sum_j (Lam_t H_{t-1}^T)[idx_k[j]][j] d_t[j], goes
+// through the Jacobian of softmax(logits_t / tau).
+//
+// The adjoint Lam_t = dLoss/dH_t runs backwards:
+//   Lam_t = Lam'_t + C_t dy_t^T,  Lam'_{t-1} = A_t^T Lam_t  ((A^T Lam)[j] = d[j] Lam[idx[j]]),
+// and the step's gradients are
+//   dC_t = H_t dy_t, dB_t = Lam_t x_t, dx_t = Lam_t^T B_t, dd_t[j] = <Lam_t[idx_{s_t}[j]], H_{t-1}[j]>.
+//
+// One block per (batch, head) sequence. A forward sweep stores the state every
+// kTb steps (O(L N P / kTb) memory, O(L N) for kTb >= P); the reverse sweep
+// recomputes each kTb-step stretch from its checkpoint into a per-sequence
+// scratch and walks it backwards. Three N x P buffers in shared memory (rows
+// padded by one word) hold the adjoint, H_t and H_{t-1}.
+#include "launch.h"
+
+namespace pdssm {
+
+namespace {
+
+constexpr int kBT = 256;  // threads per block
+constexpr int kTb = 16;   // steps between checkpoints
+
+struct BParams {
+  int64_t L, H, N, P, K, nCk;
+  float tau;
+  int logits_bf16, dy_bf16;
+  const int32_t *s;
+  const int32_t *idx;  // sanitised [K][N]
+  const int32_t *off;  // [K][N+1]
+  const int32_t *src;  // [K][N]
+  const void *logits, *d, *B, *C, *x, *dy;
+  const float *h0, *dh_final;
+  float *ckpt;     // [Bt*H][nCk][N][P]
+  float *scratch;  // [Bt*H][kTb][N][P]
+  float *dlogits, *dd, *dB, *dC, *dx, *dh0;
+  uint32_t *err;
+};
+
+__device__ __forceinline__ float ld_flag(const void *p, int64_t i, int bf16) {
+  return bf16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]) : static_cast<const float *>(p)[i];
+}
+
+template <typename TD, typename TIn>
+__global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int N = (int)a.N, P = (int)a.P, K = (int)a.K, PS = P + 1;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+
+  float *buf0 = reinterpret_cast<float *>(smem);  // three [N][PS] buffers
+  float *buf1 = buf0 + N * PS;
+  float *buf2 = buf1 + N * PS;
+  float *dsh = buf2 + N * PS;  // [N]
+  float *Bsh = dsh + N;        // [N]
+  float *Csh = Bsh + N;        // [N]
+  float *xsh = Csh + N;        // [P]
+  float *dysh = xsh + P;       // [P]
+  float *dpi = dysh + P;       // [K]
+  int *offsh = reinterpret_cast<int *>(dpi + K);  // [N+1] preimage lists of the step's entry
+  int *srcsh = offsh + N + 1;                     // [N]
+  uint8_t *idxsh = reinterpret_cast<uint8_t *>(srcsh + N);  // [K][N] dictionary
+
+  for (int e = tid; e < K * N; e += kBT) idxsh[e] = (uint8_t)a.idx[e];
+
+  const TD *dg = static_cast<const TD *>(a.d);
+  const TIn *Bg = static_cast<const TIn *>(a.B);
+  const TIn *Cg = static_cast<const TIn *>(a.C);
+  const TIn *xg = static_cast<const TIn *>(a.x);
+  float *ck = a.ckpt + bh * a.nCk * N * P;
+  float *scr = a.scratch + bh * (int64_t)kTb * N * P;
+
+  // element loop over a dense [N][P] array: thread tid starts at element tid
+  const int di = kBT / P, dp = kBT - di * P;
+  const int i_start = tid / P, p_start = tid - i_start * P;
+#define FOR_NP(i, p)                                                           \
+  for (int i = i_start, p = p_start; i < N; i += di, p += dp, (p >= P ? (p -= P, ++i) : 0))
+
+  auto row_of = [&](int64_t t) { return (b * a.L + t) * a.H + h; };
+  auto load_s = [&](int64_t row) {
+    int st = a.s[row];
+    if (st < 0 || st >= K) {
+      flag_error(a.err, kErrSRange);
+      st = 0;
+    }
+    return st;
+  };
+  // the step's d, B, x and the preimage lists of its entry (for a forward step)
+  auto stage_fwd = [&](int64_t t) {
+    const int64_t row = row_of(t);
+    const int st = load_s(row);
+    for (int j = tid; j < N; j += kBT) {
+      dsh[j] = to_f32(dg[row * N + j]);
+      Bsh[j] = to_f32(Bg[row * N + j]);
+      srcsh[j] = a.src[(int64_t)st * N + j];
+    }
+    for (int j = tid; j <= N; j += kBT) offsh[j] = a.off[(int64_t)st * (N + 1) + j];
+    for (int p = tid; p < P; p += kBT) xsh[p] = to_f32(xg[row * P + p]);
+  };
+  // Hn = A_t Hc + B_t x_t^T (after stage_fwd(t) and a barrier)
+  auto step_fwd = [&](const float *Hc, float *Hn) {
+    FOR_NP(i, p) {
+      float acc = Bsh[i] * xsh[p];
+      const int r1 = offsh[i + 1];
+      for (int r = offsh[i]; r < r1; ++r) {
+        const int j = srcsh[r];
+        acc = fmaf(dsh[j], Hc[j * PS + p], acc);
+      }
+      Hn[i * PS + p] = acc;
+    }
+  };
+  auto store_dense = [&](const float *S, float *g) {
+    FOR_NP(i, p) { g[i * P + p] = S[i * PS + p]; }
+  };
+  auto load_dense = [&](const float *g, float *S) {
+    FOR_NP(i, p) { S[i * PS + p] = g[i * P + p]; }
+  };
+
+  // ---- forward sweep: checkpoints every kTb steps
+  float *Hc = buf0, *Hn = buf1;
+  FOR_NP(i, p) { Hc[i * PS + p] = a.h0 ? a.h0[(bh * N + i) * P + p] : 0.f; }
+  for (int64_t t = 0; t < a.L; ++t) {
+    __syncthreads();  // Hc complete; the staged vectors are no longer read
+    if (t % kTb == 0) store_dense(Hc, ck + (t / kTb) * N * P);
+    stage_fwd(t);
+    __syncthreads();
+    step_fwd(Hc, Hn);
+    float *tmp = Hc;
+    Hc = Hn;
+    Hn = tmp;
+  }
+
+  // ---- reverse sweep
+  float *Lam = buf2;
+  __syncthreads();
+  FOR_NP(i, p) { Lam[i * PS + p] = a.dh_final ? a.dh_final[(bh * N + i) * P + p] : 0.f; }
+  for (int64_t c = a.nCk - 1; c >= 0; --c) {
+    const int64_t t0 = c * kTb, t1 = t0 + kTb < a.L ? t0 + kTb : a.L;
+    // recompute the stretch: scratch[t - t0] = H_{t-1}; Hc ends as H_{t1-1}
+    Hc = (Lam == buf0) ? buf1 : buf0;
+    Hn = (Lam == buf2) ? buf1 : buf2;
+    if (Lam == buf1) Hn = buf2;
+    __syncthreads();
+    load_dense(ck + c * N * P, Hc);
+    for (int64_t t = t0; t < t1; ++t) {
+      __syncthreads();
+      store_dense(Hc, scr + (t - t0) * N * P);
+      stage_fwd(t);
+      __syncthreads();
+      step_fwd(Hc, Hn);
+      float *tmp = Hc;
+      Hc = Hn;
+      Hn = tmp;
+    }
+    float *Hp = Hn;  // receives H_{t-1}
+    for (int64_t t = t1 - 1; t >= t0; --t) {
+      const int64_t row = row_of(t);
+      __syncthreads();  // [A] the previous step is done with every buffer and vector
+      const int st = load_s(row);
+      for (int j = tid; j < N; j += kBT) {
+        dsh[j] = to_f32(dg[row * N + j]);
+        Bsh[j] = to_f32(Bg[row * N + j]);
+        Csh[j] = to_f32(Cg[row * N + j]);
+      }
+      for (int p = tid; p < P; p += kBT) {
+        xsh[p] = to_f32(xg[row * P + p]);
+        dysh[p] = ld_flag(a.dy, row * P + p, a.dy_bf16);
+      }
+      load_dense(scr + (t - t0) * N * P, Hp);
+      __syncthreads();
+      // [B] Lam_t = Lam'_t + C_t dy_t^T
+      FOR_NP(i, p) { Lam[i * PS + p] = fmaf(Csh[i], dysh[p], Lam[i * PS + p]); }
+      __syncthreads();
+      // [C] dB_t, dC_t, and per entry k: <Lam_t[idx_k[j]], H_{t-1}[j]> (dd_t at k = s_t, dpi_t[k])
+      if (tid < N) {
+        float acc = 0.f;
+        for (int p = 0; p < P; ++p) acc = fmaf(Lam[tid * PS + p], xsh[p], acc);
+        a.dB[row * N + tid] = acc;
+      }
+      if (tid >= 128 && tid - 128 < N) {
+        const int i = tid - 128;
+        float acc = 0.f;
+        for (int p = 0; p < P; ++p) acc = fmaf(Hc[i * PS + p], dysh[p], acc);
+        a.dC[row * N + i] = acc;
+      }
+      for (int k = warp; k < K; k += kBT / 32) {
+        float part = 0.f;
+        for (int j = lane; j < N; j += 32) {
+          const int r = idxsh[k * N + j];
+          float q = 0.f;
+          for (int p = 0; p < P; ++p) q = fmaf(Lam[r * PS + p], Hp[j * PS + p], q);
+          if (k == st) a.dd[row * N + j] = q;
+          part = fmaf(dsh[j], q, part);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) dpi[k] = part;
+      }
+      __syncthreads();
+      // [D] logits through the tempered softmax (warp 0); Lam'_{t-1} = A_t^T Lam_t into
+      // Hc's buffer; dx_t
+      if (warp == 0 && a.dlogits) {
+        const float v0 = lane < K ? ld_flag(a.logits, row * K + lane, a.logits_bf16) / a.tau : -INFINITY;
+        const float v1 = lane + 32 < K ? ld_flag(a.logits, row * K + lane + 32, a.logits_bf16) / a.tau : -INFINITY;
+        float m = fmaxf(v0, v1);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float e0 = lane < K ? expf(v0 - m) : 0.f, e1 = lane + 32 < K ? expf(v1 - m) : 0.f;
+        float sum = e0 + e1;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const float p0 = e0 / sum, p1 = e1 / sum;
+        const float g0 = lane < K ? dpi[lane] : 0.f, g1 = lane + 32 < K ? dpi[lane + 32] : 0.f;
+        float dot = p0 * g0 + p1 * g1;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (lane < K) a.dlogits[row * K + lane] = p0 * (g0 - dot) / a.tau;
+        if (lane + 32 < K) a.dlogits[row * K + lane + 32] = p1 * (g1 - dot) / a.tau;
+      }
+      FOR_NP(j, p) { Hc[j * PS + p] = dsh[j] * Lam[idxsh[st * N + j] * PS + p]; }
+      if (tid >= 32 && tid - 32 < P) {
+        const int p = tid - 32;
+        float acc = 0.f;
+        for (int i = 0; i < N; ++i) acc = fmaf(Lam[i * PS + p], Bsh[i], acc);
+        a.dx[row * P + p] = acc;
+      }
+      // rotate: the new adjoint is in Hc's buffer, H_{t-1} becomes the next step's H_t
+      float *old = Lam;
+      Lam = Hc;
+      Hc = Hp;
+      Hp = old;
+    }
+  }
+  __syncthreads();
+  if (a.dh0) {
+    FOR_NP(i, p) { a.dh0[(bh * N + i) * P + p] = Lam[i * PS + p]; }
+  }
+#undef FOR_NP
+}
+
+}  // namespace
+
+size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t K) {
+  return (size_t)(3 * N * (P + 1) + 3 * N + 2 * P + K) * 4 + (size_t)(2 * N + 1) * 4 + (size_t)(K * N);
+}
+
+int64_t scan_bwd_checkpoints(int64_t L) { return (L + kTb - 1) / kTb; }
+int64_t scan_bwd_scratch_steps() { return kTb; }
+
+cudaError_t launch_scan_bwd(const ScanBwdArgs &s, cudaStream_t st) {
+  BParams a;
+  a.L = s.L; a.H = s.H; a.N = s.N; a.P = s.P; a.K = s.K;
+  a.nCk = scan_bwd_checkpoints(s.L);
+  a.tau = s.tau;
+  a.logits_bf16 = s.logits_t == PDSSM_BF16;
+  a.dy_bf16 = s.out_t == PDSSM_BF16;
+  a.s = s.s; a.idx = s.ws.idx; a.off = s.ws.csr_off; a.src = s.ws.csr_src;
+  a.logits = s.logits; a.d = s.d; a.B = s.B; a.C = s.C; a.x = s.x; a.dy = s.dy;
+  a.h0 = s.h0; a.dh_final = s.dh_final;
+  a.ckpt = s.ckpt; a.scratch = s.scratch;
+  a.dlogits = s.dlogits; a.dd = s.dd; a.dB = s.dB; a.dC = s.dC; a.dx = s.dx; a.dh0 = s.dh0;
+  a.err = s.ws.err;
+  const size_t smem = scan_bwd_smem_bytes(s.N, s.P, s.K);
+  auto kern = s.d_t == PDSSM_BF16 ? (s.in_t == PDSSM_BF16 ? scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16>
+                                                          : scan_bwd_kernel<__nv_bfloat16, float>)
+                                  : (s.in_t == PDSSM_BF16 ? scan_bwd_kernel<float, __nv_bfloat16>
+                                                          : scan_bwd_kernel<float, float>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if ((e = trace_before(st, "scan_bwd")) != cudaSuccess) return e;
+  kern<<<(unsigned)(s.Bt * s.H), kBT, smem, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return trace_after(st);
+}
+
+}  // namespace pdssm

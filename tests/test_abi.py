@@ -195,3 +195,28 @@ def test_default_chunk_keeps_the_workspace_below_the_fixed_chunk_one():
         assert ws(chunk=0, **kw) <= fixed, kw
     many = dict(batch=16, heads=64, seqlen=8192, N=128, P=64, K=64)
     assert ws(chunk=0, **many) < ws(chunk=64, **many)
+
+
+def test_backward_validation():
+    """pdssm_scan_bwd rejects a complex state, a non-positive temperature, logits without
+    dlogits (and the reverse), missing pointers and a small workspace, before any launch."""
+    n = ctypes.c_size_t(0)
+    assert pd._lib.pdssm_bwd_workspace_size(ctypes.byref(_pb(state_t=pd.C64, d_t=pd.C64, out_t=pd.C64)),
+                                            ctypes.byref(n)) == 2  # PDSSM_ERR_UNSUPPORTED
+    pb = _pb()
+    assert pd._lib.pdssm_bwd_workspace_size(ctypes.byref(pb), ctypes.byref(n)) == OK and n.value > 0
+    fake = ctypes.c_void_p(4096)
+
+    def call(tau=1.0, logits=fake, dlogits=fake, ws_bytes=None, **drop):
+        ptr = dict(s=fake, idx=fake, d=fake, B=fake, C=fake, x=fake, dy=fake, dd=fake, dB=fake, dC=fake, dx=fake)
+        for k in drop:
+            ptr[k] = None
+        return pd._lib.pdssm_scan_bwd(ctypes.byref(pb), logits, ptr["s"], ptr["idx"], ptr["d"], ptr["B"], ptr["C"],
+                                      ptr["x"], None, ptr["dy"], None, ctypes.c_float(tau), dlogits, ptr["dd"],
+                                      ptr["dB"], ptr["dC"], ptr["dx"], None, fake,
+                                      n.value if ws_bytes is None else ws_bytes, None)
+    assert call(tau=0.0) == 1 and call(tau=-1.0) == 1 and call(tau=float("inf")) == 1
+    assert call(logits=None) == 1 and call(dlogits=None) == 1
+    for k in ("s", "idx", "d", "B", "C", "x", "dy", "dd", "dB", "dC", "dx"):
+        assert call(**{k: True}) == 1, k
+    assert call(ws_bytes=n.value - 1) == 3  # PDSSM_ERR_WORKSPACE

@@ -1,0 +1,95 @@
+"""Parity of the backward pass (pdssm_scan_bwd through the C ABI) with the backward
+oracle (oracle/backward.py) on seeded workloads: every gradient, per (batch, head)
+slice, within 1e-4 of the slice's largest value."""
+import numpy as np
+import pytest
+import torch
+
+import structured_sparse_selective_b200 as pd
+import workloads
+from oracle import backward as bwd
+
+TOL = 1e-4
+
+
+def _slices(t):
+    """[Bt, L, H, X] -> [Bt*H, L, X] fp64 numpy"""
+    Bt, L, H, X = t.shape
+    return t.permute(0, 2, 1, 3).reshape(Bt * H, L, X).double().cpu().numpy()
+
+
+def _rel(got, ref):
+    scale = np.abs(ref).max(axis=tuple(range(1, ref.ndim)), keepdims=True)
+    return float((np.abs(got - ref) / np.maximum(scale, 1e-30)).max()) if ref.size else 0.0
+
+
+def _run(recipe, kw, dev, seed=0, with_h0=True, with_dh=True, with_logits=True, tau=0.7):
+    sp = workloads.spec(recipe, **kw)
+    inp = workloads.generate(sp, seed=seed)
+    g = {k: v.to(dev) for k, v in inp.items()}
+    # the forward pass gives the selections (they do not depend on h0)
+    fwd = pd.forward(g["logits"], g["idx"], g["d"], g["B"], g["C"], g["x"], want_s=True, want_prod=False)
+    Bt, L, H, N = inp["B"].shape
+    P = inp["x"].shape[-1]
+    gen = torch.Generator().manual_seed(100 + seed)
+    dy = torch.randn(Bt, L, H, P, generator=gen).to(fwd["y"].dtype)
+    h0 = torch.randn(Bt, H, N, P, generator=gen) if with_h0 else None
+    dh = torch.randn(Bt, H, N, P, generator=gen) if with_dh else None
+    out = pd.backward(g["logits"] if with_logits else None, fwd["s"], g["idx"], g["d"], g["B"], g["C"], g["x"],
+                      dy.to(dev), h0=None if h0 is None else h0.to(dev), dh_final=None if dh is None else dh.to(dev),
+                      tau=tau)
+    torch.cuda.synchronize(dev)
+    S = Bt * H
+    ref = bwd.scan_backward(_slices(inp["logits"]), inp["idx"].numpy(), _slices(inp["d"]), _slices(inp["B"]),
+                            _slices(inp["C"]), _slices(inp["x"]), _slices(dy),
+                            None if dh is None else dh.reshape(S, N, P).double().numpy(),
+                            None if h0 is None else h0.reshape(S, N, P).double().numpy(), tau=tau)
+    s_slices = fwd["s"].cpu().permute(0, 2, 1).reshape(S, L).numpy()
+    assert np.array_equal(s_slices, ref["s"])
+    errs = {}
+    for k in ("dd", "dB", "dC", "dx") + (("dlogits",) if with_logits else ()):
+        errs[k] = _rel(_slices(out[k].cpu()), ref[k])
+    errs["dh0"] = _rel(out["dh0"].cpu().reshape(S, N, P).double().numpy(), ref["dh0"])
+    return errs
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("recipe,kw", [
+    ("tiny", dict()),
+    ("tiny", dict(seqlen=1)),
+    ("tiny", dict(seqlen=15)),
+    ("z5", dict(batch=3, seqlen=37)),
+    ("lm", dict(batch=1, seqlen=70, heads=2)),
+    ("long", dict(batch=1, seqlen=53, heads=2)),
+])
+def test_backward_matches_oracle(cuda_device, recipe, kw):
+    errs = _run(recipe, kw, cuda_device)
+    assert all(v <= TOL for v in errs.values()), errs
+
+
+@pytest.mark.gpu
+def test_backward_without_initial_state_final_gradient_or_logits(cuda_device):
+    errs = _run("lm", dict(batch=1, seqlen=33, heads=2), cuda_device, seed=3, with_h0=False, with_dh=False,
+                with_logits=False)
+    assert all(v <= TOL for v in errs.values()), errs
+
+
+@pytest.mark.gpu
+def test_backward_maximum_sizes(cuda_device):
+    """N = P = 128, K = 64: the largest shared-memory footprint of the backward block."""
+    sp = dict(batch=1, seqlen=20, heads=1, N=128, P=128, K=64)
+    errs = _run("tiny", sp, cuda_device, seed=4)
+    assert all(v <= TOL for v in errs.values()), errs
+
+
+@pytest.mark.gpu
+def test_backward_empty_sequence_passes_the_final_gradient_through(cuda_device):
+    dev = cuda_device
+    Bt, H, N, P, K = 2, 3, 8, 4, 4
+    z = lambda *s: torch.zeros(*s, device=dev)
+    dh = torch.randn(Bt, H, N, P, device=dev)
+    out = pd.backward(z(Bt, 0, H, K), torch.zeros(Bt, 0, H, dtype=torch.int32, device=dev),
+                      torch.zeros(K, N, dtype=torch.int32, device=dev), z(Bt, 0, H, N), z(Bt, 0, H, N),
+                      z(Bt, 0, H, N), z(Bt, 0, H, P), z(Bt, 0, H, P), dh_final=dh)
+    torch.cuda.synchronize(dev)
+    assert torch.equal(out["dh0"], dh)
