@@ -93,19 +93,44 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
     }
     return st;
   };
-  // the step's d, B, x and the preimage lists of its entry (for a forward step)
-  auto stage_fwd = [&](int64_t t) {
-    const int64_t row = row_of(t);
-    const int st = load_s(row);
-    for (int j = tid; j < N; j += kBT) {
-      dsh[j] = to_f32(dg[row * N + j]);
-      Bsh[j] = to_f32(Bg[row * N + j]);
-      srcsh[j] = a.src[(int64_t)st * N + j];
-    }
-    for (int j = tid; j <= N; j += kBT) offsh[j] = a.off[(int64_t)st * (N + 1) + j];
-    for (int p = tid; p < P; p += kBT) xsh[p] = to_f32(xg[row * P + p]);
+  // A step's vectors, fetched into registers a step ahead: thread tid holds entry
+  // tid of d, B, C (and of the entry's preimage lists), of x and dy (N, P <= 128 <
+  // kBT, so one entry each) and s.
+  struct Vec {
+    float d, B, C, x, dy;
+    int src, off, st;
   };
-  // Hn = A_t Hc + B_t x_t^T (after stage_fwd(t) and a barrier)
+  auto fetch = [&](int64_t t, bool rev) {
+    Vec v;
+    const int64_t row = row_of(t);
+    v.st = load_s(row);
+    if (tid < N) {
+      v.d = to_f32(dg[row * N + tid]);
+      v.B = to_f32(Bg[row * N + tid]);
+      if (rev) v.C = to_f32(Cg[row * N + tid]);
+      else v.src = a.src[(int64_t)v.st * N + tid];
+    }
+    if (!rev && tid <= N) v.off = a.off[(int64_t)v.st * (N + 1) + tid];
+    if (tid < P) {
+      v.x = to_f32(xg[row * P + tid]);
+      if (rev) v.dy = ld_flag(a.dy, row * P + tid, a.dy_bf16);
+    }
+    return v;
+  };
+  auto commit = [&](const Vec &v, bool rev) {
+    if (tid < N) {
+      dsh[tid] = v.d;
+      Bsh[tid] = v.B;
+      if (rev) Csh[tid] = v.C;
+      else srcsh[tid] = v.src;
+    }
+    if (!rev && tid <= N) offsh[tid] = v.off;
+    if (tid < P) {
+      xsh[tid] = v.x;
+      if (rev) dysh[tid] = v.dy;
+    }
+  };
+  // Hn = A_t Hc + B_t x_t^T (after commit of step t's vectors and a barrier)
   auto step_fwd = [&](const float *Hc, float *Hn) {
     FOR_NP(i, p) {
       float acc = Bsh[i] * xsh[p];
@@ -127,10 +152,12 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
   // ---- forward sweep: checkpoints every kTb steps
   float *Hc = buf0, *Hn = buf1;
   FOR_NP(i, p) { Hc[i * PS + p] = a.h0 ? a.h0[(bh * N + i) * P + p] : 0.f; }
+  Vec nv = fetch(0, false);
   for (int64_t t = 0; t < a.L; ++t) {
     __syncthreads();  // Hc complete; the staged vectors are no longer read
     if (t % kTb == 0) store_dense(Hc, ck + (t / kTb) * N * P);
-    stage_fwd(t);
+    commit(nv, false);
+    if (t + 1 < a.L) nv = fetch(t + 1, false);
     __syncthreads();
     step_fwd(Hc, Hn);
     float *tmp = Hc;
@@ -150,10 +177,12 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
     if (Lam == buf1) Hn = buf2;
     __syncthreads();
     load_dense(ck + c * N * P, Hc);
+    nv = fetch(t0, false);
     for (int64_t t = t0; t < t1; ++t) {
       __syncthreads();
       store_dense(Hc, scr + (t - t0) * N * P);
-      stage_fwd(t);
+      commit(nv, false);
+      if (t + 1 < t1) nv = fetch(t + 1, false);
       __syncthreads();
       step_fwd(Hc, Hn);
       float *tmp = Hc;
@@ -161,19 +190,13 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
       Hn = tmp;
     }
     float *Hp = Hn;  // receives H_{t-1}
+    Vec rv = fetch(t1 - 1, true);
     for (int64_t t = t1 - 1; t >= t0; --t) {
       const int64_t row = row_of(t);
       __syncthreads();  // [A] the previous step is done with every buffer and vector
-      const int st = load_s(row);
-      for (int j = tid; j < N; j += kBT) {
-        dsh[j] = to_f32(dg[row * N + j]);
-        Bsh[j] = to_f32(Bg[row * N + j]);
-        Csh[j] = to_f32(Cg[row * N + j]);
-      }
-      for (int p = tid; p < P; p += kBT) {
-        xsh[p] = to_f32(xg[row * P + p]);
-        dysh[p] = ld_flag(a.dy, row * P + p, a.dy_bf16);
-      }
+      const int st = rv.st;
+      commit(rv, true);
+      if (t > t0) rv = fetch(t - 1, true);
       load_dense(scr + (t - t0) * N * P, Hp);
       __syncthreads();
       // [B] Lam_t = Lam'_t + C_t dy_t^T
@@ -196,6 +219,7 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
         for (int j = lane; j < N; j += 32) {
           const int r = idxsh[k * N + j];
           float q = 0.f;
+#pragma unroll 4
           for (int p = 0; p < P; ++p) q = fmaf(Lam[r * PS + p], Hp[j * PS + p], q);
           if (k == st) a.dd[row * N + j] = q;
           part = fmaf(dsh[j], q, part);
