@@ -1,6 +1,7 @@
 """Benchmark of the Flash PD-SSM forward pass on B200 (one process per GPU).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload lm]
+                    [--pass forward|backward] [--tau T]
 
 A step is one pdssm_forward call (selection + dictionary preparation + the
 whole chunked scan) over one batch of the LM-layer workload (batch 8, L 2048,
@@ -11,6 +12,8 @@ synchronise on every rank, and the slowest rank's time is reported.
 
 Rank 0 prints one JSON line. ``--impl reference`` times the dense CPU oracle
 on the host cores on a bounded sample of the same workload instead.
+``--pass backward`` measures the backward pass (pdssm_scan_bwd, real states)
+the same way instead of the forward pass; the default is the forward pass.
 """
 from __future__ import annotations
 
@@ -31,6 +34,7 @@ if ROOT not in sys.path:
 import workloads  # noqa: E402
 
 METRIC = "PD-SSM forward scan tokens·heads/s at LM shape; achieved HBM GB/s vs B200 peak"
+BWD_METRIC = "PD-SSM backward scan tokens·heads/s (straight-through tempered softmax); achieved HBM GB/s"
 UNIT = "token·heads/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
@@ -378,6 +382,132 @@ def run_ours(args, rank, world, local):
     return result
 
 
+# ------------------------------------------------------------ backward pass
+
+def bwd_bytes_per_token_head(sp: workloads.Spec) -> int:
+    """Bytes the backward pass must move per (b, t, h): s, logits, d, B, C, x and dy read once,
+    dd, dB, dC, dx and dlogits (float32) written once."""
+    def sz(dt):
+        return torch.empty((), dtype=dt).element_size()
+    reads = 4 + sp.K * sz(sp.logits_dtype) + sp.N * sz(sp.d_dtype) + 2 * sp.N * sz(sp.in_dtype)
+    reads += sp.P * sz(sp.in_dtype) + sp.P * sz(sp.out_dtype)
+    return reads + (3 * sp.N + sp.P + sp.K) * 4
+
+
+def run_ours_backward(args, rank, world, local):
+    import structured_sparse_selective_b200 as pd
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    sp = workloads.spec(args.workload)
+    if sp.state_complex:
+        raise SystemExit("the backward pass is built for real states only")
+    inp = {k: v.to(device) for k, v in workloads.generate(sp, seed=shard_seed(rank)).items()}
+    fwd = pd.forward(inp["logits"], inp["idx"], inp["d"], inp["B"], inp["C"], inp["x"], want_s=True,
+                     want_prod=False)
+    gen = torch.Generator(device=device).manual_seed(shard_seed(rank))
+    dy = torch.randn(fwd["y"].shape, generator=gen, device=device).to(fwd["y"].dtype)
+    pb = pd.make_problem(inp["logits"], inp["d"], inp["B"], inp["x"], out_dtype=dy.dtype)
+    Bt, L, H, N = inp["B"].shape
+    P = inp["x"].shape[-1]
+    f32 = dict(dtype=torch.float32, device=device)
+    gr = {"dlogits": torch.empty(Bt, L, H, sp.K, **f32), "dd": torch.empty(Bt, L, H, N, **f32),
+          "dB": torch.empty(Bt, L, H, N, **f32), "dC": torch.empty(Bt, L, H, N, **f32),
+          "dx": torch.empty(Bt, L, H, P, **f32), "dh0": torch.empty(Bt, H, N, P, **f32)}
+    ws = torch.empty(max(1, pd.pdssm_bwd_workspace_size(pb)), dtype=torch.uint8, device=device)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        pd.pdssm_scan_bwd(pb, inp["logits"], fwd["s"], inp["idx"], inp["d"], inp["B"], inp["C"], inp["x"], None,
+                          dy, None, args.tau, gr["dlogits"], gr["dd"], gr["dB"], gr["dC"], gr["dx"], gr["dh0"], ws,
+                          stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    traces = [pd.KernelTrace(max_launches=8) for _ in range(args.steps)]
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            with traces[i]:
+                step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(device)
+    barrier(world, device)
+    check = pd.pdssm_read_device_check(ws)
+    if check:
+        raise RuntimeError(f"device check status {check} after the timed steps")
+    ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)) / args.steps, world, device)
+    per_kernel = {}
+    launches = 0
+    for tr in traces:
+        for name, t in tr.timings():
+            per_kernel.setdefault(name, []).append(t)
+            launches += 1
+    dom_ms = sum(per_kernel["scan_bwd"]) / len(per_kernel["scan_bwd"])
+    units = sp.token_heads
+    alg = units * bwd_bytes_per_token_head(sp)
+    peaks = load_peaks()
+    achieved = alg / (dom_ms / 1e3) / 1e9
+    if rank != 0:
+        return None
+    return {
+        "metric": BWD_METRIC, "pass": "backward", "value": round(units * world / (ms / 1e3), 1), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(sp, 0, world), tau=args.tau),
+        "roofline": {"bound": "hbm", "kernel": "scan_bwd", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "peak_source": peaks["source"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 5),
+                     "traffic": None, "algorithmic_bytes_per_launch": int(alg), "launch_ms": round(dom_ms, 4)},
+        "kernels_ms_per_step": {k: round(sum(v) / args.steps, 5) for k, v in per_kernel.items()},
+        "gpu_launches": launches, "clocks": clocks.summary(),
+    }
+
+
+def run_reference_backward(args, rank, world):
+    """The backward oracle (numpy, dense fp64, one thread) on whole (batch, head) slices."""
+    if rank != 0:
+        return None
+    from oracle import backward as obwd
+    sp = workloads.spec(args.workload)
+    if sp.state_complex:
+        raise SystemExit("the backward pass is built for real states only")
+    idx = workloads.generate_idx(sp).numpy()
+    n = 2
+    picks = [(i // sp.heads % sp.batch, i % sp.heads) for i in range(n)]
+    sls = [workloads.generate_slice(sp, b, h) for b, h in picks]
+    stack = {k: torch.stack([s_[k] for s_ in sls]).double().numpy() for k in sls[0]}
+    dy = torch.randn(n, sp.seqlen, sp.P, generator=torch.Generator().manual_seed(0)).to(sp.out_dtype).double().numpy()
+
+    def step():
+        obwd.scan_backward(stack["logits"], idx, stack["d"], stack["B"], stack["C"], stack["x"], dy, tau=args.tau)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    sec = (time.perf_counter() - t0) / args.steps
+    units = n * sp.seqlen
+    value = units / sec
+    sample = (f"each step: {n} whole (batch, head) slices x L={sp.seqlen} of the {sp.recipe} workload "
+              f"({units} token-heads), dense fp64 backward oracle (numpy, one thread)")
+    return {
+        "impl": "reference", "metric": BWD_METRIC, "pass": "backward", "value": round(value, 1), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(workload_config(sp, 0, world), tau=args.tau),
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 # ------------------------------------------------------------ reference arm
 
 def run_reference(args, rank, world):
@@ -425,17 +555,24 @@ def main(argv=None):
     ap.add_argument("--workload", default="lm", choices=list(workloads.RECIPES))
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward")
+    ap.add_argument("--tau", type=float, default=1.0, help="softmax temperature of the backward pass")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local = dist_env()
     if args.impl == "reference":
-        res = run_reference(args, rank, world)
+        res = (run_reference_backward if args.pass_ == "backward" else run_reference)(args, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
         return 0
     init_dist(world, "nccl")
     try:
+        if args.pass_ == "backward":
+            res = run_ours_backward(args, rank, world, local)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return 0
         res = run_ours(args, rank, world, local)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:

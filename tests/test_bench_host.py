@@ -78,3 +78,27 @@ def test_bench_rejects_short_warmup():
     r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--warmup", "2"],
                        capture_output=True, text=True, timeout=120)
     assert r.returncode != 0 and "at least 3" in r.stderr
+
+
+def test_reference_arm_of_the_backward_pass():
+    """``--impl reference --pass backward`` times the backward oracle and prints one line."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--pass", "backward",
+                        "--workload", "tiny", "--steps", "2", "--warmup", "3", "--tau", "0.5"],
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    res = json.loads(lines[0])
+    assert res["pass"] == "backward" and res["impl"] == "reference" and res["value"] > 0
+    assert res["config"]["tau"] == 0.5 and res["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_backward_bytes_per_token_head():
+    """LM workload: s 4 + logits 16 x 2 + d, B, C 3 x 64 x 2 + x, dy 2 x 64 x 2 read, and
+    dd, dB, dC, dx, dlogits (3 x 64 + 64 + 16) x 4 written."""
+    import workloads
+    assert bench.bwd_bytes_per_token_head(workloads.spec("lm")) == 4 + 32 + 384 + 256 + 272 * 4
