@@ -220,3 +220,17 @@ def test_backward_validation():
     for k in ("s", "idx", "d", "B", "C", "x", "dy", "dd", "dB", "dC", "dx"):
         assert call(**{k: True}) == 1, k
     assert call(ws_bytes=n.value - 1) == 3  # PDSSM_ERR_WORKSPACE
+
+
+def test_package_refuses_to_load_without_its_cuda_library(tmp_path):
+    """No CPU fallback: a copy of the package without libpdssm.so raises on import."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "structured_sparse_selective_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(os.path.dirname(pd.__file__), "__init__.py"), pkg / "__init__.py")
+    r = subprocess.run([sys.executable, "-c", "import structured_sparse_selective_b200"], cwd=tmp_path,
+                       capture_output=True, text=True, timeout=120,
+                       env=dict(os.environ, PYTHONPATH=str(tmp_path)))
+    assert r.returncode != 0 and "ImportError" in r.stderr and "libpdssm.so" in r.stderr
