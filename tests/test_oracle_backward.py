@@ -163,9 +163,9 @@ def test_logit_gradients_sum_to_zero_and_scale_with_temperature():
 
 
 @pytest.mark.parametrize("mutation", [
-    ("lam = A[t].T @ lam", "lam = A[t] @ lam"),                                  # adjoint not transposed
+    ("lam = np.conj(A[t]).T @ lam", "lam = np.conj(A[t]) @ lam"),                # adjoint not transposed
     ("lam = lam + np.outer(C[t], dy[t])", "lam = lam + 0 * np.outer(C[t], dy[t])"),  # output term dropped
-    ("dA = lam @ Hprev.T", "dA = lam @ Ht.T"),                                   # state one step late
+    ("dA = lam @ np.conj(Hprev).T", "dA = lam @ np.conj(Ht).T"),                 # state one step late
     ('out["dd"][t] = dA[idx[s[t]], np.arange(N)]', 'out["dd"][t] = dA[np.arange(N), idx[s[t]]]'),  # transposed pick
     ("(np.diag(pit) - np.outer(pit, pit)) @ dpi / tau", "(np.diag(pit) - np.outer(pit, pit)) @ dpi"),  # no 1/tau
 ])
@@ -178,3 +178,93 @@ def test_a_planted_mistake_fails_the_automatic_differentiation_pin(mutation):
     got = ns["slice_backward"](**pr, tau=0.5)
     ref = _autograd(pr, 0.5)
     assert any(not np.allclose(got[k], v, rtol=1e-8, atol=1e-9) for k, v in ref.items())
+
+
+# ---------------------------------------------------------------- complex states
+
+def _cproblem(L, N, P, K, seed):
+    g = np.random.default_rng(seed)
+    pr = _problem(L, N, P, K, seed)
+    r = g.uniform(0.5, 1.0, (L, N))
+    pr["d"] = r * np.exp(1j * g.uniform(0, 2 * np.pi, (L, N)))
+    pr["dy"] = g.standard_normal((L, P)) + 1j * g.standard_normal((L, P))
+    pr["dh_final"] = g.standard_normal((N, P)) + 1j * g.standard_normal((N, P))
+    pr["h0"] = g.standard_normal((N, P)) + 1j * g.standard_normal((N, P))
+    return pr
+
+
+def _autograd_complex(pr, tau):
+    """Complex autograd (PyTorch's gradient dL/du + i dL/dv of a real loss) of the dense
+    forward with straight-through selection weights."""
+    real = ("logits", "B", "C", "x")
+    t = {k: torch.tensor(v, dtype=torch.float64 if k in real else torch.complex128,
+                         requires_grad=k in real + ("d", "h0")) for k, v in pr.items() if k != "idx"}
+    L, K = t["logits"].shape
+    N = t["B"].shape[1]
+    Pk = torch.zeros(K, N, N, dtype=torch.complex128)
+    for k in range(K):
+        Pk[k, torch.as_tensor(pr["idx"][k]), torch.arange(N)] = 1.0
+    soft = torch.softmax(t["logits"] / tau, dim=-1)
+    hard = torch.nn.functional.one_hot(t["logits"].argmax(dim=-1), K).to(torch.float64)
+    pi = (hard + soft - soft.detach()).to(torch.complex128)
+    H = t["h0"]
+    loss = torch.zeros((), dtype=torch.float64)
+    for s in range(L):
+        A = torch.einsum("k,kij->ij", pi[s], Pk) * t["d"][s][None, :]
+        H = A @ H + torch.outer(t["B"][s], t["x"][s]).to(torch.complex128)
+        y = H.T @ t["C"][s].to(torch.complex128)
+        loss = loss + (t["dy"][s].conj() * y).sum().real
+    loss = loss + (t["dh_final"].conj() * H).sum().real
+    names = ["logits", "d", "B", "C", "x", "h0"]
+    grads = torch.autograd.grad(loss, [t[k] for k in names])
+    return {"d" + k: g.numpy() for k, g in zip(names, grads)}
+
+
+@pytest.mark.parametrize("L,N,P,K", [(1, 3, 2, 2), (11, 5, 3, 4), (20, 8, 4, 6)])
+def test_complex_matches_automatic_differentiation(L, N, P, K):
+    pr = _cproblem(L, N, P, K, seed=L + N)
+    got = bwd.slice_backward(**pr, tau=0.6)
+    for k, v in _autograd_complex(pr, 0.6).items():
+        np.testing.assert_allclose(got[k], v, rtol=1e-10, atol=1e-11, err_msg=k)
+
+
+@pytest.mark.parametrize("name", ["d", "h0"])
+def test_complex_matches_differences_of_real_and_imaginary_parts(name):
+    """dL/du + i dL/dv by central differences of the C forward oracle (complex mode)."""
+    pr = _cproblem(8, 4, 2, 3, seed=21)
+
+    def loss(q):
+        S = lambda a: a[None]
+        r = oracle.scan_slices(S(q["logits"]), q["idx"].astype(np.int32), S(q["d"]), S(q["B"]), S(q["C"]),
+                               S(q["x"]), S(q["h0"]), want_prod=False)
+        return float(np.real(np.sum(np.conj(q["dy"]) * r["y"][0]) + np.sum(np.conj(q["dh_final"]) * r["h_final"][0])))
+
+    got = bwd.slice_backward(**pr)["d" + name]
+    base = pr[name]
+    fd = np.zeros_like(base)
+    eps = 1e-6
+    for i in np.ndindex(base.shape):
+        parts = []
+        for step in (eps, 1j * eps):
+            hi, lo = dict(pr), dict(pr)
+            hi[name], lo[name] = base.copy(), base.copy()
+            hi[name][i] += step
+            lo[name][i] -= step
+            parts.append((loss(hi) - loss(lo)) / (2 * eps))
+        fd[i] = parts[0] + 1j * parts[1]
+    np.testing.assert_allclose(got, fd, rtol=1e-6, atol=1e-7)
+
+
+def test_conjugating_every_complex_input_conjugates_the_complex_gradients():
+    """With B, C, x real, conj(d, h0, dy, dh_final) leaves the loss unchanged and
+    conjugates y and H, so dd and dh0 conjugate and the real gradients stay."""
+    pr = _cproblem(15, 5, 3, 4, seed=8)
+    a = bwd.slice_backward(**pr)
+    pc = dict(pr)
+    for k in ("d", "h0", "dy", "dh_final"):
+        pc[k] = np.conj(pr[k])
+    b = bwd.slice_backward(**pc)
+    np.testing.assert_allclose(b["dd"], np.conj(a["dd"]), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(b["dh0"], np.conj(a["dh0"]), rtol=1e-12, atol=1e-13)
+    for k in ("dB", "dC", "dx", "dlogits"):
+        np.testing.assert_allclose(b[k], a[k], rtol=1e-12, atol=1e-13, err_msg=k)
