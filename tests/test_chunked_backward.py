@@ -37,3 +37,17 @@ def test_chunked_adjoint_without_initial_state_or_final_gradient():
     got = chunked_backward(**pr, T=6)
     for k in ("dd", "dB", "dC", "dx", "dlogits", "dh0"):
         np.testing.assert_allclose(got[k], ref[k], rtol=1e-10, atol=1e-11, err_msg=k)
+
+
+@pytest.mark.parametrize("T", [1, 4, 16, 50])
+def test_chunked_adjoint_equals_sequential_for_complex_states(T):
+    g = np.random.default_rng(T)
+    pr = _problem(33, 6, 3, 4, seed=T)
+    pr["d"] = g.uniform(0.5, 1.0, (33, 6)) * np.exp(1j * g.uniform(0, 2 * np.pi, (33, 6)))
+    pr["dy"] = g.standard_normal((33, 3)) + 1j * g.standard_normal((33, 3))
+    pr["dh_final"] = g.standard_normal((6, 3)) + 1j * g.standard_normal((6, 3))
+    pr["h0"] = g.standard_normal((6, 3)) + 1j * g.standard_normal((6, 3))
+    ref = bwd.slice_backward(**pr, tau=0.9)
+    got = chunked_backward(**pr, T=T, tau=0.9)
+    for k in ("dd", "dB", "dC", "dx", "dlogits", "dh0"):
+        np.testing.assert_allclose(got[k], ref[k], rtol=1e-10, atol=1e-11, err_msg=k)
