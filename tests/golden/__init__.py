@@ -47,5 +47,11 @@ def load(name):
         "prod_val": [float(v) for v in fields["prod_val"].split()],
         "s": letters,
     }
+    for k in ("bwd_dC", "bwd_dB", "bwd_dd"):  # [L][N], rows separated by |
+        if k in fields:
+            exp[k] = [[float(v) for v in row.split()] for row in fields[k].split("|")]
+    for k in ("bwd_dx", "bwd_dh0"):
+        if k in fields:
+            exp[k] = [float(v) for v in fields[k].split()]
     assert len(idx) == K and all(len(r) == N for r in idx) and len(exp["y"]) == L
     return inp, exp

@@ -38,3 +38,21 @@ def test_a_planted_transposition_is_caught():
         A = Pk.T @ np.diag(d[t])                # the transposed operand
         H = A @ H + inp["B"][0, t, 0].numpy()
     assert H.tolist() != exp["h_final"]
+
+
+@pytest.mark.parametrize("name", [n for n in golden.names() if "bwd_dB" in golden.load(n)[1]])
+def test_backward_oracle_reproduces_the_hand_worked_gradients(name):
+    """The loss sum_t y_t (dy = 1, no final-state gradient) on the weighted automaton:
+    every gradient worked by hand in the fixture header."""
+    import numpy as np
+    from oracle import backward as bwd
+    inp, exp = golden.load(name)
+    sl = lambda t: t[0, :, 0].double().numpy()
+    L, P = inp["x"].shape[1], inp["x"].shape[-1]
+    r = bwd.slice_backward(sl(inp["logits"]), inp["idx"].numpy(), sl(inp["d"]), sl(inp["B"]), sl(inp["C"]),
+                           sl(inp["x"]), np.ones((L, P)))
+    assert r["dC"].tolist() == exp["bwd_dC"]
+    assert r["dB"].tolist() == exp["bwd_dB"]
+    assert r["dd"].tolist() == exp["bwd_dd"]
+    assert r["dx"][:, 0].tolist() == exp["bwd_dx"]
+    assert r["dh0"][:, 0].tolist() == exp["bwd_dh0"]
