@@ -111,8 +111,18 @@ const char *pdssm_version(void);
 
 /*
  * Workspace bytes that pdssm_scan_fwd / pdssm_forward need for `pb`
- * (written to *bytes). The size grows as O(batch*heads*seqlen*(N+P)) -- the
- * O(L*N) memory of Methodology 1 -- and never with N*N.
+ * (written to *bytes). The size follows the path the problem takes:
+ *   - the fused single-kernel path (real state, N = P = 64, bf16 d/B/C/x,
+ *     K * sizeof(logit) a multiple of 16, chunk 0 or 16, no
+ *     PDSSM_FLAG_REFERENCE_PATH) needs only the 4-byte error word (256 bytes
+ *     are reported), provided logits (or s), d, B, C and x are 16-byte aligned;
+ *   - every other problem takes the three-kernel path, whose workspace grows as
+ *     O(batch*heads*seqlen*(N+P)) -- the O(L*N) memory of Methodology 1 -- and
+ *     never with N*N.
+ * A fused-path problem whose inputs are not 16-byte aligned runs on the
+ * three-kernel path and needs the size reported for the same problem with
+ * PDSSM_FLAG_REFERENCE_PATH set; with a smaller workspace the call returns
+ * PDSSM_ERR_WORKSPACE before anything is enqueued.
  * Errors: PDSSM_ERR_INVALID_ARG / PDSSM_ERR_UNSUPPORTED as for the calls.
  */
 pdssm_status pdssm_workspace_size(const pdssm_problem *pb, size_t *bytes);
@@ -122,6 +132,9 @@ pdssm_status pdssm_workspace_size(const pdssm_problem *pb, size_t *bytes);
  * logits[b][t][h][k] == max_k' logits[b][t][h][k']. +0 and -0 compare equal;
  * a NaN counts as the maximum and the first NaN wins. Bit-exact.
  * logits: device, logits_t; s: device int32 output. No workspace.
+ * One row is reduced by a group of lanes of a warp; rows whose size is a
+ * multiple of 16 bytes (and a 16-byte aligned logits pointer) are read with
+ * 128-bit loads.
  */
 pdssm_status pdssm_select(const pdssm_problem *pb, const void *logits, int32_t *s,
                           pdssm_stream_t stream);
@@ -175,9 +188,11 @@ pdssm_status pdssm_forward(const pdssm_problem *pb, const void *logits, const in
  *   held by every GPU that loads the library until the process exits.
  *   Problems whose pdssm_workspace_size exceeds 32 MiB return
  *   PDSSM_ERR_WORKSPACE before anything is enqueued.
- *   The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any
- *   stream capture.
+ *   The first call on a device looks up the array's device address (with that
+ *   device current) and keeps it; make that first call before any stream
+ *   capture. A lookup that fails returns PDSSM_ERR_CUDA and is retried by the
+ *   next call. Problems served by the fused kernel use only the array's error
+ *   word; the 32 MiB limit matters for the three-kernel path.
  *   All calls on a device share the array and it keeps the last call's
  *   contents: calls that overlap on the GPU race and must be ordered by the
  *   caller (one stream, or events). pdssm_read_device_check cannot read this

@@ -28,6 +28,7 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 struct Plan {
   int64_t Bt, L, H, N, P, K, T, nC, rows;
   bool cplx;
+  bool fused;         // the fused kernel serves the problem: the workspace is the error word only
   size_t state_size;  // bytes per state element (4 or 8)
   // workspace offsets
   size_t o_err, o_idx, o_off, o_src, o_s, o_cstate, o_cidx, o_cval, o_yloc, total;
@@ -46,7 +47,11 @@ int64_t default_chunk(const pdssm_problem *pb) {
   return std::max<int64_t>(T, pb->P);
 }
 
-pdssm_status make_plan(const pdssm_problem *pb, Plan *pl) {
+// Validates the problem and lays out its workspace. The layout follows the path
+// the problem takes: the fused kernel (when it applies and `three_kernel` is
+// false) needs only the error word; the three-kernel path needs the chunk
+// states, pairs and local outputs as well.
+pdssm_status make_plan(const pdssm_problem *pb, Plan *pl, bool three_kernel = false) {
   if (!pb) return PDSSM_ERR_INVALID_ARG;
   if (pb->batch < 0 || pb->seqlen < 0 || pb->heads < 0 || pb->N < 1 || pb->P < 1 || pb->K < 1 ||
       pb->chunk < 0)
@@ -77,8 +82,15 @@ pdssm_status make_plan(const pdssm_problem *pb, Plan *pl) {
   if (p.nC > INT32_MAX) return PDSSM_ERR_UNSUPPORTED;
   p.rows = rows;
   int64_t nchunks = bh * p.nC;
+  p.fused = !three_kernel && fused_scan_applies(pb);
   size_t o = 0;
   p.o_err = o; o = align256(o + 4);
+  if (p.fused) {
+    p.o_idx = p.o_off = p.o_src = p.o_s = p.o_cstate = p.o_cidx = p.o_cval = p.o_yloc = o;
+    p.total = o;
+    *pl = p;
+    return PDSSM_OK;
+  }
   p.o_idx = o; o = align256(o + (size_t)(p.K * p.N) * 4);
   p.o_off = o; o = align256(o + (size_t)(p.K * (p.N + 1)) * 4);
   p.o_src = o; o = align256(o + (size_t)(p.K * p.N) * 4);
@@ -145,16 +157,25 @@ pdssm_status finish(const pdssm_problem *pb, const Workspace &w, cudaStream_t st
   return PDSSM_OK;
 }
 
-pdssm_status run_scan(const pdssm_problem *pb, const Plan &p, const int32_t *s,
+pdssm_status run_scan(const pdssm_problem *pb, const Plan &plan, const int32_t *s,
                       const void *logits, int32_t *s_out, const int32_t *idx, const void *d,
                       const void *B, const void *C, const void *x, const void *h0, void *y,
                       void *h_final, int32_t *prod_idx, void *prod_val, void *workspace,
-                      cudaStream_t stream) {
+                      size_t workspace_bytes, cudaStream_t stream) {
+  Plan p = plan;
+  ScanArgs a;
+  a.s = s; a.logits = logits; a.d = d; a.B = B; a.C = C; a.x = x;
+  if (p.fused && !fused_scan_pointers_ok(a)) {
+    // inputs the fused kernel's 16-byte loads cannot read: the three-kernel
+    // path runs instead and needs its own (larger) workspace
+    pdssm_status st = make_plan(pb, &p, true);
+    if (st != PDSSM_OK) return st;
+    if (workspace_bytes < p.total) return PDSSM_ERR_WORKSPACE;
+  }
   Workspace w = carve(p, workspace);
   if (cudaMemsetAsync(w.err, 0, 4, stream) != cudaSuccess) return PDSSM_ERR_CUDA;
   pdssm_status st = PDSSM_OK;
 
-  ScanArgs a;
   a.Bt = p.Bt; a.L = p.L; a.H = p.H; a.N = p.N; a.P = p.P; a.K = p.K; a.T = p.T; a.nC = p.nC;
   a.d_t = pb->d_t; a.in_t = pb->in_t; a.out_t = pb->out_t; a.logits_t = pb->logits_t;
   a.cplx = p.cplx;
@@ -167,8 +188,7 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &p, const int32_t *s,
     st = cuda_status(launch_empty_outputs(a, stream));
     return st != PDSSM_OK ? st : finish(pb, w, stream);
   }
-  const bool fused_chunk = pb->chunk == 0 || pb->chunk == 16;
-  if (!(pb->flags & PDSSM_FLAG_REFERENCE_PATH) && fused_chunk && fused_scan_supported(a)) {
+  if (p.fused) {
     // the fused kernel validates idx itself and needs no preimage lists
     st = cuda_status(launch_fused_scan(a, stream));
     return st != PDSSM_OK ? st : finish(pb, w, stream);
@@ -196,9 +216,10 @@ struct BwdPlan {
 
 pdssm_status make_bwd_plan(const pdssm_problem *pb, BwdPlan *bp) {
   Plan p;
-  pdssm_status st = make_plan(pb, &p);
+  pdssm_status st = make_plan(pb, &p, true);
   if (st != PDSSM_OK) return st;
   if (p.cplx) return PDSSM_ERR_UNSUPPORTED;
+  if (scan_bwd_smem_bytes(p.N, p.P, p.K) > (size_t)227 * 1024) return PDSSM_ERR_UNSUPPORTED;
   BwdPlan q;
   q.Bt = p.Bt; q.L = p.L; q.H = p.H; q.N = p.N; q.P = p.P; q.K = p.K; q.rows = p.rows;
   q.nCk = scan_bwd_checkpoints(p.L);
@@ -328,7 +349,7 @@ pdssm_status pdssm_scan_fwd(const pdssm_problem *pb, const int32_t *s, const int
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if ((st = bind_device(cs)) != PDSSM_OK) return st;
   return run_scan(pb, p, s, nullptr, nullptr, idx, d, B, C, x, h0, y, h_final, prod_idx, prod_val,
-                  workspace, cs);
+                  workspace, workspace_bytes, cs);
 }
 
 pdssm_status pdssm_forward(const pdssm_problem *pb, const void *logits, const int32_t *idx,
@@ -347,7 +368,7 @@ pdssm_status pdssm_forward(const pdssm_problem *pb, const void *logits, const in
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if ((st = bind_device(cs)) != PDSSM_OK) return st;
   return run_scan(pb, p, nullptr, logits, s_out, idx, d, B, C, x, h0, y, h_final, prod_idx,
-                  prod_val, workspace, cs);
+                  prod_val, workspace, workspace_bytes, cs);
 }
 
 pdssm_status pdssm_bwd_workspace_size(const pdssm_problem *pb, size_t *bytes) {
@@ -453,22 +474,26 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
 
-std::once_flag g_static_ws_once[kMaxDevices];
+std::mutex g_static_ws_mutex;
 void *g_static_ws_ptr[kMaxDevices] = {};
-cudaError_t g_static_ws_err[kMaxDevices] = {};
 
 // Device address of the static workspace on the current device. In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// with that device current and cached. Only a successful lookup is cached: a
+// call that fails (for instance inside a stream capture, where the lookup may
+// be refused) returns PDSSM_ERR_CUDA and the next call tries again.
 pdssm_status static_workspace(void **ptr) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PDSSM_ERR_CUDA;
-  std::call_once(g_static_ws_once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (!g_static_ws_ptr[dev]) {
     void *p = nullptr;
-    g_static_ws_err[dev] = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || !p) {
+      cudaGetLastError();  // the failure is reported by status; leave no sticky runtime error behind
+      return PDSSM_ERR_CUDA;
+    }
     g_static_ws_ptr[dev] = p;
-  });
-  if (g_static_ws_err[dev] != cudaSuccess || !g_static_ws_ptr[dev]) return PDSSM_ERR_CUDA;
+  }
   *ptr = g_static_ws_ptr[dev];
   return PDSSM_OK;
 }
@@ -494,5 +519,5 @@ extern "C" pdssm_status pdssm_forward_noalloc(const pdssm_problem *pb, const voi
                        kStaticWorkspaceBytes);
   if (st != PDSSM_OK) return st;
   return run_scan(pb, p, nullptr, logits, s_out, idx, d, B, C, x, h0, y, h_final, prod_idx,
-                  prod_val, ws, cs);
+                  prod_val, ws, kStaticWorkspaceBytes, cs);
 }

@@ -36,7 +36,11 @@ cudaError_t launch_prep_dict(const int32_t *idx, int K, int N, const Workspace &
 // The plain three-kernel chunked scan (phases A, B, C as separate launches).
 cudaError_t launch_chunked_scan(const ScanArgs &a, cudaStream_t st);
 // The fused single-kernel forward pass (real state, N = P = 64, bf16 d/B/C/x).
-bool fused_scan_supported(const ScanArgs &a);
+// fused_scan_applies decides from the problem alone (shape, dtypes, chunk,
+// flags); fused_scan_pointers_ok checks the 16-byte alignment its vector
+// loads need. The fused kernel needs no workspace beyond the error word.
+bool fused_scan_applies(const pdssm_problem *pb);
+bool fused_scan_pointers_ok(const ScanArgs &a);
 cudaError_t launch_fused_scan(const ScanArgs &a, cudaStream_t st);
 // Outputs of an empty sequence (L == 0): h_final = h0 (or 0), prod = identity.
 cudaError_t launch_empty_outputs(const ScanArgs &a, cudaStream_t st);

@@ -967,11 +967,16 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
 
 }  // namespace
 
-bool fused_scan_supported(const ScanArgs &s) {
-  if (s.cplx || s.N != kN || s.P != kP) return false;
-  if (s.d_t != PDSSM_BF16 || s.in_t != PDSSM_BF16) return false;
-  const int lsz = s.logits_t == PDSSM_BF16 ? 2 : 4;
-  if ((s.K * lsz) % 16 != 0) return false;
+bool fused_scan_applies(const pdssm_problem *pb) {
+  if (pb->flags & PDSSM_FLAG_REFERENCE_PATH) return false;
+  if (pb->chunk != 0 && pb->chunk != kT) return false;
+  if (pb->state_t != PDSSM_F32 || pb->N != kN || pb->P != kP) return false;
+  if (pb->d_t != PDSSM_BF16 || pb->in_t != PDSSM_BF16) return false;
+  const int lsz = pb->logits_t == PDSSM_BF16 ? 2 : 4;
+  return (pb->K * lsz) % 16 == 0;
+}
+
+bool fused_scan_pointers_ok(const ScanArgs &s) {
   if (!s.logits && !s.s) return false;
   auto al16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   return (!s.logits || al16(s.logits)) && al16(s.d) && al16(s.B) && al16(s.C) && al16(s.x);

@@ -18,3 +18,16 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Largest parity errors of the session (per-slice max-norm and elementwise relative)."""
+    try:
+        from tests.parity import REPORT
+    except Exception:
+        return
+    if not REPORT:
+        return
+    terminalreporter.write_sep("-", "largest parity errors against the oracle")
+    for (dtype, name), v in sorted(REPORT.items()):
+        terminalreporter.write_line(f"{dtype:>10}  {name:<22} {v:.3e}")

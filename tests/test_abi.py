@@ -121,6 +121,23 @@ def test_workspace_is_linear_in_length_and_never_quadratic_in_N():
     assert abs(b - 2 * a) < 2 * 4096
 
 
+def test_workspace_follows_the_path():
+    """The fused single-kernel path (real state, N = P = 64, bf16 d/B/C/x) needs only the
+    error word; the three-kernel path (any other problem, or the reference flag) needs its
+    chunk states and local outputs."""
+    lm = dict(batch=8, seqlen=2048, heads=32, N=64, P=64, K=16, logits_t=pd.BF16, in_t=pd.BF16,
+              d_t=pd.BF16, out_t=pd.BF16)
+    rc, fused = _ws(_pb(**lm))
+    assert rc == OK and fused == 256
+    assert _ws(_pb(**dict(lm, chunk=16))) == (OK, 256)
+    assert _ws(_pb(**dict(lm, out_t=pd.F32))) == (OK, 256)
+    rc, ref = _ws(_pb(**dict(lm, flags=pd.FLAG_REFERENCE_PATH)))
+    assert rc == OK and ref > 100 << 20
+    for kw in (dict(chunk=64), dict(K=5), dict(N=32), dict(P=32), dict(d_t=pd.F32), dict(in_t=pd.F32)):
+        rc, n = _ws(_pb(**dict(lm, **kw)))
+        assert rc == OK and n > 1 << 20, kw
+
+
 def _call_scan(pb, ws_bytes, **ptrs):
     null = None
     fake = ctypes.c_void_p(4096)  # never reaches a launch: every call below fails validation first

@@ -93,3 +93,23 @@ def test_backward_empty_sequence_passes_the_final_gradient_through(cuda_device):
                       z(Bt, 0, H, N), z(Bt, 0, H, P), z(Bt, 0, H, P), dh_final=dh)
     torch.cuda.synchronize(dev)
     assert torch.equal(out["dh0"], dh)
+
+
+@pytest.mark.parametrize("name", ["fsa_advance_merge_weighted"])
+def test_backward_reproduces_the_hand_worked_gradients(cuda_device, name):
+    """pdssm_scan_bwd on the weighted automaton fixture (loss sum_t y_t: dy = 1, no final-state
+    gradient, no logits): every gradient is a small integer worked by hand in the fixture header
+    and exact in fp32, so the C ABI must return it exactly."""
+    from tests import golden
+    inp, exp = golden.load(name)
+    g = {k: v.to(cuda_device) for k, v in inp.items()}
+    fwd = pd.forward(g["logits"], g["idx"], g["d"], g["B"], g["C"], g["x"], want_s=True, want_prod=False)
+    assert fwd["s"][0, :, 0].tolist() == exp["s"]
+    dy = torch.ones_like(fwd["y"])
+    out = pd.backward(None, fwd["s"], g["idx"], g["d"], g["B"], g["C"], g["x"], dy)
+    torch.cuda.synchronize()
+    assert out["dC"][0, :, 0].tolist() == exp["bwd_dC"]
+    assert out["dB"][0, :, 0].tolist() == exp["bwd_dB"]
+    assert out["dd"][0, :, 0].tolist() == exp["bwd_dd"]
+    assert out["dx"][0, :, 0, 0].tolist() == exp["bwd_dx"]
+    assert out["dh0"][0, 0, :, 0].tolist() == exp["bwd_dh0"]

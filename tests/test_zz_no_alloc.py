@@ -8,9 +8,11 @@ after call, because every call reuses the same array.
 This file is named to be collected last, so a run that stops at the first
 failure has run every other test before it.
 """
+import numpy as np
 import pytest
 import torch
 
+import oracle
 import structured_sparse_selective_b200 as pd
 import workloads
 from tests.parity import TOL, bhl_to_slices, slice_rel_err, to_np
@@ -36,7 +38,9 @@ def _outputs(sp, dev):
 ])
 def test_noalloc_matches_forward_on_consecutive_calls(cuda_device, recipe, kw):
     sp = workloads.spec(recipe, **kw)
-    inp = {k: v.to(cuda_device) for k, v in workloads.generate(sp, seed=21).items()}
+    host = workloads.generate(sp, seed=21)
+    inp = {k: v.to(cuda_device) for k, v in host.items()}
+    r = oracle.scan(host["logits"], host["idx"], host["d"], host["B"], host["C"], host["x"])
     pb = pd.make_problem(inp["logits"], inp["d"], inp["B"], inp["x"])
     ref = _outputs(sp, cuda_device)
     ws = pd.alloc_workspace(pb, cuda_device)
@@ -54,9 +58,16 @@ def test_noalloc_matches_forward_on_consecutive_calls(cuda_device, recipe, kw):
         assert slice_rel_err(bhl_to_slices(to_np(out["y"])), bhl_to_slices(to_np(ref["y"]))) <= TOL[sp.out_dtype]
         for k in ("h_final", "prod_val"):
             assert slice_rel_err(to_np(out[k]).reshape(S, -1), to_np(ref[k]).reshape(S, -1)) <= 1e-4, (call, k)
+        # and against the oracle itself
+        assert np.array_equal(to_np(out["s"]), r["s"]), call
+        assert np.array_equal(to_np(out["prod_idx"]), r["prod_idx"]), call
+        assert slice_rel_err(bhl_to_slices(to_np(out["y"])), bhl_to_slices(r["y"])) <= TOL[sp.out_dtype], call
+        for k in ("h_final", "prod_val"):
+            assert slice_rel_err(to_np(out[k]).reshape(S, -1), r[k].reshape(S, -1)) <= 1e-4, (call, k)
 
 
 def test_noalloc_rejects_problems_beyond_its_workspace(cuda_device):
+    """A three-kernel problem whose workspace exceeds the built-in array is refused before launch."""
     # real, full-size buffers: nothing here can make a kernel touch memory it does not own
     sp = workloads.spec("lm", batch=8, seqlen=2048, heads=8)
     g = torch.Generator(device=cuda_device).manual_seed(0)
@@ -68,10 +79,33 @@ def test_noalloc_rejects_problems_beyond_its_workspace(cuda_device):
         "C": torch.zeros(sp.batch, sp.seqlen, sp.heads, sp.N, dtype=torch.bfloat16, device=cuda_device),
         "x": torch.zeros(sp.batch, sp.seqlen, sp.heads, sp.P, dtype=torch.bfloat16, device=cuda_device),
     }
-    pb = pd.make_problem(inp["logits"], inp["d"], inp["B"], inp["x"])
+    # the three-kernel path needs far more than the built-in 32 MiB at this size
+    pb = pd.make_problem(inp["logits"], inp["d"], inp["B"], inp["x"], flags=pd.FLAG_REFERENCE_PATH)
     assert pd.pdssm_workspace_size(pb) > 32 << 20
     out = _outputs(sp, cuda_device)
     with pytest.raises(pd.PdssmError) as e:
         pd.pdssm_forward_noalloc(pb, inp["logits"], inp["idx"], inp["d"], inp["B"], inp["C"], inp["x"], None,
                                  out["y"], out["h_final"], out["prod_idx"], out["prod_val"], out["s"])
     assert e.value.status == 3  # PDSSM_ERR_WORKSPACE, before anything is enqueued
+
+
+def test_noalloc_serves_full_size_fused_problems(cuda_device):
+    """The fused kernel needs only the error word, so the full LM-layer problem (batch 8, L 2048,
+    heads 32) runs allocation-free; its outputs equal pdssm_forward's bit for bit (the fused
+    kernel is deterministic), call after call."""
+    sp = workloads.spec("lm")
+    inp = {k: v.to(cuda_device) for k, v in workloads.generate(sp, seed=5).items()}
+    pb = pd.make_problem(inp["logits"], inp["d"], inp["B"], inp["x"])
+    assert pd.pdssm_workspace_size(pb) <= 256
+    ref = _outputs(sp, cuda_device)
+    ws = pd.alloc_workspace(pb, cuda_device)
+    pd.pdssm_forward(pb, inp["logits"], inp["idx"], inp["d"], inp["B"], inp["C"], inp["x"], None, ref["y"],
+                     ref["h_final"], ref["prod_idx"], ref["prod_val"], ref["s"], ws)
+    torch.cuda.synchronize()
+    for call in range(2):
+        out = _outputs(sp, cuda_device)
+        pd.pdssm_forward_noalloc(pb, inp["logits"], inp["idx"], inp["d"], inp["B"], inp["C"], inp["x"], None,
+                                 out["y"], out["h_final"], out["prod_idx"], out["prod_val"], out["s"])
+        torch.cuda.synchronize()
+        for k in ref:
+            assert torch.equal(out[k], ref[k]), (call, k)
