@@ -44,12 +44,20 @@
 // of time) and four 16-column output slots. R = 3 for bf16 output; for fp32
 // output R = 2 and the third region holds S_lo.
 //
-// Roles (256 threads): warps 0-3 each prepare every fourth sub-chunk's
-// operands; warps 4-7 (one per tensor-memory quarter) advance the carry state
-// and write y, and one thread of warp 4 issues the MMAs. Every wait is
-// bounded; a timeout sets an error bit, makes every role leave its loop,
-// drains outstanding MMAs and copies, and frees tensor memory.
+// Roles (352 threads, 11 warps):
+//   warps 0-5   three prep pairs; pair w prepares sub-chunks w, w + 3, ... into
+//               operand stage (sub-chunk mod nst). In a pair, warp A (even)
+//               runs the suffix recursion Psi_sigma (B-hat scatter, and at its
+//               end Phi_{T-1}: the carry records and S_a's order); warp B (odd)
+//               runs the readout recursion R_sigma = A_{sigma+1}^T R_{sigma+1}
+//               (the G entries, and one step further, Ct = R_{-1}).
+//   warps 6-9   carry the state (one per tensor-memory lane quarter) and write y
+//               two sub-chunks behind the carry.
+//   warp 10     one thread issues the MMAs.
+// Every wait is bounded; a timeout sets an error bit, makes every role leave its
+// loop, drains outstanding MMAs and copies, and frees tensor memory.
 #include <algorithm>
+#include <climits>
 #include <type_traits>
 
 #include "launch.h"
@@ -64,13 +72,14 @@ namespace {
 constexpr int kN = 64;   // state rows
 constexpr int kP = 64;   // state columns
 constexpr int kT = 16;   // sub-chunk length
-constexpr int kNW = 4;   // prep warp pairs; pair w prepares sub-chunks w, w + 4, ...
+constexpr int kNW = 3;   // prep warp pairs; pair w prepares sub-chunks w, w + kNW, ...
 constexpr int kPrepWarps = 2 * kNW;
-constexpr int kCarryWarp0 = kPrepWarps;  // warps 8-11 carry the state (one per tensor-memory quarter)
-constexpr int kIssuerWarp = kCarryWarp0 + 4;  // warp 12: one thread issues the MMAs
+constexpr int kCarryWarp0 = kPrepWarps;  // warps 6-9 carry the state (one per tensor-memory quarter)
+constexpr int kIssuerWarp = kCarryWarp0 + 4;  // warp 10: one thread issues the MMAs
 constexpr int kMaxStages = 6;  // operand stages (sub-chunk a uses stage a mod nst, nst >= kNW)
 constexpr int kNY = 4;   // output accumulator slots
-constexpr int kThreads = 32 * (kPrepWarps + 5);  // 8 prep warps, 4 carry warps, 1 MMA-issuing warp
+constexpr int kYLag = 2;  // the carry step of sub-chunk a writes the output of sub-chunk a - kYLag
+constexpr int kThreads = 32 * (kPrepWarps + 5);  // 6 prep warps, 4 carry warps, 1 MMA-issuing warp
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
 
 // tensor-memory columns: 64-column state regions (a ring of 3, or 2 plus S_lo
@@ -107,17 +116,27 @@ __host__ __device__ constexpr int op_stage_bytes(bool precise) { return kOffCtLo
 constexpr int kMetaKeep = 1 << 8;
 constexpr int kMetaEnd = 1 << 9;
 constexpr int kMetaOrdShift = 10;
+constexpr int kOrdNone = 127;  // ordinal field of positions whose total another thread writes
 
-// per-prep-warp scratch (bytes)
-constexpr int kScrBins = 0;                   // int [2][N] fixed-point accumulators (by sigma parity)
-constexpr int kScrCnt = 512;                  // int [N] sources per target
-constexpr int kScrCntLo = 768;                // int [N] sources j < 32 per target
-constexpr int kScrOffs = 1024;                // int [N] first position of each target's group
-constexpr int kScrBytes = 1280;
+// per-pair scratch (bytes)
+constexpr int kRPitch = 80;                   // readout tile row: 16 fp32 columns + 16 bytes pad
+constexpr int kQPitch = 144;                  // partial-sum tile row (one per lane): 2 x 16 fp32 + pad
+constexpr int kScrR = 0;                      // float [N][20]: rows of R_sigma (warp B)
+constexpr int kScrQ = kScrR + kN * kRPitch;   // float [32][36]: per-lane partial G of two sigma (warp B)
+constexpr int kScrBins = kScrQ + 32 * kQPitch;  // int [2][N] fixed-point accumulators (warp A)
+constexpr int kScrCnt = kScrBins + 512;       // int [N] sources per target
+constexpr int kScrCntLo = kScrCnt + 256;      // int [N] sources j < 32 per target
+constexpr int kScrOffs = kScrCntLo + 256;     // int [N] first position of each target's group
+constexpr int kScrPsi = kScrOffs + 256;       // int [N] Psi_sigma index by source row
+constexpr int kScrW = kScrPsi + 256;          // float [N] Psi_sigma value by source row
+constexpr int kScrPosB = kScrW + 256;         // uint8 [N] position of row i in S_{a+1}'s order
+constexpr int kScrPosA = kScrPosB + 64;       // uint8 [N] position of row j in S_a's order
+constexpr int kScrSel = kScrPosA + 64;        // int [2T] selections of this and the next sub-chunk
+constexpr int kScrBytes = ((kScrSel + 4 * 2 * kT) + 127) & ~127;
 
-// input stage layout: logits [T][K] raw, d/B/C [T][N] bf16, x canonical
+// input stage layout: logits [T][K] raw (this and the next sub-chunk), d/B/C [T][N] bf16
 struct InLayout {
-  int logits, nlogits, d, B, C, x, bytes;  // nlogits: the next sub-chunk's logits
+  int logits, nlogits, d, B, C, bytes;
 };
 
 struct FParams {
@@ -217,22 +236,20 @@ __device__ __forceinline__ void st_bf16_split(uint8_t *hi, uint8_t *lo, int off,
 
 // ---------------------------------------------------------------- loads
 
-// cp.async of one sub-chunk's inputs (and the next sub-chunk's logits) into an
-// input stage by one warp; rows past the end of the sequence are zero-filled.
-template <typename TL>
+// cp.async of one sub-chunk's d, B, C and logits (and the next sub-chunk's
+// logits) into an input stage by one warp; rows past the end of the sequence
+// are zero-filled.
 __device__ __forceinline__ void load_inputs(const FParams &a, uint8_t *st, int64_t b, int64_t h, int sub,
                                             int lane) {
   const int t0 = sub * kT;
   const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
   const int nnext = (int)(a.L - t0 - kT < kT ? (a.L - t0 - kT > 0 ? a.L - t0 - kT : 0) : kT);
   const int64_t row0 = (b * a.L + t0) * a.H + h;  // row of token t0 in [Bt][L][H]
-  // d, B, C, x: 16 rows of 128 B (8 chunks of 16 B); lane takes chunk lane % 8 of
-  // rows lane / 8 + 4c, c = 0..3
+  // 16 rows of 128 B (8 chunks of 16 B); lane takes chunk lane % 8 of rows lane / 8 + 4c
   const int ch = lane & 7, tau0 = lane >> 3;
   const int64_t e0 = (row0 + (int64_t)tau0 * a.H) * kN + ch * 8;  // element offset of (tau0, ch)
   const int64_t estep = (int64_t)4 * a.H * kN;                    // 4 rows further
   const int so = tau0 * 128 + ch * 16;                            // row-major stage offset
-  const int sx = (tau0 & 7) * 16 + ch * 128;                      // x: (tau%8)*16 + (tau/8)*1024 + (p/8)*128
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     const int tau = tau0 + 4 * c;
@@ -240,18 +257,15 @@ __device__ __forceinline__ void load_inputs(const FParams &a, uint8_t *st, int64
     uint8_t *dd = st + a.in.d + so + c * 512;
     uint8_t *db = st + a.in.B + so + c * 512;
     uint8_t *dc = st + a.in.C + so + c * 512;
-    uint8_t *dx = st + a.in.x + sx + ((tau0 + 4 * c) >> 3) * 1024 + ((4 * c) & 7) * 16;
     if (tau < nvalid) {
       cp_async16(dd, a.d + ge);
       cp_async16(db, a.B + ge);
       cp_async16(dc, a.C + ge);
-      cp_async16(dx, a.x + ge);  // P == N
     } else {
       const uint4 z = make_uint4(0, 0, 0, 0);
       *reinterpret_cast<uint4 *>(dd) = z;
       *reinterpret_cast<uint4 *>(db) = z;
       *reinterpret_cast<uint4 *>(dc) = z;
-      *reinterpret_cast<uint4 *>(dx) = z;
     }
   }
   if (a.logits) {
@@ -271,29 +285,105 @@ __device__ __forceinline__ void load_inputs(const FParams &a, uint8_t *st, int64
   }
 }
 
-// Hard selection of one token from its logits row: the largest value, the lowest
-// k among ties, and the first NaN if there is one. Reads 16-byte chunks.
+// cp.async of one sub-chunk's x straight into its operand stage (bf16 MN-major,
+// mn = p, k = tau: (tau % 8) * 16 + (tau / 8) * 1024 + (p / 8) * 128 + (p % 8) * 2).
+__device__ __forceinline__ void load_x(const FParams &a, uint8_t *opx, int64_t b, int64_t h, int sub, int lane) {
+  const int t0 = sub * kT;
+  const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
+  const int64_t row0 = (b * a.L + t0) * a.H + h;
+  const int ch = lane & 7, tau0 = lane >> 3;
+  const int64_t e0 = (row0 + (int64_t)tau0 * a.H) * kP + ch * 8;
+  const int64_t estep = (int64_t)4 * a.H * kP;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int tau = tau0 + 4 * c;
+    uint8_t *dx = opx + (tau & 7) * 16 + (tau >> 3) * 1024 + ch * 128;
+    if (tau < nvalid)
+      cp_async16(dx, a.x + e0 + c * estep);
+    else
+      *reinterpret_cast<uint4 *>(dx) = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// (value, k) candidates of one logits row, merged so that the result is the
+// lowest k holding the maximum: a NaN beats every number and the lowest NaN
+// wins; +0 and -0 tie. k == INT_MAX marks "no candidate yet". The merge is
+// associative and commutative.
+__device__ __forceinline__ void sel_merge(float &v, int &k, float ov, int ok) {
+  const bool n = v != v, on = ov != ov;
+  bool take;
+  if (ok == INT_MAX)
+    take = false;
+  else if (k == INT_MAX)
+    take = true;
+  else if (n || on)
+    take = on && (!n || ok < k);
+  else
+    take = ov > v || (ov == v && ok < k);
+  if (take) {
+    v = ov;
+    k = ok;
+  }
+}
+
+// Hard selection of token lane / 2 of a stage's logits block: the two lanes of
+// a token each scan every other 16-byte chunk of its row, then merge.
 template <typename TL>
-__device__ __forceinline__ int argmax_row(const uint8_t *row, int K) {
+__device__ __forceinline__ int argmax_pair(const uint8_t *rows, int K, int lane) {
   constexpr int kPer = 16 / (int)sizeof(TL);
-  float best = 0.f;
-  int bi = 0, nan_at = -1;
-  for (int c = 0; c < K; c += kPer) {
-    const uint4 q = *reinterpret_cast<const uint4 *>(row + c * sizeof(TL));
+  const uint8_t *row = rows + (lane >> 1) * K * (int)sizeof(TL);
+  float bv = 0.f;
+  int bk = INT_MAX;
+  for (int c = lane & 1; c * kPer < K; c += 2) {
+    const uint4 q = *reinterpret_cast<const uint4 *>(row + c * 16);
     const TL *e = reinterpret_cast<const TL *>(&q);
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const float v = to_f32(e[u]);
-      const int k = c + u;
-      if (v != v && nan_at < 0) nan_at = k;
-      if (k == 0 || v > best) {
-        best = v;
-        bi = k;
-      }
-    }
+    for (int u = 0; u < kPer; ++u) sel_merge(bv, bk, to_f32(e[u]), c * kPer + u);
   }
-  return nan_at >= 0 ? nan_at : bi;
+  sel_merge(bv, bk, __shfl_xor_sync(0xffffffffu, bv, 1), __shfl_xor_sync(0xffffffffu, bk, 1));
+  return bk;
 }
+
+// packed fp32 pair arithmetic (one instruction for two lanes of data)
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<uint64_t *>(&a)),
+      "l"(*reinterpret_cast<uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&r);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(*reinterpret_cast<uint64_t *>(&a)),
+      "l"(*reinterpret_cast<uint64_t *>(&b)), "l"(*reinterpret_cast<uint64_t *>(&c)));
+  return *reinterpret_cast<float2 *>(&r);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<uint64_t *>(&a)),
+      "l"(*reinterpret_cast<uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&r);
+}
+// float4 = two float2 halves
+__device__ __forceinline__ float4 scale4(float4 v, float s) {
+  const float2 ss = make_float2(s, s);
+  const float2 lo = mul2(make_float2(v.x, v.y), ss), hi = mul2(make_float2(v.z, v.w), ss);
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+__device__ __forceinline__ float4 dot2_4(float b0, float4 g0, float b1, float4 g1) {  // b0 g0 + b1 g1
+  const float2 s0 = make_float2(b0, b0), s1 = make_float2(b1, b1);
+  const float2 lo = fma2(make_float2(g1.x, g1.y), s1, mul2(make_float2(g0.x, g0.y), s0));
+  const float2 hi = fma2(make_float2(g1.z, g1.w), s1, mul2(make_float2(g0.z, g0.w), s0));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+__device__ __forceinline__ float4 add4(float4 a, float4 b) {
+  const float2 lo = add2(make_float2(a.x, a.y), make_float2(b.x, b.y));
+  const float2 hi = add2(make_float2(a.z, a.w), make_float2(b.z, b.w));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+// bf16 pair (as loaded, element 0 in the low half) -> floats
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // Positions of the 64 sources j0 = lane, j1 = lane + 32 of an index map when the
 // sources are grouped by target row (targets ascending, sources ascending in a
@@ -346,7 +436,7 @@ __device__ __forceinline__ bool pair_and(uint32_t id, bool v) {
 // ------------------------------------------------------------- MMA issue
 
 // U_u into state region (u + 1) mod R and the intra-sub-chunk part of Y_u
-// (written, not accumulated). The region held S_{u+1-R}: this is issued only
+// (written, not accumulated). G is bf16 for bf16 output and hi + lo otherwise. The region held S_{u+1-R}: this is issued only
 // after the carry step of sub-chunk u+1-R is complete and its readout has been
 // issued (tensor-core operations of one thread execute in issue order).
 template <bool kPrecise>
@@ -360,7 +450,7 @@ __device__ __noinline__ void mma_issue_input(Bars *bars, uint32_t ob, int nst, u
   mma_bf16(dU, dX, smem_desc(o + kOffBhHi, kBhLbo, kBhSbo), kIdU, 0);
   mma_bf16(dU, dX, smem_desc(o + kOffBhLo, kBhLbo, kBhSbo), kIdU, 1);
   mma_bf16(dY, dX, smem_desc(o + kOffGtHi, 128, 256), kIdG, 0);
-  mma_bf16(dY, dX, smem_desc(o + kOffGtLo, 128, 256), kIdG, 1);
+  if constexpr (kPrecise) mma_bf16(dY, dX, smem_desc(o + kOffGtLo, 128, 256), kIdG, 1);
   mma_commit(&bars->ufull[(u + 1) % kRing]);
 }
 
@@ -441,115 +531,140 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
 
   if (warp < kPrepWarps) {
     // ================================================================ prep
-    // Warp pair w prepares sub-chunks w, w + kNW, ... (sub-chunk a into operand
-    // stage a mod nst). Role 0 loads the inputs and builds the composites, the
-    // forward chain (Ct), the carry records and the suffix scatter (Bh); role 1
-    // the backward readouts and G. Lanes own rows j0 = lane and j1 = lane + 32.
+    // Pair w prepares sub-chunks w, w + kNW, ... (sub-chunk a into operand stage
+    // a mod nst). Warp A (role 0) loads the inputs, composes the next sub-chunk's
+    // indices (S_{a+1}'s order), runs the suffix recursion
+    //   Psi_{sigma-1} = Psi_sigma A_sigma,  Bh_sigma = Psi_sigma B_sigma (scatter)
+    // whose end Psi_{-1} = Phi_{T-1} gives S_a's order and the carry records.
+    // Warp B (role 1) runs the readout recursion
+    //   R_sigma = A_{sigma+1}^T R_{sigma+1} with column sigma = C_sigma,
+    //   G[tau][sigma] = B_sigma . R_sigma[:, tau],
+    // and one step further R_{-1}[:, tau] = Phi_tau^T C_tau = Ct_tau.
     const int pair = warp >> 1, role = warp & 1;
     const uint32_t pbar = 1 + pair;
     uint8_t *in = in_base + pair * a.in.bytes;
     uint8_t *ws = scr + pair * kScrBytes;
-    int *bins = reinterpret_cast<int *>(ws + kScrBins);
+    int *sel = reinterpret_cast<int *>(ws + kScrSel);
+    uint8_t *posBt = ws + kScrPosB;
+    uint8_t *posAt = ws + kScrPosA;
     if (role == 0) {
+      int *bins = reinterpret_cast<int *>(ws + kScrBins);
 #pragma unroll
       for (int c = 0; c < 4; ++c) bins[lane + 32 * c] = 0;
     }
-    const int j0 = lane, j1 = lane + 32;
     for (int sub = pair; sub < nsub; sub += kNW) {
       const int stg = sub % a.nst;
       uint8_t *op = op_base + stg * kOpStage;
       const int t0 = sub * kT;
       const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
       const int nnext = (int)(a.L - t0 - kT < kT ? (a.L - t0 - kT > 0 ? a.L - t0 - kT : 0) : kT);
-      // the inputs load while the stage is being released
+      // the inputs load while the operand stage is being released
       if (role == 0) {
-        load_inputs<TL>(a, in, b, h, sub, lane);
+        load_inputs(a, in, b, h, sub, lane);
         cp_async_commit();
       }
-      bool ok = wait_bar_warp(bars, &bars->opfree[stg], ((sub / a.nst) & 1) ^ 1, a.err);
-      if (role == 0) cp_async_wait<0>();
+      const bool ok = wait_bar_warp(bars, &bars->opfree[stg], ((sub / a.nst) & 1) ^ 1, a.err);
+      if (role == 0) {
+        if (ok) load_x(a, op + kOffX, b, h, sub, lane);
+        cp_async_commit();
+        if (ok) cp_async_wait<1>(); else cp_async_wait<0>();
+      }
       // one decision for the pair; the barrier also publishes the loaded inputs
       if (!pair_and(pbar, ok)) break;
 
-      // selections: lanes 0-15 take this sub-chunk's tokens, lanes 16-31 the next one's
-      int s_lane = 0;
+      // selections, two lanes per token: warp B this sub-chunk's, warp A the next one's
       {
-        const int tok = lane & 15;
-        const bool nx = lane >= 16;
-        if (tok < (nx ? nnext : nvalid)) {
-          if (a.logits) {
-            s_lane = argmax_row<TL>(in + (nx ? a.in.nlogits : a.in.logits) + tok * a.K * a.logit_size, a.K);
-          } else {
-            s_lane = a.s_in[(b * a.L + t0 + (nx ? kT : 0) + tok) * a.H + h];
-            if (s_lane < 0 || s_lane >= a.K) {
-              flag_error(a.err, kErrSRange);
-              s_lane = 0;
-            }
+        const bool nx = role == 0;
+        const int tok = lane >> 1;
+        int s_tok = 0;
+        if (a.logits) {
+          s_tok = argmax_pair<TL>(in + (nx ? a.in.nlogits : a.in.logits), a.K, lane);
+        } else if (tok < (nx ? nnext : nvalid)) {
+          s_tok = a.s_in[(b * a.L + t0 + (nx ? kT : 0) + tok) * a.H + h];
+          if (s_tok < 0 || s_tok >= a.K) {
+            flag_error(a.err, kErrSRange);
+            s_tok = 0;
           }
-          if (role == 0 && !nx && a.s_out) a.s_out[(b * a.L + t0 + tok) * a.H + h] = s_lane;
+        }
+        if (tok >= (nx ? nnext : nvalid)) s_tok = 0;
+        if ((lane & 1) == 0) {
+          sel[(nx ? kT : 0) + tok] = s_tok;
+          if (!nx && a.s_out && tok < nvalid) a.s_out[(b * a.L + t0 + tok) * a.H + h] = s_tok;
         }
       }
-
+      pair_sync(pbar);
 
       const uint8_t *din = in + a.in.d, *Bin = in + a.in.B, *Cin = in + a.in.C;
       if (role == 0) {
-        // x into the operand stage (2 KB)
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          reinterpret_cast<uint4 *>(op + kOffX)[lane + 32 * c] = reinterpret_cast<const uint4 *>(in + a.in.x)[lane + 32 * c];
-
-        // ---- the next sub-chunk's composite (indices only) -> the order of S_{a+1}
-        int posB0, posB1;
+        const int j0 = lane, j1 = lane + 32;
+        int *bins = reinterpret_cast<int *>(ws + kScrBins);
+        int *psiT = reinterpret_cast<int *>(ws + kScrPsi);
+        float *WT = reinterpret_cast<float *>(ws + kScrW);
+        // ---- the next sub-chunk's composite (indices only) -> positions of S_{a+1}'s order
         {
           int n0 = j0, n1 = j1;
           for (int tau = 0; tau < nnext; ++tau) {
-            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, 16 + tau) * kN;
+            const uint8_t *dk = dict + sel[kT + tau] * kN;
             n0 = dk[n0];
             n1 = dk[n1];
           }
-          { const int2 pp = group_positions(n0, n1, ws, lane); posB0 = pp.x; posB1 = pp.y; }
+          const int2 pp = group_positions(n0, n1, ws, lane);
+          posBt[j0] = (uint8_t)pp.x;
+          posBt[j1] = (uint8_t)pp.y;
         }
+        // ---- suffix recursion: Bh_sigma = Psi_sigma B_sigma, summed as exact
+        //      fixed-point integers (order-independent) at the target's position in
+        //      S_{a+1}'s order; Psi over the steps past the end of the sequence is
+        //      the identity (their B rows were zero-filled)
+        int p0 = j0, p1 = j1;      // Psi_sigma(j): target row
+        float w0 = 1.f, w1 = 1.f;  // Psi_sigma(j): value
+        psiT[j0] = j0;
+        psiT[j1] = j1;
+        WT[j0] = 1.f;
+        WT[j1] = 1.f;
         __syncwarp();
-
-        // ---- Phi_{T-1} (indices): the positions of S_a's order
-        int posA0, posA1, i0 = j0, i1 = j1;
-        for (int tau = 0; tau < nvalid; ++tau) {
-          const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
-          i0 = dk[i0];
-          i1 = dk[i1];
-        }
-        { const int2 pp = group_positions(i0, i1, ws, lane); posA0 = pp.x; posA1 = pp.y; }
-        // ---- forward chain: Phi_tau and Ct_tau = Phi_tau^T C_tau at the positions of S_a's order
-        float v0 = 1.f, v1 = 1.f;
-        {
-          const int o0 = kOffCt + off_ct_pos(posA0), o1 = kOffCt + off_ct_pos(posA1);
-          int f0 = j0, f1 = j1;
 #pragma unroll 1
-          for (int tau = 0; tau < kT; ++tau) {
-            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, tau) * kN;
-            float c0 = 0.f, c1 = 0.f;
-            if (tau < nvalid) {
-              v0 *= ld_bf16(din, tau * kN + f0);
-              v1 *= ld_bf16(din, tau * kN + f1);
-              f0 = dk[f0];
-              f1 = dk[f1];
-              c0 = v0 * ld_bf16(Cin, tau * kN + f0);
-              c1 = v1 * ld_bf16(Cin, tau * kN + f1);
-            }
-            float *c0p = reinterpret_cast<float *>(op + o0 + off_ct_tau(tau));
-            float *c1p = reinterpret_cast<float *>(op + o1 + off_ct_tau(tau));
-            if constexpr (kPrecise) {  // hi as fp32 (read as tf32), lo = the rest
-              c0p[0] = c0;
-              c1p[0] = c1;
-              c0p[(kOffCtLo - kOffCt) / 4] = c0 - tf32_trunc(c0);
-              c1p[(kOffCtLo - kOffCt) / 4] = c1 - tf32_trunc(c1);
-            } else {
-              c0p[0] = tf32_rn(c0);
-              c1p[0] = tf32_rn(c1);
-            }
+        for (int sg = kT - 1; sg >= 0; --sg) {
+          int *bn = bins + (sg & 1) * kN;  // the other parity's accumulators are being cleared
+          const float v0 = w0 * ld_bf16(Bin, sg * kN + j0), v1 = w1 * ld_bf16(Bin, sg * kN + j1);
+          const unsigned mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(v0), fabsf(v1))));
+          // |v| < 2^ex; 64 terms of magnitude < 2^24 stay below 2^30
+          const int ex = (int)((mb >> 23) & 0xff) - 126;
+          const int e = mb ? 24 - ex : 0;
+          const float up = exp2i(e);
+          atomicAdd(&bn[posBt[p0]], __float2int_rn(v0 * up));
+          atomicAdd(&bn[posBt[p1]], __float2int_rn(v1 * up));
+          if (sg < nvalid) {
+            // Psi_{sg-1}(j) = Psi_sg(idx_sg[j]), value d_sg[j] * W_sg(idx_sg[j])
+            const uint8_t *dk = dict + sel[sg] * kN;
+            const int r0 = dk[j0], r1 = dk[j1];
+            const int np0 = psiT[r0], np1 = psiT[r1];
+            const float nw0 = WT[r0] * ld_bf16(din, sg * kN + j0), nw1 = WT[r1] * ld_bf16(din, sg * kN + j1);
+            __syncwarp();
+            psiT[j0] = np0;
+            psiT[j1] = np1;
+            WT[j0] = nw0;
+            WT[j1] = nw1;
+            p0 = np0;
+            p1 = np1;
+            w0 = nw0;
+            w1 = nw1;
           }
+          __syncwarp();
+          const float dn = exp2i(-e);
+          const float bh0 = (float)bn[j0] * dn, bh1 = (float)bn[j1] * dn;  // positions j0, j1
+          bn[j0] = 0;
+          bn[j1] = 0;
+          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(j0, sg), bh0);
+          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(j1, sg), bh1);
         }
-        // ---- Phi_{T-1} = (i, v): carry-step records
+        // ---- Psi_{-1} = Phi_{T-1} = (p, w): positions of S_a's order, carry records
+        const int i0 = p0, i1 = p1;
+        const float v0 = w0, v1 = w1;
+        const int2 pa = group_positions(i0, i1, ws, lane);
+        const int posA0 = pa.x, posA1 = pa.y;
+        posAt[j0] = (uint8_t)posA0;
+        posAt[j1] = (uint8_t)posA1;
         {
           const int *cnt = reinterpret_cast<const int *>(ws + kScrCnt);
           const int *offs = reinterpret_cast<const int *>(ws + kScrOffs);
@@ -567,21 +682,25 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           const int g0 = __shfl_sync(0xffffffffu, gex, i0 >> 1), h0 = __shfl_sync(0xffffffffu, na, i0 >> 1);
           const int g1 = __shfl_sync(0xffffffffu, gex, i1 >> 1), h1 = __shfl_sync(0xffffffffu, na, i1 >> 1);
           const int e0 = g0 + ((i0 & 1) ? h0 : 0), e1 = g1 + ((i1 & 1) ? h1 : 0);
-          // the target's column in the next order: posB of row i (held by lane i & 31)
-          const int pb0a = __shfl_sync(0xffffffffu, posB0, i0 & 31), pb0b = __shfl_sync(0xffffffffu, posB1, i0 & 31);
-          const int pb1a = __shfl_sync(0xffffffffu, posB0, i1 & 31), pb1b = __shfl_sync(0xffffffffu, posB1, i1 & 31);
           const int f0 = offs[i0], f1 = offs[i1];
           const bool keep0 = posA0 != f0, keep1 = posA1 != f1;
           const bool end0 = posA0 == f0 + cnt[i0] - 1, end1 = posA1 == f1 + cnt[i1] - 1;
+          // the group that continues across positions 31 | 32 (or -1): its positions
+          // below 32 carry ordinal kOrdNone, so that only the upper half's thread
+          // writes the group's total (the lower half's part is added by shuffle)
+          const int c32 = posA0 == 32 ? (keep0 ? e0 : -1) : (posA1 == 32 ? (keep1 ? e1 : -1) : -2);
+          const int ecross = __reduce_max_sync(0xffffffffu, c32);
+          const int o0 = (posA0 < 32 && e0 == ecross) ? kOrdNone : e0;
+          const int o1 = (posA1 < 32 && e1 == ecross) ? kOrdNone : e1;
           int *meta = reinterpret_cast<int *>(op + kOffMeta);
-          meta[posA0] = (keep0 ? kMetaKeep : 0) | (end0 ? kMetaEnd : 0) | (e0 << kMetaOrdShift);
-          meta[posA1] = (keep1 ? kMetaKeep : 0) | (end1 ? kMetaEnd : 0) | (e1 << kMetaOrdShift);
-          if (end0) op[kOffGDst + e0] = (uint8_t)(i0 < 32 ? pb0a : pb0b);
-          if (end1) op[kOffGDst + e1] = (uint8_t)(i1 < 32 ? pb1a : pb1b);
+          meta[posA0] = (keep0 ? kMetaKeep : 0) | (end0 ? kMetaEnd : 0) | (o0 << kMetaOrdShift);
+          meta[posA1] = (keep1 ? kMetaKeep : 0) | (end1 ? kMetaEnd : 0) | (o1 << kMetaOrdShift);
+          // the target's column in the next order
+          if (end0) op[kOffGDst + e0] = posBt[i0];
+          if (end1) op[kOffGDst + e1] = posBt[i1];
           int *hdr = reinterpret_cast<int *>(op + kOffHdr);
           if (lane == 0) hdr[0] = n_img;
-          if (posA0 == 32) hdr[1] = keep0 ? e0 : -1;
-          if (posA1 == 32) hdr[1] = keep1 ? e1 : -1;
+          if (lane == 0) hdr[1] = ecross;
           reinterpret_cast<float *>(op + kOffNu)[posA0] = v0;
           reinterpret_cast<float *>(op + kOffNu)[posA1] = v1;
           reinterpret_cast<int *>(op + kOffSrc)[posA0] = j0;
@@ -591,126 +710,117 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           reinterpret_cast<float *>(op + kOffPhiVal)[j0] = v0;
           reinterpret_cast<float *>(op + kOffPhiVal)[j1] = v1;
         }
-
-
-        // ---- backward: the suffix Psi_sigma and Bh_sigma = Psi_sigma B_sigma as an
-        //      exact fixed-point sum (integer adds are order-independent), written at
-        //      the target's position in S_{a+1}'s order. Steps past the end of the
-        //      sequence are the identity; their B rows were zero-filled.
-        int k0 = j0, k1 = j1;          // Psi_sigma
-        float m0 = 1.f, m1 = 1.f;
-#pragma unroll 1
-        for (int sg = kT - 1; sg >= 0; --sg) {
-          const bool sv = sg < nvalid;
-          const float bs0 = ld_bf16(Bin, sg * kN + j0), bs1 = ld_bf16(Bin, sg * kN + j1);
-          int *bn = bins + (sg & 1) * kN;  // the other parity's accumulators serve the next step
-          const float w0 = m0 * bs0, w1 = m1 * bs1;
-          const unsigned mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(w0), fabsf(w1))));
-          // |w| < 2^ex; 64 terms of magnitude < 2^24 stay below 2^30
-          const int ex = (int)((mb >> 23) & 0xff) - 126;
-          const int e = mb ? 24 - ex : 0;
-          const float up = exp2i(e), dn = exp2i(-e);
-          atomicAdd(&bn[k0], __float2int_rn(w0 * up));
-          atomicAdd(&bn[k1], __float2int_rn(w1 * up));
-          // Psi_{sg-1} = Psi_sg A_sg: column j <- d[j] * column idx[j]
-          {
-            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, sg) * kN;
-            const int r0 = sv ? dk[j0] : j0, r1 = sv ? dk[j1] : j1;
-            const float d0 = sv ? ld_bf16(din, sg * kN + j0) : 1.f, d1 = sv ? ld_bf16(din, sg * kN + j1) : 1.f;
-            const int ka = __shfl_sync(0xffffffffu, k0, r0 & 31), kb = __shfl_sync(0xffffffffu, k1, r0 & 31);
-            const float ma = __shfl_sync(0xffffffffu, m0, r0 & 31), mb2 = __shfl_sync(0xffffffffu, m1, r0 & 31);
-            const int kc = __shfl_sync(0xffffffffu, k0, r1 & 31), kd = __shfl_sync(0xffffffffu, k1, r1 & 31);
-            const float mc = __shfl_sync(0xffffffffu, m0, r1 & 31), md = __shfl_sync(0xffffffffu, m1, r1 & 31);
-            k0 = r0 < 32 ? ka : kb;
-            m0 = (r0 < 32 ? ma : mb2) * d0;
-            k1 = r1 < 32 ? kc : kd;
-            m1 = (r1 < 32 ? mc : md) * d1;
-          }
-          __syncwarp();
-          const float bh0 = (float)bn[j0] * dn, bh1 = (float)bn[j1] * dn;
-          bn[j0] = 0;
-          bn[j1] = 0;
-          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB0, sg), bh0);
-          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(posB1, sg), bh1);
-        }
+        pair_sync(pbar);  // S_a's order is published to warp B
+        cp_async_wait<0>();  // x has landed in the operand stage
       } else {
-        // ---- backward readouts R_sigma[j][tau] = (A_tau...A_{sigma+1})^T C_tau and
-        //      G[tau][sigma] = B_sigma . R_sigma[:, tau]. Columns tau < sigma are zero
-        //      and stay zero under the gathers; rows past the end of the sequence
-        //      were zero-filled, so their columns stay zero too.
+        // ---- readout recursion. Lane owns rows j0 = 2 lane, j1 = 2 lane + 1; a row of
+        //      R is 16 fp32 columns in the pair's tile, gathered whole (four 16-byte
+        //      chunks) by the row index of the next step's map. Columns tau < sigma of
+        //      R_sigma are zero; chunk c of R_sigma is written only for c >= sigma / 4.
+        //      Partial G of two consecutive sigma are reduced over the lanes together.
+        float *Rt = reinterpret_cast<float *>(ws + kScrR);
+        float *Qt = reinterpret_cast<float *>(ws + kScrQ);
+        const int j0 = 2 * lane, j1 = 2 * lane + 1;
         reinterpret_cast<uint4 *>(op + kOffGtHi)[lane] = make_uint4(0, 0, 0, 0);  // G^T above the diagonal
-        reinterpret_cast<uint4 *>(op + kOffGtHi)[lane + 32] = make_uint4(0, 0, 0, 0);
-        float R0[kT], R1[kT];
-#pragma unroll
-        for (int c = 0; c < kT; ++c) R0[c] = R1[c] = 0.f;
-        // lo_c: readout columns [lo, T) can be nonzero (sigma >= lo)
-        auto readout_step = [&](auto lo_c, int sg) {
-          constexpr int lo = decltype(lo_c)::value;
-          const float bs0 = ld_bf16(Bin, sg * kN + j0), bs1 = ld_bf16(Bin, sg * kN + j1);
-          // R_sg = A_{sg+1}^T R_{sg+1} on the columns tau > sg
-          {
-            const int sn = sg + 1 < kT ? sg + 1 : sg;
-            const uint8_t *dk = dict + __shfl_sync(0xffffffffu, s_lane, sn) * kN;
-            const int r0 = dk[j0], r1 = dk[j1];
-            const float d0 = ld_bf16(din, sn * kN + j0), d1 = ld_bf16(din, sn * kN + j1);
-#pragma unroll
-            for (int tau = lo + 1; tau < kT; ++tau) {
-              const float a0 = __shfl_sync(0xffffffffu, R0[tau], r0 & 31);
-              const float a1 = __shfl_sync(0xffffffffu, R1[tau], r0 & 31);
-              const float c0 = __shfl_sync(0xffffffffu, R0[tau], r1 & 31);
-              const float c1 = __shfl_sync(0xffffffffu, R1[tau], r1 & 31);
-              R0[tau] = d0 * (r0 < 32 ? a0 : a1);
-              R1[tau] = d1 * (r1 < 32 ? c0 : c1);
-            }
-          }
-          // R_sg[:, sg] = C_sg (sg is in [lo, lo + 8))
-          {
-            const float c0 = ld_bf16(Cin, sg * kN + j0), c1 = ld_bf16(Cin, sg * kN + j1);
-#pragma unroll
-            for (int tau = lo; tau < lo + 8; ++tau) {
-              R0[tau] = tau == sg ? c0 : R0[tau];
-              R1[tau] = tau == sg ? c1 : R1[tau];
-            }
-          }
-          // G[tau][sg] for tau in [8 * rnd, 8 * rnd + 8): partials, then a
-          // reduce-scatter of 8 values over 32 lanes
-#pragma unroll
-          for (int rnd = lo / 8; rnd < 2; ++rnd) {
-            float g[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) g[c] = bs0 * R0[8 * rnd + c] + bs1 * R1[8 * rnd + c];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const bool upr = lane & 16;
-              const float send = upr ? g[c] : g[c + 4];
-              const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-              g[c] = (upr ? g[c + 4] : g[c]) + recv;
-            }
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const bool upr = lane & 8;
-              const float send = upr ? g[c] : g[c + 2];
-              const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
-              g[c] = (upr ? g[c + 2] : g[c]) + recv;
-            }
-            {
-              const bool upr = lane & 4;
-              const float send = upr ? g[0] : g[1];
-              const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
-              g[0] = (upr ? g[1] : g[0]) + recv;
-            }
-            g[0] += __shfl_xor_sync(0xffffffffu, g[0], 2);
-            g[0] += __shfl_xor_sync(0xffffffffu, g[0], 1);
-            if ((lane & 3) == 0) {
-              const int tau = 8 * rnd + ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-              st_bf16_split(op + kOffGtHi, op + kOffGtLo, off_gt(tau, sg), g[0]);
-            }
-          }
-        };
+        if constexpr (kPrecise) reinterpret_cast<uint4 *>(op + kOffGtLo)[lane] = make_uint4(0, 0, 0, 0);
+        float4 g0[4], g1[4];
 #pragma unroll 1
-        for (int sg = kT - 1; sg >= 8; --sg) readout_step(std::integral_constant<int, 8>(), sg);
-#pragma unroll 1
-        for (int sg = 7; sg >= 0; --sg) readout_step(std::integral_constant<int, 0>(), sg);
+        for (int sg = kT - 1; sg >= -1; --sg) {
+          const int c0 = sg >= 0 ? sg >> 2 : 0;
+          // chunk c0 of R_{sg+1} was never written when sg is the last column of its chunk
+          const bool fresh = sg >= 0 && (sg & 3) == 3;
+          const bool have_next = sg < kT - 1;
+          float d0 = 0.f, d1 = 0.f;
+          int i0 = 0, i1 = 0;
+          if (have_next) {
+            const uint32_t ip = *reinterpret_cast<const uint16_t *>(dict + sel[sg + 1] * kN + j0);
+            i0 = ip & 0xff;
+            i1 = ip >> 8;
+            const uint32_t dp = *reinterpret_cast<const uint32_t *>(din + ((sg + 1) * kN + j0) * 2);
+            d0 = bf_lo(dp);
+            d1 = bf_hi(dp);
+          }
+          __syncwarp();  // the rows written by the previous step
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            if (have_next && (c > c0 || (c == c0 && !fresh))) {
+              g0[c] = scale4(*reinterpret_cast<const float4 *>(Rt + i0 * (kRPitch / 4) + 4 * c), d0);
+              g1[c] = scale4(*reinterpret_cast<const float4 *>(Rt + i1 * (kRPitch / 4) + 4 * c), d1);
+            } else {
+              g0[c] = g1[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+          }
+          __syncwarp();  // every gather of this step is done before rows are overwritten
+          if (sg < 0) break;  // g0, g1 hold rows j0, j1 of R_{-1} = Ct
+          const uint32_t bp = *reinterpret_cast<const uint32_t *>(Bin + (sg * kN + j0) * 2);
+          const uint32_t cp = *reinterpret_cast<const uint32_t *>(Cin + (sg * kN + j0) * 2);
+          const float b0 = bf_lo(bp), b1 = bf_hi(bp), cv0 = bf_lo(cp), cv1 = bf_hi(cp);
+          float *q = Qt + lane * (kQPitch / 4) + (sg & 1) * kT;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            if (c >= c0) {
+              *reinterpret_cast<float4 *>(Rt + j0 * (kRPitch / 4) + 4 * c) = g0[c];
+              *reinterpret_cast<float4 *>(Rt + j1 * (kRPitch / 4) + 4 * c) = g1[c];
+              *reinterpret_cast<float4 *>(q + 4 * c) = dot2_4(b0, g0[c], b1, g1[c]);
+            }
+          }
+          // column sigma: C_sigma (its gathered value is zero), and G's diagonal term
+          Rt[j0 * (kRPitch / 4) + sg] = cv0;
+          Rt[j1 * (kRPitch / 4) + sg] = cv1;
+          q[sg] = fmaf(b1, cv1, b0 * cv0);
+          if ((sg & 1) == 0) {
+            // G[tau][sigma] for sigma = sg + 1 (slot 1) and sg (slot 0): lane (rb, cc)
+            // sums chunk cc & 3 of slot cc >> 2 over lanes 8 rb .. 8 rb + 7, then the
+            // four rb groups are reduced by two butterfly exchanges
+            __syncwarp();
+            const int cc = lane & 7, rb = lane >> 3, slot = cc >> 2, c = cc & 3;
+            const float *qs = Qt + (8 * rb) * (kQPitch / 4) + slot * kT + 4 * c;
+            float4 acc = *reinterpret_cast<const float4 *>(qs);
+#pragma unroll
+            for (int i = 1; i < 8; ++i) acc = add4(acc, *reinterpret_cast<const float4 *>(qs + i * (kQPitch / 4)));
+            const bool b4 = lane & 16, b3 = lane & 8;
+            float k0 = b4 ? acc.z : acc.x, k1 = b4 ? acc.w : acc.y;
+            const float s0 = b4 ? acc.x : acc.z, s1 = b4 ? acc.y : acc.w;
+            k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+            k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+            float gv = b3 ? k1 : k0;
+            gv += __shfl_xor_sync(0xffffffffu, b3 ? k0 : k1, 8);
+            const int tau = 4 * c + (b4 ? 2 : 0) + (b3 ? 1 : 0);
+            const int sig = sg + slot;
+            if (tau >= sig) {
+              if constexpr (kPrecise) {
+                st_bf16_split(op + kOffGtHi, op + kOffGtLo, off_gt(tau, sig), gv);
+              } else {
+                *reinterpret_cast<__nv_bfloat16 *>(op + kOffGtHi + off_gt(tau, sig)) = __float2bfloat16_rn(gv);
+              }
+            }
+          }
+        }
+        // ---- Ct_tau = R_{-1}[:, tau], written at the source's position in S_a's order
+        pair_sync(pbar);  // warp A has published S_a's order
+        {
+          const int o0 = kOffCt + off_ct_pos(posAt[j0]), o1 = kOffCt + off_ct_pos(posAt[j1]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float r0[4] = {g0[c].x, g0[c].y, g0[c].z, g0[c].w};
+            const float r1[4] = {g1[c].x, g1[c].y, g1[c].z, g1[c].w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int tau = 4 * c + u;
+              float *c0p = reinterpret_cast<float *>(op + o0 + off_ct_tau(tau));
+              float *c1p = reinterpret_cast<float *>(op + o1 + off_ct_tau(tau));
+              if constexpr (kPrecise) {  // hi as fp32 (read as tf32), lo = the rest
+                c0p[0] = r0[u];
+                c1p[0] = r1[u];
+                c0p[(kOffCtLo - kOffCt) / 4] = r0[u] - tf32_trunc(r0[u]);
+                c1p[(kOffCtLo - kOffCt) / 4] = r1[u] - tf32_trunc(r1[u]);
+              } else {
+                c0p[0] = tf32_rn(r0[u]);
+                c1p[0] = tf32_rn(r1[u]);
+              }
+            }
+          }
+        }
       }
 
       fence_proxy_async_smem();
@@ -720,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       pair_sync(pbar);
     }
   } else if (warp < kIssuerWarp) {
-    // ============================================ carry state and output (warps 8-11)
+    // ============================================ carry state and output (warps 6-9)
     const int q = warp & 3;                 // tensor-memory quarter
     const bool act = lane < 16;
     const int p = 16 * q + lane;            // state column owned by this lane
@@ -767,15 +877,16 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       if (!__all_sync(0xffffffffu, ok)) break;
       const int st = sub % a.nst;
       const uint8_t *op = op_base + st * kOpStage;
+      const int ys = sub - kYLag;  // the sub-chunk whose output rides on this step
       if (!wait_bar_warp(bars, &bars->ufull[(sub + 1) % kRing], (sub / kRing) & 1, a.err)) break;
       if (!wait_bar_warp(bars, &bars->full[st], (sub / a.nst) & 1, a.err)) break;
-      if (sub > 0 && !wait_bar_warp(bars, &bars->yfull[(sub - 1) % kNY], ((sub - 1) / kNY) & 1, a.err)) break;
+      if (ys >= 0 && !wait_bar_warp(bars, &bars->yfull[ys % kNY], (ys / kNY) & 1, a.err)) break;
       tc_fence_after();
       const uint32_t RS = tbase + lanebase + col_state(sub % kRing);
       const uint32_t RU = tbase + lanebase + col_state((sub + 1) % kRing);
       const int4 *meta4 = reinterpret_cast<const int4 *>(op + kOffMeta);
       const float4 *nu4 = reinterpret_cast<const float4 *>(op + kOffNu);
-      // running whole-sequence product (warp 4 keeps it; sub-chunks arrive in order)
+      // running whole-sequence product (the quarter-0 carry warp keeps it; sub-chunks arrive in order)
       if (q == 0) {
         const int *pi = reinterpret_cast<const int *>(op + kOffPhiIdx);
         const float *pv = reinterpret_cast<const float *>(op + kOffPhiVal);
@@ -792,13 +903,11 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       // tensor-memory round trip.
       {
         const int hh = lane >> 4, pl = lane & 15;
-        float v[32];
-        tmem_ld_x2_32<32>(RS, v);
-        float yv[8];
-        if (sub > 0) tmem_ld_x2_8<8>(tbase + lanebase + kColY + ((sub - 1) % kNY) * kT, yv);
-        tmem_wait_ld();
-        if (sub > 0) {
-          const int tp = (sub - 1) * kT;
+        if (ys >= 0) {
+          float yv[8];
+          tmem_ld_x2_8<8>(tbase + lanebase + kColY + (ys % kNY) * kT, yv);
+          tmem_wait_ld();
+          const int tp = ys * kT;
           const int nv = (int)(a.L - tp < kT ? a.L - tp : kT);
           TO *yrow = yout + ((b * a.L + tp + 8 * hh) * a.H + h) * kP + 16 * q + pl;
           const int64_t ystep = a.H * kP;
@@ -807,44 +916,51 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
             if (8 * hh + i < nv) store_out(yrow + i * ystep, yv[i]);
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->yfree[(sub - 1) % kNY]);
+          if (lane == 0) mbar_arrive(&bars->yfree[ys % kNY]);
         }
         const int *hdr = reinterpret_cast<const int *>(op + kOffHdr);
         const int n_img = hdr[0], ecross = hdr[1];
-        // group totals go through this warp's 1 KB of the stage's Bh area (its MMA
-        // completed before ufull was signalled)
-        float *cs = reinterpret_cast<float *>(const_cast<uint8_t *>(op) + kOffBhHi) + q * 256;
+        // group totals go through this warp's 17 x 16 floats of the stage's Bh area
+        // (its MMA completed before ufull was signalled): rows 0-15 for the groups
+        // of this pass, row 16 absorbs the stores of every other position
+        float *cs = reinterpret_cast<float *>(const_cast<uint8_t *>(op) + kOffBhHi) + q * 17 * 16 + pl;
+#pragma unroll 1
         for (int base = 0; base < n_img; base += 16) {
+          // running sum over the group's positions, stored at every position into the
+          // group's row: the last store of a group, at its end, leaves its total
           float run = 0.f;
+#pragma unroll 1
+          for (int r = 0; r < 4; ++r) {
+            float v[8];
+            tmem_ld_x2_8<32>(RS + 8 * r, v);
+            const int4 ma = meta4[8 * hh + 2 * r], mb = meta4[8 * hh + 2 * r + 1];
+            const float4 na = nu4[8 * hh + 2 * r], nb = nu4[8 * hh + 2 * r + 1];
+            const int mt[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+            const float nu[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
+            tmem_wait_ld();
 #pragma unroll
-          for (int r4 = 0; r4 < 8; ++r4) {
-            const int4 m4 = meta4[8 * hh + r4];
-            const float4 n4 = nu4[8 * hh + r4];
-            const int mt[4] = {m4.x, m4.y, m4.z, m4.w};
-            const float nu[4] = {n4.x, n4.y, n4.z, n4.w};
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 8; ++c) {
               run = (mt[c] & kMetaKeep) ? run : 0.f;
-              run = fmaf(nu[c], v[4 * r4 + c], run);
+              run = fmaf(nu[c], v[c], run);
               const unsigned e = (unsigned)((mt[c] >> kMetaOrdShift) - base);
-              if ((mt[c] & kMetaEnd) && e < 16u) cs[e * 16 + pl] = run;
+              cs[(e < 16u ? e : 16u) * 16] = run;
             }
           }
           // the group that crosses positions 31 | 32 gets the lower half's part
           const float tail = __shfl_sync(0xffffffffu, run, pl);
           const unsigned ec = (unsigned)(ecross - base);
-          if (hh == 1 && ecross >= 0 && ec < 16u) cs[ec * 16 + pl] += tail;
           __syncwarp();
-          // U at the group ends += group totals, eight at a time
+          if (hh == 1 && ecross >= 0 && ec < 16u) cs[ec * 16] += tail;
+          __syncwarp();
+          // U at the group ends += group totals
+          const int ne = n_img - base < 16 ? n_img - base : 16;
 #pragma unroll 1
-          for (int e8 = base; e8 < base + 16 && e8 < n_img; e8 += 8) {
-            float u[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) tmem_ld1_if(RU + op[kOffGDst + e8 + e], u[e], e8 + e < n_img);
+          for (int e = 0; e < ne; ++e) {
+            const uint32_t col = RU + op[kOffGDst + base + e];
+            float u;
+            tmem_ld1(col, u);
             tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              tmem_st1_if(RU + op[kOffGDst + e8 + e], u[e] + cs[(e8 - base + e) * 16 + pl], e8 + e < n_img);
+            tmem_st1(col, u + cs[e * 16]);
           }
           __syncwarp();
         }
@@ -870,14 +986,16 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       }
       done = sub + 1;
     }
-    // output of the last sub-chunk
-    if (__all_sync(0xffffffffu, ok) && done == nsub && nsub > 0 &&
-        wait_bar_warp(bars, &bars->yfull[(nsub - 1) % kNY], ((nsub - 1) / kNY) & 1, a.err)) {
+    // outputs of the last kYLag sub-chunks
+    for (int ys = nsub - kYLag > 0 ? nsub - kYLag : 0; ys < nsub; ++ys) {
+      if (!(__all_sync(0xffffffffu, ok) && done == nsub &&
+            wait_bar_warp(bars, &bars->yfull[ys % kNY], (ys / kNY) & 1, a.err)))
+        break;
       tc_fence_after();
       float v[16];
-      tmem_ld16(tbase + lanebase + kColY + ((nsub - 1) % kNY) * kT, v);
+      tmem_ld16(tbase + lanebase + kColY + (ys % kNY) * kT, v);
       tmem_wait_ld();
-      store_y(nsub - 1, v);
+      store_y(ys, v);
     }
     const bool clean = !*(volatile int *)&bars->abort;
     if (q == 0 && clean) {
@@ -904,7 +1022,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     __syncwarp();
 
   } else if (lane == 0) {
-    // ============================================ MMA issue (warp 12, one thread)
+    // ============================================ MMA issue (warp 10, one thread)
     const uint32_t ob = smem_u32(op_base);
     auto issue_u_now = [&](int u) { mma_issue_input<kPrecise>(bars, ob, a.nst, tbase, u); };
     auto issue_y_now = [&](int s_) { mma_issue_readout<kPrecise>(bars, ob, a.nst, tbase, s_); };
@@ -967,13 +1085,47 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
 
 }  // namespace
 
+namespace {
+
+// Shared-memory plan of one CTA: as many operand stages as fit two CTAs per SM
+// (at least one per prep pair). Returns false when even that does not fit.
+constexpr int kTwoCtaBytes = 228 * 1024 / 2 - 1024;  // per-CTA share of an SM, less the reserved 1 KB
+bool plan_smem(int K, int logit_size, bool have_logits, bool precise, FParams *a, int *bytes) {
+  int o = 0;
+  a->in.logits = o; o += have_logits ? kT * K * logit_size : 0; o = (o + 127) & ~127;
+  a->in.nlogits = o; o += have_logits ? kT * K * logit_size : 0; o = (o + 127) & ~127;
+  a->in.d = o; o += kT * kN * 2;
+  a->in.B = o; o += kT * kN * 2;
+  a->in.C = o; o += kT * kN * 2;
+  a->in.bytes = (o + 127) & ~127;
+  for (a->nst = kMaxStages; a->nst >= kNW; --a->nst) {
+    int off = 0;
+    a->off_op = off; off += a->nst * op_stage_bytes(precise); off = (off + 1023) & ~1023;
+    a->off_in = off; off += kNW * a->in.bytes;
+    a->off_dict = off; off += (K * kN + 127) & ~127;
+    a->off_scr = off; off += kNW * kScrBytes;
+    off = (off + 127) & ~127;
+    a->off_bar = off; off += (int)sizeof(Bars);
+    if (off <= kTwoCtaBytes) {
+      *bytes = off;
+      return true;
+    }
+  }
+  return false;
+}
+
+}  // namespace
+
 bool fused_scan_applies(const pdssm_problem *pb) {
   if (pb->flags & PDSSM_FLAG_REFERENCE_PATH) return false;
   if (pb->chunk != 0 && pb->chunk != kT) return false;
   if (pb->state_t != PDSSM_F32 || pb->N != kN || pb->P != kP) return false;
   if (pb->d_t != PDSSM_BF16 || pb->in_t != PDSSM_BF16) return false;
   const int lsz = pb->logits_t == PDSSM_BF16 ? 2 : 4;
-  return (pb->K * lsz) % 16 == 0;
+  if ((pb->K * lsz) % 16 != 0) return false;
+  FParams a;
+  int bytes = 0;
+  return plan_smem((int)pb->K, lsz, true, pb->out_t != PDSSM_BF16, &a, &bytes);
 }
 
 bool fused_scan_pointers_ok(const ScanArgs &s) {
@@ -1003,31 +1155,9 @@ cudaError_t launch_fused_scan(const ScanArgs &s, cudaStream_t st) {
   a.prod_val = static_cast<float *>(s.prod_val);
   a.s_out = s.s_out;
   a.err = s.ws.err;
-  // input stage
-  int o = 0;
-  a.in.logits = o; o += s.logits ? kT * a.K * a.logit_size : 0; o = (o + 127) & ~127;
-  a.in.nlogits = o; o += s.logits ? kT * a.K * a.logit_size : 0; o = (o + 127) & ~127;
-  a.in.d = o; o += kT * kN * 2;
-  a.in.B = o; o += kT * kN * 2;
-  a.in.C = o; o += kT * kN * 2;
-  a.in.x = o; o += kT * kP * 2;
-  a.in.bytes = (o + 127) & ~127;
-  // smem
-  // As many operand stages as fit two CTAs per SM (at least one per prep warp).
   const bool precise = s.out_t != PDSSM_BF16;
-  constexpr int kTwoCtaBytes = 228 * 1024 / 2 - 1024;  // per-CTA share of an SM, less the reserved 1 KB
   int off = 0;
-  for (a.nst = kMaxStages; a.nst >= kNW; --a.nst) {
-    off = 0;
-    a.off_op = off; off += a.nst * op_stage_bytes(precise); off = (off + 1023) & ~1023;
-    a.off_in = off; off += kNW * a.in.bytes;
-    a.off_dict = off; off += (int)((s.K * kN + 127) & ~127);
-    a.off_scr = off; off += kNW * kScrBytes;
-    off = (off + 127) & ~127;
-    a.off_bar = off; off += (int)sizeof(Bars);
-    if (off <= kTwoCtaBytes) break;
-  }
-  if (a.nst < kNW) a.nst = kNW;  // the last layout computed (nst = kNW) is kept
+  if (!plan_smem(a.K, a.logit_size, s.logits != nullptr, precise, &a, &off)) return cudaErrorInvalidConfiguration;
 
   cudaError_t e;
   auto kern = (s.logits_t == PDSSM_BF16)
