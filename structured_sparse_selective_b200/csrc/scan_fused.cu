@@ -118,21 +118,22 @@ constexpr int kMetaEnd = 1 << 9;
 constexpr int kMetaOrdShift = 10;
 constexpr int kOrdNone = 127;  // ordinal field of positions whose total another thread writes
 
-// per-pair scratch (bytes)
-constexpr int kRPitch = 80;                   // readout tile row: 16 fp32 columns + 16 bytes pad
-constexpr int kQPitch = 144;                  // partial-sum tile row (one per lane): 2 x 16 fp32 + pad
-constexpr int kScrR = 0;                      // float [N][20]: rows of R_sigma (warp B)
-constexpr int kScrQ = kScrR + kN * kRPitch;   // float [32][36]: per-lane partial G of two sigma (warp B)
-constexpr int kScrBins = kScrQ + 32 * kQPitch;  // int [2][N] fixed-point accumulators (warp A)
-constexpr int kScrCnt = kScrBins + 512;       // int [N] sources per target
-constexpr int kScrCntLo = kScrCnt + 256;      // int [N] sources j < 32 per target
-constexpr int kScrOffs = kScrCntLo + 256;     // int [N] first position of each target's group
-constexpr int kScrPsi = kScrOffs + 256;       // int [N] Psi_sigma index by source row
-constexpr int kScrW = kScrPsi + 256;          // float [N] Psi_sigma value by source row
-constexpr int kScrPosB = kScrW + 256;         // uint8 [N] position of row i in S_{a+1}'s order
+// per-pair scratch (bytes); warp X = the pair's even warp, warp Y the odd one
+constexpr int kQBytes = 2 * kT * 32 * 4;      // float [2 slots][16 tau][32 lanes] partial G
+constexpr int kScrQX = 0;                     // partial G of warp X's walks
+constexpr int kScrQY = kScrQX + kQBytes;      // partial G of warp Y's walks
+constexpr int kScrBinsX = kScrQY + kQBytes;   // int [2][N] fixed-point accumulators of warp X
+constexpr int kScrBinsY = kScrBinsX + 512;    // int [2][N] of warp Y
+constexpr int kScrGrpX = kScrBinsY + 512;     // warp X's grouping scratch (counts, offsets: 768 B)
+constexpr int kScrGrpY = kScrGrpX + 768;      // warp Y's grouping scratch
+constexpr int kScrPosB = kScrGrpY + 768;      // uint8 [N] position of row i in S_{a+1}'s order
 constexpr int kScrPosA = kScrPosB + 64;       // uint8 [N] position of row j in S_a's order
 constexpr int kScrSel = kScrPosA + 64;        // int [2T] selections of this and the next sub-chunk
 constexpr int kScrBytes = ((kScrSel + 4 * 2 * kT) + 127) & ~127;
+// offsets inside a grouping scratch (group_positions)
+constexpr int kScrCnt = 0;                    // int [N] sources per target
+constexpr int kScrCntLo = 256;                // int [N] sources j < 32 per target
+constexpr int kScrOffs = 512;                 // int [N] first position of each target's group
 
 // input stage layout: logits [T][K] raw (this and the next sub-chunk), d/B/C [T][N] bf16
 struct InLayout {
@@ -232,6 +233,14 @@ __device__ __forceinline__ void st_bf16_split(uint8_t *hi, uint8_t *lo, int off,
   const __nv_bfloat16 h = __float2bfloat16_rn(v);
   *reinterpret_cast<__nv_bfloat16 *>(hi + off) = h;
   *reinterpret_cast<__nv_bfloat16 *>(lo + off) = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
+// two adjacent values as bf16 hi + lo pairs (one 4-byte store per part)
+__device__ __forceinline__ void st_bf16x2_split(uint8_t *hi, uint8_t *lo, int off, float v0, float v1) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+  const float2 hf = __bfloat1622float2(h);
+  *reinterpret_cast<__nv_bfloat162 *>(hi + off) = h;
+  *reinterpret_cast<__nv_bfloat162 *>(lo + off) = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
 }
 
 // ---------------------------------------------------------------- loads
@@ -532,14 +541,17 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
   if (warp < kPrepWarps) {
     // ================================================================ prep
     // Pair w prepares sub-chunks w, w + kNW, ... (sub-chunk a into operand stage
-    // a mod nst). Warp A (role 0) loads the inputs, composes the next sub-chunk's
-    // indices (S_{a+1}'s order), runs the suffix recursion
-    //   Psi_{sigma-1} = Psi_sigma A_sigma,  Bh_sigma = Psi_sigma B_sigma (scatter)
-    // whose end Psi_{-1} = Phi_{T-1} gives S_a's order and the carry records.
-    // Warp B (role 1) runs the readout recursion
-    //   R_sigma = A_{sigma+1}^T R_{sigma+1} with column sigma = C_sigma,
-    //   G[tau][sigma] = B_sigma . R_sigma[:, tau],
-    // and one step further R_{-1}[:, tau] = Phi_tau^T C_tau = Ct_tau.
+    // a mod nst). Both of its warps run "walkers": a walker (sigma, j) starts at
+    // row j just after step sigma and follows the row through the maps of the
+    // steps sigma + 1 ... (the last valid step), carrying the product of the d it
+    // passes times B_sigma[j]. On its way it meets C_tau at its current row, which
+    // is its part of G[tau][sigma] = C_tau^T A_tau...A_{sigma+1} B_sigma; at the end
+    // its row is Psi_sigma(j) and its value the part of Bh_sigma = Psi_sigma B_sigma
+    // that lands there. Walkers of sigma = -1 (no B) give Ct_tau = Phi_tau^T C_tau
+    // and, at the end, Phi_{T-1}: the carry records. Lanes own rows j and j + 32
+    // and walk two sigma at once (four independent walkers per lane).
+    //   warp X: S_{a+1}'s order, walks sigma = 0,1 | 4,5 | 8,9 | 12,13
+    //   warp Y: S_a's order, the sigma = -1 walk and the records, walks 2,3 | ... | 14,15
     const int pair = warp >> 1, role = warp & 1;
     const uint32_t pbar = 1 + pair;
     uint8_t *in = in_base + pair * a.in.bytes;
@@ -547,17 +559,19 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     int *sel = reinterpret_cast<int *>(ws + kScrSel);
     uint8_t *posBt = ws + kScrPosB;
     uint8_t *posAt = ws + kScrPosA;
-    if (role == 0) {
-      int *bins = reinterpret_cast<int *>(ws + kScrBins);
+    float *Qt = reinterpret_cast<float *>(ws + (role ? kScrQY : kScrQX));
+    int *bins = reinterpret_cast<int *>(ws + (role ? kScrBinsY : kScrBinsX));
+    uint8_t *grp = ws + (role ? kScrGrpY : kScrGrpX);
+    const int j0 = lane, j1 = lane + 32;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) bins[lane + 32 * c] = 0;
-    }
+    for (int c = 0; c < 4; ++c) bins[lane + 32 * c] = 0;
     for (int sub = pair; sub < nsub; sub += kNW) {
       const int stg = sub % a.nst;
       uint8_t *op = op_base + stg * kOpStage;
       const int t0 = sub * kT;
       const int nvalid = (int)(a.L - t0 < kT ? a.L - t0 : kT);
       const int nnext = (int)(a.L - t0 - kT < kT ? (a.L - t0 - kT > 0 ? a.L - t0 - kT : 0) : kT);
+      const int tend = nvalid - 1;  // last valid step of the sub-chunk
       // the inputs load while the operand stage is being released
       if (role == 0) {
         load_inputs(a, in, b, h, sub, lane);
@@ -565,14 +579,15 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       }
       const bool ok = wait_bar_warp(bars, &bars->opfree[stg], ((sub / a.nst) & 1) ^ 1, a.err);
       if (role == 0) {
-        if (ok) load_x(a, op + kOffX, b, h, sub, lane);
+        cp_async_wait<0>();
+      } else if (ok) {
+        load_x(a, op + kOffX, b, h, sub, lane);
         cp_async_commit();
-        if (ok) cp_async_wait<1>(); else cp_async_wait<0>();
       }
       // one decision for the pair; the barrier also publishes the loaded inputs
       if (!pair_and(pbar, ok)) break;
 
-      // selections, two lanes per token: warp B this sub-chunk's, warp A the next one's
+      // selections, two lanes per token: warp Y this sub-chunk's, warp X the next one's
       {
         const bool nx = role == 0;
         const int tok = lane >> 1;
@@ -595,79 +610,62 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
       pair_sync(pbar);
 
       const uint8_t *din = in + a.in.d, *Bin = in + a.in.B, *Cin = in + a.in.C;
-      if (role == 0) {
-        const int j0 = lane, j1 = lane + 32;
-        int *bins = reinterpret_cast<int *>(ws + kScrBins);
-        int *psiT = reinterpret_cast<int *>(ws + kScrPsi);
-        float *WT = reinterpret_cast<float *>(ws + kScrW);
-        // ---- the next sub-chunk's composite (indices only) -> positions of S_{a+1}'s order
-        {
-          int n0 = j0, n1 = j1;
-          for (int tau = 0; tau < nnext; ++tau) {
-            const uint8_t *dk = dict + sel[kT + tau] * kN;
-            n0 = dk[n0];
-            n1 = dk[n1];
-          }
-          const int2 pp = group_positions(n0, n1, ws, lane);
-          posBt[j0] = (uint8_t)pp.x;
-          posBt[j1] = (uint8_t)pp.y;
+      // ---- orders of the states: X the next sub-chunk's (S_{a+1}), Y this one's (S_a)
+      int phi0 = j0, phi1 = j1;  // warp Y: Phi_{T-1} indices
+      {
+        int n0 = j0, n1 = j1;
+        const int nsteps = role == 0 ? nnext : nvalid;
+        const int *ss = sel + (role == 0 ? kT : 0);
+        for (int tau = 0; tau < nsteps; ++tau) {
+          const uint8_t *dk = dict + ss[tau] * kN;
+          n0 = dk[n0];
+          n1 = dk[n1];
         }
-        // ---- suffix recursion: Bh_sigma = Psi_sigma B_sigma, summed as exact
-        //      fixed-point integers (order-independent) at the target's position in
-        //      S_{a+1}'s order; Psi over the steps past the end of the sequence is
-        //      the identity (their B rows were zero-filled)
-        int p0 = j0, p1 = j1;      // Psi_sigma(j): target row
-        float w0 = 1.f, w1 = 1.f;  // Psi_sigma(j): value
-        psiT[j0] = j0;
-        psiT[j1] = j1;
-        WT[j0] = 1.f;
-        WT[j1] = 1.f;
-        __syncwarp();
+        const int2 pp = group_positions(n0, n1, grp, lane);
+        uint8_t *pt = role == 0 ? posBt : posAt;
+        pt[j0] = (uint8_t)pp.x;
+        pt[j1] = (uint8_t)pp.y;
+        phi0 = n0;
+        phi1 = n1;
+        if (role == 0) {  // G^T above the diagonal stays zero
+          reinterpret_cast<uint4 *>(op + kOffGtHi)[lane] = make_uint4(0, 0, 0, 0);
+          if constexpr (kPrecise) reinterpret_cast<uint4 *>(op + kOffGtLo)[lane] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      pair_sync(pbar);  // both orders are published
+
+      if (role == 1) {
+        // ---- the sigma = -1 walk: Ct_tau at the source's position in S_a's order,
+        //      then Phi_{T-1} = (row, value) and the carry records
+        const int posA0 = posAt[j0], posA1 = posAt[j1];
+        const int o0 = kOffCt + off_ct_pos(posA0), o1 = kOffCt + off_ct_pos(posA1);
+        int r0 = j0, r1 = j1;
+        float v0 = 1.f, v1 = 1.f;
 #pragma unroll 1
-        for (int sg = kT - 1; sg >= 0; --sg) {
-          int *bn = bins + (sg & 1) * kN;  // the other parity's accumulators are being cleared
-          const float v0 = w0 * ld_bf16(Bin, sg * kN + j0), v1 = w1 * ld_bf16(Bin, sg * kN + j1);
-          const unsigned mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(v0), fabsf(v1))));
-          // |v| < 2^ex; 64 terms of magnitude < 2^24 stay below 2^30
-          const int ex = (int)((mb >> 23) & 0xff) - 126;
-          const int e = mb ? 24 - ex : 0;
-          const float up = exp2i(e);
-          atomicAdd(&bn[posBt[p0]], __float2int_rn(v0 * up));
-          atomicAdd(&bn[posBt[p1]], __float2int_rn(v1 * up));
-          if (sg < nvalid) {
-            // Psi_{sg-1}(j) = Psi_sg(idx_sg[j]), value d_sg[j] * W_sg(idx_sg[j])
-            const uint8_t *dk = dict + sel[sg] * kN;
-            const int r0 = dk[j0], r1 = dk[j1];
-            const int np0 = psiT[r0], np1 = psiT[r1];
-            const float nw0 = WT[r0] * ld_bf16(din, sg * kN + j0), nw1 = WT[r1] * ld_bf16(din, sg * kN + j1);
-            __syncwarp();
-            psiT[j0] = np0;
-            psiT[j1] = np1;
-            WT[j0] = nw0;
-            WT[j1] = nw1;
-            p0 = np0;
-            p1 = np1;
-            w0 = nw0;
-            w1 = nw1;
+        for (int tau = 0; tau <= tend; ++tau) {
+          const uint8_t *dk = dict + sel[tau] * kN;
+          v0 *= ld_bf16(din, tau * kN + r0);
+          v1 *= ld_bf16(din, tau * kN + r1);
+          r0 = dk[r0];
+          r1 = dk[r1];
+          const float c0 = v0 * ld_bf16(Cin, tau * kN + r0), c1 = v1 * ld_bf16(Cin, tau * kN + r1);
+          float *c0p = reinterpret_cast<float *>(op + o0 + off_ct_tau(tau));
+          float *c1p = reinterpret_cast<float *>(op + o1 + off_ct_tau(tau));
+          if constexpr (kPrecise) {  // hi as fp32 (read as tf32), lo = the rest
+            c0p[0] = c0;
+            c1p[0] = c1;
+            c0p[(kOffCtLo - kOffCt) / 4] = c0 - tf32_trunc(c0);
+            c1p[(kOffCtLo - kOffCt) / 4] = c1 - tf32_trunc(c1);
+          } else {
+            c0p[0] = tf32_rn(c0);
+            c1p[0] = tf32_rn(c1);
           }
-          __syncwarp();
-          const float dn = exp2i(-e);
-          const float bh0 = (float)bn[j0] * dn, bh1 = (float)bn[j1] * dn;  // positions j0, j1
-          bn[j0] = 0;
-          bn[j1] = 0;
-          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(j0, sg), bh0);
-          st_bf16_split(op + kOffBhHi, op + kOffBhLo, off_bh(j1, sg), bh1);
         }
-        // ---- Psi_{-1} = Phi_{T-1} = (p, w): positions of S_a's order, carry records
-        const int i0 = p0, i1 = p1;
-        const float v0 = w0, v1 = w1;
-        const int2 pa = group_positions(i0, i1, ws, lane);
-        const int posA0 = pa.x, posA1 = pa.y;
-        posAt[j0] = (uint8_t)posA0;
-        posAt[j1] = (uint8_t)posA1;
+        // records of Phi_{T-1} = (i, v) for the carry step
+        const int i0 = phi0, i1 = phi1;
         {
-          const int *cnt = reinterpret_cast<const int *>(ws + kScrCnt);
-          const int *offs = reinterpret_cast<const int *>(ws + kScrOffs);
+          const int *cnt = reinterpret_cast<const int *>(grp + kScrCnt);
+          const int *offs = reinterpret_cast<const int *>(grp + kScrOffs);
           // ordinal of each nonempty target group (targets ascending): target t's is
           // the exclusive count of nonempty targets below t
           const int na = cnt[2 * lane] > 0, nb = cnt[2 * lane + 1] > 0;
@@ -690,17 +688,19 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           // writes the group's total (the lower half's part is added by shuffle)
           const int c32 = posA0 == 32 ? (keep0 ? e0 : -1) : (posA1 == 32 ? (keep1 ? e1 : -1) : -2);
           const int ecross = __reduce_max_sync(0xffffffffu, c32);
-          const int o0 = (posA0 < 32 && e0 == ecross) ? kOrdNone : e0;
-          const int o1 = (posA1 < 32 && e1 == ecross) ? kOrdNone : e1;
+          const int q0 = (posA0 < 32 && e0 == ecross) ? kOrdNone : e0;
+          const int q1 = (posA1 < 32 && e1 == ecross) ? kOrdNone : e1;
           int *meta = reinterpret_cast<int *>(op + kOffMeta);
-          meta[posA0] = (keep0 ? kMetaKeep : 0) | (end0 ? kMetaEnd : 0) | (o0 << kMetaOrdShift);
-          meta[posA1] = (keep1 ? kMetaKeep : 0) | (end1 ? kMetaEnd : 0) | (o1 << kMetaOrdShift);
+          meta[posA0] = (keep0 ? kMetaKeep : 0) | (end0 ? kMetaEnd : 0) | (q0 << kMetaOrdShift);
+          meta[posA1] = (keep1 ? kMetaKeep : 0) | (end1 ? kMetaEnd : 0) | (q1 << kMetaOrdShift);
           // the target's column in the next order
           if (end0) op[kOffGDst + e0] = posBt[i0];
           if (end1) op[kOffGDst + e1] = posBt[i1];
           int *hdr = reinterpret_cast<int *>(op + kOffHdr);
-          if (lane == 0) hdr[0] = n_img;
-          if (lane == 0) hdr[1] = ecross;
+          if (lane == 0) {
+            hdr[0] = n_img;
+            hdr[1] = ecross;
+          }
           reinterpret_cast<float *>(op + kOffNu)[posA0] = v0;
           reinterpret_cast<float *>(op + kOffNu)[posA1] = v1;
           reinterpret_cast<int *>(op + kOffSrc)[posA0] = j0;
@@ -710,118 +710,89 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           reinterpret_cast<float *>(op + kOffPhiVal)[j0] = v0;
           reinterpret_cast<float *>(op + kOffPhiVal)[j1] = v1;
         }
-        pair_sync(pbar);  // S_a's order is published to warp B
-        cp_async_wait<0>();  // x has landed in the operand stage
-      } else {
-        // ---- readout recursion. Lane owns rows j0 = 2 lane, j1 = 2 lane + 1; a row of
-        //      R is 16 fp32 columns in the pair's tile, gathered whole (four 16-byte
-        //      chunks) by the row index of the next step's map. Columns tau < sigma of
-        //      R_sigma are zero; chunk c of R_sigma is written only for c >= sigma / 4.
-        //      Partial G of two consecutive sigma are reduced over the lanes together.
-        float *Rt = reinterpret_cast<float *>(ws + kScrR);
-        float *Qt = reinterpret_cast<float *>(ws + kScrQ);
-        const int j0 = 2 * lane, j1 = 2 * lane + 1;
-        reinterpret_cast<uint4 *>(op + kOffGtHi)[lane] = make_uint4(0, 0, 0, 0);  // G^T above the diagonal
-        if constexpr (kPrecise) reinterpret_cast<uint4 *>(op + kOffGtLo)[lane] = make_uint4(0, 0, 0, 0);
-        float4 g0[4], g1[4];
-#pragma unroll 1
-        for (int sg = kT - 1; sg >= -1; --sg) {
-          const int c0 = sg >= 0 ? sg >> 2 : 0;
-          // chunk c0 of R_{sg+1} was never written when sg is the last column of its chunk
-          const bool fresh = sg >= 0 && (sg & 3) == 3;
-          const bool have_next = sg < kT - 1;
-          float d0 = 0.f, d1 = 0.f;
-          int i0 = 0, i1 = 0;
-          if (have_next) {
-            const uint32_t ip = *reinterpret_cast<const uint16_t *>(dict + sel[sg + 1] * kN + j0);
-            i0 = ip & 0xff;
-            i1 = ip >> 8;
-            const uint32_t dp = *reinterpret_cast<const uint32_t *>(din + ((sg + 1) * kN + j0) * 2);
-            d0 = bf_lo(dp);
-            d1 = bf_hi(dp);
-          }
-          __syncwarp();  // the rows written by the previous step
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (have_next && (c > c0 || (c == c0 && !fresh))) {
-              g0[c] = scale4(*reinterpret_cast<const float4 *>(Rt + i0 * (kRPitch / 4) + 4 * c), d0);
-              g1[c] = scale4(*reinterpret_cast<const float4 *>(Rt + i1 * (kRPitch / 4) + 4 * c), d1);
-            } else {
-              g0[c] = g1[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-          }
-          __syncwarp();  // every gather of this step is done before rows are overwritten
-          if (sg < 0) break;  // g0, g1 hold rows j0, j1 of R_{-1} = Ct
-          const uint32_t bp = *reinterpret_cast<const uint32_t *>(Bin + (sg * kN + j0) * 2);
-          const uint32_t cp = *reinterpret_cast<const uint32_t *>(Cin + (sg * kN + j0) * 2);
-          const float b0 = bf_lo(bp), b1 = bf_hi(bp), cv0 = bf_lo(cp), cv1 = bf_hi(cp);
-          float *q = Qt + lane * (kQPitch / 4) + (sg & 1) * kT;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (c >= c0) {
-              *reinterpret_cast<float4 *>(Rt + j0 * (kRPitch / 4) + 4 * c) = g0[c];
-              *reinterpret_cast<float4 *>(Rt + j1 * (kRPitch / 4) + 4 * c) = g1[c];
-              *reinterpret_cast<float4 *>(q + 4 * c) = dot2_4(b0, g0[c], b1, g1[c]);
-            }
-          }
-          // column sigma: C_sigma (its gathered value is zero), and G's diagonal term
-          Rt[j0 * (kRPitch / 4) + sg] = cv0;
-          Rt[j1 * (kRPitch / 4) + sg] = cv1;
-          q[sg] = fmaf(b1, cv1, b0 * cv0);
-          if ((sg & 1) == 0) {
-            // G[tau][sigma] for sigma = sg + 1 (slot 1) and sg (slot 0): lane (rb, cc)
-            // sums chunk cc & 3 of slot cc >> 2 over lanes 8 rb .. 8 rb + 7, then the
-            // four rb groups are reduced by two butterfly exchanges
-            __syncwarp();
-            const int cc = lane & 7, rb = lane >> 3, slot = cc >> 2, c = cc & 3;
-            const float *qs = Qt + (8 * rb) * (kQPitch / 4) + slot * kT + 4 * c;
-            float4 acc = *reinterpret_cast<const float4 *>(qs);
-#pragma unroll
-            for (int i = 1; i < 8; ++i) acc = add4(acc, *reinterpret_cast<const float4 *>(qs + i * (kQPitch / 4)));
-            const bool b4 = lane & 16, b3 = lane & 8;
-            float k0 = b4 ? acc.z : acc.x, k1 = b4 ? acc.w : acc.y;
-            const float s0 = b4 ? acc.x : acc.z, s1 = b4 ? acc.y : acc.w;
-            k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
-            k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-            float gv = b3 ? k1 : k0;
-            gv += __shfl_xor_sync(0xffffffffu, b3 ? k0 : k1, 8);
-            const int tau = 4 * c + (b4 ? 2 : 0) + (b3 ? 1 : 0);
-            const int sig = sg + slot;
-            if (tau >= sig) {
-              if constexpr (kPrecise) {
-                st_bf16_split(op + kOffGtHi, op + kOffGtLo, off_gt(tau, sig), gv);
-              } else {
-                *reinterpret_cast<__nv_bfloat16 *>(op + kOffGtHi + off_gt(tau, sig)) = __float2bfloat16_rn(gv);
-              }
-            }
-          }
-        }
-        // ---- Ct_tau = R_{-1}[:, tau], written at the source's position in S_a's order
-        pair_sync(pbar);  // warp A has published S_a's order
-        {
-          const int o0 = kOffCt + off_ct_pos(posAt[j0]), o1 = kOffCt + off_ct_pos(posAt[j1]);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const float r0[4] = {g0[c].x, g0[c].y, g0[c].z, g0[c].w};
-            const float r1[4] = {g1[c].x, g1[c].y, g1[c].z, g1[c].w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int tau = 4 * c + u;
-              float *c0p = reinterpret_cast<float *>(op + o0 + off_ct_tau(tau));
-              float *c1p = reinterpret_cast<float *>(op + o1 + off_ct_tau(tau));
-              if constexpr (kPrecise) {  // hi as fp32 (read as tf32), lo = the rest
-                c0p[0] = r0[u];
-                c1p[0] = r1[u];
-                c0p[(kOffCtLo - kOffCt) / 4] = r0[u] - tf32_trunc(r0[u]);
-                c1p[(kOffCtLo - kOffCt) / 4] = r1[u] - tf32_trunc(r1[u]);
-              } else {
-                c0p[0] = tf32_rn(r0[u]);
-                c1p[0] = tf32_rn(r1[u]);
-              }
-            }
-          }
-        }
       }
+
+      // ---- walks of the sigma pairs (sa, sa + 1): warp X takes sa = 0, 4, 6, 8 and
+      //      warp Y (which also ran the sigma = -1 walk) sa = 2, 10, 12, 14; a pair
+      //      (sa, sa + 1) takes 14 - sa joint steps
+#pragma unroll 1
+      for (int m = 0; m < 4; ++m) {
+        const int sa = role ? (m == 0 ? 2 : 8 + 2 * m) : (m == 0 ? 0 : 2 + 2 * m), sb = sa + 1;
+        float *q = Qt + lane;  // element (slot, tau) of this lane at q[(slot * kT + tau) * 32]
+        // B of both starts at the lane's rows, and G's diagonal terms
+        const float ba0 = ld_bf16(Bin, sa * kN + j0), ba1 = ld_bf16(Bin, sa * kN + j1);
+        const float bb0 = ld_bf16(Bin, sb * kN + j0), bb1 = ld_bf16(Bin, sb * kN + j1);
+        q[sa * 32] = fmaf(ba1, ld_bf16(Cin, sa * kN + j1), ba0 * ld_bf16(Cin, sa * kN + j0));
+        q[(kT + sb) * 32] = fmaf(bb1, ld_bf16(Cin, sb * kN + j1), bb0 * ld_bf16(Cin, sb * kN + j0));
+        int ra0 = j0, ra1 = j1, rb0 = j0, rb1 = j1;
+        float wa0 = ba0, wa1 = ba1, wb0 = bb0, wb1 = bb1;
+        if (sb <= tend) {  // walker a's first step (sb): b starts after it
+          const uint8_t *dk = dict + sel[sb] * kN;
+          wa0 *= ld_bf16(din, sb * kN + ra0);
+          wa1 *= ld_bf16(din, sb * kN + ra1);
+          ra0 = dk[ra0];
+          ra1 = dk[ra1];
+          q[sb * 32] = fmaf(wa1, ld_bf16(Cin, sb * kN + ra1), wa0 * ld_bf16(Cin, sb * kN + ra0));
+        }
+#pragma unroll 1
+        for (int tau = sb + 1; tau <= tend; ++tau) {
+          const uint8_t *dk = dict + sel[tau] * kN;
+          const uint8_t *dr = din + tau * kN * 2, *cr = Cin + tau * kN * 2;
+          wa0 *= ld_bf16(dr, ra0);
+          wa1 *= ld_bf16(dr, ra1);
+          wb0 *= ld_bf16(dr, rb0);
+          wb1 *= ld_bf16(dr, rb1);
+          ra0 = dk[ra0];
+          ra1 = dk[ra1];
+          rb0 = dk[rb0];
+          rb1 = dk[rb1];
+          q[tau * 32] = fmaf(wa1, ld_bf16(cr, ra1), wa0 * ld_bf16(cr, ra0));
+          q[(kT + tau) * 32] = fmaf(wb1, ld_bf16(cr, rb1), wb0 * ld_bf16(cr, rb0));
+        }
+        // Bh_sa and Bh_sb: the walkers' values summed as exact fixed-point integers
+        // (order-independent) at their rows' positions in S_{a+1}'s order
+        int *bna = bins, *bnb = bins + kN;
+        const unsigned mxa = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(wa0), fabsf(wa1))));
+        const unsigned mxb = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(wb0), fabsf(wb1))));
+        // |w| < 2^ex; 64 terms of magnitude < 2^24 stay below 2^30
+        const int ea = mxa ? 24 - ((int)((mxa >> 23) & 0xff) - 126) : 0;
+        const int eb = mxb ? 24 - ((int)((mxb >> 23) & 0xff) - 126) : 0;
+        const float upa = exp2i(ea), upb = exp2i(eb);
+        atomicAdd(&bna[posBt[ra0]], __float2int_rn(wa0 * upa));
+        atomicAdd(&bna[posBt[ra1]], __float2int_rn(wa1 * upa));
+        atomicAdd(&bnb[posBt[rb0]], __float2int_rn(wb0 * upb));
+        atomicAdd(&bnb[posBt[rb1]], __float2int_rn(wb1 * upb));
+        __syncwarp();  // the walks' partial G and the scatter are complete
+        {
+          // Bh at positions 2 lane and 2 lane + 1 (adjacent in the operand: one
+          // packed store per part)
+          const float dna = exp2i(-ea), dnb = exp2i(-eb);
+          const int2 ia = reinterpret_cast<const int2 *>(bna)[lane], ib = reinterpret_cast<const int2 *>(bnb)[lane];
+          reinterpret_cast<int2 *>(bna)[lane] = make_int2(0, 0);
+          reinterpret_cast<int2 *>(bnb)[lane] = make_int2(0, 0);
+          st_bf16x2_split(op + kOffBhHi, op + kOffBhLo, off_bh(2 * lane, sa), (float)ia.x * dna, (float)ia.y * dna);
+          st_bf16x2_split(op + kOffBhHi, op + kOffBhLo, off_bh(2 * lane, sb), (float)ib.x * dnb, (float)ib.y * dnb);
+        }
+        // G[tau][sigma]: lane (slot, tau) sums its row of the partial tile, reading the
+        // eight 16-byte chunks in a lane-rotated order (no bank conflicts)
+        {
+          const int slot = lane >> 4, tau = lane & 15, sig = sa + slot;
+          const float4 *row = reinterpret_cast<const float4 *>(Qt + lane * 32);
+          float4 acc = row[lane & 7];
+#pragma unroll
+          for (int c = 1; c < 8; ++c) acc = add4(acc, row[(lane + c) & 7]);
+          const float g = (acc.x + acc.y) + (acc.z + acc.w);
+          if (tau >= sig && tau <= tend) {
+            if constexpr (kPrecise) {
+              st_bf16_split(op + kOffGtHi, op + kOffGtLo, off_gt(tau, sig), g);
+            } else {
+              *reinterpret_cast<__nv_bfloat16 *>(op + kOffGtHi + off_gt(tau, sig)) = __float2bfloat16_rn(g);
+            }
+          }
+        }
+        __syncwarp();  // the tile and the accumulators are free for the next pair
+      }
+      if (role == 1) cp_async_wait<0>();  // x has landed in the operand stage
 
       fence_proxy_async_smem();
       __syncwarp();
