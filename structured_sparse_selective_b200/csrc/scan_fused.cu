@@ -111,12 +111,18 @@ constexpr int kOffHdr = kOffGDst + 64;           // int [4]: number of groups, t
 constexpr int kOffCtLo = kOffHdr + 16;           // low part of Ct (fp32 output only), as kOffCt
 __host__ __device__ constexpr int op_stage_bytes(bool precise) { return kOffCtLo + (precise ? 2 * kCtSbo : 0); }
 
-// carry-step record of a position: whether it continues a target group (else
-// it starts one), whether it ends it, and the group's ordinal
-constexpr int kMetaKeep = 1 << 8;
-constexpr int kMetaEnd = 1 << 9;
-constexpr int kMetaOrdShift = 10;
-constexpr int kOrdNone = 127;  // ordinal field of positions whose total another thread writes
+// carry-step record of a position: bit 0 = it continues a target group (else it
+// starts one); bits 8-14 = the group's ordinal (kOrdNone: another thread writes the
+// group's total); bits 16-31 = the byte offset, in a carry warp's group-total
+// rows, where the first pass (groups 0-15) stores the position's running sum
+// (row 16 absorbs the positions of other groups)
+constexpr int kMetaKeep = 1;
+constexpr int kMetaOrdShift = 8;
+constexpr int kMetaOffShift = 16;
+constexpr int kOrdNone = 127;
+__host__ __device__ constexpr int meta_word(bool keep, int ord) {
+  return (keep ? kMetaKeep : 0) | (ord << kMetaOrdShift) | ((ord < 16 ? ord : 16) * 64 << kMetaOffShift);
+}
 
 // per-pair scratch (bytes); warp X = the pair's even warp, warp Y the odd one
 constexpr int kQBytes = 2 * kT * 32 * 4;      // float [2 slots][16 tau][32 lanes] partial G
@@ -691,8 +697,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           const int q0 = (posA0 < 32 && e0 == ecross) ? kOrdNone : e0;
           const int q1 = (posA1 < 32 && e1 == ecross) ? kOrdNone : e1;
           int *meta = reinterpret_cast<int *>(op + kOffMeta);
-          meta[posA0] = (keep0 ? kMetaKeep : 0) | (end0 ? kMetaEnd : 0) | (q0 << kMetaOrdShift);
-          meta[posA1] = (keep1 ? kMetaKeep : 0) | (end1 ? kMetaEnd : 0) | (q1 << kMetaOrdShift);
+          meta[posA0] = meta_word(keep0, q0);
+          meta[posA1] = meta_word(keep1, q1);
           // the target's column in the next order
           if (end0) op[kOffGDst + e0] = posBt[i0];
           if (end1) op[kOffGDst + e1] = posBt[i1];
@@ -841,6 +847,9 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           if (tau < nvalid) store_out(yout + ((b * a.L + t0 + tau) * a.H + h) * kP + p, v[tau]);
       }
     };
+    // this thread's output column and rows (8 hh + i) of sub-chunk 0; rows are ystep apart
+    const int64_t ystep = a.H * kP;
+    TO *const ybase = yout + ((b * a.L + 8 * (lane >> 4)) * a.H + h) * kP + 16 * q + (lane & 15);
     int pidx0 = lane, pidx1 = lane + 32;
     float pval0 = 1.f, pval1 = 1.f;
     int done = 0;  // sub-chunks whose carry step completed
@@ -880,8 +889,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
           tmem_wait_ld();
           const int tp = ys * kT;
           const int nv = (int)(a.L - tp < kT ? a.L - tp : kT);
-          TO *yrow = yout + ((b * a.L + tp + 8 * hh) * a.H + h) * kP + 16 * q + pl;
-          const int64_t ystep = a.H * kP;
+          TO *yrow = ybase + (int64_t)tp * ystep;
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             if (8 * hh + i < nv) store_out(yrow + i * ystep, yv[i]);
@@ -909,12 +917,21 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
             const int mt[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
             const float nu[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
             tmem_wait_ld();
+            if (base == 0) {  // the store offsets of the first pass are precomputed
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              run = (mt[c] & kMetaKeep) ? run : 0.f;
-              run = fmaf(nu[c], v[c], run);
-              const unsigned e = (unsigned)((mt[c] >> kMetaOrdShift) - base);
-              cs[(e < 16u ? e : 16u) * 16] = run;
+              for (int c = 0; c < 8; ++c) {
+                run = (mt[c] & kMetaKeep) ? run : 0.f;
+                run = fmaf(nu[c], v[c], run);
+                *reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(cs) + (mt[c] >> kMetaOffShift)) = run;
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                run = (mt[c] & kMetaKeep) ? run : 0.f;
+                run = fmaf(nu[c], v[c], run);
+                const unsigned e = (unsigned)(((mt[c] >> kMetaOrdShift) & 127) - base);
+                cs[(e < 16u ? e : 16u) * 16] = run;
+              }
             }
           }
           // the group that crosses positions 31 | 32 gets the lower half's part
