@@ -38,7 +38,8 @@
  * Layouts (row-major, contiguous, element-aligned):
  *   logits [batch][seqlen][heads][K]          s    [batch][seqlen][heads] int32
  *   idx    [K][N] int32, shared by all heads  (idx[k][j] = row of the nonzero
- *                                              of column j of P_k, in [0, N))
+ *                                              of column j of P_k, in [0, N));
+ *          [heads][K][N] with PDSSM_FLAG_HEAD_DICTS
  *   d, B, C [batch][seqlen][heads][N]         x, y [batch][seqlen][heads][P]
  *   h0, h_final [batch][heads][N][P]          prod_idx, prod_val [batch][heads][N]
  *   Complex values (PDSSM_C64) are interleaved (re, im) float pairs, the
@@ -83,6 +84,18 @@ typedef enum { PDSSM_F32 = 0, PDSSM_BF16 = 1, PDSSM_C64 = 2 } pdssm_dtype;
 /* flags */
 #define PDSSM_FLAG_DEVICE_CHECK 1u   /* synchronise and return PDSSM_ERR_DEVICE_CHECK on bad idx/s */
 #define PDSSM_FLAG_REFERENCE_PATH 2u /* use the plain three-kernel chunked path (no fused kernel) */
+/* Failure-detection testing: the fused kernel's bounded device waits (one role
+ * waiting for another) give up after about 1 microsecond instead of 2 seconds.
+ * A wait that gives up records PDSSM_ERR_TIMEOUT in the workspace's error word,
+ * every role leaves its loop and the kernel returns: nothing faults or hangs, and
+ * the outputs of that call are unspecified. The final wait for the kernel's own
+ * tensor-core work keeps its long limit. No effect on the three-kernel path. */
+#define PDSSM_FLAG_SHORT_WAITS 4u
+/* Per-head dictionaries (Flash PD-SSM page, Methodology 4: multi-head layers;
+ * each head may hold its own dictionary): idx is [heads][K][N] instead of the
+ * shared [K][N]; head h's step t uses P_{s_t} of its own dictionary
+ * idx[h][s_t]. Workspace sizes grow by the dictionary's size only. */
+#define PDSSM_FLAG_HEAD_DICTS 8u
 
 /*
  * Problem description. Supported dtype combinations:

@@ -125,6 +125,7 @@ def _to_slices(t: torch.Tensor) -> torch.Tensor:
 
 def scan(logits, idx, d, B, C, x, h0=None, want_prod: bool = True) -> Dict[str, np.ndarray]:
     """Dense recurrence on full [Bt, L, H, *] arrays; outputs in the same layout.
+    ``idx`` is the shared dictionary [K, N] or per-head dictionaries [H, K, N].
 
     Returns y [Bt,L,H,P], h_final [Bt,H,N,P], s [Bt,L,H] and optionally
     prod_idx [Bt,H,N], prod_val [Bt,H,N].
@@ -133,8 +134,22 @@ def scan(logits, idx, d, B, C, x, h0=None, want_prod: bool = True) -> Dict[str, 
     N = B.shape[-1]
     P = x.shape[-1]
     h0s = None if h0 is None else h0.reshape(Bt * H, N, P)
-    r = scan_slices(_to_slices(logits), idx, _to_slices(d), _to_slices(B), _to_slices(C),
-                    _to_slices(x), h0s, want_prod)
+    if getattr(idx, "ndim", 2) == 3:
+        # per-head dictionaries idx[H][K][N]: the slices of head h use idx[h]
+        sl = {k: _to_slices(v) for k, v in (("logits", logits), ("d", d), ("B", B), ("C", C), ("x", x))}
+        parts = []
+        for hh in range(H):
+            rows = list(range(hh, Bt * H, H))
+            parts.append((rows, scan_slices(sl["logits"][rows], idx[hh], sl["d"][rows], sl["B"][rows],
+                                            sl["C"][rows], sl["x"][rows],
+                                            None if h0s is None else h0s[rows], want_prod)))
+        r = {k: np.empty((Bt * H,) + v.shape[1:], dtype=v.dtype) for k, v in parts[0][1].items()}
+        for rows, part in parts:
+            for k, v in part.items():
+                r[k][rows] = v
+    else:
+        r = scan_slices(_to_slices(logits), idx, _to_slices(d), _to_slices(B), _to_slices(C),
+                        _to_slices(x), h0s, want_prod)
     out = {
         "y": r["y"].reshape(Bt, H, L, P).transpose(0, 2, 1, 3),
         "h_final": r["h_final"].reshape(Bt, H, N, P),

@@ -108,9 +108,11 @@ def slice_backward(logits, idx, d, B, C, x, dy, dh_final=None, h0=None, tau: flo
 
 
 def scan_backward(logits, idx, d, B, C, x, dy, dh_final=None, h0=None, tau: float = 1.0) -> Dict[str, np.ndarray]:
-    """Gradients of S slices given slice-major arrays; returns slice-major arrays."""
+    """Gradients of S slices given slice-major arrays; returns slice-major arrays. ``idx`` is
+    one dictionary [K, N] for every slice, or one per slice [S, K, N]."""
     S = np.asarray(logits).shape[0]
-    res = [slice_backward(logits[i], idx, d[i], B[i], C[i], x[i], dy[i],
+    idx = np.asarray(idx)
+    res = [slice_backward(logits[i], idx[i] if idx.ndim == 3 else idx, d[i], B[i], C[i], x[i], dy[i],
                           None if dh_final is None else dh_final[i], None if h0 is None else h0[i], tau)
            for i in range(S)]
     return {k: np.stack([r[k] for r in res]) for k in res[0]}

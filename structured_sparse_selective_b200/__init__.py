@@ -29,7 +29,8 @@ from typing import Dict, Optional
 import torch
 
 __all__ = [
-    "PdssmError", "Problem", "F32", "BF16", "C64", "FLAG_DEVICE_CHECK", "FLAG_REFERENCE_PATH",
+    "PdssmError", "Problem", "F32", "BF16", "C64", "FLAG_DEVICE_CHECK", "FLAG_REFERENCE_PATH", "FLAG_SHORT_WAITS",
+    "FLAG_HEAD_DICTS",
     "library_path", "make_problem", "pdssm_workspace_size", "pdssm_select", "pdssm_scan_fwd",
     "pdssm_forward", "pdssm_read_device_check", "pdssm_status_string", "forward", "EXPORTED_SYMBOLS",
     "KernelTrace", "alloc_workspace", "pdssm_forward_noalloc", "pdssm_bwd_workspace_size", "pdssm_scan_bwd",
@@ -39,6 +40,8 @@ __all__ = [
 F32, BF16, C64 = 0, 1, 2
 FLAG_DEVICE_CHECK = 1
 FLAG_REFERENCE_PATH = 2
+FLAG_SHORT_WAITS = 4
+FLAG_HEAD_DICTS = 8
 MAX_N, MAX_P, MAX_K = 128, 128, 64
 
 EXPORTED_SYMBOLS = (
@@ -258,6 +261,17 @@ class KernelTrace:
         return [(nm, self.events[2 * i].elapsed_time(self.events[2 * i + 1])) for i, nm in enumerate(self.names)]
 
 
+def _dict_flags(idx: torch.Tensor, heads: int, K: int, N: int) -> int:
+    """FLAG_HEAD_DICTS for a per-head dictionary [heads, K, N]; 0 for a shared [K, N] one."""
+    if idx.dim() == 3:
+        if tuple(idx.shape) != (heads, K, N):
+            raise ValueError(f"per-head dictionary must be [{heads}, {K}, {N}], got {tuple(idx.shape)}")
+        return FLAG_HEAD_DICTS
+    if tuple(idx.shape) != (K, N):
+        raise ValueError(f"dictionary must be [{K}, {N}], got {tuple(idx.shape)}")
+    return 0
+
+
 def alloc_workspace(pb: Problem, device) -> torch.Tensor:
     return torch.empty(max(1, pdssm_workspace_size(pb)), dtype=torch.uint8, device=device)
 
@@ -267,7 +281,9 @@ def forward(logits: torch.Tensor, idx: torch.Tensor, d: torch.Tensor, B: torch.T
             out_dtype: Optional[torch.dtype] = None, chunk: int = 0, flags: int = 0,
             want_prod: bool = True, want_s: bool = False, workspace: Optional[torch.Tensor] = None,
             stream=None) -> Dict[str, torch.Tensor]:
-    """Allocates the outputs (torch) and runs ``pdssm_forward`` on the inputs' device."""
+    """Allocates the outputs (torch) and runs ``pdssm_forward`` on the inputs' device.
+    A 3-D ``idx`` [heads, K, N] is a per-head dictionary (PDSSM_FLAG_HEAD_DICTS)."""
+    flags |= _dict_flags(idx, B.shape[2], logits.shape[-1], B.shape[-1])
     pb = make_problem(logits, d, B, x, out_dtype=out_dtype, chunk=chunk, flags=flags)
     dev = B.device
     Bt, L, H, N = B.shape
@@ -295,8 +311,9 @@ def backward(logits: Optional[torch.Tensor], s: torch.Tensor, idx: torch.Tensor,
              want_dh0: bool = True, workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
     """Allocates the gradients (float32) and runs ``pdssm_scan_bwd``; ``s`` are the forward's
     selections, ``dy`` has the forward output's dtype. No logits -> no ``dlogits``."""
-    K = logits.shape[-1] if logits is not None else int(idx.shape[0])
-    pb = make_problem(logits, d, B, x, out_dtype=dy.dtype, K=K)
+    K = logits.shape[-1] if logits is not None else int(idx.shape[-2])
+    pb = make_problem(logits, d, B, x, out_dtype=dy.dtype, K=K,
+                      flags=_dict_flags(idx, B.shape[2], K, B.shape[-1]))
     dev = B.device
     Bt, L, H, N = B.shape
     P = x.shape[-1]

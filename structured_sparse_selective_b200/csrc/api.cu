@@ -27,6 +27,7 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Plan {
   int64_t Bt, L, H, N, P, K, T, nC, rows;
+  int64_t Kd;         // dictionary entries: K, or heads * K with per-head dictionaries
   bool cplx;
   bool fused;         // the fused kernel serves the problem: the workspace is the error word only
   size_t state_size;  // bytes per state element (4 or 8)
@@ -68,7 +69,9 @@ pdssm_status make_plan(const pdssm_problem *pb, Plan *pl, bool three_kernel = fa
   } else {
     return PDSSM_ERR_UNSUPPORTED;
   }
-  if (pb->flags & ~(PDSSM_FLAG_DEVICE_CHECK | PDSSM_FLAG_REFERENCE_PATH)) return PDSSM_ERR_INVALID_ARG;
+  if (pb->flags & ~(PDSSM_FLAG_DEVICE_CHECK | PDSSM_FLAG_REFERENCE_PATH | PDSSM_FLAG_SHORT_WAITS |
+                    PDSSM_FLAG_HEAD_DICTS))
+    return PDSSM_ERR_INVALID_ARG;
 
   Plan p;
   p.Bt = pb->batch; p.L = pb->seqlen; p.H = pb->heads; p.N = pb->N; p.P = pb->P; p.K = pb->K;
@@ -81,6 +84,7 @@ pdssm_status make_plan(const pdssm_problem *pb, Plan *pl, bool three_kernel = fa
   if (!mul_ok(rows, std::max(std::max(p.N, p.P), p.K) * 8, &tmp)) return PDSSM_ERR_UNSUPPORTED;
   if (p.nC > INT32_MAX) return PDSSM_ERR_UNSUPPORTED;
   p.rows = rows;
+  p.Kd = (pb->flags & PDSSM_FLAG_HEAD_DICTS) ? p.H * p.K : p.K;
   int64_t nchunks = bh * p.nC;
   p.fused = !three_kernel && fused_scan_applies(pb);
   size_t o = 0;
@@ -91,9 +95,9 @@ pdssm_status make_plan(const pdssm_problem *pb, Plan *pl, bool three_kernel = fa
     *pl = p;
     return PDSSM_OK;
   }
-  p.o_idx = o; o = align256(o + (size_t)(p.K * p.N) * 4);
-  p.o_off = o; o = align256(o + (size_t)(p.K * (p.N + 1)) * 4);
-  p.o_src = o; o = align256(o + (size_t)(p.K * p.N) * 4);
+  p.o_idx = o; o = align256(o + (size_t)(p.Kd * p.N) * 4);
+  p.o_off = o; o = align256(o + (size_t)(p.Kd * (p.N + 1)) * 4);
+  p.o_src = o; o = align256(o + (size_t)(p.Kd * p.N) * 4);
   p.o_s = o; o = align256(o + (size_t)rows * 4);
   p.o_cstate = o; o = align256(o + (size_t)nchunks * p.N * p.P * p.state_size);
   p.o_cidx = o; o = align256(o + (size_t)nchunks * p.N * 4);
@@ -182,6 +186,8 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &plan, const int32_t *
   a.s = s; a.logits = logits; a.s_out = s_out; a.idx = idx;
   a.d = d; a.B = B; a.C = C; a.x = x; a.h0 = h0; a.y = y; a.h_final = h_final;
   a.prod_idx = prod_idx; a.prod_val = prod_val; a.ws = w;
+  a.short_waits = (pb->flags & PDSSM_FLAG_SHORT_WAITS) != 0;
+  a.head_dicts = (pb->flags & PDSSM_FLAG_HEAD_DICTS) != 0;
 
   if (p.Bt * p.H == 0) return finish(pb, w, stream);
   if (p.L == 0) {
@@ -193,7 +199,7 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &plan, const int32_t *
     st = cuda_status(launch_fused_scan(a, stream));
     return st != PDSSM_OK ? st : finish(pb, w, stream);
   }
-  st = cuda_status(launch_prep_dict(idx, (int)p.K, (int)p.N, w, stream));
+  st = cuda_status(launch_prep_dict(idx, (int)p.Kd, (int)p.N, w, stream));
   if (st != PDSSM_OK) return st;
   if (!a.s) {
     // unfused selection into s_out (or the workspace)
@@ -210,7 +216,7 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &plan, const int32_t *
 // Workspace of the backward pass: error word, dictionary preimage lists,
 // checkpoints [Bt][H][nCk][N][P] and the per-slice scratch [Bt][H][16][N][P].
 struct BwdPlan {
-  int64_t Bt, L, H, N, P, K, rows, nCk;
+  int64_t Bt, L, H, N, P, K, rows, nCk, Kd;
   size_t o_err, o_idx, o_off, o_src, o_ckpt, o_scr, total;
 };
 
@@ -221,7 +227,7 @@ pdssm_status make_bwd_plan(const pdssm_problem *pb, BwdPlan *bp) {
   if (p.cplx) return PDSSM_ERR_UNSUPPORTED;
   if (scan_bwd_smem_bytes(p.N, p.P, p.K) > (size_t)227 * 1024) return PDSSM_ERR_UNSUPPORTED;
   BwdPlan q;
-  q.Bt = p.Bt; q.L = p.L; q.H = p.H; q.N = p.N; q.P = p.P; q.K = p.K; q.rows = p.rows;
+  q.Bt = p.Bt; q.L = p.L; q.H = p.H; q.N = p.N; q.P = p.P; q.K = p.K; q.rows = p.rows; q.Kd = p.Kd;
   q.nCk = scan_bwd_checkpoints(p.L);
   int64_t slices = p.Bt * p.H, per_slice, tot;
   if (!mul_ok(p.N * p.P, q.nCk + scan_bwd_scratch_steps(), &per_slice) || !mul_ok(slices, per_slice, &tot) ||
@@ -229,9 +235,9 @@ pdssm_status make_bwd_plan(const pdssm_problem *pb, BwdPlan *bp) {
     return PDSSM_ERR_UNSUPPORTED;
   size_t o = 0;
   q.o_err = o; o = align256(o + 4);
-  q.o_idx = o; o = align256(o + (size_t)(p.K * p.N) * 4);
-  q.o_off = o; o = align256(o + (size_t)(p.K * (p.N + 1)) * 4);
-  q.o_src = o; o = align256(o + (size_t)(p.K * p.N) * 4);
+  q.o_idx = o; o = align256(o + (size_t)(p.Kd * p.N) * 4);
+  q.o_off = o; o = align256(o + (size_t)(p.Kd * (p.N + 1)) * 4);
+  q.o_src = o; o = align256(o + (size_t)(p.Kd * p.N) * 4);
   q.o_ckpt = o; o = align256(o + (size_t)(slices * q.nCk * p.N * p.P) * 4);
   q.o_scr = o; o = align256(o + (size_t)(slices * scan_bwd_scratch_steps() * p.N * p.P) * 4);
   q.total = o;
@@ -422,9 +428,10 @@ pdssm_status pdssm_scan_bwd(const pdssm_problem *pb, const void *logits, const i
     }
     return finish(pb, w, cs);
   }
-  st = cuda_status(launch_prep_dict(idx, (int)q.K, (int)q.N, w, cs));
+  st = cuda_status(launch_prep_dict(idx, (int)q.Kd, (int)q.N, w, cs));
   if (st != PDSSM_OK) return st;
   ScanBwdArgs a;
+  a.head_dicts = (pb->flags & PDSSM_FLAG_HEAD_DICTS) != 0;
   a.Bt = q.Bt; a.L = q.L; a.H = q.H; a.N = q.N; a.P = q.P; a.K = q.K;
   a.d_t = pb->d_t; a.in_t = pb->in_t; a.out_t = pb->out_t; a.logits_t = pb->logits_t;
   a.tau = tau;

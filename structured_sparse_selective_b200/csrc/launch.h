@@ -23,6 +23,8 @@ struct ScanArgs {
   int32_t *prod_idx;
   void *prod_val;
   Workspace ws;
+  bool short_waits = false;  // PDSSM_FLAG_SHORT_WAITS: the fused kernel's role waits give up after ~1 us
+  bool head_dicts = false;   // PDSSM_FLAG_HEAD_DICTS: idx is [H][K][N]; head h's entry k is h * K + k
 };
 
 // Records the caller's trace events around a launch (no-op unless tracing).
@@ -56,6 +58,7 @@ struct ScanBwdArgs {
   float *ckpt, *scratch;
   float *dlogits, *dd, *dB, *dC, *dx, *dh0;
   Workspace ws;  // err, idx, csr_off, csr_src
+  bool head_dicts = false;  // PDSSM_FLAG_HEAD_DICTS: dictionary entries h * K + k
 };
 // Shared memory of one backward block, checkpoints of a sequence, and the steps
 // between checkpoints (the per-sequence scratch holds that many states).

@@ -33,6 +33,7 @@ struct BParams {
   int64_t L, H, N, P, K, nCk;
   float tau;
   int logits_bf16, dy_bf16;
+  bool head_dicts;  // idx/off/src hold heads * K entries, head h's from h * K
   const int32_t *s;
   const int32_t *idx;  // sanitised [K][N]
   const int32_t *off;  // [K][N+1]
@@ -69,7 +70,8 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
   int *srcsh = offsh + N + 1;                     // [N]
   uint8_t *idxsh = reinterpret_cast<uint8_t *>(srcsh + N);  // [K][N] dictionary
 
-  for (int e = tid; e < K * N; e += kBT) idxsh[e] = (uint8_t)a.idx[e];
+  const int64_t kh = a.head_dicts ? h * K : 0;  // this head's first dictionary entry
+  for (int e = tid; e < K * N; e += kBT) idxsh[e] = (uint8_t)a.idx[kh * N + e];
 
   const TD *dg = static_cast<const TD *>(a.d);
   const TIn *Bg = static_cast<const TIn *>(a.B);
@@ -108,9 +110,9 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
       v.d = to_f32(dg[row * N + tid]);
       v.B = to_f32(Bg[row * N + tid]);
       if (rev) v.C = to_f32(Cg[row * N + tid]);
-      else v.src = a.src[(int64_t)v.st * N + tid];
+      else v.src = a.src[(kh + v.st) * N + tid];
     }
-    if (!rev && tid <= N) v.off = a.off[(int64_t)v.st * (N + 1) + tid];
+    if (!rev && tid <= N) v.off = a.off[(kh + v.st) * (N + 1) + tid];
     if (tid < P) {
       v.x = to_f32(xg[row * P + tid]);
       if (rev) v.dy = ld_flag(a.dy, row * P + tid, a.dy_bf16);
@@ -292,6 +294,7 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs &s, cudaStream_t st) {
   a.ckpt = s.ckpt; a.scratch = s.scratch;
   a.dlogits = s.dlogits; a.dd = s.dd; a.dB = s.dB; a.dC = s.dC; a.dx = s.dx; a.dh0 = s.dh0;
   a.err = s.ws.err;
+  a.head_dicts = s.head_dicts;
   const size_t smem = scan_bwd_smem_bytes(s.N, s.P, s.K);
   auto kern = s.d_t == PDSSM_BF16 ? (s.in_t == PDSSM_BF16 ? scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16>
                                                           : scan_bwd_kernel<__nv_bfloat16, float>)

@@ -32,6 +32,7 @@ constexpr int kMaxRows = 16;  // rows per thread at most
 
 struct KParams {
   int64_t L, H, N, P, K, T, nC;
+  int64_t Kh;   // dictionary entries per head with per-head dictionaries (else 0)
   int64_t nPB;  // column blocks (columns are independent)
   const int32_t *s;
   const int32_t *idx;  // sanitised [K][N]
@@ -43,13 +44,14 @@ struct KParams {
   uint32_t *err;
 };
 
-__device__ __forceinline__ int load_s(const KParams &a, int64_t row) {
+// Dictionary entry of row `row` (head h): the selection, validated, plus h * Kh.
+__device__ __forceinline__ int load_s(const KParams &a, int64_t row, int64_t h) {
   int st = a.s[row];
   if (st < 0 || st >= a.K) {
     flag_error(a.err, kErrSRange);
     st = 0;
   }
-  return st;
+  return st + (int)(h * a.Kh);
 }
 
 // ------------------------------------------------------------------ phase A
@@ -96,7 +98,7 @@ __global__ void __launch_bounds__(RG * kPB) phase_a_kernel(KParams a) {
   auto fetch = [&](int64_t t) {
     StepVec<T> v;
     const int64_t row = (b * a.L + t) * a.H + h;
-    v.st = load_s(a, row);
+    v.st = load_s(a, row, h);
     if (tid < N) {
       v.d = LoadD<CPLX, TD>::ld(dg + row * N + tid);
       v.B = ldf(Bg + row * N + tid);
@@ -351,7 +353,7 @@ __global__ void __launch_bounds__(RG * kPB) phase_c_kernel(KParams a) {
     if (tid < N) {
       dn = LoadD<CPLX, TD>::ld(dg + row * N + tid);
       cn = ldf(Cg + row * N + tid);
-      sn = load_s(a, row);
+      sn = load_s(a, row, h);
     }
   };
   T ylv = Nm::zero();  // y_loc of the step being finished, fetched a step ahead
@@ -407,6 +409,7 @@ __global__ void empty_outputs_kernel(KParams a, int64_t slices) {
 KParams make_params(const ScanArgs &s) {
   KParams k;
   k.L = s.L; k.H = s.H; k.N = s.N; k.P = s.P; k.K = s.K; k.T = s.T; k.nC = s.nC;
+  k.Kh = s.head_dicts ? s.K : 0;
   k.nPB = (s.P + kPB - 1) / kPB;
   k.s = s.s; k.idx = s.ws.idx; k.off = s.ws.csr_off; k.src = s.ws.csr_src;
   k.d = s.d; k.B = s.B; k.C = s.C; k.x = s.x; k.h0 = s.h0;

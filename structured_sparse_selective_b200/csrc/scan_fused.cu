@@ -81,6 +81,7 @@ constexpr int kNY = 4;   // output accumulator slots
 constexpr int kYLag = 2;  // the carry step of sub-chunk a writes the output of sub-chunk a - kYLag
 constexpr int kThreads = 32 * (kPrepWarps + 5);  // 6 prep warps, 4 carry warps, 1 MMA-issuing warp
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
+constexpr uint64_t kShortTimeoutNs = 1000ull;     // 1 us (failure-detection testing)
 
 // tensor-memory columns: 64-column state regions (a ring of 3, or 2 plus S_lo
 // at column 128), then the output slots
@@ -163,6 +164,8 @@ struct FParams {
   uint32_t *err;
   InLayout in;
   int nst;  // operand stages
+  bool short_waits;
+  bool head_dicts;  // idx is [H][K][N]
   int off_in, off_op, off_dict, off_scr, off_bar;
 };
 
@@ -174,6 +177,7 @@ struct Bars {
   uint64_t ufull[3], sready[4], slofree, drain;
   uint32_t tmem_base;
   int abort;
+  uint64_t wait_ns;  // limit of the roles' waits (the final drain always uses kTimeoutNs)
 };
 
 __device__ __forceinline__ uint64_t now_ns() {
@@ -187,9 +191,9 @@ __device__ __noinline__ bool wait_bar(Bars *bars, uint64_t *bar, uint32_t parity
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = now_ns();
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
+    if (mbar_try_wait_sleep(bar, parity, bars->wait_ns < 20000 ? (uint32_t)bars->wait_ns : 20000u)) return true;
     if (*(volatile int *)&bars->abort) return false;
-    if (now_ns() - t0 > kTimeoutNs) {
+    if (now_ns() - t0 > bars->wait_ns) {
       *(volatile int *)&bars->abort = 1;
       flag_error(err, kErrTimeout);
       return false;
@@ -525,10 +529,12 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     mbar_init(&bars->slofree, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
+    bars->wait_ns = a.short_waits ? kShortTimeoutNs : kTimeoutNs;
     mbar_fence_init();
   }
+  const int32_t *idx_h = a.idx + (a.head_dicts ? h * a.K * kN : 0);
   for (int e = tid; e < a.K * kN; e += kThreads) {
-    int v = a.idx[e];
+    int v = idx_h[e];
     if (v < 0 || v >= kN) {
       flag_error(a.err, kErrIdxRange);
       v = 0;
@@ -590,8 +596,12 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         load_x(a, op + kOffX, b, h, sub, lane);
         cp_async_commit();
       }
-      // one decision for the pair; the barrier also publishes the loaded inputs
-      if (!pair_and(pbar, ok)) break;
+      // one decision for the pair; the barrier also publishes the loaded inputs. A
+      // pair that stops waits for its own copies still in flight first.
+      if (!pair_and(pbar, ok)) {
+        cp_async_wait<0>();
+        break;
+      }
 
       // selections, two lanes per token: warp Y this sub-chunk's, warp X the next one's
       {
@@ -1143,6 +1153,8 @@ cudaError_t launch_fused_scan(const ScanArgs &s, cudaStream_t st) {
   a.prod_val = static_cast<float *>(s.prod_val);
   a.s_out = s.s_out;
   a.err = s.ws.err;
+  a.short_waits = s.short_waits;
+  a.head_dicts = s.head_dicts;
   const bool precise = s.out_t != PDSSM_BF16;
   int off = 0;
   if (!plan_smem(a.K, a.logit_size, s.logits != nullptr, precise, &a, &off)) return cudaErrorInvalidConfiguration;

@@ -70,6 +70,8 @@ def run_gpu(inp, device, chunk=0, h0=None, via_scan=False, flags=0, want_s=True)
         out = pd.forward(g["logits"], g["idx"], g["d"], g["B"], g["C"], g["x"], h0=h0d, chunk=chunk,
                          flags=flags, want_s=want_s)
     else:
+        if g["idx"].dim() == 3:  # per-head dictionaries
+            flags |= pd.FLAG_HEAD_DICTS
         pb = pd.make_problem(g["logits"], g["d"], g["B"], g["x"], chunk=chunk, flags=flags)
         Bt, L, H, N = g["B"].shape
         P = g["x"].shape[-1]

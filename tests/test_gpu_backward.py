@@ -23,9 +23,12 @@ def _rel(got, ref):
     return float((np.abs(got - ref) / np.maximum(scale, 1e-30)).max()) if ref.size else 0.0
 
 
-def _run(recipe, kw, dev, seed=0, with_h0=True, with_dh=True, with_logits=True, tau=0.7):
+def _run(recipe, kw, dev, seed=0, with_h0=True, with_dh=True, with_logits=True, tau=0.7, head_dicts=False):
     sp = workloads.spec(recipe, **kw)
     inp = workloads.generate(sp, seed=seed)
+    if head_dicts:  # a dictionary per head [H, K, N]
+        g = torch.Generator().manual_seed(40 + seed)
+        inp["idx"] = torch.randint(0, sp.N, (sp.heads, sp.K, sp.N), generator=g).to(torch.int32)
     g = {k: v.to(dev) for k, v in inp.items()}
     # the forward pass gives the selections (they do not depend on h0)
     fwd = pd.forward(g["logits"], g["idx"], g["d"], g["B"], g["C"], g["x"], want_s=True, want_prod=False)
@@ -40,7 +43,10 @@ def _run(recipe, kw, dev, seed=0, with_h0=True, with_dh=True, with_logits=True, 
                       tau=tau)
     torch.cuda.synchronize(dev)
     S = Bt * H
-    ref = bwd.scan_backward(_slices(inp["logits"]), inp["idx"].numpy(), _slices(inp["d"]), _slices(inp["B"]),
+    idx_ref = inp["idx"].numpy()
+    if idx_ref.ndim == 3:  # slice b * H + h uses head h's dictionary
+        idx_ref = np.stack([idx_ref[i % H] for i in range(Bt * H)])
+    ref = bwd.scan_backward(_slices(inp["logits"]), idx_ref, _slices(inp["d"]), _slices(inp["B"]),
                             _slices(inp["C"]), _slices(inp["x"]), _slices(dy),
                             None if dh is None else dh.reshape(S, N, P).double().numpy(),
                             None if h0 is None else h0.reshape(S, N, P).double().numpy(), tau=tau)
@@ -113,3 +119,10 @@ def test_backward_reproduces_the_hand_worked_gradients(cuda_device, name):
     assert out["dd"][0, :, 0].tolist() == exp["bwd_dd"]
     assert out["dx"][0, :, 0, 0].tolist() == exp["bwd_dx"]
     assert out["dh0"][0, 0, :, 0].tolist() == exp["bwd_dh0"]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("recipe,kw", [("lm", dict(batch=2, seqlen=40, heads=3)), ("tiny", dict(heads=2, seqlen=50))])
+def test_backward_with_per_head_dictionaries(cuda_device, recipe, kw):
+    errs = _run(recipe, kw, cuda_device, seed=6, head_dicts=True)
+    assert all(v <= TOL for v in errs.values()), errs

@@ -350,3 +350,24 @@ def test_hand_worked_automaton_runs(cuda_device, chunk, via_scan):
         assert out["h_final"][0, 0, :, 0].tolist() == exp["h_final"], name
         assert out["prod_idx"][0, 0].tolist() == exp["prod_idx"], name
         assert out["prod_val"][0, 0].tolist() == exp["prod_val"], name
+
+
+# ------------------------------------------------------- per-head dictionaries
+
+@pytest.mark.parametrize("recipe,kw,chunk", [
+    ("lm", dict(batch=2, seqlen=300, heads=3), 0),            # the fused kernel
+    ("lm", dict(batch=1, seqlen=100, heads=2), 7),            # the three-kernel path
+    ("tiny", dict(batch=2, seqlen=90, heads=3), 0),
+    ("long", dict(batch=1, seqlen=130, heads=3), 16),
+    ("complex", dict(batch=1, seqlen=60, heads=2, N=16, P=8, K=5), 0),
+])
+def test_per_head_dictionaries_match_oracle(cuda_device, recipe, kw, chunk):
+    """Methodology 4 (multi-head layers): a dictionary per head, idx [H, K, N]."""
+    sp = workloads.spec(recipe, **kw)
+    inp = workloads.generate(sp, seed=9)
+    g = torch.Generator().manual_seed(5)
+    inp["idx"] = torch.randint(0, sp.N, (sp.heads, sp.K, sp.N), generator=g).to(torch.int32)
+    out = run_gpu(inp, cuda_device, chunk=chunk)
+    compare_full(inp, out)
+    # the selection-given entry point too
+    compare_full(inp, run_gpu(inp, cuda_device, chunk=chunk, via_scan=True))
