@@ -101,6 +101,7 @@ def test_backward_empty_sequence_passes_the_final_gradient_through(cuda_device):
     assert torch.equal(out["dh0"], dh)
 
 
+@pytest.mark.gpu
 @pytest.mark.parametrize("name", ["fsa_advance_merge_weighted"])
 def test_backward_reproduces_the_hand_worked_gradients(cuda_device, name):
     """pdssm_scan_bwd on the weighted automaton fixture (loss sum_t y_t: dy = 1, no final-state
