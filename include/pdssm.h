@@ -218,6 +218,84 @@ pdssm_status pdssm_forward_noalloc(const pdssm_problem *pb, const void *logits, 
                                    void *prod_val, int32_t *s_out, pdssm_stream_t stream);
 
 /*
+ * Dictionary construction (Flash PD-SSM page, Technical Summary, Methodology 1:
+ * the dictionary's K sparse matrices are pre-computed; the original PD-SSM makes
+ * a matrix sparse by a column-wise hardmax): for each dense matrix M_k and
+ * column j, idx[k][j] = the lowest i with M[k][i][j] == max_i' M[k][i'][j]
+ * (a NaN counts as the maximum and the first NaN wins). Bit-exact.
+ *   M    device float [K][N][N], row-major (M[k][i][j] at (k * N + i) * N + j);
+ *        K may count heads x entries to build per-head dictionaries [heads][K][N]
+ *   idx  device int32 [K][N] output, in [0, N)
+ * Errors: PDSSM_ERR_INVALID_ARG for null pointers, K < 0, N < 1, misaligned
+ * pointers; PDSSM_ERR_UNSUPPORTED for N > PDSSM_MAX_N. No workspace.
+ */
+pdssm_status pdssm_dict_hardmax(int64_t K, int64_t N, const float *M, int32_t *idx, pdssm_stream_t stream);
+
+/*
+ * Fused projection and selection (Methodology 1: the input u_t generates the K
+ * scores by a linear transformation; Methodology 2: hard argmax). For each row
+ * r = b * seqlen + t and head h:
+ *   logits[r][h][k] = sum_d u[r][d] * W[d][h * K + k]
+ *   s[r][h]         = the lowest k with logits[r][h][k] == max_k' logits[r][h][k']
+ * The products are exact (bf16 x bf16) and the sums are fp32, accumulated on the
+ * tensor cores in tensor memory; the argmax runs in the epilogue that reads the
+ * accumulator, so the logits need not be written at all.
+ *   pb      batch, seqlen, heads, K (N, P, chunk and the dtypes are not used)
+ *   D       width of u (the embedding dimension): a positive multiple of 64
+ *   u       device bf16 [batch * seqlen][D], 16-byte aligned
+ *   W       device bf16 [D][heads * K], 16-byte aligned
+ *   s       device int32 [batch][seqlen][heads] output (the layout pdssm_scan_fwd reads)
+ *   logits  device float [batch][seqlen][heads][K] output, or NULL
+ *   workspace >= 256 bytes (error word; pdssm_read_device_check reads it)
+ * Requirements: K a power of two; heads * K a multiple of 32 and either at most
+ * 256 or a multiple of 256. Others return PDSSM_ERR_UNSUPPORTED.
+ */
+pdssm_status pdssm_select_proj(const pdssm_problem *pb, int64_t D, const void *u, const void *W, int32_t *s,
+                               float *logits, void *workspace, size_t workspace_bytes, pdssm_stream_t stream);
+
+/*
+ * The original PD-SSM's selection (Flash PD-SSM page, Technical Summary,
+ * Methodology 1, "Original PD-SSM"; Problem Statement: its O(L N^2) memory and
+ * 40x slowdown are what Flash PD-SSM removes). Built here as the contrast the
+ * pages measure against: each step's transition is the column-wise hardmax of a
+ * convex combination of K dense dictionary matrices,
+ *   pi_t = softmax(logits_t / tau),  idx_t[j] = argmax_i sum_k pi_t[k] M_k[i][j]
+ * (lowest i on ties). The mixtures are never written to memory: for 128 steps of
+ * one head they are one tensor-core product [steps x K] x [K x N^2] (pi and M
+ * split into bf16 hi + lo, about 16 bits) whose epilogue takes the argmax.
+ *   logits    device logits_t [batch][seqlen][heads][K]
+ *   M         device float [K][N][N] ([heads][K][N][N] with PDSSM_FLAG_HEAD_DICTS)
+ *   tau       > 0
+ *   idx_steps device uint8 [batch][seqlen][heads][N] output: row of the nonzero
+ *             of column j of step t's transition
+ *   workspace pdssm_soft_select_workspace_size bytes, 256-byte aligned (the error
+ *             word and the dictionary in the tensor cores' bf16 layout)
+ * Requirements: N a power of two in [16, 128]; K <= 64. Near-ties of the
+ * mixture (within its ~2^-16 relative precision) may resolve differently from an
+ * exact computation.
+ */
+pdssm_status pdssm_soft_select_workspace_size(const pdssm_problem *pb, size_t *bytes);
+pdssm_status pdssm_soft_select(const pdssm_problem *pb, const void *logits, const float *M, float tau,
+                               uint8_t *idx_steps, void *workspace, size_t workspace_bytes,
+                               pdssm_stream_t stream);
+
+/*
+ * The scan with a transition given for every step (the original PD-SSM's
+ * per-step matrices from pdssm_soft_select, or any per-step one-hot-column
+ * transitions): H_t = P_t diag(d_t) H_{t-1} + B_t x_t^T, y_t = H_t^T C_t with
+ * P_t[idx_steps[t][j]][j] = 1. Arguments as pdssm_scan_fwd with idx_steps
+ * (device uint8 [batch][seqlen][heads][N], 16-byte aligned; values >= N are
+ * replaced by 0 and flagged) in place of s and idx; pb->K, pb->logits_t and
+ * PDSSM_FLAG_HEAD_DICTS are not used. Served by the fused kernel only (N = P =
+ * 64, bf16 d/B/C/x, real state): other problems return PDSSM_ERR_UNSUPPORTED.
+ * The workspace is 256 bytes (the error word).
+ */
+pdssm_status pdssm_scan_fwd_steps(const pdssm_problem *pb, const uint8_t *idx_steps, const void *d,
+                                  const void *B, const void *C, const void *x, const void *h0, void *y,
+                                  void *h_final, int32_t *prod_idx, void *prod_val, void *workspace,
+                                  size_t workspace_bytes, pdssm_stream_t stream);
+
+/*
  * Backward pass (real state): workspace bytes for pdssm_scan_bwd. Checkpoints
  * of the state every 16 steps plus a 16-step scratch per (batch, head) slice:
  * 4 * N * P * batch * heads * (ceil(L / 16) + 16) bytes, plus the dictionary's

@@ -159,3 +159,29 @@ def scan(logits, idx, d, B, C, x, h0=None, want_prod: bool = True) -> Dict[str, 
         out["prod_idx"] = r["prod_idx"].reshape(Bt, H, N)
         out["prod_val"] = r["prod_val"].reshape(Bt, H, N)
     return out
+
+
+def scan_steps(idx_steps, d, B, C, x, h0=None, want_prod: bool = True) -> Dict[str, np.ndarray]:
+    """The recurrence with a transition given per step (the original PD-SSM's per-step
+    matrices): step t of slice (b, h) applies P_t with P_t[idx_steps[b, t, h, j]][j] = 1.
+    Each slice is the dense loop above with its L step rows as the dictionary and step t
+    selecting row t. idx_steps [Bt, L, H, N]; other arrays as in scan()."""
+    st = np.asarray(idx_steps.cpu() if isinstance(idx_steps, torch.Tensor) else idx_steps).astype(np.int32)
+    Bt, L, H, N = st.shape
+    P = x.shape[-1]
+    pick = np.eye(L)  # logits: step t selects dictionary row t
+    out = {"y": None}
+    ys, hfs, pis, pvs = [], [], [], []
+    for b in range(Bt):
+        for h in range(H):
+            r = scan_slices(pick[None], st[b, :, h], d[b:b + 1, :, h], B[b:b + 1, :, h], C[b:b + 1, :, h],
+                            x[b:b + 1, :, h], None if h0 is None else h0[b:b + 1, h], want_prod)
+            ys.append(r["y"][0]); hfs.append(r["h_final"][0])
+            if want_prod:
+                pis.append(r["prod_idx"][0]); pvs.append(r["prod_val"][0])
+    out["y"] = np.stack(ys).reshape(Bt, H, L, P).transpose(0, 2, 1, 3)
+    out["h_final"] = np.stack(hfs).reshape(Bt, H, N, P)
+    if want_prod:
+        out["prod_idx"] = np.stack(pis).reshape(Bt, H, N)
+        out["prod_val"] = np.stack(pvs).reshape(Bt, H, N)
+    return out

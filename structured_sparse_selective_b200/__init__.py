@@ -34,7 +34,9 @@ __all__ = [
     "library_path", "make_problem", "pdssm_workspace_size", "pdssm_select", "pdssm_scan_fwd",
     "pdssm_forward", "pdssm_read_device_check", "pdssm_status_string", "forward", "EXPORTED_SYMBOLS",
     "KernelTrace", "alloc_workspace", "pdssm_forward_noalloc", "pdssm_bwd_workspace_size", "pdssm_scan_bwd",
-    "backward",
+    "backward", "pdssm_dict_hardmax", "pdssm_select_proj", "dict_hardmax", "select_proj",
+    "pdssm_soft_select_workspace_size", "pdssm_soft_select", "pdssm_scan_fwd_steps", "soft_select",
+    "forward_steps",
 ]
 
 F32, BF16, C64 = 0, 1, 2
@@ -48,7 +50,8 @@ EXPORTED_SYMBOLS = (
     "pdssm_status_string", "pdssm_version", "pdssm_workspace_size", "pdssm_select",
     "pdssm_scan_fwd", "pdssm_forward", "pdssm_read_device_check", "pdssm_trace_begin",
     "pdssm_trace_end", "pdssm_trace_kernel_name", "pdssm_forward_noalloc", "pdssm_bwd_workspace_size",
-    "pdssm_scan_bwd",
+    "pdssm_scan_bwd", "pdssm_dict_hardmax", "pdssm_select_proj", "pdssm_soft_select_workspace_size",
+    "pdssm_soft_select", "pdssm_scan_fwd_steps",
 )
 
 _DIR = os.path.dirname(os.path.abspath(__file__))
@@ -102,6 +105,16 @@ def _load() -> ctypes.CDLL:
     lib.pdssm_scan_bwd.argtypes = [pb, vp, i32p, i32p, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float,
                                    vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.pdssm_scan_bwd.restype = ctypes.c_int
+    lib.pdssm_dict_hardmax.argtypes = [ctypes.c_int64, ctypes.c_int64, vp, vp, vp]
+    lib.pdssm_dict_hardmax.restype = ctypes.c_int
+    lib.pdssm_select_proj.argtypes = [pb, ctypes.c_int64, vp, vp, vp, vp, vp, sz, vp]
+    lib.pdssm_select_proj.restype = ctypes.c_int
+    lib.pdssm_soft_select_workspace_size.argtypes = [pb, ctypes.POINTER(sz)]
+    lib.pdssm_soft_select_workspace_size.restype = ctypes.c_int
+    lib.pdssm_soft_select.argtypes = [pb, vp, vp, ctypes.c_float, vp, vp, sz, vp]
+    lib.pdssm_soft_select.restype = ctypes.c_int
+    lib.pdssm_scan_fwd_steps.argtypes = [pb, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.pdssm_scan_fwd_steps.restype = ctypes.c_int
     lib.pdssm_read_device_check.argtypes = [vp, vp]
     lib.pdssm_read_device_check.restype = ctypes.c_int
     lib.pdssm_trace_begin.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
@@ -226,6 +239,105 @@ def pdssm_scan_bwd(pb: Problem, logits, s, idx, d, B, C, x, h0, dy, dh_final, ta
         _ptr(C, dev), _ptr(x, dev), _ptr(h0, dev), _ptr(dy, dev), _ptr(dh_final, dev), float(tau),
         _ptr(dlogits, dev), _ptr(dd, dev), _ptr(dB, dev), _ptr(dC, dev), _ptr(dx, dev), _ptr(dh0, dev),
         _ptr(workspace, dev), ws_bytes, _stream(stream, dev)), "pdssm_scan_bwd")
+
+
+def pdssm_dict_hardmax(K: int, N: int, M: torch.Tensor, idx: torch.Tensor, stream=None) -> None:
+    dev = M.device
+    _check(_lib.pdssm_dict_hardmax(int(K), int(N), _ptr(M, dev), _ptr(idx, dev), _stream(stream, dev)),
+           "pdssm_dict_hardmax")
+
+
+def pdssm_select_proj(pb: Problem, D: int, u, W, s, logits, workspace, stream=None) -> None:
+    dev = u.device
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pdssm_select_proj(ctypes.byref(pb), int(D), _ptr(u, dev), _ptr(W, dev), _ptr(s, dev),
+                                  _ptr(logits, dev), _ptr(workspace, dev), ws_bytes, _stream(stream, dev)),
+           "pdssm_select_proj")
+
+
+def dict_hardmax(M: torch.Tensor, stream=None) -> torch.Tensor:
+    """Column-wise hardmax of dense matrices M [..., N, N] (float32): idx [..., N] int32."""
+    N = M.shape[-1]
+    K = M.numel() // (N * N)
+    idx = torch.empty(M.shape[:-2] + (N,), dtype=torch.int32, device=M.device)
+    pdssm_dict_hardmax(K, N, M.contiguous(), idx, stream)
+    return idx
+
+
+def select_proj(u: torch.Tensor, W: torch.Tensor, heads: int, K: int, want_logits: bool = False,
+                stream=None) -> Dict[str, torch.Tensor]:
+    """u [Bt, L, D] bf16, W [D, heads * K] bf16 -> s [Bt, L, heads] int32 (and logits [Bt, L, heads, K])."""
+    Bt, L, D = u.shape
+    pb = Problem(batch=Bt, seqlen=L, heads=heads, N=1, P=1, K=K, chunk=0, logits_t=BF16, in_t=BF16, d_t=BF16,
+                 state_t=F32, out_t=BF16, flags=0)
+    out = {"s": torch.empty(Bt, L, heads, dtype=torch.int32, device=u.device)}
+    if want_logits:
+        out["logits"] = torch.empty(Bt, L, heads, K, dtype=torch.float32, device=u.device)
+    ws = torch.zeros(256, dtype=torch.uint8, device=u.device)
+    pdssm_select_proj(pb, D, u.contiguous(), W.contiguous(), out["s"], out.get("logits"), ws, stream)
+    out["workspace"] = ws
+    return out
+
+
+def pdssm_soft_select_workspace_size(pb: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.pdssm_soft_select_workspace_size(ctypes.byref(pb), ctypes.byref(n)),
+           "pdssm_soft_select_workspace_size")
+    return int(n.value)
+
+
+def pdssm_soft_select(pb: Problem, logits, M, tau: float, idx_steps, workspace, stream=None) -> None:
+    dev = logits.device
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pdssm_soft_select(ctypes.byref(pb), _ptr(logits, dev), _ptr(M, dev), float(tau), _ptr(idx_steps, dev),
+                                  _ptr(workspace, dev), ws_bytes, _stream(stream, dev)), "pdssm_soft_select")
+
+
+def pdssm_scan_fwd_steps(pb: Problem, idx_steps, d, B, C, x, h0, y, h_final, prod_idx, prod_val, workspace,
+                         stream=None) -> None:
+    dev = d.device
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pdssm_scan_fwd_steps(
+        ctypes.byref(pb), _ptr(idx_steps, dev), _ptr(d, dev), _ptr(B, dev), _ptr(C, dev), _ptr(x, dev),
+        _ptr(h0, dev), _ptr(y, dev), _ptr(h_final, dev), _ptr(prod_idx, dev), _ptr(prod_val, dev),
+        _ptr(workspace, dev), ws_bytes, _stream(stream, dev)), "pdssm_scan_fwd_steps")
+
+
+def soft_select(logits: torch.Tensor, M: torch.Tensor, tau: float = 1.0, N: Optional[int] = None,
+                stream=None) -> Dict[str, torch.Tensor]:
+    """The original PD-SSM's per-step transitions: idx_steps [Bt, L, H, N] uint8 from logits
+    [Bt, L, H, K] and dense dictionary matrices M [K, N, N] (or per head [H, K, N, N])."""
+    Bt, L, H, K = logits.shape
+    N = M.shape[-1]
+    flags = FLAG_HEAD_DICTS if M.dim() == 4 else 0
+    pb = Problem(batch=Bt, seqlen=L, heads=H, N=N, P=1, K=K, chunk=0, logits_t=_DT[logits.dtype], in_t=F32,
+                 d_t=F32, state_t=F32, out_t=F32, flags=flags)
+    ws = torch.empty(pdssm_soft_select_workspace_size(pb), dtype=torch.uint8, device=logits.device)
+    steps = torch.empty(Bt, L, H, N, dtype=torch.uint8, device=logits.device)
+    pdssm_soft_select(pb, logits.contiguous(), M.contiguous(), tau, steps, ws, stream)
+    return {"idx_steps": steps, "workspace": ws}
+
+
+def forward_steps(idx_steps: torch.Tensor, d: torch.Tensor, B: torch.Tensor, C: torch.Tensor, x: torch.Tensor,
+                  h0: Optional[torch.Tensor] = None, out_dtype: Optional[torch.dtype] = None, flags: int = 0,
+                  stream=None) -> Dict[str, torch.Tensor]:
+    """The scan with a transition per step (idx_steps [Bt, L, H, N] uint8), e.g. from soft_select."""
+    Bt, L, H, N = B.shape
+    P = x.shape[-1]
+    if out_dtype is None:
+        out_dtype = B.dtype
+    pb = Problem(batch=Bt, seqlen=L, heads=H, N=N, P=P, K=1, chunk=0, logits_t=BF16, in_t=_DT[B.dtype],
+                 d_t=_DT[d.dtype], state_t=F32, out_t=_DT[out_dtype], flags=flags)
+    dev = B.device
+    out = {"y": torch.empty(Bt, L, H, P, dtype=out_dtype, device=dev),
+           "h_final": torch.empty(Bt, H, N, P, dtype=torch.float32, device=dev),
+           "prod_idx": torch.empty(Bt, H, N, dtype=torch.int32, device=dev),
+           "prod_val": torch.empty(Bt, H, N, dtype=torch.float32, device=dev)}
+    ws = alloc_workspace(pb, dev)
+    pdssm_scan_fwd_steps(pb, idx_steps, d, B, C, x, h0, out["y"], out["h_final"], out["prod_idx"], out["prod_val"],
+                         ws, stream)
+    out["workspace"] = ws
+    return out
 
 
 def pdssm_read_device_check(workspace: torch.Tensor, stream=None) -> int:

@@ -165,10 +165,11 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &plan, const int32_t *
                       const void *logits, int32_t *s_out, const int32_t *idx, const void *d,
                       const void *B, const void *C, const void *x, const void *h0, void *y,
                       void *h_final, int32_t *prod_idx, void *prod_val, void *workspace,
-                      size_t workspace_bytes, cudaStream_t stream) {
+                      size_t workspace_bytes, cudaStream_t stream, const uint8_t *steps = nullptr) {
   Plan p = plan;
   ScanArgs a;
-  a.s = s; a.logits = logits; a.d = d; a.B = B; a.C = C; a.x = x;
+  a.s = s; a.logits = logits; a.d = d; a.B = B; a.C = C; a.x = x; a.steps = steps;
+  if (steps && (!p.fused || !fused_scan_pointers_ok(a))) return PDSSM_ERR_UNSUPPORTED;
   if (p.fused && !fused_scan_pointers_ok(a)) {
     // inputs the fused kernel's 16-byte loads cannot read: the three-kernel
     // path runs instead and needs its own (larger) workspace
@@ -183,7 +184,7 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &plan, const int32_t *
   a.Bt = p.Bt; a.L = p.L; a.H = p.H; a.N = p.N; a.P = p.P; a.K = p.K; a.T = p.T; a.nC = p.nC;
   a.d_t = pb->d_t; a.in_t = pb->in_t; a.out_t = pb->out_t; a.logits_t = pb->logits_t;
   a.cplx = p.cplx;
-  a.s = s; a.logits = logits; a.s_out = s_out; a.idx = idx;
+  a.s = s; a.logits = logits; a.s_out = s_out; a.idx = idx; a.steps = steps;
   a.d = d; a.B = B; a.C = C; a.x = x; a.h0 = h0; a.y = y; a.h_final = h_final;
   a.prod_idx = prod_idx; a.prod_val = prod_val; a.ws = w;
   a.short_waits = (pb->flags & PDSSM_FLAG_SHORT_WAITS) != 0;
@@ -375,6 +376,98 @@ pdssm_status pdssm_forward(const pdssm_problem *pb, const void *logits, const in
   if ((st = bind_device(cs)) != PDSSM_OK) return st;
   return run_scan(pb, p, nullptr, logits, s_out, idx, d, B, C, x, h0, y, h_final, prod_idx,
                   prod_val, workspace, workspace_bytes, cs);
+}
+
+pdssm_status pdssm_dict_hardmax(int64_t K, int64_t N, const float *M, int32_t *idx, pdssm_stream_t stream) {
+  if (K < 0 || N < 1) return PDSSM_ERR_INVALID_ARG;
+  if (N > PDSSM_MAX_N) return PDSSM_ERR_UNSUPPORTED;
+  if (K == 0) return PDSSM_OK;
+  if (!M || !idx || !aligned(M, 4) || !aligned(idx, 4)) return PDSSM_ERR_INVALID_ARG;
+  int64_t kn;
+  if (!mul_ok(K, N * N, &kn)) return PDSSM_ERR_UNSUPPORTED;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  pdssm_status st = bind_device(cs);
+  if (st != PDSSM_OK) return st;
+  return cuda_status(launch_dict_hardmax(K, (int)N, M, idx, cs));
+}
+
+pdssm_status pdssm_select_proj(const pdssm_problem *pb, int64_t D, const void *u, const void *W, int32_t *s,
+                               float *logits, void *workspace, size_t workspace_bytes, pdssm_stream_t stream) {
+  if (!pb || pb->batch < 0 || pb->seqlen < 0 || pb->heads < 1 || pb->K < 1 || D < 1) return PDSSM_ERR_INVALID_ARG;
+  if (pb->K > PDSSM_MAX_K || pb->heads > 65535 || !proj_select_supported(D, pb->heads, pb->K))
+    return PDSSM_ERR_UNSUPPORTED;
+  int64_t rows;
+  if (!mul_ok(pb->batch, pb->seqlen, &rows)) return PDSSM_ERR_UNSUPPORTED;
+  if (rows > 0 && (!u || !W || !s)) return PDSSM_ERR_INVALID_ARG;
+  if (!aligned(u, 16) || !aligned(W, 16) || !aligned(s, 4) || !aligned(logits, 16)) return PDSSM_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < 4) return PDSSM_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return PDSSM_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  pdssm_status st = bind_device(cs);
+  if (st != PDSSM_OK) return st;
+  uint32_t *err = static_cast<uint32_t *>(workspace);
+  if (cudaMemsetAsync(err, 0, 4, cs) != cudaSuccess) return PDSSM_ERR_CUDA;
+  if (rows == 0) return PDSSM_OK;
+  return cuda_status(launch_proj_select(rows, D, pb->heads, pb->K, u, W, s, logits, err, cs));
+}
+
+pdssm_status pdssm_soft_select_workspace_size(const pdssm_problem *pb, size_t *bytes) {
+  if (!bytes) return PDSSM_ERR_INVALID_ARG;
+  Plan p;
+  pdssm_status st = make_plan(pb, &p, true);
+  if (st != PDSSM_OK) return st;
+  if (!soft_select_supported(p.N, p.K)) return PDSSM_ERR_UNSUPPORTED;
+  *bytes = 256 + soft_select_ws_bytes((pb->flags & PDSSM_FLAG_HEAD_DICTS) ? p.H : 1, p.N, p.K);
+  return PDSSM_OK;
+}
+
+pdssm_status pdssm_soft_select(const pdssm_problem *pb, const void *logits, const float *M, float tau,
+                               uint8_t *idx_steps, void *workspace, size_t workspace_bytes,
+                               pdssm_stream_t stream) {
+  size_t need = 0;
+  pdssm_status st = pdssm_soft_select_workspace_size(pb, &need);
+  if (st != PDSSM_OK) return st;
+  if (!(tau > 0.f) || !(tau < INFINITY)) return PDSSM_ERR_INVALID_ARG;
+  Plan p;
+  make_plan(pb, &p, true);
+  if (p.rows > 0 && (!logits || !M || !idx_steps)) return PDSSM_ERR_INVALID_ARG;
+  if (!aligned(logits, dtype_size(pb->logits_t)) || !aligned(M, 4)) return PDSSM_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < need) return PDSSM_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return PDSSM_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = bind_device(cs)) != PDSSM_OK) return st;
+  uint32_t *err = static_cast<uint32_t *>(workspace);
+  if (cudaMemsetAsync(err, 0, 4, cs) != cudaSuccess) return PDSSM_ERR_CUDA;
+  if (p.rows == 0) return PDSSM_OK;
+  return cuda_status(launch_soft_select(p.Bt * p.L, p.H, p.N, p.K, pb->logits_t, logits, M,
+                                        (pb->flags & PDSSM_FLAG_HEAD_DICTS) != 0, tau,
+                                        static_cast<char *>(workspace) + 256, idx_steps, err, cs));
+}
+
+pdssm_status pdssm_scan_fwd_steps(const pdssm_problem *pb, const uint8_t *idx_steps, const void *d, const void *B,
+                                  const void *C, const void *x, const void *h0, void *y, void *h_final,
+                                  int32_t *prod_idx, void *prod_val, void *workspace, size_t workspace_bytes,
+                                  pdssm_stream_t stream) {
+  if (!pb) return PDSSM_ERR_INVALID_ARG;
+  // there are no logits and no dictionary: K and logits_t are not used
+  pdssm_problem q = *pb;
+  q.K = 16;
+  q.logits_t = PDSSM_BF16;
+  q.flags &= ~PDSSM_FLAG_HEAD_DICTS;
+  pb = &q;
+  Plan p;
+  pdssm_status st = make_plan(pb, &p);
+  if (st != PDSSM_OK) return st;
+  if (!p.fused) return PDSSM_ERR_UNSUPPORTED;
+  if (p.rows > 0 && (!idx_steps || !aligned(idx_steps, 16))) return PDSSM_ERR_INVALID_ARG;
+  // the dictionary argument of the shared checks is unused here
+  st = check_scan_args(pb, p, reinterpret_cast<const int32_t *>(idx_steps ? (const void *)idx_steps : d), d, B, C,
+                       x, h0, y, h_final, prod_idx, prod_val, workspace, workspace_bytes);
+  if (st != PDSSM_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = bind_device(cs)) != PDSSM_OK) return st;
+  return run_scan(pb, p, nullptr, nullptr, nullptr, nullptr, d, B, C, x, h0, y, h_final, prod_idx, prod_val,
+                  workspace, workspace_bytes, cs, idx_steps);
 }
 
 pdssm_status pdssm_bwd_workspace_size(const pdssm_problem *pb, size_t *bytes) {

@@ -1,6 +1,8 @@
 // Device-side helpers shared by the libpdssm kernels (sm_100a).
 #pragma once
 
+#include <climits>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -28,6 +30,27 @@ __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162flo
 template <typename T>
 __device__ __forceinline__ float ldf(const T *p) {
   return to_f32(*p);
+}
+
+// (value, k) candidates of one argmax, merged so that the result is the lowest k
+// holding the maximum: a NaN beats every number and the lowest NaN wins; +0 and
+// -0 tie. k == INT_MAX marks "no candidate yet" (it loses to anything). The merge
+// is associative and commutative, so partial winners may be combined in any tree.
+__device__ __forceinline__ void sel_merge(float &v, int &k, float ov, int ok) {
+  const bool n = v != v, on = ov != ov;
+  bool take;
+  if (ok == INT_MAX)
+    take = false;
+  else if (k == INT_MAX)
+    take = true;
+  else if (n || on)
+    take = on && (!n || ok < k);
+  else
+    take = ov > v || (ov == v && ok < k);
+  if (take) {
+    v = ov;
+    k = ok;
+  }
 }
 
 // ---------------------------------------------------- real / complex state

@@ -17,6 +17,7 @@ struct ScanArgs {
   const int32_t *s;        // selections (device; null when the scan selects from logits)
   const int32_t *idx;      // caller's dictionary [K][N]
   const void *logits;      // logits when the scan selects by itself (may be null)
+  const uint8_t *steps = nullptr;  // per-step transitions [Bt][L][H][N] (the original PD-SSM), or null
   int32_t *s_out;          // where a fused select stores s (may be null)
   const void *d, *B, *C, *x, *h0;
   void *y, *h_final;
@@ -46,6 +47,20 @@ bool fused_scan_pointers_ok(const ScanArgs &a);
 cudaError_t launch_fused_scan(const ScanArgs &a, cudaStream_t st);
 // Outputs of an empty sequence (L == 0): h_final = h0 (or 0), prod = identity.
 cudaError_t launch_empty_outputs(const ScanArgs &a, cudaStream_t st);
+
+// Fused projection and selection on the tensor cores, and dictionary construction
+// by column-wise hardmax (csrc/select_gemm.cu).
+bool proj_select_supported(int64_t D, int64_t H, int64_t K);
+size_t proj_select_smem_bytes(int64_t H, int64_t K);
+cudaError_t launch_proj_select(int64_t rows, int64_t D, int64_t H, int64_t K, const void *u, const void *W,
+                               int32_t *s, float *logits, uint32_t *err, cudaStream_t st);
+cudaError_t launch_dict_hardmax(int64_t K, int N, const float *M, int32_t *idx, cudaStream_t st);
+// The original PD-SSM's soft selection (convex mixture + column-wise hardmax) per step.
+bool soft_select_supported(int64_t N, int64_t K);
+size_t soft_select_ws_bytes(int64_t dicts, int64_t N, int64_t K);
+cudaError_t launch_soft_select(int64_t rows, int64_t H, int64_t N, int64_t K, int logits_t, const void *logits,
+                               const float *M, bool head_dicts, float tau, void *prep, uint8_t *steps, uint32_t *err,
+                               cudaStream_t st);
 
 // Everything a backward launch needs (real state); validated by the C-ABI layer.
 struct ScanBwdArgs {

@@ -151,8 +151,10 @@ struct FParams {
   int64_t L, H;
   int K, logit_size;
   int nsub;
-  const void *logits;   // null when the selections are given
+  const void *logits;   // null when the selections (or the steps' transitions) are given
   const int32_t *s_in;  // selections [Bt][L][H] (when logits is null)
+  const uint8_t *steps; // per-step transitions [Bt][L][H][N] (the original PD-SSM), or null
+  int row_bytes;        // bytes of one staged logits / transition row (0: selections given)
   const int32_t *idx;
   const __nv_bfloat16 *d, *B, *C, *x;
   const float *h0;
@@ -287,9 +289,10 @@ __device__ __forceinline__ void load_inputs(const FParams &a, uint8_t *st, int64
       *reinterpret_cast<uint4 *>(dc) = z;
     }
   }
-  if (a.logits) {
-    const int lchunks = a.K * a.logit_size / 16;  // 16-byte chunks per logits row
-    const uint8_t *lg = static_cast<const uint8_t *>(a.logits);
+  if (a.row_bytes) {
+    // logits rows, or the steps' transition rows (one byte per column j)
+    const int lchunks = a.row_bytes / 16;  // 16-byte chunks per row
+    const uint8_t *lg = a.steps ? a.steps : static_cast<const uint8_t *>(a.logits);
 #pragma unroll 1
     for (int e = lane; e < 2 * kT * lchunks; e += 32) {
       const int nx = e >= kT * lchunks;
@@ -324,26 +327,6 @@ __device__ __forceinline__ void load_x(const FParams &a, uint8_t *opx, int64_t b
   }
 }
 
-// (value, k) candidates of one logits row, merged so that the result is the
-// lowest k holding the maximum: a NaN beats every number and the lowest NaN
-// wins; +0 and -0 tie. k == INT_MAX marks "no candidate yet". The merge is
-// associative and commutative.
-__device__ __forceinline__ void sel_merge(float &v, int &k, float ov, int ok) {
-  const bool n = v != v, on = ov != ov;
-  bool take;
-  if (ok == INT_MAX)
-    take = false;
-  else if (k == INT_MAX)
-    take = true;
-  else if (n || on)
-    take = on && (!n || ok < k);
-  else
-    take = ov > v || (ov == v && ok < k);
-  if (take) {
-    v = ov;
-    k = ok;
-  }
-}
 
 // Hard selection of token lane / 2 of a stage's logits block: the two lanes of
 // a token each scan every other 16-byte chunk of its row, then merge.
@@ -533,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
     mbar_fence_init();
   }
   const int32_t *idx_h = a.idx + (a.head_dicts ? h * a.K * kN : 0);
-  for (int e = tid; e < a.K * kN; e += kThreads) {
+  for (int e = tid; e < (a.steps ? 0 : a.K * kN); e += kThreads) {
     int v = idx_h[e];
     if (v < 0 || v >= kN) {
       flag_error(a.err, kErrIdxRange);
@@ -603,8 +586,24 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         break;
       }
 
-      // selections, two lanes per token: warp Y this sub-chunk's, warp X the next one's
-      {
+      // selections, two lanes per token: warp Y this sub-chunk's, warp X the next one's.
+      // With per-step transitions the "dictionary" is the stage's table of the 2T
+      // steps' rows and step tau selects row tau (values >= N are replaced by 0).
+      if (a.steps) {
+        uint4 *rows = reinterpret_cast<uint4 *>(in + a.in.logits + (role == 0 ? kT * kN : 0));
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint4 v = rows[lane + 32 * c];
+          if (((v.x | v.y | v.z | v.w) & 0xC0C0C0C0u) != 0) {  // a byte >= 64 = N
+            uint8_t *bv = reinterpret_cast<uint8_t *>(&v);
+            for (int q = 0; q < 16; ++q)
+              if (bv[q] >= kN) bv[q] = 0;
+            rows[lane + 32 * c] = v;
+            flag_error(a.err, kErrIdxRange);
+          }
+        }
+        if (lane < kT) sel[(role == 0 ? kT : 0) + lane] = (role == 0 ? kT : 0) + lane;
+      } else {
         const bool nx = role == 0;
         const int tok = lane >> 1;
         int s_tok = 0;
@@ -624,6 +623,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         }
       }
       pair_sync(pbar);
+      const uint8_t *dict_p = a.steps ? in + a.in.logits : dict;  // rows indexed by sel
 
       const uint8_t *din = in + a.in.d, *Bin = in + a.in.B, *Cin = in + a.in.C;
       // ---- orders of the states: X the next sub-chunk's (S_{a+1}), Y this one's (S_a)
@@ -633,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         const int nsteps = role == 0 ? nnext : nvalid;
         const int *ss = sel + (role == 0 ? kT : 0);
         for (int tau = 0; tau < nsteps; ++tau) {
-          const uint8_t *dk = dict + ss[tau] * kN;
+          const uint8_t *dk = dict_p + ss[tau] * kN;
           n0 = dk[n0];
           n1 = dk[n1];
         }
@@ -659,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         float v0 = 1.f, v1 = 1.f;
 #pragma unroll 1
         for (int tau = 0; tau <= tend; ++tau) {
-          const uint8_t *dk = dict + sel[tau] * kN;
+          const uint8_t *dk = dict_p + sel[tau] * kN;
           v0 *= ld_bf16(din, tau * kN + r0);
           v1 *= ld_bf16(din, tau * kN + r1);
           r0 = dk[r0];
@@ -743,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         int ra0 = j0, ra1 = j1, rb0 = j0, rb1 = j1;
         float wa0 = ba0, wa1 = ba1, wb0 = bb0, wb1 = bb1;
         if (sb <= tend) {  // walker a's first step (sb): b starts after it
-          const uint8_t *dk = dict + sel[sb] * kN;
+          const uint8_t *dk = dict_p + sel[sb] * kN;
           wa0 *= ld_bf16(din, sb * kN + ra0);
           wa1 *= ld_bf16(din, sb * kN + ra1);
           ra0 = dk[ra0];
@@ -752,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_scan_kernel(FParams a) {
         }
 #pragma unroll 1
         for (int tau = sb + 1; tau <= tend; ++tau) {
-          const uint8_t *dk = dict + sel[tau] * kN;
+          const uint8_t *dk = dict_p + sel[tau] * kN;
           const uint8_t *dr = din + tau * kN * 2, *cr = Cin + tau * kN * 2;
           wa0 *= ld_bf16(dr, ra0);
           wa1 *= ld_bf16(dr, ra1);
@@ -1088,10 +1088,10 @@ namespace {
 // Shared-memory plan of one CTA: as many operand stages as fit two CTAs per SM
 // (at least one per prep pair). Returns false when even that does not fit.
 constexpr int kTwoCtaBytes = 228 * 1024 / 2 - 1024;  // per-CTA share of an SM, less the reserved 1 KB
-bool plan_smem(int K, int logit_size, bool have_logits, bool precise, FParams *a, int *bytes) {
+bool plan_smem(int K, int row_bytes, bool precise, FParams *a, int *bytes) {
   int o = 0;
-  a->in.logits = o; o += have_logits ? kT * K * logit_size : 0; o = (o + 127) & ~127;
-  a->in.nlogits = o; o += have_logits ? kT * K * logit_size : 0; o = (o + 127) & ~127;
+  a->in.logits = o; o += kT * row_bytes; o = (o + 127) & ~127;
+  a->in.nlogits = o; o += kT * row_bytes; o = (o + 127) & ~127;
   a->in.d = o; o += kT * kN * 2;
   a->in.B = o; o += kT * kN * 2;
   a->in.C = o; o += kT * kN * 2;
@@ -1123,11 +1123,13 @@ bool fused_scan_applies(const pdssm_problem *pb) {
   if ((pb->K * lsz) % 16 != 0) return false;
   FParams a;
   int bytes = 0;
-  return plan_smem((int)pb->K, lsz, true, pb->out_t != PDSSM_BF16, &a, &bytes);
+  return plan_smem((int)pb->K, (int)pb->K * lsz, pb->out_t != PDSSM_BF16, &a, &bytes) &&
+         plan_smem((int)pb->K, kN, pb->out_t != PDSSM_BF16, &a, &bytes);
 }
 
 bool fused_scan_pointers_ok(const ScanArgs &s) {
-  if (!s.logits && !s.s) return false;
+  if (!s.logits && !s.s && !s.steps) return false;
+  if (s.steps && (reinterpret_cast<uintptr_t>(s.steps) & 15) != 0) return false;
   auto al16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   return (!s.logits || al16(s.logits)) && al16(s.d) && al16(s.B) && al16(s.C) && al16(s.x);
 }
@@ -1140,7 +1142,9 @@ cudaError_t launch_fused_scan(const ScanArgs &s, cudaStream_t st) {
   a.logit_size = s.logits_t == PDSSM_BF16 ? 2 : 4;
   a.nsub = (int)((s.L + kT - 1) / kT);
   a.logits = s.logits;
-  a.s_in = s.logits ? nullptr : s.s;
+  a.steps = s.steps;
+  a.s_in = (s.logits || s.steps) ? nullptr : s.s;
+  a.row_bytes = s.steps ? kN : (s.logits ? a.K * a.logit_size : 0);
   a.idx = s.idx;
   a.d = static_cast<const __nv_bfloat16 *>(s.d);
   a.B = static_cast<const __nv_bfloat16 *>(s.B);
@@ -1157,7 +1161,7 @@ cudaError_t launch_fused_scan(const ScanArgs &s, cudaStream_t st) {
   a.head_dicts = s.head_dicts;
   const bool precise = s.out_t != PDSSM_BF16;
   int off = 0;
-  if (!plan_smem(a.K, a.logit_size, s.logits != nullptr, precise, &a, &off)) return cudaErrorInvalidConfiguration;
+  if (!plan_smem(a.K, a.row_bytes, precise, &a, &off)) return cudaErrorInvalidConfiguration;
 
   cudaError_t e;
   auto kern = (s.logits_t == PDSSM_BF16)

@@ -19,27 +19,6 @@
 
 namespace pdssm {
 
-// (value, k) candidates of one row, combined so that the result is the lowest k
-// holding the maximum: a NaN beats every number and the lowest NaN wins; +0 and
-// -0 tie. The combination is associative and commutative, so lanes may merge
-// their partial winners in any tree order.
-// k == INT_MAX marks a lane that holds no logit yet (it loses to anything).
-__device__ __forceinline__ void sel_merge(float &v, int &k, float ov, int ok) {
-  const bool n = v != v, on = ov != ov;
-  bool take;
-  if (ok == INT_MAX)
-    take = false;
-  else if (k == INT_MAX)
-    take = true;
-  else if (n || on)
-    take = on && (!n || ok < k);
-  else
-    take = ov > v || (ov == v && ok < k);
-  if (take) {
-    v = ov;
-    k = ok;
-  }
-}
 
 // Warp-level selection. A row of K logits occupies G = 2^g lanes of a warp
 // (32 / G rows per warp and pass). Vector form (kVec): the row is a whole
