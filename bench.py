@@ -10,8 +10,13 @@ torchrun every rank runs its own batch (weak scaling; the batch shards need no
 collective), the timed region is bracketed by a barrier and a device
 synchronise on every rank, and the slowest rank's time is reported.
 
-Rank 0 prints one JSON line. ``--impl reference`` times the dense CPU oracle
-on the host cores on a bounded sample of the same workload instead.
+Rank 0 prints one JSON line. On one GPU the LM line also carries, unless
+``--no-extras``: ``per_config`` (the tiny, Z5, long and complex workloads, each
+with its dominant kernel's roofline and the oracle beside it), the original
+PD-SSM's soft selection timed against the Flash path at the LM shape
+(``contrast_original_pdssm``), and the fused projection + selection GEMM
+(``projection``). ``--impl reference`` times the dense CPU oracle on the host
+cores on a bounded sample of the same workload instead.
 ``--pass backward`` measures the backward pass (pdssm_scan_bwd, real states)
 the same way instead of the forward pass; the default is the forward pass.
 """
@@ -212,16 +217,24 @@ def workload_config(sp: workloads.Spec, chunk: int, world: int):
     }
 
 
-def cpu_baseline(sp: workloads.Spec, target_s: float = 12.0):
-    """The oracle as it stands, on the host cores, on whole (batch, head) slices of the workload."""
+def cpu_baseline(sp: workloads.Spec, target_s: float = 12.0, seqlen_cap: int = 0):
+    """The oracle as it stands, on the host cores, on (batch, head) slices of the workload:
+    whole slices, or their first ``seqlen_cap`` steps (the oracle's cost per step does not
+    depend on the position in the sequence)."""
     import oracle
     cores = oracle.threads()
     idx = workloads.generate_idx(sp)
     picks = []
     total = 0.0
     n = max(1, cores)
+    Ls = min(sp.seqlen, seqlen_cap) if seqlen_cap else sp.seqlen
+
+    def slice_of(b, h):
+        sl_ = workloads.generate_slice(sp, b, h)
+        return {k: v[:Ls] for k, v in sl_.items()}
+
     # one calibration slice, then enough slices for ~target_s of work
-    sl = [workloads.generate_slice(sp, 0, 0)]
+    sl = [slice_of(0, 0)]
     t0 = time.perf_counter()
     oracle.scan_slices(sl[0]["logits"][None], idx, sl[0]["d"][None], sl[0]["B"][None], sl[0]["C"][None],
                        sl[0]["x"][None], want_prod=False)
@@ -230,15 +243,211 @@ def cpu_baseline(sp: workloads.Spec, target_s: float = 12.0):
     n = max(1, (n // cores) * cores) if n >= cores else n
     for i in range(n):
         picks.append((i // sp.heads % sp.batch, i % sp.heads))
-    sls = [workloads.generate_slice(sp, b, h) for b, h in picks]
+    sls = [slice_of(b, h) for b, h in picks]
     stack = {k: torch.stack([s[k] for s in sls]) for k in sls[0]}
     t0 = time.perf_counter()
     oracle.scan_slices(stack["logits"], idx, stack["d"], stack["B"], stack["C"], stack["x"], want_prod=False)
     total = time.perf_counter() - t0
-    units = n * sp.seqlen
+    units = n * Ls
+    what = "whole (batch, head) slices" if Ls == sp.seqlen else f"(batch, head) slices cut to their first {Ls} steps"
     return {"value": units / total, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{n} whole (batch, head) slices x L={sp.seqlen} of the {sp.recipe} workload "
+            "sample": f"{n} {what} x L={Ls} of the {sp.recipe} workload "
                       f"({units} token-heads), dense fp64 oracle, {total:.1f} s wall"}
+
+
+def kernel_alg_bytes(sp: workloads.Spec, kernel: str):
+    """Algorithmic bytes of one launch of ``kernel`` on the whole workload (None if unknown):
+    what the kernel must read and write once, never workspace traffic."""
+    def sz(dt):
+        return torch.empty((), dtype=dt).element_size()
+    units = sp.token_heads
+    with_logits = sp.K * sz(sp.logits_dtype)
+    return {
+        "fused_scan": units * sp.algorithmic_bytes_per_token_head(with_logits=True),
+        # phase A reads s, d, B, C and x of every token-head (its y_loc and chunk-state
+        # writes are workspace traffic, not algorithmic)
+        "chunked_phase_a": units * (sp.algorithmic_bytes_per_token_head(with_logits=False) - sp.P * sz(sp.out_dtype)),
+        "chunked_phase_c": units * (4 + sp.N * (sz(sp.d_dtype) + sz(sp.in_dtype)) + sp.P * sz(sp.out_dtype)),
+        "select": units * (with_logits + 4),
+    }.get(kernel)
+
+
+def time_forward(sp, inp, device, steps: int, warmup: int, flush: torch.Tensor, chunk: int = 0):
+    """Device time of pdssm_forward on ``inp`` (already on the device): mean ms per step,
+    per-kernel ms per step (CUDA events the library records around its launches), launches."""
+    import structured_sparse_selective_b200 as pd
+    pb = pd.make_problem(inp["logits"], inp["d"], inp["B"], inp["x"], chunk=chunk)
+    Bt, L, H, N = inp["B"].shape
+    P = inp["x"].shape[-1]
+    sdt = torch.complex64 if sp.state_complex else torch.float32
+    out = {"y": torch.empty(Bt, L, H, P, dtype=sp.out_dtype, device=device),
+           "h_final": torch.empty(Bt, H, N, P, dtype=sdt, device=device)}
+    ws = pd.alloc_workspace(pb, device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        pd.pdssm_forward(pb, inp["logits"], inp["idx"], inp["d"], inp["B"], inp["C"], inp["x"], None, out["y"],
+                         out["h_final"], None, None, None, ws, stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    traces = [pd.KernelTrace(max_launches=16) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        with traces[i]:
+            step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(device)
+    check = pd.pdssm_read_device_check(ws)
+    if check:
+        raise RuntimeError(f"device check status {check} on the {sp.recipe} workload")
+    per_kernel = {}
+    launches = 0
+    for tr in traces:
+        for name, t in tr.timings():
+            per_kernel.setdefault(name, []).append(t)
+            launches += 1
+    ms = sum(s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)) / steps
+    return ms, {k: sum(v) / steps for k, v in per_kernel.items()}, launches
+
+
+def roofline_entry(sp, per_kernel_ms, peaks, traffic=None, traffic_source=None):
+    dominant = max(per_kernel_ms, key=per_kernel_ms.get)
+    alg = kernel_alg_bytes(sp, dominant)
+    if alg is None:
+        return None
+    dom_ms = per_kernel_ms[dominant]
+    achieved = alg / (dom_ms / 1e3) / 1e9
+    return {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+            "peak_source": peaks["source"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic, "traffic_source": traffic_source, "algorithmic_bytes_per_launch": int(alg),
+            "launch_ms": round(dom_ms, 4)}
+
+
+def per_config(device, flush, names=("tiny", "z5", "long", "complex"), steps: int = 5, warmup: int = 3):
+    """Throughput and roofline of the other configurations (one GPU), with the oracle beside each."""
+    peaks = load_peaks()
+    res = {}
+    for name in names:
+        sp = workloads.spec(name)
+        on_host = sp.token_heads * sp.algorithmic_bytes_per_token_head() < 2e9
+        inp = (workloads.generate(sp, seed=7) if on_host else workloads.generate_on_device(sp, seed=7, device=device))
+        inp = {k: v.to(device) for k, v in inp.items()}
+        ms, kms, launches = time_forward(sp, inp, device, steps, warmup, flush)
+        del inp
+        torch.cuda.empty_cache()
+        res[name] = {
+            "workload": workload_config(sp, 0, 1)["workload"],
+            "inputs": "host recipe (workloads.generate)" if on_host else "drawn on the device (same recipe)",
+            "value": round(sp.token_heads / (ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(ms, 4),
+            "steps": steps, "warmup": warmup, "kernels_ms_per_step": {k: round(v, 4) for k, v in kms.items()},
+            "gpu_launches": launches,
+            "roofline": roofline_entry(sp, kms, peaks),
+            "cpu_baseline": cpu_baseline(sp, target_s=2.0, seqlen_cap=0 if name != "complex" else 128),
+        }
+    return res
+
+
+def contrast_original(device, flush, flash_ms: float, steps: int = 5, warmup: int = 3):
+    """The original PD-SSM's selection (soft mixture of dense dictionary matrices + column-wise
+    hardmax, then the scan with per-step transitions) at the LM-layer shape, timed like the
+    Flash PD-SSM forward pass, and the memory each needs for its transitions."""
+    import structured_sparse_selective_b200 as pd
+    sp = workloads.spec("lm")
+    inp = {k: v.to(device) for k, v in workloads.generate_on_device(sp, seed=8, device=device).items()}
+    g = torch.Generator(device=device).manual_seed(9)
+    M = torch.randn(sp.K, sp.N, sp.N, generator=g, device=device)
+    Bt, L, H, N, P = sp.batch, sp.seqlen, sp.heads, sp.N, sp.P
+    pbs = pd.Problem(batch=Bt, seqlen=L, heads=H, N=N, P=1, K=sp.K, chunk=0, logits_t=pd.BF16, in_t=pd.F32,
+                     d_t=pd.F32, state_t=pd.F32, out_t=pd.F32, flags=0)
+    wss = torch.empty(pd.pdssm_soft_select_workspace_size(pbs), dtype=torch.uint8, device=device)
+    steps_t = torch.empty(Bt, L, H, N, dtype=torch.uint8, device=device)
+    pb = pd.Problem(batch=Bt, seqlen=L, heads=H, N=N, P=P, K=16, chunk=0, logits_t=pd.BF16, in_t=pd.BF16,
+                    d_t=pd.BF16, state_t=pd.F32, out_t=pd.BF16, flags=0)
+    ws = pd.alloc_workspace(pb, device)
+    y = torch.empty(Bt, L, H, P, dtype=torch.bfloat16, device=device)
+    hf = torch.empty(Bt, H, N, P, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        pd.pdssm_soft_select(pbs, inp["logits"], M, 1.0, steps_t, wss, stream)
+        pd.pdssm_scan_fwd_steps(pb, steps_t, inp["d"], inp["B"], inp["C"], inp["x"], None, y, hf, None, None, ws,
+                                stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    traces = [pd.KernelTrace(max_launches=8) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        with traces[i]:
+            step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(device)
+    if pd.pdssm_read_device_check(wss) or pd.pdssm_read_device_check(ws):
+        raise RuntimeError("device check failed in the original PD-SSM contrast")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    kms = {}
+    for tr in traces:
+        for name, t in tr.timings():
+            kms[name] = kms.get(name, 0.0) + t / steps
+    units = sp.token_heads
+    return {
+        "what": "original PD-SSM: softmax mixture of K dense N x N dictionary matrices + column-wise hardmax "
+                "per step (tensor cores), then the scan with per-step transitions; LM-layer shape",
+        "original_ms_per_step": round(ms, 4), "flash_ms_per_step": round(flash_ms, 4),
+        "original_over_flash": round(ms / flash_ms, 3),
+        "original_value": round(units / (ms / 1e3), 1), "unit": UNIT,
+        "kernels_ms_per_step": {k: round(v, 4) for k, v in kms.items()},
+        "transition_bytes": {
+            "dense_mixtures_if_materialised": units * N * N * 4,
+            "original_per_step_index_arrays": units * N,
+            "flash_dictionary": sp.K * N * 4,
+            "flash_selections": units * 4,
+        },
+    }
+
+
+def projection_entry(device, steps: int = 10, warmup: int = 3, D: int = 1024):
+    """The fused projection + selection GEMM (u [Bt*L, D] x W [D, H*K], argmax epilogue) at the
+    LM-layer shape with an embedding width D, against the measured bf16 tensor-core peak."""
+    import structured_sparse_selective_b200 as pd
+    sp = workloads.spec("lm")
+    rows, HK = sp.batch * sp.seqlen, sp.heads * sp.K
+    g = torch.Generator(device=device).manual_seed(10)
+    u = torch.randn(sp.batch, sp.seqlen, D, generator=g, device=device).to(torch.bfloat16)
+    W = (torch.randn(D, HK, generator=g, device=device) / D ** 0.5).to(torch.bfloat16)
+    pb = pd.Problem(batch=sp.batch, seqlen=sp.seqlen, heads=sp.heads, N=1, P=1, K=sp.K, chunk=0, logits_t=pd.BF16,
+                    in_t=pd.BF16, d_t=pd.BF16, state_t=pd.F32, out_t=pd.BF16, flags=0)
+    s = torch.empty(sp.batch, sp.seqlen, sp.heads, dtype=torch.int32, device=device)
+    ws = torch.zeros(256, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(warmup):
+        pd.pdssm_select_proj(pb, D, u, W, s, None, ws, stream)
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        pd.pdssm_select_proj(pb, D, u, W, s, None, ws, stream)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    if pd.pdssm_read_device_check(ws):
+        raise RuntimeError("device check failed in the projection")
+    ms = a.elapsed_time(b) / steps
+    peaks = load_peaks()
+    tflops = 2.0 * rows * D * HK / (ms / 1e3) / 1e12
+    return {"what": f"s = argmax_k (u W) per head: rows {rows}, D {D}, heads x K {HK} (bf16, fp32 accumulate)",
+            "ms": round(ms, 4), "roofline": {"bound": "tensor", "achieved": round(tflops, 1),
+                                              "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                              "frac": round(tflops / peaks["bf16_tflops"], 4),
+                                              "peak_source": peaks["source"]},
+            "inputs_l2_resident": "u and W (34 MB) stay in L2 across the back-to-back launches"}
 
 
 # ------------------------------------------------------------- our arm
@@ -322,12 +531,15 @@ def run_ours(args, rank, world, local):
     }.get(dominant)
     peaks = load_peaks()
     traffic = recorded_traffic(dominant, args.workload)
+    traffic_source = (f"profiles/{dominant}_{args.workload}.md (ncu capture of the same kernel sources)"
+                      if traffic is not None else None)
     roofline = None
     if alg_bytes is not None:
         achieved = alg_bytes / (dom_ms / 1e3) / 1e9
         roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1),
                     "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                    "traffic_source": traffic_source,
                     "algorithmic_bytes_per_launch": int(alg_bytes), "launch_ms": round(dom_ms, 4)}
 
     # ---- end to end through the public API with host buffers
@@ -555,6 +767,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="lm", choices=list(workloads.RECIPES))
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other configurations, the original PD-SSM contrast and the projection")
     ap.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward")
     ap.add_argument("--tau", type=float, default=1.0, help="softmax temperature of the backward pass")
     args = ap.parse_args(argv)
@@ -577,6 +791,12 @@ def main(argv=None):
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
                 res["cpu_baseline"] = cpu_baseline(workloads.spec(args.workload))
+            if world == 1 and not args.no_extras and args.workload == "lm":
+                dev = torch.device("cuda", local)
+                flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+                res["per_config"] = per_config(dev, flush)
+                res["contrast_original_pdssm"] = contrast_original(dev, flush, res["ms_per_step"])
+                res["projection"] = projection_entry(dev)
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:

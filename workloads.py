@@ -184,3 +184,44 @@ def generate(sp: Spec, seed: int = 0, device: Optional[torch.device] = None) -> 
         for k, v in sl.items():
             out[k][b, :, h].copy_(v, non_blocking=False)
     return out
+
+
+def generate_on_device(sp: Spec, seed: int = 0, device: Optional[torch.device] = None) -> Dict[str, torch.Tensor]:
+    """The workload's recipe drawn directly on ``device`` (one generator there, whole
+    tensors at once): the same shapes, dtypes, structure and distributions as
+    ``generate`` but not the same numbers. For timing the largest workloads without
+    building them on the host; parity tests use ``generate``."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    Bt, L, H, N, P, K = sp.batch, sp.seqlen, sp.heads, sp.N, sp.P, sp.K
+    g = torch.Generator(device=dev)
+    g.manual_seed(_mix(seed, _SALT[sp.recipe], 0xDE71CE))
+    out = {"idx": generate_idx(sp, seed).to(dev)}
+    if sp.recipe == "z5":
+        tokens = torch.randint(0, K, (Bt, L, H), generator=g, device=dev)
+        out["logits"] = torch.nn.functional.one_hot(tokens, K).to(sp.logits_dtype)
+        out["d"] = torch.ones(Bt, L, H, N, device=dev).to(sp.d_dtype)
+        Bv = torch.zeros(Bt, L, H, N, device=dev)
+        Bv[:, 0, :, 0] = 1.0
+        out["B"] = Bv.to(sp.in_dtype)
+        out["C"] = torch.nn.functional.one_hot(torch.arange(L, device=dev) % N, N).to(sp.in_dtype)[None, :, None, :] \
+            .expand(Bt, L, H, N).contiguous()
+        out["x"] = torch.ones(Bt, L, H, P, device=dev).to(sp.in_dtype)
+        return out
+    out["logits"] = torch.randn(Bt, L, H, K, generator=g, device=dev).to(sp.logits_dtype)
+    z = torch.randn(Bt, L, H, N, generator=g, device=dev)
+    if sp.recipe == "tiny":
+        d = 0.5 + 0.5 * torch.rand(Bt, L, H, N, generator=g, device=dev)
+    elif sp.recipe == "complex":
+        r = torch.exp(-torch.nn.functional.softplus(z))
+        d = torch.polar(r, 2.0 * math.pi * torch.rand(Bt, L, H, N, generator=g, device=dev))
+    else:
+        d = torch.exp(-torch.nn.functional.softplus(z))
+    out["d"] = d.to(sp.d_dtype)
+    del z, d
+    std = 1.0 / math.sqrt(N) if sp.recipe == "lm" else 1.0
+    for k, X in (("B", N), ("C", N), ("x", P)):
+        v = torch.randn(Bt, L, H, X, generator=g, device=dev)
+        if k != "x":
+            v.mul_(std)
+        out[k] = v.to(sp.in_dtype)
+    return out
