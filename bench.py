@@ -17,7 +17,7 @@ PD-SSM's soft selection timed against the Flash path at the LM shape
 (``contrast_original_pdssm``), and the fused projection + selection GEMM
 (``projection``). ``--impl reference`` times the dense CPU oracle on the host
 cores on a bounded sample of the same workload instead.
-``--pass backward`` measures the backward pass (pdssm_scan_bwd, real states)
+``--pass backward`` measures the backward pass (pdssm_scan_bwd, real or complex states)
 the same way instead of the forward pass; the default is the forward pass.
 """
 from __future__ import annotations
@@ -603,7 +603,8 @@ def bwd_bytes_per_token_head(sp: workloads.Spec) -> int:
         return torch.empty((), dtype=dt).element_size()
     reads = 4 + sp.K * sz(sp.logits_dtype) + sp.N * sz(sp.d_dtype) + 2 * sp.N * sz(sp.in_dtype)
     reads += sp.P * sz(sp.in_dtype) + sp.P * sz(sp.out_dtype)
-    return reads + (3 * sp.N + sp.P + sp.K) * 4
+    state = 8 if sp.state_complex else 4  # dd has the state's type
+    return reads + sp.N * state + (2 * sp.N + sp.P + sp.K) * 4
 
 
 def run_ours_backward(args, rank, world, local):
@@ -612,20 +613,23 @@ def run_ours_backward(args, rank, world, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     sp = workloads.spec(args.workload)
-    if sp.state_complex:
-        raise SystemExit("the backward pass is built for real states only")
-    inp = {k: v.to(device) for k, v in workloads.generate(sp, seed=shard_seed(rank)).items()}
+    if sp.state_complex:  # ~10 GB of inputs: drawn on the device (same recipe, other numbers)
+        inp = workloads.generate_on_device(sp, seed=shard_seed(rank), device=device)
+    else:
+        inp = {k: v.to(device) for k, v in workloads.generate(sp, seed=shard_seed(rank)).items()}
     fwd = pd.forward(inp["logits"], inp["idx"], inp["d"], inp["B"], inp["C"], inp["x"], want_s=True,
                      want_prod=False)
     gen = torch.Generator(device=device).manual_seed(shard_seed(rank))
-    dy = torch.randn(fwd["y"].shape, generator=gen, device=device).to(fwd["y"].dtype)
+    sdt = torch.complex64 if sp.state_complex else torch.float32
+    dy = torch.randn(fwd["y"].shape, generator=gen, device=device, dtype=sdt).to(fwd["y"].dtype)
     pb = pd.make_problem(inp["logits"], inp["d"], inp["B"], inp["x"], out_dtype=dy.dtype)
     Bt, L, H, N = inp["B"].shape
     P = inp["x"].shape[-1]
     f32 = dict(dtype=torch.float32, device=device)
-    gr = {"dlogits": torch.empty(Bt, L, H, sp.K, **f32), "dd": torch.empty(Bt, L, H, N, **f32),
+    fst = dict(dtype=sdt, device=device)
+    gr = {"dlogits": torch.empty(Bt, L, H, sp.K, **f32), "dd": torch.empty(Bt, L, H, N, **fst),
           "dB": torch.empty(Bt, L, H, N, **f32), "dC": torch.empty(Bt, L, H, N, **f32),
-          "dx": torch.empty(Bt, L, H, P, **f32), "dh0": torch.empty(Bt, H, N, P, **f32)}
+          "dx": torch.empty(Bt, L, H, P, **f32), "dh0": torch.empty(Bt, H, N, P, **fst)}
     ws = torch.empty(max(1, pd.pdssm_bwd_workspace_size(pb)), dtype=torch.uint8, device=device)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
@@ -672,7 +676,8 @@ def run_ours_backward(args, rank, world, local):
     return {
         "metric": BWD_METRIC, "pass": "backward", "value": round(units * world / (ms / 1e3), 1), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "c64" if sp.state_complex else "f32", "data": "synthetic",
         "config": dict(workload_config(sp, 0, world), tau=args.tau),
         "roofline": {"bound": "hbm", "kernel": "scan_bwd", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "peak_source": peaks["source"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 5),

@@ -296,10 +296,13 @@ pdssm_status pdssm_scan_fwd_steps(const pdssm_problem *pb, const uint8_t *idx_st
                                   size_t workspace_bytes, pdssm_stream_t stream);
 
 /*
- * Backward pass (real state): workspace bytes for pdssm_scan_bwd. Checkpoints
- * of the state every 16 steps plus a 16-step scratch per (batch, head) slice:
- * 4 * N * P * batch * heads * (ceil(L / 16) + 16) bytes, plus the dictionary's
- * preimage lists. PDSSM_ERR_UNSUPPORTED for a complex state.
+ * Backward pass: workspace bytes for pdssm_scan_bwd. Checkpoints of the state
+ * every 16 steps plus a 16-step scratch per (batch, head) slice:
+ * E * N * P * batch * heads * (ceil(L / 16) + 16) bytes (E = 4 for a real state,
+ * 8 for a complex one), plus the dictionary's preimage lists.
+ * PDSSM_ERR_UNSUPPORTED when one block's shared memory (three N x (P + 1)
+ * state buffers and the dictionary) exceeds 227 KiB: every real problem up to
+ * N = P = 128, K = 64 fits, and complex ones up to N = 128, P = 64, K = 64.
  */
 pdssm_status pdssm_bwd_workspace_size(const pdssm_problem *pb, size_t *bytes);
 
@@ -307,27 +310,32 @@ pdssm_status pdssm_bwd_workspace_size(const pdssm_problem *pb, size_t *bytes);
  * Backward pass of the scan (Flash PD-SSM page, Technical Summary,
  * Methodology 2 "Gradient Propagation": hard argmax forward, tempered softmax
  * backward through a straight-through estimator). Gradients of
- *   Loss = sum_t <dy_t, y_t> + <dh_final, H_{L-1}>
- * where y, H are the forward pass of pdssm_scan_fwd on the same arguments:
- *   dd, dB, dC  float [batch][seqlen][heads][N]: exact derivatives;
- *   dx          float [batch][seqlen][heads][P]: exact derivative;
- *   dh0         float [batch][heads][N][P] or NULL: derivative in h0;
+ *   Loss = Re[ sum_t <dy_t, y_t> + <dh_final, H_{L-1}> ],  <a, b> = sum conj(a) b,
+ * where y, H are the forward pass of pdssm_scan_fwd on the same arguments. For
+ * a complex quantity z = u + i v the gradient is dLoss/du + i dLoss/dv (for a
+ * real state every conjugate and real part is the identity):
+ *   dd          state type [batch][seqlen][heads][N]: exact derivative,
+ *               dd_t[j] = sum_p Lam_t[idx[s_t][j]][p] conj(H_{t-1}[j][p]);
+ *   dB, dC      float [batch][seqlen][heads][N]: exact derivatives (real parts);
+ *   dx          float [batch][seqlen][heads][P]: exact derivative (real part);
+ *   dh0         state type [batch][heads][N][P] or NULL: derivative in h0;
  *   dlogits     float [batch][seqlen][heads][K] or NULL (then `logits` is NULL
  *               too): with pit = softmax(logits_t / tau) and
- *               dpi_t[k] = sum_j (Lam_t H_{t-1}^T)[idx[k][j]][j] d_t[j]
+ *               dpi_t[k] = Re sum_j conj((Lam_t H_{t-1}^H)[idx[k][j]][j]) d_t[j]
  *               (Lam_t = dLoss/dH_t), dlogits_t = pit * (dpi_t - <pit, dpi_t>) / tau.
+ * "State type" is float for state_t = PDSSM_F32 and interleaved (re, im) float
+ * pairs for state_t = PDSSM_C64.
  * Inputs: s (device int32 [batch][seqlen][heads], the forward's selections),
- * idx, d, B, C, x, h0 as for pdssm_scan_fwd (h0 float or NULL); dy in the
- * problem's out_t ([batch][seqlen][heads][P]); dh_final float
- * [batch][heads][N][P] or NULL (zero); logits in logits_t; tau > 0.
- * Real state only (state_t = PDSSM_F32); every gradient is float.
+ * idx, d, B, C, x, h0 as for pdssm_scan_fwd (h0 of the state type or NULL); dy
+ * in the problem's out_t ([batch][seqlen][heads][P]); dh_final of the state
+ * type [batch][heads][N][P] or NULL (zero); logits in logits_t; tau > 0.
  * Errors as pdssm_scan_fwd; the workspace is pdssm_bwd_workspace_size bytes.
  */
 pdssm_status pdssm_scan_bwd(const pdssm_problem *pb, const void *logits, const int32_t *s,
                             const int32_t *idx, const void *d, const void *B, const void *C,
-                            const void *x, const float *h0, const void *dy, const float *dh_final,
-                            float tau, float *dlogits, float *dd, float *dB, float *dC, float *dx,
-                            float *dh0, void *workspace, size_t workspace_bytes,
+                            const void *x, const void *h0, const void *dy, const void *dh_final,
+                            float tau, float *dlogits, void *dd, float *dB, float *dC, float *dx,
+                            void *dh0, void *workspace, size_t workspace_bytes,
                             pdssm_stream_t stream);
 
 /*

@@ -421,8 +421,9 @@ def backward(logits: Optional[torch.Tensor], s: torch.Tensor, idx: torch.Tensor,
              B: torch.Tensor, C: torch.Tensor, x: torch.Tensor, dy: torch.Tensor,
              h0: Optional[torch.Tensor] = None, dh_final: Optional[torch.Tensor] = None, tau: float = 1.0,
              want_dh0: bool = True, workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
-    """Allocates the gradients (float32) and runs ``pdssm_scan_bwd``; ``s`` are the forward's
-    selections, ``dy`` has the forward output's dtype. No logits -> no ``dlogits``."""
+    """Allocates the gradients and runs ``pdssm_scan_bwd``; ``s`` are the forward's selections,
+    ``dy`` has the forward output's dtype. dd and dh0 have the state's dtype (float32, or
+    complex64 for a complex ``d``), the others are float32. No logits -> no ``dlogits``."""
     K = logits.shape[-1] if logits is not None else int(idx.shape[-2])
     pb = make_problem(logits, d, B, x, out_dtype=dy.dtype, K=K,
                       flags=_dict_flags(idx, B.shape[2], K, B.shape[-1]))
@@ -430,12 +431,13 @@ def backward(logits: Optional[torch.Tensor], s: torch.Tensor, idx: torch.Tensor,
     Bt, L, H, N = B.shape
     P = x.shape[-1]
     f = dict(dtype=torch.float32, device=dev)
-    out = {"dd": torch.empty(Bt, L, H, N, **f), "dB": torch.empty(Bt, L, H, N, **f),
+    fs = dict(dtype=torch.complex64 if d.is_complex() else torch.float32, device=dev)
+    out = {"dd": torch.empty(Bt, L, H, N, **fs), "dB": torch.empty(Bt, L, H, N, **f),
            "dC": torch.empty(Bt, L, H, N, **f), "dx": torch.empty(Bt, L, H, P, **f)}
     if logits is not None:
         out["dlogits"] = torch.empty(Bt, L, H, K, **f)
     if want_dh0:
-        out["dh0"] = torch.empty(Bt, H, N, P, **f)
+        out["dh0"] = torch.empty(Bt, H, N, P, **fs)
     ws = workspace if workspace is not None else torch.empty(max(1, pdssm_bwd_workspace_size(pb)),
                                                               dtype=torch.uint8, device=dev)
     pdssm_scan_bwd(pb, logits, s, idx, d, B, C, x, h0, dy, dh_final, tau, out.get("dlogits"), out["dd"], out["dB"],

@@ -217,7 +217,7 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &plan, const int32_t *
 // Workspace of the backward pass: error word, dictionary preimage lists,
 // checkpoints [Bt][H][nCk][N][P] and the per-slice scratch [Bt][H][16][N][P].
 struct BwdPlan {
-  int64_t Bt, L, H, N, P, K, rows, nCk, Kd;
+  int64_t Bt, L, H, N, P, K, rows, nCk, Kd, state_size;
   size_t o_err, o_idx, o_off, o_src, o_ckpt, o_scr, total;
 };
 
@@ -225,22 +225,22 @@ pdssm_status make_bwd_plan(const pdssm_problem *pb, BwdPlan *bp) {
   Plan p;
   pdssm_status st = make_plan(pb, &p, true);
   if (st != PDSSM_OK) return st;
-  if (p.cplx) return PDSSM_ERR_UNSUPPORTED;
-  if (scan_bwd_smem_bytes(p.N, p.P, p.K) > (size_t)227 * 1024) return PDSSM_ERR_UNSUPPORTED;
+  if (scan_bwd_smem_bytes(p.N, p.P, p.K, p.cplx) > (size_t)227 * 1024) return PDSSM_ERR_UNSUPPORTED;
   BwdPlan q;
+  q.state_size = p.state_size;
   q.Bt = p.Bt; q.L = p.L; q.H = p.H; q.N = p.N; q.P = p.P; q.K = p.K; q.rows = p.rows; q.Kd = p.Kd;
   q.nCk = scan_bwd_checkpoints(p.L);
   int64_t slices = p.Bt * p.H, per_slice, tot;
   if (!mul_ok(p.N * p.P, q.nCk + scan_bwd_scratch_steps(), &per_slice) || !mul_ok(slices, per_slice, &tot) ||
-      !mul_ok(tot, 4, &tot))
+      !mul_ok(tot, p.state_size, &tot))
     return PDSSM_ERR_UNSUPPORTED;
   size_t o = 0;
   q.o_err = o; o = align256(o + 4);
   q.o_idx = o; o = align256(o + (size_t)(p.Kd * p.N) * 4);
   q.o_off = o; o = align256(o + (size_t)(p.Kd * (p.N + 1)) * 4);
   q.o_src = o; o = align256(o + (size_t)(p.Kd * p.N) * 4);
-  q.o_ckpt = o; o = align256(o + (size_t)(slices * q.nCk * p.N * p.P) * 4);
-  q.o_scr = o; o = align256(o + (size_t)(slices * scan_bwd_scratch_steps() * p.N * p.P) * 4);
+  q.o_ckpt = o; o = align256(o + (size_t)(slices * q.nCk * p.N * p.P) * p.state_size);
+  q.o_scr = o; o = align256(o + (size_t)(slices * scan_bwd_scratch_steps() * p.N * p.P) * p.state_size);
   q.total = o;
   *bp = q;
   return PDSSM_OK;
@@ -481,9 +481,9 @@ pdssm_status pdssm_bwd_workspace_size(const pdssm_problem *pb, size_t *bytes) {
 
 pdssm_status pdssm_scan_bwd(const pdssm_problem *pb, const void *logits, const int32_t *s,
                             const int32_t *idx, const void *d, const void *B, const void *C,
-                            const void *x, const float *h0, const void *dy, const float *dh_final,
-                            float tau, float *dlogits, float *dd, float *dB, float *dC, float *dx,
-                            float *dh0, void *workspace, size_t workspace_bytes,
+                            const void *x, const void *h0, const void *dy, const void *dh_final,
+                            float tau, float *dlogits, void *dd, float *dB, float *dC, float *dx,
+                            void *dh0, void *workspace, size_t workspace_bytes,
                             pdssm_stream_t stream) {
   BwdPlan q;
   pdssm_status st = make_bwd_plan(pb, &q);
@@ -493,10 +493,11 @@ pdssm_status pdssm_scan_bwd(const pdssm_problem *pb, const void *logits, const i
   if (q.rows > 0 && (!s || !d || !B || !C || !x || !dy || !dd || !dB || !dC || !dx))
     return PDSSM_ERR_INVALID_ARG;
   const size_t es_in = dtype_size(pb->in_t), es_d = dtype_size(pb->d_t), es_o = dtype_size(pb->out_t);
+  const size_t es_s = (size_t)q.state_size;
   if (!aligned(idx, 4) || !aligned(s, 4) || !aligned(d, es_d) || !aligned(B, es_in) || !aligned(C, es_in) ||
       !aligned(x, es_in) || !aligned(dy, es_o) || !aligned(logits, dtype_size(pb->logits_t)) ||
-      !aligned(h0, 4) || !aligned(dh_final, 4) || !aligned(dlogits, 4) || !aligned(dd, 4) ||
-      !aligned(dB, 4) || !aligned(dC, 4) || !aligned(dx, 4) || !aligned(dh0, 4))
+      !aligned(h0, es_s) || !aligned(dh_final, es_s) || !aligned(dlogits, 4) || !aligned(dd, es_s) ||
+      !aligned(dB, 4) || !aligned(dC, 4) || !aligned(dx, 4) || !aligned(dh0, es_s))
     return PDSSM_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < q.total) return PDSSM_ERR_WORKSPACE;
   if (!aligned(workspace, 16)) return PDSSM_ERR_INVALID_ARG;
@@ -514,7 +515,7 @@ pdssm_status pdssm_scan_bwd(const pdssm_problem *pb, const void *logits, const i
   if (slices == 0) return finish(pb, w, cs);
   if (q.L == 0) {  // no steps: the final state is the initial one
     if (dh0) {
-      const size_t n = (size_t)(slices * q.N * q.P) * 4;
+      const size_t n = (size_t)(slices * q.N * q.P) * es_s;
       cudaError_t e = dh_final ? cudaMemcpyAsync(dh0, dh_final, n, cudaMemcpyDeviceToDevice, cs)
                                : cudaMemsetAsync(dh0, 0, n, cs);
       if (e != cudaSuccess) return PDSSM_ERR_CUDA;
@@ -530,8 +531,8 @@ pdssm_status pdssm_scan_bwd(const pdssm_problem *pb, const void *logits, const i
   a.tau = tau;
   a.s = s; a.logits = logits; a.d = d; a.B = B; a.C = C; a.x = x; a.dy = dy;
   a.h0 = h0; a.dh_final = dh_final;
-  a.ckpt = reinterpret_cast<float *>(base + q.o_ckpt);
-  a.scratch = reinterpret_cast<float *>(base + q.o_scr);
+  a.ckpt = base + q.o_ckpt;
+  a.scratch = base + q.o_scr;
   a.dlogits = dlogits; a.dd = dd; a.dB = dB; a.dC = dC; a.dx = dx; a.dh0 = dh0;
   a.ws = w;
   st = cuda_status(launch_scan_bwd(a, cs));

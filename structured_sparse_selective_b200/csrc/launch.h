@@ -62,22 +62,24 @@ cudaError_t launch_soft_select(int64_t rows, int64_t H, int64_t N, int64_t K, in
                                const float *M, bool head_dicts, float tau, void *prep, uint8_t *steps, uint32_t *err,
                                cudaStream_t st);
 
-// Everything a backward launch needs (real state); validated by the C-ABI layer.
+// Everything a backward launch needs (real or complex state; h0, dh_final, dd,
+// dh0 and the checkpoints are of the state type); validated by the C-ABI layer.
 struct ScanBwdArgs {
   int64_t Bt, L, H, N, P, K;
   int d_t, in_t, out_t, logits_t;
   float tau;
   const int32_t *s;
   const void *logits, *d, *B, *C, *x, *dy;
-  const float *h0, *dh_final;
-  float *ckpt, *scratch;
-  float *dlogits, *dd, *dB, *dC, *dx, *dh0;
+  const void *h0, *dh_final;
+  void *ckpt, *scratch;
+  float *dlogits, *dB, *dC, *dx;
+  void *dd, *dh0;
   Workspace ws;  // err, idx, csr_off, csr_src
   bool head_dicts = false;  // PDSSM_FLAG_HEAD_DICTS: dictionary entries h * K + k
 };
 // Shared memory of one backward block, checkpoints of a sequence, and the steps
 // between checkpoints (the per-sequence scratch holds that many states).
-size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t K);
+size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t K, bool cplx);
 int64_t scan_bwd_checkpoints(int64_t L);
 int64_t scan_bwd_scratch_steps();
 cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t st);

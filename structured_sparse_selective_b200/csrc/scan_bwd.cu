@@ -1,25 +1,28 @@
-// Backward pass of the PD scan (real state): gradients of the loss
-//   sum_t <dy_t, y_t> + <dh_final, H_{L-1}>
+// Backward pass of the PD scan (real or complex state): gradients of the loss
+//   Re[ sum_t <dy_t, y_t> + <dh_final, H_{L-1}> ],  <a, b> = sum conj(a) b,
 // with respect to d, B, C, x, h0 and, through the straight-through estimator
-// with a tempered softmax, the selection logits.
+// with a tempered softmax, the selection logits. For a complex quantity
+// z = u + i v the gradient is dLoss/du + i dLoss/dv; for a real state every
+// conjugate and real part below is the identity.
 //
 // Flash PD-SSM page, Technical Summary, Methodology 2 ("Gradient Propagation"):
 // the forward pass uses the hard argmax; the backward pass approximates the
 // selection by a tempered softmax. The step's transition is read as the mixture
 // A_t = sum_k pi_k P_k diag(d_t), one-hot at s_t in the forward pass; the gradient
-// in the weights, dpi_t[k] = sum_j (Lam_t H_{t-1}^T)[idx_k[j]][j] d_t[j], goes
-// through the Jacobian of softmax(logits_t / tau).
+// in the weights, dpi_t[k] = Re sum_j conj((Lam_t H_{t-1}^H)[idx_k[j]][j]) d_t[j],
+// goes through the Jacobian of softmax(logits_t / tau).
 //
 // The adjoint Lam_t = dLoss/dH_t runs backwards:
-//   Lam_t = Lam'_t + C_t dy_t^T,  Lam'_{t-1} = A_t^T Lam_t  ((A^T Lam)[j] = d[j] Lam[idx[j]]),
+//   Lam_t = Lam'_t + C_t dy_t^T,  Lam'_{t-1} = A_t^H Lam_t  ((A^H Lam)[j] = conj(d[j]) Lam[idx[j]]),
 // and the step's gradients are
-//   dC_t = H_t dy_t, dB_t = Lam_t x_t, dx_t = Lam_t^T B_t, dd_t[j] = <Lam_t[idx_{s_t}[j]], H_{t-1}[j]>.
+//   dC_t = Re(H_t conj(dy_t)), dB_t = Re(Lam_t) x_t, dx_t = Re(Lam_t)^T B_t,
+//   dd_t[j] = sum_p Lam_t[idx_{s_t}[j]][p] conj(H_{t-1}[j][p]).
 //
 // One block per (batch, head) sequence. A forward sweep stores the state every
 // kTb steps (O(L N P / kTb) memory, O(L N) for kTb >= P); the reverse sweep
 // recomputes each kTb-step stretch from its checkpoint into a per-sequence
 // scratch and walks it backwards. Three N x P buffers in shared memory (rows
-// padded by one word) hold the adjoint, H_t and H_{t-1}.
+// padded by one element) hold the adjoint, H_t and H_{t-1}.
 #include "launch.h"
 
 namespace pdssm {
@@ -39,10 +42,11 @@ struct BParams {
   const int32_t *off;  // [K][N+1]
   const int32_t *src;  // [K][N]
   const void *logits, *d, *B, *C, *x, *dy;
-  const float *h0, *dh_final;
-  float *ckpt;     // [Bt*H][nCk][N][P]
-  float *scratch;  // [Bt*H][kTb][N][P]
-  float *dlogits, *dd, *dB, *dC, *dx, *dh0;
+  const void *h0, *dh_final;  // state type
+  void *ckpt;     // [Bt*H][nCk][N][P], state type
+  void *scratch;  // [Bt*H][kTb][N][P], state type
+  float *dlogits, *dB, *dC, *dx;
+  void *dd, *dh0;  // state type
   uint32_t *err;
 };
 
@@ -50,22 +54,44 @@ __device__ __forceinline__ float ld_flag(const void *p, int64_t i, int bf16) {
   return bf16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]) : static_cast<const float *>(p)[i];
 }
 
-template <typename TD, typename TIn>
+// Conjugates and real parts of the state type (identities for a real state).
+__device__ __forceinline__ float conj_of(float v) { return v; }
+__device__ __forceinline__ float2 conj_of(float2 v) { return make_float2(v.x, -v.y); }
+__device__ __forceinline__ float re_of(float v) { return v; }
+__device__ __forceinline__ float re_of(float2 v) { return v.x; }
+// c + a conj(b)
+__device__ __forceinline__ float fma_conj(float a, float b, float c) { return fmaf(a, b, c); }
+__device__ __forceinline__ float2 fma_conj(float2 a, float2 b, float2 c) {
+  return make_float2(fmaf(a.x, b.x, fmaf(a.y, b.y, c.x)), fmaf(a.y, b.x, fmaf(-a.x, b.y, c.y)));
+}
+// c + Re(a conj(b))
+__device__ __forceinline__ float fma_re_conj(float a, float b, float c) { return fmaf(a, b, c); }
+__device__ __forceinline__ float fma_re_conj(float2 a, float2 b, float c) { return fmaf(a.x, b.x, fmaf(a.y, b.y, c)); }
+
+// dy as stored: f32 / bf16 for a real state, complex64 for a complex one.
+__device__ __forceinline__ void ld_dy(const void *p, int64_t i, int bf16, float *v) { *v = ld_flag(p, i, bf16); }
+__device__ __forceinline__ void ld_dy(const void *p, int64_t i, int, float2 *v) {
+  *v = static_cast<const float2 *>(p)[i];
+}
+
+template <bool CPLX, typename TD, typename TIn>
 __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
+  using NT = Num<CPLX>;
+  using T = typename NT::T;
   extern __shared__ __align__(16) unsigned char smem[];
   const int N = (int)a.N, P = (int)a.P, K = (int)a.K, PS = P + 1;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
 
-  float *buf0 = reinterpret_cast<float *>(smem);  // three [N][PS] buffers
-  float *buf1 = buf0 + N * PS;
-  float *buf2 = buf1 + N * PS;
-  float *dsh = buf2 + N * PS;  // [N]
-  float *Bsh = dsh + N;        // [N]
-  float *Csh = Bsh + N;        // [N]
-  float *xsh = Csh + N;        // [P]
-  float *dysh = xsh + P;       // [P]
-  float *dpi = dysh + P;       // [K]
+  T *buf0 = reinterpret_cast<T *>(smem);  // three [N][PS] buffers
+  T *buf1 = buf0 + N * PS;
+  T *buf2 = buf1 + N * PS;
+  T *dsh = buf2 + N * PS;  // [N]
+  T *dysh = dsh + N;       // [P]
+  float *Bsh = reinterpret_cast<float *>(dysh + P);  // [N]
+  float *Csh = Bsh + N;                              // [N]
+  float *xsh = Csh + N;                              // [P]
+  float *dpi = xsh + P;                              // [K]
   int *offsh = reinterpret_cast<int *>(dpi + K);  // [N+1] preimage lists of the step's entry
   int *srcsh = offsh + N + 1;                     // [N]
   uint8_t *idxsh = reinterpret_cast<uint8_t *>(srcsh + N);  // [K][N] dictionary
@@ -77,8 +103,11 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
   const TIn *Bg = static_cast<const TIn *>(a.B);
   const TIn *Cg = static_cast<const TIn *>(a.C);
   const TIn *xg = static_cast<const TIn *>(a.x);
-  float *ck = a.ckpt + bh * a.nCk * N * P;
-  float *scr = a.scratch + bh * (int64_t)kTb * N * P;
+  const T *h0g = static_cast<const T *>(a.h0);
+  const T *dhg = static_cast<const T *>(a.dh_final);
+  T *ddg = static_cast<T *>(a.dd);
+  T *ck = static_cast<T *>(a.ckpt) + bh * a.nCk * N * P;
+  T *scr = static_cast<T *>(a.scratch) + bh * (int64_t)kTb * N * P;
 
   // element loop over a dense [N][P] array: thread tid starts at element tid
   const int di = kBT / P, dp = kBT - di * P;
@@ -99,7 +128,8 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
   // tid of d, B, C (and of the entry's preimage lists), of x and dy (N, P <= 128 <
   // kBT, so one entry each) and s.
   struct Vec {
-    float d, B, C, x, dy;
+    T d, dy;
+    float B, C, x;
     int src, off, st;
   };
   auto fetch = [&](int64_t t, bool rev) {
@@ -107,7 +137,7 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
     const int64_t row = row_of(t);
     v.st = load_s(row);
     if (tid < N) {
-      v.d = to_f32(dg[row * N + tid]);
+      v.d = LoadD<CPLX, TD>::ld(dg + row * N + tid);
       v.B = to_f32(Bg[row * N + tid]);
       if (rev) v.C = to_f32(Cg[row * N + tid]);
       else v.src = a.src[(kh + v.st) * N + tid];
@@ -115,7 +145,7 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
     if (!rev && tid <= N) v.off = a.off[(kh + v.st) * (N + 1) + tid];
     if (tid < P) {
       v.x = to_f32(xg[row * P + tid]);
-      if (rev) v.dy = ld_flag(a.dy, row * P + tid, a.dy_bf16);
+      if (rev) ld_dy(a.dy, row * P + tid, a.dy_bf16, &v.dy);
     }
     return v;
   };
@@ -133,27 +163,27 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
     }
   };
   // Hn = A_t Hc + B_t x_t^T (after commit of step t's vectors and a barrier)
-  auto step_fwd = [&](const float *Hc, float *Hn) {
+  auto step_fwd = [&](const T *Hc, T *Hn) {
     FOR_NP(i, p) {
-      float acc = Bsh[i] * xsh[p];
+      T acc = NT::from_real(Bsh[i] * xsh[p]);
       const int r1 = offsh[i + 1];
       for (int r = offsh[i]; r < r1; ++r) {
         const int j = srcsh[r];
-        acc = fmaf(dsh[j], Hc[j * PS + p], acc);
+        acc = NT::fma(dsh[j], Hc[j * PS + p], acc);
       }
       Hn[i * PS + p] = acc;
     }
   };
-  auto store_dense = [&](const float *S, float *g) {
+  auto store_dense = [&](const T *S, T *g) {
     FOR_NP(i, p) { g[i * P + p] = S[i * PS + p]; }
   };
-  auto load_dense = [&](const float *g, float *S) {
+  auto load_dense = [&](const T *g, T *S) {
     FOR_NP(i, p) { S[i * PS + p] = g[i * P + p]; }
   };
 
   // ---- forward sweep: checkpoints every kTb steps
-  float *Hc = buf0, *Hn = buf1;
-  FOR_NP(i, p) { Hc[i * PS + p] = a.h0 ? a.h0[(bh * N + i) * P + p] : 0.f; }
+  T *Hc = buf0, *Hn = buf1;
+  FOR_NP(i, p) { Hc[i * PS + p] = h0g ? h0g[(bh * N + i) * P + p] : NT::zero(); }
   Vec nv = fetch(0, false);
   for (int64_t t = 0; t < a.L; ++t) {
     __syncthreads();  // Hc complete; the staged vectors are no longer read
@@ -162,15 +192,15 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
     if (t + 1 < a.L) nv = fetch(t + 1, false);
     __syncthreads();
     step_fwd(Hc, Hn);
-    float *tmp = Hc;
+    T *tmp = Hc;
     Hc = Hn;
     Hn = tmp;
   }
 
   // ---- reverse sweep
-  float *Lam = buf2;
+  T *Lam = buf2;
   __syncthreads();
-  FOR_NP(i, p) { Lam[i * PS + p] = a.dh_final ? a.dh_final[(bh * N + i) * P + p] : 0.f; }
+  FOR_NP(i, p) { Lam[i * PS + p] = dhg ? dhg[(bh * N + i) * P + p] : NT::zero(); }
   for (int64_t c = a.nCk - 1; c >= 0; --c) {
     const int64_t t0 = c * kTb, t1 = t0 + kTb < a.L ? t0 + kTb : a.L;
     // recompute the stretch: scratch[t - t0] = H_{t-1}; Hc ends as H_{t1-1}
@@ -187,11 +217,11 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
       if (t + 1 < t1) nv = fetch(t + 1, false);
       __syncthreads();
       step_fwd(Hc, Hn);
-      float *tmp = Hc;
+      T *tmp = Hc;
       Hc = Hn;
       Hn = tmp;
     }
-    float *Hp = Hn;  // receives H_{t-1}
+    T *Hp = Hn;  // receives H_{t-1}
     Vec rv = fetch(t1 - 1, true);
     for (int64_t t = t1 - 1; t >= t0; --t) {
       const int64_t row = row_of(t);
@@ -202,36 +232,37 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
       load_dense(scr + (t - t0) * N * P, Hp);
       __syncthreads();
       // [B] Lam_t = Lam'_t + C_t dy_t^T
-      FOR_NP(i, p) { Lam[i * PS + p] = fmaf(Csh[i], dysh[p], Lam[i * PS + p]); }
+      FOR_NP(i, p) { Lam[i * PS + p] = NT::fma_r(Csh[i], dysh[p], Lam[i * PS + p]); }
       __syncthreads();
-      // [C] dB_t, dC_t, and per entry k: <Lam_t[idx_k[j]], H_{t-1}[j]> (dd_t at k = s_t, dpi_t[k])
+      // [C] dB_t, dC_t, and per entry k: sum_p Lam_t[idx_k[j]][p] conj(H_{t-1}[j][p])
+      // (dd_t at k = s_t, dpi_t[k])
       if (tid < N) {
         float acc = 0.f;
-        for (int p = 0; p < P; ++p) acc = fmaf(Lam[tid * PS + p], xsh[p], acc);
+        for (int p = 0; p < P; ++p) acc = fmaf(re_of(Lam[tid * PS + p]), xsh[p], acc);
         a.dB[row * N + tid] = acc;
       }
       if (tid >= 128 && tid - 128 < N) {
         const int i = tid - 128;
         float acc = 0.f;
-        for (int p = 0; p < P; ++p) acc = fmaf(Hc[i * PS + p], dysh[p], acc);
+        for (int p = 0; p < P; ++p) acc = fma_re_conj(Hc[i * PS + p], dysh[p], acc);
         a.dC[row * N + i] = acc;
       }
       for (int k = warp; k < K; k += kBT / 32) {
         float part = 0.f;
         for (int j = lane; j < N; j += 32) {
           const int r = idxsh[k * N + j];
-          float q = 0.f;
+          T q = NT::zero();
 #pragma unroll 4
-          for (int p = 0; p < P; ++p) q = fmaf(Lam[r * PS + p], Hp[j * PS + p], q);
-          if (k == st) a.dd[row * N + j] = q;
-          part = fmaf(dsh[j], q, part);
+          for (int p = 0; p < P; ++p) q = fma_conj(Lam[r * PS + p], Hp[j * PS + p], q);
+          if (k == st) ddg[row * N + j] = q;
+          part = fma_re_conj(dsh[j], q, part);  // Re(conj(q) d_j)
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
         if (lane == 0) dpi[k] = part;
       }
       __syncthreads();
-      // [D] logits through the tempered softmax (warp 0); Lam'_{t-1} = A_t^T Lam_t into
+      // [D] logits through the tempered softmax (warp 0); Lam'_{t-1} = A_t^H Lam_t into
       // Hc's buffer; dx_t
       if (warp == 0 && a.dlogits) {
         const float v0 = lane < K ? ld_flag(a.logits, row * K + lane, a.logits_bf16) / a.tau : -INFINITY;
@@ -251,15 +282,15 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
         if (lane < K) a.dlogits[row * K + lane] = p0 * (g0 - dot) / a.tau;
         if (lane + 32 < K) a.dlogits[row * K + lane + 32] = p1 * (g1 - dot) / a.tau;
       }
-      FOR_NP(j, p) { Hc[j * PS + p] = dsh[j] * Lam[idxsh[st * N + j] * PS + p]; }
+      FOR_NP(j, p) { Hc[j * PS + p] = NT::mul(conj_of(dsh[j]), Lam[idxsh[st * N + j] * PS + p]); }
       if (tid >= 32 && tid - 32 < P) {
         const int p = tid - 32;
         float acc = 0.f;
-        for (int i = 0; i < N; ++i) acc = fmaf(Lam[i * PS + p], Bsh[i], acc);
+        for (int i = 0; i < N; ++i) acc = fmaf(re_of(Lam[i * PS + p]), Bsh[i], acc);
         a.dx[row * P + p] = acc;
       }
       // rotate: the new adjoint is in Hc's buffer, H_{t-1} becomes the next step's H_t
-      float *old = Lam;
+      T *old = Lam;
       Lam = Hc;
       Hc = Hp;
       Hp = old;
@@ -267,15 +298,18 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
   }
   __syncthreads();
   if (a.dh0) {
-    FOR_NP(i, p) { a.dh0[(bh * N + i) * P + p] = Lam[i * PS + p]; }
+    T *dh0g = static_cast<T *>(a.dh0);
+    FOR_NP(i, p) { dh0g[(bh * N + i) * P + p] = Lam[i * PS + p]; }
   }
 #undef FOR_NP
 }
 
 }  // namespace
 
-size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t K) {
-  return (size_t)(3 * N * (P + 1) + 3 * N + 2 * P + K) * 4 + (size_t)(2 * N + 1) * 4 + (size_t)(K * N);
+size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t K, bool cplx) {
+  const size_t es = cplx ? 8 : 4;
+  return (size_t)(3 * N * (P + 1) + N + P) * es + (size_t)(2 * N + P + K) * 4 + (size_t)(2 * N + 1) * 4 +
+         (size_t)(K * N);
 }
 
 int64_t scan_bwd_checkpoints(int64_t L) { return (L + kTb - 1) / kTb; }
@@ -295,11 +329,16 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs &s, cudaStream_t st) {
   a.dlogits = s.dlogits; a.dd = s.dd; a.dB = s.dB; a.dC = s.dC; a.dx = s.dx; a.dh0 = s.dh0;
   a.err = s.ws.err;
   a.head_dicts = s.head_dicts;
-  const size_t smem = scan_bwd_smem_bytes(s.N, s.P, s.K);
-  auto kern = s.d_t == PDSSM_BF16 ? (s.in_t == PDSSM_BF16 ? scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16>
-                                                          : scan_bwd_kernel<__nv_bfloat16, float>)
-                                  : (s.in_t == PDSSM_BF16 ? scan_bwd_kernel<float, __nv_bfloat16>
-                                                          : scan_bwd_kernel<float, float>);
+  const bool cplx = s.d_t == PDSSM_C64;
+  const size_t smem = scan_bwd_smem_bytes(s.N, s.P, s.K, cplx);
+  void (*kern)(BParams);
+  if (cplx)
+    kern = s.in_t == PDSSM_BF16 ? scan_bwd_kernel<true, float2, __nv_bfloat16> : scan_bwd_kernel<true, float2, float>;
+  else if (s.d_t == PDSSM_BF16)
+    kern = s.in_t == PDSSM_BF16 ? scan_bwd_kernel<false, __nv_bfloat16, __nv_bfloat16>
+                                : scan_bwd_kernel<false, __nv_bfloat16, float>;
+  else
+    kern = s.in_t == PDSSM_BF16 ? scan_bwd_kernel<false, float, __nv_bfloat16> : scan_bwd_kernel<false, float, float>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if ((e = trace_before(st, "scan_bwd")) != cudaSuccess) return e;

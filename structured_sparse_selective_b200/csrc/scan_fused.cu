@@ -46,11 +46,14 @@
 //
 // Roles (352 threads, 11 warps):
 //   warps 0-5   three prep pairs; pair w prepares sub-chunks w, w + 3, ... into
-//               operand stage (sub-chunk mod nst). In a pair, warp A (even)
-//               runs the suffix recursion Psi_sigma (B-hat scatter, and at its
-//               end Phi_{T-1}: the carry records and S_a's order); warp B (odd)
-//               runs the readout recursion R_sigma = A_{sigma+1}^T R_{sigma+1}
-//               (the G entries, and one step further, Ct = R_{-1}).
+//               operand stage (sub-chunk mod nst). Both warps of a pair run
+//               "walkers": walker (sigma, j) starts at row j after step sigma and
+//               follows it through the later steps' maps, carrying B_sigma[j] times
+//               the d it passes; it meets C_tau on its way (its part of
+//               G[tau][sigma]) and ends at Psi_sigma(j) (its part of Bh_sigma).
+//               The walkers of sigma = -1 give Ct and Phi_{T-1} (the carry records
+//               and S_a's order). Warp X (even) also orders S_{a+1}; warp Y (odd)
+//               orders S_a and runs the sigma = -1 walk.
 //   warps 6-9   carry the state (one per tensor-memory lane quarter) and write y
 //               two sub-chunks behind the carry.
 //   warp 10     one thread issues the MMAs.

@@ -1,6 +1,6 @@
 """Parity of the backward pass (pdssm_scan_bwd through the C ABI) with the backward
-oracle (oracle/backward.py) on seeded workloads: every gradient, per (batch, head)
-slice, within 1e-4 of the slice's largest value."""
+oracle (oracle/backward.py) on seeded workloads, real and complex states: every
+gradient, per (batch, head) slice, within 1e-4 of the slice's largest value."""
 import numpy as np
 import pytest
 import torch
@@ -12,10 +12,16 @@ from oracle import backward as bwd
 TOL = 1e-4
 
 
+def _np64(t):
+    """fp64 (or complex128) numpy copy of a tensor"""
+    t = t.detach().cpu()
+    return (t.to(torch.complex128) if t.is_complex() else t.double()).numpy()
+
+
 def _slices(t):
-    """[Bt, L, H, X] -> [Bt*H, L, X] fp64 numpy"""
+    """[Bt, L, H, X] -> [Bt*H, L, X] fp64 / complex128 numpy"""
     Bt, L, H, X = t.shape
-    return t.permute(0, 2, 1, 3).reshape(Bt * H, L, X).double().cpu().numpy()
+    return _np64(t.permute(0, 2, 1, 3).reshape(Bt * H, L, X))
 
 
 def _rel(got, ref):
@@ -35,9 +41,10 @@ def _run(recipe, kw, dev, seed=0, with_h0=True, with_dh=True, with_logits=True, 
     Bt, L, H, N = inp["B"].shape
     P = inp["x"].shape[-1]
     gen = torch.Generator().manual_seed(100 + seed)
-    dy = torch.randn(Bt, L, H, P, generator=gen).to(fwd["y"].dtype)
-    h0 = torch.randn(Bt, H, N, P, generator=gen) if with_h0 else None
-    dh = torch.randn(Bt, H, N, P, generator=gen) if with_dh else None
+    sdt = torch.complex64 if sp.state_complex else torch.float32  # complex draws have both parts
+    dy = torch.randn(Bt, L, H, P, generator=gen, dtype=sdt).to(fwd["y"].dtype)
+    h0 = torch.randn(Bt, H, N, P, generator=gen, dtype=sdt) if with_h0 else None
+    dh = torch.randn(Bt, H, N, P, generator=gen, dtype=sdt) if with_dh else None
     out = pd.backward(g["logits"] if with_logits else None, fwd["s"], g["idx"], g["d"], g["B"], g["C"], g["x"],
                       dy.to(dev), h0=None if h0 is None else h0.to(dev), dh_final=None if dh is None else dh.to(dev),
                       tau=tau)
@@ -48,14 +55,19 @@ def _run(recipe, kw, dev, seed=0, with_h0=True, with_dh=True, with_logits=True, 
         idx_ref = np.stack([idx_ref[i % H] for i in range(Bt * H)])
     ref = bwd.scan_backward(_slices(inp["logits"]), idx_ref, _slices(inp["d"]), _slices(inp["B"]),
                             _slices(inp["C"]), _slices(inp["x"]), _slices(dy),
-                            None if dh is None else dh.reshape(S, N, P).double().numpy(),
-                            None if h0 is None else h0.reshape(S, N, P).double().numpy(), tau=tau)
+                            None if dh is None else _np64(dh.reshape(S, N, P)),
+                            None if h0 is None else _np64(h0.reshape(S, N, P)), tau=tau)
     s_slices = fwd["s"].cpu().permute(0, 2, 1).reshape(S, L).numpy()
     assert np.array_equal(s_slices, ref["s"])
     errs = {}
     for k in ("dd", "dB", "dC", "dx") + (("dlogits",) if with_logits else ()):
-        errs[k] = _rel(_slices(out[k].cpu()), ref[k])
-    errs["dh0"] = _rel(out["dh0"].cpu().reshape(S, N, P).double().numpy(), ref["dh0"])
+        errs[k] = _rel(_slices(out[k]), ref[k])
+    errs["dh0"] = _rel(_np64(out["dh0"].reshape(S, N, P)), ref["dh0"])
+    if sp.state_complex:  # the complex gradients carry imaginary parts, the rest are real
+        assert out["dd"].dtype == torch.complex64 and out["dh0"].dtype == torch.complex64
+        assert np.abs(ref["dd"].imag).max() > 1e-3 * np.abs(ref["dd"]).max()
+        assert np.abs(ref["dh0"].imag).max() > 1e-3 * np.abs(ref["dh0"]).max()
+        assert all(out[k].dtype == torch.float32 for k in ("dB", "dC", "dx"))
     return errs
 
 
@@ -67,6 +79,8 @@ def _run(recipe, kw, dev, seed=0, with_h0=True, with_dh=True, with_logits=True, 
     ("z5", dict(batch=3, seqlen=37)),
     ("lm", dict(batch=1, seqlen=70, heads=2)),
     ("long", dict(batch=1, seqlen=53, heads=2)),
+    ("complex", dict(batch=1, seqlen=45, heads=2, N=16, P=8, K=8)),
+    ("complex", dict(batch=2, seqlen=17, heads=1, N=40, P=24, K=12)),
 ])
 def test_backward_matches_oracle(cuda_device, recipe, kw):
     errs = _run(recipe, kw, cuda_device)
@@ -85,6 +99,21 @@ def test_backward_maximum_sizes(cuda_device):
     """N = P = 128, K = 64: the largest shared-memory footprint of the backward block."""
     sp = dict(batch=1, seqlen=20, heads=1, N=128, P=128, K=64)
     errs = _run("tiny", sp, cuda_device, seed=4)
+    assert all(v <= TOL for v in errs.values()), errs
+
+
+@pytest.mark.gpu
+def test_backward_complex_maximum_sizes(cuda_device):
+    """Complex state at N = 128, P = 64, K = 64 (the complex-diagonal layer's head shape): the
+    largest complex footprint the backward block holds (three 128 x 65 complex buffers)."""
+    errs = _run("complex", dict(batch=1, seqlen=20, heads=1), cuda_device, seed=8)
+    assert all(v <= TOL for v in errs.values()), errs
+
+
+@pytest.mark.gpu
+def test_backward_complex_without_initial_state_or_logits(cuda_device):
+    errs = _run("complex", dict(batch=1, seqlen=33, heads=2, N=32, P=16, K=8), cuda_device, seed=9,
+                with_h0=False, with_dh=False, with_logits=False)
     assert all(v <= TOL for v in errs.values()), errs
 
 
@@ -123,7 +152,8 @@ def test_backward_reproduces_the_hand_worked_gradients(cuda_device, name):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("recipe,kw", [("lm", dict(batch=2, seqlen=40, heads=3)), ("tiny", dict(heads=2, seqlen=50))])
+@pytest.mark.parametrize("recipe,kw", [("lm", dict(batch=2, seqlen=40, heads=3)), ("tiny", dict(heads=2, seqlen=50)),
+                                       ("complex", dict(batch=1, seqlen=30, heads=3, N=16, P=8, K=8))])
 def test_backward_with_per_head_dictionaries(cuda_device, recipe, kw):
     errs = _run(recipe, kw, cuda_device, seed=6, head_dicts=True)
     assert all(v <= TOL for v in errs.values()), errs
