@@ -29,7 +29,7 @@ namespace pdssm {
 
 namespace {
 
-constexpr int kBT = 256;  // threads per block
+constexpr int kBT = 512;  // threads per block (two blocks per SM: at most 64 registers a thread)
 constexpr int kTb = 16;   // steps between checkpoints
 
 struct BParams {
@@ -75,7 +75,7 @@ __device__ __forceinline__ void ld_dy(const void *p, int64_t i, int, float2 *v) 
 }
 
 template <bool CPLX, typename TD, typename TIn>
-__global__ void __launch_bounds__(kBT) scan_bwd_kernel(BParams a) {
+__global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
   using NT = Num<CPLX>;
   using T = typename NT::T;
   extern __shared__ __align__(16) unsigned char smem[];

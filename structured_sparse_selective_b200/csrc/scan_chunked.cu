@@ -10,15 +10,17 @@
 // Scannable Models abstract): (idx, val) o (idx', val') = (idx[idx'], val[idx']*val').
 //
 // A block owns up to 32 columns of one (batch, head) state and all N rows, in
-// shared memory (the gather index is dynamic). Its threads are RG row groups of
-// 32 columns (RG = 1, 2 or 8, so that a thread has at most 16 rows): thread
-// (g, p) updates rows i = g, g + RG, ... of column p, so a warp always reads one
-// state row across 32 consecutive columns (no bank conflicts) and the CSR work
-// of a step is spread over the row groups. New rows are held in registers until
-// every thread has read the old state, so one state buffer suffices. Per-step
-// vectors (d, B, C, x and the selected entry's preimage lists) are fetched into
-// registers one step ahead and staged in shared memory; a column's output is
-// the sum of the row groups' parts.
+// shared memory (the gather index is dynamic). In phases B and C its threads are
+// RG row groups of 32 columns (RG = 1, 2 or 8, so that a thread has at most 16
+// rows): thread (g, p) updates rows i = g, g + RG, ... of column p, so a warp
+// always reads one state row across 32 consecutive columns (no bank conflicts).
+// In phase A, the per-token recurrence, a thread owns a 16-byte run of columns
+// (4 real or 2 complex) of its rows instead, so that each row's preimage list is
+// read once for the whole run and the state moves in 16-byte loads. New rows are
+// held in registers until every thread has read the old state, so one state
+// buffer suffices. Per-step vectors (d, B, C, x and the selected entry's preimage
+// lists) are fetched into registers one step ahead and staged in shared memory; a
+// column's output is the sum of the row groups' parts.
 #include <algorithm>
 
 #include "launch.h"
@@ -64,20 +66,53 @@ struct StepVec {  // one thread's share of a step's vectors (entry j = tid)
   int src, off, st;
 };
 
+// Columns a phase-A thread owns: one 16-byte run (4 real or 2 complex values), so
+// that the preimage lists of a row are read once for several columns and eight
+// consecutive lanes read 128 contiguous bytes of a state row (no bank conflicts).
+template <typename T>
+struct ColRun {
+  static constexpr int VW = 16 / (int)sizeof(T);  // columns per thread
+  static constexpr int TPR = kPB / VW;            // threads per row group
+  static constexpr int MR = 16 / VW;              // rows per thread at most (RG * MR >= N)
+};
+
+__device__ __forceinline__ float shfl_xor(float v, int o) { return __shfl_xor_sync(0xffffffffu, v, o); }
+__device__ __forceinline__ float2 shfl_xor(float2 v, int o) {
+  return make_float2(__shfl_xor_sync(0xffffffffu, v.x, o), __shfl_xor_sync(0xffffffffu, v.y, o));
+}
+
+__device__ __forceinline__ void ld_run(const float *p, float (&v)[4]) {
+  const float4 w = *reinterpret_cast<const float4 *>(p);
+  v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
+}
+__device__ __forceinline__ void ld_run(const float2 *p, float2 (&v)[2]) {
+  const float4 w = *reinterpret_cast<const float4 *>(p);
+  v[0] = make_float2(w.x, w.y); v[1] = make_float2(w.z, w.w);
+}
+__device__ __forceinline__ void st_run(float *p, const float (&v)[4]) {
+  *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void st_run(float2 *p, const float2 (&v)[2]) {
+  *reinterpret_cast<float4 *>(p) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+}
+
+// Threads: RG row groups of TPR threads; thread (g, cl) updates rows g, g + RG, ...
+// of columns [cl * VW, cl * VW + VW) of the block's kPB columns.
 template <int RG, bool CPLX, typename TD, typename TIn>
-__global__ void __launch_bounds__(RG * kPB) phase_a_kernel(KParams a) {
+__global__ void __launch_bounds__(RG * ColRun<typename Num<CPLX>::T>::TPR) phase_a_kernel(KParams a) {
   using Nm = Num<CPLX>;
   using T = typename Nm::T;
-  constexpr int NT = RG * kPB;
+  constexpr int VW = ColRun<T>::VW, TPR = ColRun<T>::TPR, MR = ColRun<T>::MR, NT = RG * TPR, NW = NT / 32;
+  static_assert(NT % 32 == 0 && 32 % TPR == 0, "row groups tile whole warps");
   extern __shared__ __align__(16) unsigned char smem[];
-  const int N = (int)a.N, tid = threadIdx.x, pl = tid % kPB, g = tid / kPB;
+  const int N = (int)a.N, tid = threadIdx.x, cl = tid % TPR, g = tid / TPR, pc = cl * VW;
   const int64_t c = blockIdx.x / a.nPB, pb = blockIdx.x % a.nPB, h = blockIdx.y, b = blockIdx.z;
   const int p0 = (int)(pb * kPB), P = (int)min((int64_t)kPB, a.P - p0), PG = (int)a.P;
   const int64_t t0 = c * a.T, t1 = min(t0 + a.T, a.L);
 
   T *Hs = reinterpret_cast<T *>(smem);  // [N][kPB]
-  T *ysh = Hs + N * kPB;                // [RG][kPB]
-  T *dsh = ysh + RG * kPB;              // [N]
+  T *ysh = Hs + N * kPB;                // [NW][kPB] per-warp parts of the output
+  T *dsh = ysh + NW * kPB;              // [N]
   float *Bsh = reinterpret_cast<float *>(dsh + N);
   float *Csh = Bsh + N;
   float *xsh = Csh + N;                 // [kPB]
@@ -94,7 +129,7 @@ __global__ void __launch_bounds__(RG * kPB) phase_a_kernel(KParams a) {
   int pidx = tid;  // chunk pair entry tid (tid < N)
   T pval = Nm::one();
 
-  // NT >= 2N: thread tid fetches entry tid of each vector (and off[N], x[tid])
+  // NT > N: thread tid fetches entry tid of each vector (and off[N], x[tid])
   auto fetch = [&](int64_t t) {
     StepVec<T> v;
     const int64_t row = (b * a.L + t) * a.H + h;
@@ -119,13 +154,13 @@ __global__ void __launch_bounds__(RG * kPB) phase_a_kernel(KParams a) {
     if (tid <= N) offsh[tid] = v.off;
     if (tid < kPB) xsh[tid] = v.x;
   };
-  // output of step t from the row groups' parts
+  // output of step t from the warps' parts (fixed order)
   auto finish_y = [&](int64_t t) {
-    if (g == 0 && pl < P) {
-      T acc = ysh[pl];
+    if (tid < P) {
+      T acc = ysh[tid];
 #pragma unroll
-      for (int q = 1; q < RG; ++q) acc = Nm::add(acc, ysh[q * kPB + pl]);
-      yl[((b * a.L + t) * a.H + h) * PG + p0 + pl] = acc;
+      for (int w = 1; w < NW; ++w) acc = Nm::add(acc, ysh[w * kPB + tid]);
+      yl[((b * a.L + t) * a.H + h) * PG + p0 + tid] = acc;
     }
   };
 
@@ -141,40 +176,55 @@ __global__ void __launch_bounds__(RG * kPB) phase_a_kernel(KParams a) {
       pval = Nm::mul(dsh[pidx], pval);
       pidx = a.idx[(int64_t)st * N + pidx];
     }
-    T nv[kMaxRows];
-    T yp = Nm::zero();
-    const float xp = xsh[pl];
+    T nv[MR][VW];
+    T yp[VW];
+    float xv[VW];
 #pragma unroll
-    for (int m = 0; m < kMaxRows; ++m) {
+    for (int e = 0; e < VW; ++e) {
+      yp[e] = Nm::zero();
+      xv[e] = xsh[pc + e];
+    }
+#pragma unroll
+    for (int m = 0; m < MR; ++m) {
       const int i = g + RG * m;
       if (i < N) {
-        T acc = Nm::from_real(Bsh[i] * xp);
-        // sources in increasing order; the first two outside the loop so that
-        // their loads overlap (most rows have at most two)
+        const float bi = Bsh[i];
+#pragma unroll
+        for (int e = 0; e < VW; ++e) nv[m][e] = Nm::from_real(bi * xv[e]);
+        // sources in increasing order (fixed summation order); the first two outside
+        // the loop so that their loads overlap (most rows have at most two)
+        auto add_src = [&](int j) {
+          const T dj = dsh[j];
+          T hv[VW];
+          ld_run(Hs + j * kPB + pc, hv);
+#pragma unroll
+          for (int e = 0; e < VW; ++e) nv[m][e] = Nm::fma(dj, hv[e], nv[m][e]);
+        };
         const int r0 = offsh[i], r1 = offsh[i + 1];
         if (r0 < r1) {
-          const int ja = srcsh[r0];
-          acc = Nm::fma(dsh[ja], Hs[ja * kPB + pl], acc);
+          add_src(srcsh[r0]);
           if (r0 + 1 < r1) {
-            const int jb = srcsh[r0 + 1];
-            acc = Nm::fma(dsh[jb], Hs[jb * kPB + pl], acc);
-            for (int r = r0 + 2; r < r1; ++r) {
-              const int j = srcsh[r];
-              acc = Nm::fma(dsh[j], Hs[j * kPB + pl], acc);
-            }
+            add_src(srcsh[r0 + 1]);
+            for (int r = r0 + 2; r < r1; ++r) add_src(srcsh[r]);
           }
         }
-        nv[m] = acc;
-        yp = Nm::fma_r(Csh[i], acc, yp);
+        const float ci = Csh[i];
+#pragma unroll
+        for (int e = 0; e < VW; ++e) yp[e] = Nm::fma_r(ci, nv[m][e], yp[e]);
       }
     }
+    // the row groups of a warp share columns: sum their parts, one per warp to memory
+#pragma unroll
+    for (int o = TPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < VW; ++e) yp[e] = Nm::add(yp[e], shfl_xor(yp[e], o));
     __syncthreads();  // every read of the old state and of the staged vectors is done
 #pragma unroll
-    for (int m = 0; m < kMaxRows; ++m) {
+    for (int m = 0; m < MR; ++m) {
       const int i = g + RG * m;
-      if (i < N) Hs[i * kPB + pl] = nv[m];
+      if (i < N) st_run(Hs + i * kPB + pc, nv[m]);
     }
-    ysh[g * kPB + pl] = yp;
+    if ((tid & 31) < TPR) st_run(ysh + (tid >> 5) * kPB + pc, yp);
     if (t + 1 < t1) {
       commit(nxt);
       st = nxt.st;
@@ -186,8 +236,10 @@ __global__ void __launch_bounds__(RG * kPB) phase_a_kernel(KParams a) {
   // chunk-end local state and chunk pair
   const int64_t slot = (b * a.H + h) * a.nC + c;
   T *cs = static_cast<T *>(a.chunk_state) + slot * N * PG;
-  if (pl < P)
-    for (int i = g; i < N; i += RG) cs[i * PG + p0 + pl] = Hs[i * kPB + pl];
+  for (int e = tid; e < N * kPB; e += NT) {
+    const int i = e / kPB, p = e % kPB;
+    if (p < P) cs[i * PG + p0 + p] = Hs[e];
+  }
   if (pb != 0 || tid >= N) return;  // every column block computes the pair; one writes it
   a.chunk_idx[slot * N + tid] = pidx;
   static_cast<T *>(a.chunk_val)[slot * N + tid] = pval;
@@ -438,12 +490,15 @@ cudaError_t run_chunked_rg(const ScanArgs &s, cudaStream_t st) {
   using T = typename Num<CPLX>::T;
   const KParams k = make_params(s);
   const size_t ts = sizeof(T), N = (size_t)s.N;
-  const size_t smem_a = N * kPB * ts + RG * kPB * ts + N * ts + 2 * N * 4 + kPB * 4 + (2 * N + 1) * 4;
+  // phase A's row groups (threads > N, RGA * MR >= N): real 32 / 8 / 4, complex
+  // 16 / 4 / 2 for N <= 128 / 32 / 16
+  constexpr int RGA = ColRun<T>::TPR == 8 ? (RG == 8 ? 32 : RG == 2 ? 8 : 4) : (RG == 8 ? 16 : RG == 2 ? 4 : 2);
+  constexpr int NTA = RGA * ColRun<T>::TPR;
+  const size_t smem_a = N * kPB * ts + (NTA / 32) * kPB * ts + N * ts + 2 * N * 4 + kPB * 4 + (2 * N + 1) * 4;
   const size_t smem_b = N * kPB * ts + N * ts + N * 4 + (2 * N + 1) * 4;
   const size_t smem_c = N * kPB * ts + RG * kPB * ts + 2 * N * ts + N * 4;
   const dim3 grid_chunks((unsigned)(s.nC * k.nPB), (unsigned)s.H, (unsigned)s.Bt);
-  cudaError_t e = launch_dyn(phase_a_kernel<RG, CPLX, TD, TIn>, "chunked_phase_a", grid_chunks, RG * kPB, smem_a,
-                             st, k);
+  cudaError_t e = launch_dyn(phase_a_kernel<RGA, CPLX, TD, TIn>, "chunked_phase_a", grid_chunks, NTA, smem_a, st, k);
   if (e != cudaSuccess) return e;
   e = launch_dyn(phase_b_kernel<RG, CPLX>, "chunked_phase_b", dim3((unsigned)(s.H * k.nPB), (unsigned)s.Bt),
                  RG * kPB, smem_b, st, k);
