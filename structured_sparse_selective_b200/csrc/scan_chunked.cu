@@ -362,85 +362,112 @@ __global__ void __launch_bounds__(RG * kPB) phase_b_kernel(KParams a) {
 // ------------------------------------------------------------------ phase C
 // y_t = y_loc_t + carry_in^T Ctil_t, Ctil_t[j] = val_t[j] * C_t[idx_t[j]], where
 // (idx_t, val_t) is the pair of the chunk's prefix up to and including t.
+// Steps go in groups of kTG: the prefix pairs give Ctil for the group's steps
+// (one thread per entry j), then each thread accumulates the group's outputs for
+// its column run over its rows, so a carry row is read once per group.
+constexpr int kTG = 8;
+
 template <int RG, bool CPLX, typename TD, typename TIn, typename TOut>
-__global__ void __launch_bounds__(RG * kPB) phase_c_kernel(KParams a) {
+__global__ void __launch_bounds__(RG * ColRun<typename Num<CPLX>::T>::TPR) phase_c_kernel(KParams a) {
   using Nm = Num<CPLX>;
   using T = typename Nm::T;
+  constexpr int VW = ColRun<T>::VW, TPR = ColRun<T>::TPR, MR = ColRun<T>::MR, NT = RG * TPR, NW = NT / 32;
   extern __shared__ __align__(16) unsigned char smem[];
-  const int N = (int)a.N, tid = threadIdx.x, pl = tid % kPB, g = tid / kPB;
+  const int N = (int)a.N, tid = threadIdx.x, cl = tid % TPR, g = tid / TPR, pc = cl * VW;
   const int64_t c = blockIdx.x / a.nPB, pb = blockIdx.x % a.nPB, h = blockIdx.y, b = blockIdx.z;
   const int p0 = (int)(pb * kPB), P = (int)min((int64_t)kPB, a.P - p0), PG = (int)a.P;
-  const bool col = pl < P;
   const int64_t t0 = c * a.T, t1 = min(t0 + a.T, a.L);
-  T *Hin = reinterpret_cast<T *>(smem);  // [N][kPB]
-  T *ysh = Hin + N * kPB;                // [RG][kPB]
-  T *ct = ysh + RG * kPB;                // [N]
+  T *Hin = reinterpret_cast<T *>(smem);  // [N][kPB] carry into the chunk
+  T *ysh = Hin + N * kPB;                // [NW][kTG][kPB] per-warp parts of the outputs
+  T *ct = ysh + NW * kTG * kPB;          // [kTG][N] Ctil of the group's steps
+  T *dsh = ct + kTG * N;                 // [kTG][N]
+  float *Csh = reinterpret_cast<float *>(dsh + kTG * N);  // [kTG][N]
+  int *ssh = reinterpret_cast<int *>(Csh + kTG * N);      // [kTG] dictionary entries
 
   const TD *dg = static_cast<const TD *>(a.d);
   const TIn *Cg = static_cast<const TIn *>(a.C);
   const T *yl = static_cast<const T *>(a.y_loc);
   TOut *yo = static_cast<TOut *>(a.y);
-  auto yoff = [&](int64_t t) { return ((b * a.L + t) * a.H + h) * PG + p0 + pl; };
+  auto yrow = [&](int64_t t) { return ((b * a.L + t) * a.H + h) * PG + p0; };
 
   const bool carry = (c > 0) || (a.h0 != nullptr);
   if (!carry) {
-    if (g == 0 && col)
-      for (int64_t t = t0; t < t1; ++t) st_out(yo + yoff(t), yl[yoff(t)]);
+    for (int64_t e = tid; e < (t1 - t0) * P; e += NT) {
+      const int64_t t = t0 + e / P;
+      const int p = (int)(e % P);
+      st_out(yo + yrow(t) + p, yl[yrow(t) + p]);
+    }
     return;
   }
   const T *hin = c > 0 ? static_cast<const T *>(a.chunk_state) + ((b * a.H + h) * a.nC + c - 1) * N * PG
                        : static_cast<const T *>(a.h0) + (b * a.H + h) * N * PG;
-  for (int i = g; i < N; i += RG) Hin[i * kPB + pl] = col ? hin[i * PG + p0 + pl] : Nm::zero();
+  for (int e = tid; e < N * kPB; e += NT) {
+    const int i = e / kPB, p = e % kPB;
+    Hin[e] = p < P ? hin[i * PG + p0 + p] : Nm::zero();
+  }
   int pidx = tid;  // prefix pair entry tid (tid < N)
   T pval = Nm::one();
-  // the prefix pair needs d_t[pidx] and C_t[idx_t[pidx]]: entries of the step's
-  // vectors that another thread may own, so the vectors go through shared memory
-  T *dsh = ct + N;                                  // [N]
-  float *Csh = reinterpret_cast<float *>(dsh + N);  // [N]
-  T dn = Nm::zero();
-  float cn = 0.f;
-  int sn = 0;
-  auto fetch = [&](int64_t t) {
-    const int64_t row = (b * a.L + t) * a.H + h;
-    if (tid < N) {
-      dn = LoadD<CPLX, TD>::ld(dg + row * N + tid);
-      cn = ldf(Cg + row * N + tid);
-      sn = load_s(a, row, h);
-    }
-  };
-  T ylv = Nm::zero();  // y_loc of the step being finished, fetched a step ahead
-  auto finish_y = [&](int64_t t) {
-    if (g == 0 && col) {
-      T acc = ylv;
-#pragma unroll
-      for (int q = 0; q < RG; ++q) acc = Nm::add(acc, ysh[q * kPB + pl]);
-      st_out(yo + yoff(t), acc);
-    }
-  };
 
-  fetch(t0);
-  for (int64_t t = t0; t < t1; ++t) {
-    if (tid < N) {
-      dsh[tid] = dn;
-      Csh[tid] = cn;
+  for (int64_t tg = t0; tg < t1; tg += kTG) {
+    const int ng = (int)min((int64_t)kTG, t1 - tg);
+    // the group's vectors: the prefix pair needs d_t[pidx] and C_t[idx_t[pidx]],
+    // entries another thread may own
+    for (int e = tid; e < ng * N; e += NT) {
+      const int tau = e / N, j = e % N;
+      const int64_t row = (b * a.L + tg + tau) * a.H + h;
+      dsh[e] = LoadD<CPLX, TD>::ld(dg + row * N + j);
+      Csh[e] = ldf(Cg + row * N + j);
     }
-    const int st = sn;
-    if (t + 1 < t1) fetch(t + 1);
-    __syncthreads();  // step t's vectors and the parts of step t - 1 are visible
-    if (t > t0) finish_y(t - 1);
-    if (g == 0 && col) ylv = yl[yoff(t)];
+    if (tid < ng) ssh[tid] = load_s(a, (b * a.L + tg + tid) * a.H + h, h);
+    __syncthreads();  // the group's vectors; the previous group's parts were read
     if (tid < N) {
-      pval = Nm::mul(dsh[pidx], pval);
-      pidx = a.idx[(int64_t)st * N + pidx];
-      ct[tid] = Nm::mul(pval, Nm::from_real(Csh[pidx]));
+      for (int tau = 0; tau < ng; ++tau) {
+        pval = Nm::mul(dsh[tau * N + pidx], pval);
+        pidx = a.idx[(int64_t)ssh[tau] * N + pidx];
+        ct[tau * N + tid] = Nm::mul(pval, Nm::from_real(Csh[tau * N + pidx]));
+      }
     }
-    __syncthreads();  // Ctil_t is complete; the parts of step t - 1 were read
-    T yp = Nm::zero();
-    for (int i = g; i < N; i += RG) yp = Nm::fma(ct[i], Hin[i * kPB + pl], yp);
-    ysh[g * kPB + pl] = yp;
+    __syncthreads();  // Ctil of the group
+    T acc[kTG][VW];
+#pragma unroll
+    for (int tau = 0; tau < kTG; ++tau)
+#pragma unroll
+      for (int e = 0; e < VW; ++e) acc[tau][e] = Nm::zero();
+#pragma unroll
+    for (int m = 0; m < MR; ++m) {
+      const int i = g + RG * m;
+      if (i < N) {
+        T hv[VW];
+        ld_run(Hin + i * kPB + pc, hv);
+#pragma unroll
+        for (int tau = 0; tau < kTG; ++tau) {
+          const T cv = ct[tau * N + i];  // stale entries past ng are never written out
+#pragma unroll
+          for (int e = 0; e < VW; ++e) acc[tau][e] = Nm::fma(cv, hv[e], acc[tau][e]);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = TPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int tau = 0; tau < kTG; ++tau)
+#pragma unroll
+        for (int e = 0; e < VW; ++e) acc[tau][e] = Nm::add(acc[tau][e], shfl_xor(acc[tau][e], o));
+    if ((tid & 31) < TPR)
+#pragma unroll
+      for (int tau = 0; tau < kTG; ++tau) st_run(ysh + ((tid >> 5) * kTG + tau) * kPB + pc, acc[tau]);
+    __syncthreads();  // the warps' parts
+    for (int e = tid; e < ng * kPB; e += NT) {
+      const int tau = e / kPB, p = e % kPB;
+      if (p < P) {
+        const int64_t o = yrow(tg + tau) + p;
+        T y = yl[o];
+#pragma unroll
+        for (int w = 0; w < NW; ++w) y = Nm::add(y, ysh[(w * kTG + tau) * kPB + p]);
+        st_out(yo + o, y);
+      }
+    }
   }
-  __syncthreads();
-  finish_y(t1 - 1);
 }
 
 // ------------------------------------------------------------ empty L == 0
@@ -496,15 +523,14 @@ cudaError_t run_chunked_rg(const ScanArgs &s, cudaStream_t st) {
   constexpr int NTA = RGA * ColRun<T>::TPR;
   const size_t smem_a = N * kPB * ts + (NTA / 32) * kPB * ts + N * ts + 2 * N * 4 + kPB * 4 + (2 * N + 1) * 4;
   const size_t smem_b = N * kPB * ts + N * ts + N * 4 + (2 * N + 1) * 4;
-  const size_t smem_c = N * kPB * ts + RG * kPB * ts + 2 * N * ts + N * 4;
+  const size_t smem_c = N * kPB * ts + (NTA / 32) * kTG * kPB * ts + 2 * kTG * N * ts + kTG * N * 4 + kTG * 4;
   const dim3 grid_chunks((unsigned)(s.nC * k.nPB), (unsigned)s.H, (unsigned)s.Bt);
   cudaError_t e = launch_dyn(phase_a_kernel<RGA, CPLX, TD, TIn>, "chunked_phase_a", grid_chunks, NTA, smem_a, st, k);
   if (e != cudaSuccess) return e;
   e = launch_dyn(phase_b_kernel<RG, CPLX>, "chunked_phase_b", dim3((unsigned)(s.H * k.nPB), (unsigned)s.Bt),
                  RG * kPB, smem_b, st, k);
   if (e != cudaSuccess) return e;
-  return launch_dyn(phase_c_kernel<RG, CPLX, TD, TIn, TOut>, "chunked_phase_c", grid_chunks, RG * kPB, smem_c, st,
-                    k);
+  return launch_dyn(phase_c_kernel<RGA, CPLX, TD, TIn, TOut>, "chunked_phase_c", grid_chunks, NTA, smem_c, st, k);
 }
 
 // Row groups: a thread updates at most kMaxRows rows, and the block's threads
