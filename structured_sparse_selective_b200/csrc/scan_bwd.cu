@@ -21,8 +21,10 @@
 // One block per (batch, head) sequence. A forward sweep stores the state every
 // kTb steps (O(L N P / kTb) memory, O(L N) for kTb >= P); the reverse sweep
 // recomputes each kTb-step stretch from its checkpoint into a per-sequence
-// scratch and walks it backwards. Three N x P buffers in shared memory (rows
-// padded by one element) hold the adjoint, H_t and H_{t-1}.
+// scratch and walks it backwards. Three N x P buffers in shared memory hold the
+// adjoint, H_t and H_{t-1}; threads move their rows in 16-byte runs (4 real or 2
+// complex values), so a row's preimage list or dictionary row is read once per
+// run.
 #include "launch.h"
 
 namespace pdssm {
@@ -74,12 +76,33 @@ __device__ __forceinline__ void ld_dy(const void *p, int64_t i, int, float2 *v) 
   *v = static_cast<const float2 *>(p)[i];
 }
 
+// 16 bytes of a state row: 4 real or 2 complex values.
+__device__ __forceinline__ void ld_run(const float *p, float (&v)[4]) {
+  const float4 w = *reinterpret_cast<const float4 *>(p);
+  v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
+}
+__device__ __forceinline__ void ld_run(const float2 *p, float2 (&v)[2]) {
+  const float4 w = *reinterpret_cast<const float4 *>(p);
+  v[0] = make_float2(w.x, w.y); v[1] = make_float2(w.z, w.w);
+}
+__device__ __forceinline__ void st_run(float *p, const float (&v)[4]) {
+  *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void st_run(float2 *p, const float2 (&v)[2]) {
+  *reinterpret_cast<float4 *>(p) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+}
+
 template <bool CPLX, typename TD, typename TIn>
 __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
   using NT = Num<CPLX>;
   using T = typename NT::T;
+  constexpr int VW = 16 / (int)sizeof(T);  // values per 16-byte run
   extern __shared__ __align__(16) unsigned char smem[];
-  const int N = (int)a.N, P = (int)a.P, K = (int)a.K, PS = P + 1;
+  const int N = (int)a.N, P = (int)a.P, K = (int)a.K;
+  // Rows hold PV = P rounded up to whole runs (the extra columns stay zero: their
+  // x and dy are zero) plus one run of padding, which keeps rows 16-byte aligned
+  // and puts consecutive rows 16 bytes apart in the banks.
+  const int NR = (P + VW - 1) / VW, PV = NR * VW, PS = PV + VW;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
 
@@ -87,17 +110,21 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
   T *buf1 = buf0 + N * PS;
   T *buf2 = buf1 + N * PS;
   T *dsh = buf2 + N * PS;  // [N]
-  T *dysh = dsh + N;       // [P]
-  float *Bsh = reinterpret_cast<float *>(dysh + P);  // [N]
-  float *Csh = Bsh + N;                              // [N]
-  float *xsh = Csh + N;                              // [P]
-  float *dpi = xsh + P;                              // [K]
+  T *dysh = dsh + N;       // [PV]
+  float *Bsh = reinterpret_cast<float *>(dysh + PV);  // [N]
+  float *Csh = Bsh + N;                               // [N]
+  float *xsh = Csh + N;                               // [PV]
+  float *dpi = xsh + PV;                              // [K]
   int *offsh = reinterpret_cast<int *>(dpi + K);  // [N+1] preimage lists of the step's entry
   int *srcsh = offsh + N + 1;                     // [N]
   uint8_t *idxsh = reinterpret_cast<uint8_t *>(srcsh + N);  // [K][N] dictionary
 
   const int64_t kh = a.head_dicts ? h * K : 0;  // this head's first dictionary entry
   for (int e = tid; e < K * N; e += kBT) idxsh[e] = (uint8_t)a.idx[kh * N + e];
+  for (int p = P + tid; p < PV; p += kBT) {  // the padding columns' x and dy stay zero
+    xsh[p] = 0.f;
+    dysh[p] = NT::zero();
+  }
 
   const TD *dg = static_cast<const TD *>(a.d);
   const TIn *Bg = static_cast<const TIn *>(a.B);
@@ -109,11 +136,11 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
   T *ck = static_cast<T *>(a.ckpt) + bh * a.nCk * N * P;
   T *scr = static_cast<T *>(a.scratch) + bh * (int64_t)kTb * N * P;
 
-  // element loop over a dense [N][P] array: thread tid starts at element tid
-  const int di = kBT / P, dp = kBT - di * P;
-  const int i_start = tid / P, p_start = tid - i_start * P;
-#define FOR_NP(i, p)                                                           \
-  for (int i = i_start, p = p_start; i < N; i += di, p += dp, (p >= P ? (p -= P, ++i) : 0))
+  // loop over the runs of a dense [N][PV] array: thread tid starts at run tid
+  const int dr = kBT / NR, dq = kBT - dr * NR;
+  const int r_start = tid / NR, q_start = tid - r_start * NR;
+#define FOR_RUNS(i, q)                                                         \
+  for (int i = r_start, q = q_start; i < N; i += dr, q += dq, (q >= NR ? (q -= NR, ++i) : 0))
 
   auto row_of = [&](int64_t t) { return (b * a.L + t) * a.H + h; };
   auto load_s = [&](int64_t row) {
@@ -164,26 +191,48 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
   };
   // Hn = A_t Hc + B_t x_t^T (after commit of step t's vectors and a barrier)
   auto step_fwd = [&](const T *Hc, T *Hn) {
-    FOR_NP(i, p) {
-      T acc = NT::from_real(Bsh[i] * xsh[p]);
+    FOR_RUNS(i, q) {
+      const int p0 = q * VW;
+      T acc[VW];
+      const float bi = Bsh[i];
+#pragma unroll
+      for (int e = 0; e < VW; ++e) acc[e] = NT::from_real(bi * xsh[p0 + e]);
       const int r1 = offsh[i + 1];
       for (int r = offsh[i]; r < r1; ++r) {
         const int j = srcsh[r];
-        acc = NT::fma(dsh[j], Hc[j * PS + p], acc);
+        const T dj = dsh[j];
+        T hv[VW];
+        ld_run(Hc + j * PS + p0, hv);
+#pragma unroll
+        for (int e = 0; e < VW; ++e) acc[e] = NT::fma(dj, hv[e], acc[e]);
       }
-      Hn[i * PS + p] = acc;
+      st_run(Hn + i * PS + p0, acc);
     }
   };
+  // [N][P] in global memory <-> [N][PV] rows in shared memory (the padding columns read as zero)
   auto store_dense = [&](const T *S, T *g) {
-    FOR_NP(i, p) { g[i * P + p] = S[i * PS + p]; }
+    FOR_RUNS(i, q) {
+      const int p0 = q * VW;
+      T v[VW];
+      ld_run(S + i * PS + p0, v);
+#pragma unroll
+      for (int e = 0; e < VW; ++e)
+        if (p0 + e < P) g[i * P + p0 + e] = v[e];
+    }
   };
   auto load_dense = [&](const T *g, T *S) {
-    FOR_NP(i, p) { S[i * PS + p] = g[i * P + p]; }
+    FOR_RUNS(i, q) {
+      const int p0 = q * VW;
+      T v[VW];
+#pragma unroll
+      for (int e = 0; e < VW; ++e) v[e] = (g && p0 + e < P) ? g[i * P + p0 + e] : NT::zero();
+      st_run(S + i * PS + p0, v);
+    }
   };
 
   // ---- forward sweep: checkpoints every kTb steps
   T *Hc = buf0, *Hn = buf1;
-  FOR_NP(i, p) { Hc[i * PS + p] = h0g ? h0g[(bh * N + i) * P + p] : NT::zero(); }
+  load_dense(h0g ? h0g + bh * N * P : nullptr, Hc);
   Vec nv = fetch(0, false);
   for (int64_t t = 0; t < a.L; ++t) {
     __syncthreads();  // Hc complete; the staged vectors are no longer read
@@ -200,7 +249,7 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
   // ---- reverse sweep
   T *Lam = buf2;
   __syncthreads();
-  FOR_NP(i, p) { Lam[i * PS + p] = dhg ? dhg[(bh * N + i) * P + p] : NT::zero(); }
+  load_dense(dhg ? dhg + bh * N * P : nullptr, Lam);
   for (int64_t c = a.nCk - 1; c >= 0; --c) {
     const int64_t t0 = c * kTb, t1 = t0 + kTb < a.L ? t0 + kTb : a.L;
     // recompute the stretch: scratch[t - t0] = H_{t-1}; Hc ends as H_{t1-1}
@@ -232,30 +281,57 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
       load_dense(scr + (t - t0) * N * P, Hp);
       __syncthreads();
       // [B] Lam_t = Lam'_t + C_t dy_t^T
-      FOR_NP(i, p) { Lam[i * PS + p] = NT::fma_r(Csh[i], dysh[p], Lam[i * PS + p]); }
+      FOR_RUNS(i, q) {
+        const int p0 = q * VW;
+        T v[VW];
+        ld_run(Lam + i * PS + p0, v);
+        const float ci = Csh[i];
+#pragma unroll
+        for (int e = 0; e < VW; ++e) v[e] = NT::fma_r(ci, dysh[p0 + e], v[e]);
+        st_run(Lam + i * PS + p0, v);
+      }
       __syncthreads();
-      // [C] dB_t, dC_t, and per entry k: sum_p Lam_t[idx_k[j]][p] conj(H_{t-1}[j][p])
-      // (dd_t at k = s_t, dpi_t[k])
+      // [C] dB_t, dC_t (a thread per row), and per entry k, lanes over j:
+      // q_kj = sum_p Lam_t[idx_k[j]][p] conj(H_{t-1}[j][p]) (dd_t at k = s_t, dpi_t[k])
       if (tid < N) {
         float acc = 0.f;
-        for (int p = 0; p < P; ++p) acc = fmaf(re_of(Lam[tid * PS + p]), xsh[p], acc);
+        for (int q = 0; q < NR; ++q) {
+          T v[VW];
+          ld_run(Lam + tid * PS + q * VW, v);
+#pragma unroll
+          for (int e = 0; e < VW; ++e) acc = fmaf(re_of(v[e]), xsh[q * VW + e], acc);
+        }
         a.dB[row * N + tid] = acc;
       }
       if (tid >= 128 && tid - 128 < N) {
         const int i = tid - 128;
         float acc = 0.f;
-        for (int p = 0; p < P; ++p) acc = fma_re_conj(Hc[i * PS + p], dysh[p], acc);
+        for (int q = 0; q < NR; ++q) {
+          T v[VW];
+          ld_run(Hc + i * PS + q * VW, v);
+#pragma unroll
+          for (int e = 0; e < VW; ++e) acc = fma_re_conj(v[e], dysh[q * VW + e], acc);
+        }
         a.dC[row * N + i] = acc;
       }
       for (int k = warp; k < K; k += kBT / 32) {
         float part = 0.f;
         for (int j = lane; j < N; j += 32) {
-          const int r = idxsh[k * N + j];
-          T q = NT::zero();
-#pragma unroll 4
-          for (int p = 0; p < P; ++p) q = fma_conj(Lam[r * PS + p], Hp[j * PS + p], q);
-          if (k == st) ddg[row * N + j] = q;
-          part = fma_re_conj(dsh[j], q, part);  // Re(conj(q) d_j)
+          const T *lr = Lam + idxsh[k * N + j] * PS, *hr = Hp + j * PS;
+          T q0 = NT::zero(), q1 = NT::zero();  // two partial sums: a shorter dependent chain
+          for (int q = 0; q < NR; ++q) {
+            T l[VW], hp[VW];
+            ld_run(lr + q * VW, l);
+            ld_run(hr + q * VW, hp);
+#pragma unroll
+            for (int e = 0; e < VW; e += 2) {
+              q0 = fma_conj(l[e], hp[e], q0);
+              q1 = fma_conj(l[e + 1], hp[e + 1], q1);
+            }
+          }
+          const T qv = NT::add(q0, q1);
+          if (k == st) ddg[row * N + j] = qv;
+          part = fma_re_conj(dsh[j], qv, part);  // Re(conj(q) d_j)
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
@@ -282,7 +358,15 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
         if (lane < K) a.dlogits[row * K + lane] = p0 * (g0 - dot) / a.tau;
         if (lane + 32 < K) a.dlogits[row * K + lane + 32] = p1 * (g1 - dot) / a.tau;
       }
-      FOR_NP(j, p) { Hc[j * PS + p] = NT::mul(conj_of(dsh[j]), Lam[idxsh[st * N + j] * PS + p]); }
+      FOR_RUNS(j, q) {
+        const int p0 = q * VW;
+        const T dc = conj_of(dsh[j]);
+        T v[VW];
+        ld_run(Lam + idxsh[st * N + j] * PS + p0, v);
+#pragma unroll
+        for (int e = 0; e < VW; ++e) v[e] = NT::mul(dc, v[e]);
+        st_run(Hc + j * PS + p0, v);
+      }
       if (tid >= 32 && tid - 32 < P) {
         const int p = tid - 32;
         float acc = 0.f;
@@ -297,19 +381,15 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
     }
   }
   __syncthreads();
-  if (a.dh0) {
-    T *dh0g = static_cast<T *>(a.dh0);
-    FOR_NP(i, p) { dh0g[(bh * N + i) * P + p] = Lam[i * PS + p]; }
-  }
-#undef FOR_NP
+  if (a.dh0) store_dense(Lam, static_cast<T *>(a.dh0) + bh * N * P);
+#undef FOR_RUNS
 }
 
 }  // namespace
 
 size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t K, bool cplx) {
-  const size_t es = cplx ? 8 : 4;
-  return (size_t)(3 * N * (P + 1) + N + P) * es + (size_t)(2 * N + P + K) * 4 + (size_t)(2 * N + 1) * 4 +
-         (size_t)(K * N);
+  const int64_t es = cplx ? 8 : 4, vw = 16 / es, pv = (P + vw - 1) / vw * vw;
+  return (size_t)((3 * N * (pv + vw) + N + pv) * es + (2 * N + pv + K) * 4 + (2 * N + 1) * 4 + K * N);
 }
 
 int64_t scan_bwd_checkpoints(int64_t L) { return (L + kTb - 1) / kTb; }

@@ -9,18 +9,20 @@
 // one-hot-column transitions (the associative-operator framing of the Prefix
 // Scannable Models abstract): (idx, val) o (idx', val') = (idx[idx'], val[idx']*val').
 //
-// A block owns up to 32 columns of one (batch, head) state and all N rows, in
-// shared memory (the gather index is dynamic). In phases B and C its threads are
-// RG row groups of 32 columns (RG = 1, 2 or 8, so that a thread has at most 16
-// rows): thread (g, p) updates rows i = g, g + RG, ... of column p, so a warp
-// always reads one state row across 32 consecutive columns (no bank conflicts).
-// In phase A, the per-token recurrence, a thread owns a 16-byte run of columns
-// (4 real or 2 complex) of its rows instead, so that each row's preimage list is
-// read once for the whole run and the state moves in 16-byte loads. New rows are
-// held in registers until every thread has read the old state, so one state
-// buffer suffices. Per-step vectors (d, B, C, x and the selected entry's preimage
-// lists) are fetched into registers one step ahead and staged in shared memory; a
-// column's output is the sum of the row groups' parts.
+// A block owns a range of columns of one (batch, head) state and all N rows, in
+// shared memory (the gather index is dynamic). In phases A and C (32 columns a
+// block) a thread owns a 16-byte run of columns (4 real or 2 complex) of the rows
+// g, g + RG, ... of its row group, so that each row's preimage list is read once
+// for the whole run, the state moves in 16-byte loads and eight consecutive
+// lanes read 128 contiguous bytes of a row (no bank conflicts). Phase B runs its
+// chunks in sequence, so its blocks are narrower (8 columns, one column a thread)
+// to spread few sequences over many blocks. New rows are held in registers until
+// every thread has read the old state, so one state buffer suffices. Per-step
+// vectors (d, B, C, x and the selected entry's preimage lists) are fetched into
+// registers one step ahead and staged in shared memory; a column's output is the
+// sum of the row groups' parts. (Complex phase A is held to 64 registers a thread
+// for occupancy, measured faster despite a few spilled bytes; real phase A has no
+// occupancy bound, minBlocks 0, which measured faster for it.)
 #include <algorithm>
 
 #include "launch.h"
@@ -30,12 +32,12 @@ namespace pdssm {
 namespace {
 
 constexpr int kPB = 32;       // columns per block (one warp per row group)
-constexpr int kMaxRows = 16;  // rows per thread at most
 
 struct KParams {
   int64_t L, H, N, P, K, T, nC;
   int64_t Kh;   // dictionary entries per head with per-head dictionaries (else 0)
-  int64_t nPB;  // column blocks (columns are independent)
+  int64_t nPB;   // column blocks of phases A and C (columns are independent)
+  int64_t nPBB;  // column blocks of phase B (narrower: its blocks run the chunks in sequence)
   const int32_t *s;
   const int32_t *idx;  // sanitised [K][N]
   const int32_t *off;  // [K][N+1]
@@ -99,7 +101,9 @@ __device__ __forceinline__ void st_run(float2 *p, const float2 (&v)[2]) {
 // Threads: RG row groups of TPR threads; thread (g, cl) updates rows g, g + RG, ...
 // of columns [cl * VW, cl * VW + VW) of the block's kPB columns.
 template <int RG, bool CPLX, typename TD, typename TIn>
-__global__ void __launch_bounds__(RG * ColRun<typename Num<CPLX>::T>::TPR) phase_a_kernel(KParams a) {
+__global__ void __launch_bounds__(RG * ColRun<typename Num<CPLX>::T>::TPR,
+                                  CPLX ? 1024 / (RG * ColRun<typename Num<CPLX>::T>::TPR) : 0)
+    phase_a_kernel(KParams a) {
   using Nm = Num<CPLX>;
   using T = typename Nm::T;
   constexpr int VW = ColRun<T>::VW, TPR = ColRun<T>::TPR, MR = ColRun<T>::MR, NT = RG * TPR, NW = NT / 32;
@@ -250,25 +254,29 @@ __global__ void __launch_bounds__(RG * ColRun<typename Num<CPLX>::T>::TPR) phase
 // apply((idx, val), H)[i] = sum_{j: idx[j] = i} val[j] H[j], sources in increasing
 // j. The carries overwrite the local states in place; h_final is the last carry
 // and (prod_idx, prod_val) the composition of all chunk pairs.
-template <int RG, bool CPLX>
-__global__ void __launch_bounds__(RG * kPB) phase_b_kernel(KParams a) {
+// A block owns PB columns (RG row groups of them, at most MRB rows a thread): 8
+// for N <= 32, so that a workload with few sequences still spreads its
+// sequential chunk loops over many blocks, else 32 (every block sorts the chunk
+// pairs' preimages, O(N) a thread).
+template <int RG, int PB, int MRB, bool CPLX>
+__global__ void __launch_bounds__(RG * PB) phase_b_kernel(KParams a) {
   using Nm = Num<CPLX>;
   using T = typename Nm::T;
-  constexpr int NT = RG * kPB;
+  constexpr int NT = RG * PB;
   extern __shared__ __align__(16) unsigned char smem[];
-  const int N = (int)a.N, tid = threadIdx.x, pl = tid % kPB, g = tid / kPB;
-  const int64_t h = blockIdx.x / a.nPB, pb = blockIdx.x % a.nPB, b = blockIdx.y;
-  const int p0 = (int)(pb * kPB), P = (int)min((int64_t)kPB, a.P - p0), PG = (int)a.P;
+  const int N = (int)a.N, tid = threadIdx.x, pl = tid % PB, g = tid / PB;
+  const int64_t h = blockIdx.x / a.nPBB, pb = blockIdx.x % a.nPBB, b = blockIdx.y;
+  const int p0 = (int)(pb * PB), P = (int)min((int64_t)PB, a.P - p0), PG = (int)a.P;
   const bool col = pl < P;
-  T *Hs = reinterpret_cast<T *>(smem);  // [N][kPB]
-  T *pv = Hs + N * kPB;                 // [N]
+  T *Hs = reinterpret_cast<T *>(smem);  // [N][PB]
+  T *pv = Hs + N * PB;                 // [N]
   int *pi = reinterpret_cast<int *>(pv + N);
   int *off = pi + N;                    // [N+1] preimage lists of the chunk pair's index map
   int *src = off + N + 1;               // [N]
 
   const T *h0 = static_cast<const T *>(a.h0);
   for (int i = g; i < N; i += RG)
-    Hs[i * kPB + pl] = (h0 && col) ? h0[((b * a.H + h) * N + i) * PG + p0 + pl] : Nm::zero();
+    Hs[i * PB + pl] = (h0 && col) ? h0[((b * a.H + h) * N + i) * PG + p0 + pl] : Nm::zero();
   int tidx = tid;  // whole-sequence product entry tid (tid < N)
   T tval = Nm::one();
   const int64_t slot0 = (b * a.H + h) * a.nC;
@@ -281,9 +289,9 @@ __global__ void __launch_bounds__(RG * kPB) phase_b_kernel(KParams a) {
 
   for (int64_t c = 0; c < a.nC; ++c) {
     T *cs = static_cast<T *>(a.chunk_state) + (slot0 + c) * N * PG + p0;
-    T nv[kMaxRows];  // the local state's rows, loaded while the lists are built
+    T nv[MRB];  // the local state's rows, loaded while the lists are built
 #pragma unroll
-    for (int m = 0; m < kMaxRows; ++m) {
+    for (int m = 0; m < MRB; ++m) {
       const int i = g + RG * m;
       if (i < N) nv[m] = col ? cs[i * PG + pl] : Nm::zero();
     }
@@ -317,20 +325,20 @@ __global__ void __launch_bounds__(RG * kPB) phase_b_kernel(KParams a) {
     if (tid < N) src[off[mine] + rank] = tid;
     __syncthreads();
 #pragma unroll
-    for (int m = 0; m < kMaxRows; ++m) {
+    for (int m = 0; m < MRB; ++m) {
       const int i = g + RG * m;
       if (i < N) {
         T acc = nv[m];
         const int r0 = off[i], r1 = off[i + 1];
         if (r0 < r1) {
           const int ja = src[r0];
-          acc = Nm::fma(pv[ja], Hs[ja * kPB + pl], acc);
+          acc = Nm::fma(pv[ja], Hs[ja * PB + pl], acc);
           if (r0 + 1 < r1) {
             const int jb = src[r0 + 1];
-            acc = Nm::fma(pv[jb], Hs[jb * kPB + pl], acc);
+            acc = Nm::fma(pv[jb], Hs[jb * PB + pl], acc);
             for (int r = r0 + 2; r < r1; ++r) {
               const int j = src[r];
-              acc = Nm::fma(pv[j], Hs[j * kPB + pl], acc);
+              acc = Nm::fma(pv[j], Hs[j * PB + pl], acc);
             }
           }
         }
@@ -339,10 +347,10 @@ __global__ void __launch_bounds__(RG * kPB) phase_b_kernel(KParams a) {
     }
     __syncthreads();  // every read of the previous carry is done
 #pragma unroll
-    for (int m = 0; m < kMaxRows; ++m) {
+    for (int m = 0; m < MRB; ++m) {
       const int i = g + RG * m;
       if (i < N) {
-        Hs[i * kPB + pl] = nv[m];
+        Hs[i * PB + pl] = nv[m];
         if (col) cs[i * PG + pl] = nv[m];
       }
     }
@@ -351,7 +359,7 @@ __global__ void __launch_bounds__(RG * kPB) phase_b_kernel(KParams a) {
 
   if (a.h_final && col) {
     T *hf = static_cast<T *>(a.h_final) + (b * a.H + h) * N * PG + p0;
-    for (int i = g; i < N; i += RG) hf[i * PG + pl] = Hs[i * kPB + pl];
+    for (int i = g; i < N; i += RG) hf[i * PG + pl] = Hs[i * PB + pl];
   }
   (void)NT;
   if (pb != 0 || tid >= N) return;
@@ -490,6 +498,8 @@ KParams make_params(const ScanArgs &s) {
   k.L = s.L; k.H = s.H; k.N = s.N; k.P = s.P; k.K = s.K; k.T = s.T; k.nC = s.nC;
   k.Kh = s.head_dicts ? s.K : 0;
   k.nPB = (s.P + kPB - 1) / kPB;
+  const int64_t pbb = s.N <= 32 ? 8 : kPB;  // phase B's columns a block (as run_chunked_n)
+  k.nPBB = (s.P + pbb - 1) / pbb;
   k.s = s.s; k.idx = s.ws.idx; k.off = s.ws.csr_off; k.src = s.ws.csr_src;
   k.d = s.d; k.B = s.B; k.C = s.C; k.x = s.x; k.h0 = s.h0;
   k.y_loc = s.ws.y_loc; k.chunk_state = s.ws.chunk_state; k.chunk_val = s.ws.chunk_val;
@@ -512,34 +522,34 @@ cudaError_t launch_dyn(Kern kern, const char *name, dim3 grid, int threads, size
   return trace_after(st);
 }
 
-template <int RG, bool CPLX, typename TD, typename TIn, typename TOut>
-cudaError_t run_chunked_rg(const ScanArgs &s, cudaStream_t st) {
+// NMAX bounds N (16, 32, 64 or 128); it sizes every phase's row groups.
+template <int NMAX, bool CPLX, typename TD, typename TIn, typename TOut>
+cudaError_t run_chunked_n(const ScanArgs &s, cudaStream_t st) {
   using T = typename Num<CPLX>::T;
   const KParams k = make_params(s);
   const size_t ts = sizeof(T), N = (size_t)s.N;
-  // phase A's row groups (threads > N, RGA * MR >= N): real 32 / 8 / 4, complex
-  // 16 / 4 / 2 for N <= 128 / 32 / 16
-  constexpr int RGA = ColRun<T>::TPR == 8 ? (RG == 8 ? 32 : RG == 2 ? 8 : 4) : (RG == 8 ? 16 : RG == 2 ? 4 : 2);
-  constexpr int NTA = RGA * ColRun<T>::TPR;
+  // phases A and C: RGA * MR >= N rows, 2 NMAX threads; phase B: RGB * MRB >= N rows
+  constexpr int RGA = NMAX / ColRun<T>::MR, NTA = RGA * ColRun<T>::TPR;
+  constexpr int PBB = NMAX <= 32 ? 8 : kPB, MRB = NMAX <= 32 ? 4 : 16, RGB = NMAX / MRB, NTB = RGB * PBB;
+  static_assert(NTA > NMAX && NTB >= NMAX, "a thread per vector entry");
   const size_t smem_a = N * kPB * ts + (NTA / 32) * kPB * ts + N * ts + 2 * N * 4 + kPB * 4 + (2 * N + 1) * 4;
-  const size_t smem_b = N * kPB * ts + N * ts + N * 4 + (2 * N + 1) * 4;
+  const size_t smem_b = N * PBB * ts + N * ts + N * 4 + (2 * N + 1) * 4;
   const size_t smem_c = N * kPB * ts + (NTA / 32) * kTG * kPB * ts + 2 * kTG * N * ts + kTG * N * 4 + kTG * 4;
   const dim3 grid_chunks((unsigned)(s.nC * k.nPB), (unsigned)s.H, (unsigned)s.Bt);
   cudaError_t e = launch_dyn(phase_a_kernel<RGA, CPLX, TD, TIn>, "chunked_phase_a", grid_chunks, NTA, smem_a, st, k);
   if (e != cudaSuccess) return e;
-  e = launch_dyn(phase_b_kernel<RG, CPLX>, "chunked_phase_b", dim3((unsigned)(s.H * k.nPB), (unsigned)s.Bt),
-                 RG * kPB, smem_b, st, k);
+  e = launch_dyn(phase_b_kernel<RGB, PBB, MRB, CPLX>, "chunked_phase_b", dim3((unsigned)(s.H * k.nPBB), (unsigned)s.Bt), NTB,
+                 smem_b, st, k);
   if (e != cudaSuccess) return e;
   return launch_dyn(phase_c_kernel<RGA, CPLX, TD, TIn, TOut>, "chunked_phase_c", grid_chunks, NTA, smem_c, st, k);
 }
 
-// Row groups: a thread updates at most kMaxRows rows, and the block's threads
-// (32 per row group) are at least twice N.
 template <bool CPLX, typename TD, typename TIn, typename TOut>
 cudaError_t run_chunked(const ScanArgs &s, cudaStream_t st) {
-  if (s.N <= 16) return run_chunked_rg<1, CPLX, TD, TIn, TOut>(s, st);
-  if (s.N <= 32) return run_chunked_rg<2, CPLX, TD, TIn, TOut>(s, st);
-  return run_chunked_rg<8, CPLX, TD, TIn, TOut>(s, st);
+  if (s.N <= 16) return run_chunked_n<16, CPLX, TD, TIn, TOut>(s, st);
+  if (s.N <= 32) return run_chunked_n<32, CPLX, TD, TIn, TOut>(s, st);
+  if (s.N <= 64) return run_chunked_n<64, CPLX, TD, TIn, TOut>(s, st);
+  return run_chunked_n<128, CPLX, TD, TIn, TOut>(s, st);
 }
 
 }  // namespace
