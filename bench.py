@@ -340,13 +340,16 @@ def per_config(device, flush, names=("tiny", "z5", "long", "complex"), steps: in
         ms, kms, launches = time_forward(sp, inp, device, steps, warmup, flush)
         del inp
         torch.cuda.empty_cache()
+        dom = max(kms, key=kms.get)
+        traffic = recorded_traffic(dom, name)
+        source = f"profiles/{dom}_{name}.md (ncu capture of the same kernel sources)" if traffic is not None else None
         res[name] = {
             "workload": workload_config(sp, 0, 1)["workload"],
             "inputs": "host recipe (workloads.generate)" if on_host else "drawn on the device (same recipe)",
             "value": round(sp.token_heads / (ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(ms, 4),
             "steps": steps, "warmup": warmup, "kernels_ms_per_step": {k: round(v, 4) for k, v in kms.items()},
             "gpu_launches": launches,
-            "roofline": roofline_entry(sp, kms, peaks),
+            "roofline": roofline_entry(sp, kms, peaks, traffic, source),
             "cpu_baseline": cpu_baseline(sp, target_s=2.0, seqlen_cap=0 if name != "complex" else 128),
         }
     return res
@@ -452,12 +455,22 @@ def projection_entry(device, steps: int = 10, warmup: int = 3, D: int = 1024):
 
 # ------------------------------------------------------------- our arm
 
+def bench_spec(args) -> workloads.Spec:
+    """The workload the command line names; --batch / --seqlen shorten it (profiling captures)."""
+    kw = {}
+    if getattr(args, "batch", 0):
+        kw["batch"] = args.batch
+    if getattr(args, "seqlen", 0):
+        kw["seqlen"] = args.seqlen
+    return workloads.spec(args.workload, **kw)
+
+
 def run_ours(args, rank, world, local):
     import structured_sparse_selective_b200 as pd
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    sp = workloads.spec(args.workload)
+    sp = bench_spec(args)
     inp = {k: v.to(device) for k, v in workloads.generate(sp, seed=shard_seed(rank)).items()}
     pb = pd.make_problem(inp["logits"], inp["d"], inp["B"], inp["x"], chunk=args.chunk)
     Bt, L, H, N = inp["B"].shape
@@ -530,7 +543,7 @@ def run_ours(args, rank, world, local):
         "select": units * (with_logits + 4),
     }.get(dominant)
     peaks = load_peaks()
-    traffic = recorded_traffic(dominant, args.workload)
+    traffic = None if (args.batch or args.seqlen) else recorded_traffic(dominant, args.workload)
     traffic_source = (f"profiles/{dominant}_{args.workload}.md (ncu capture of the same kernel sources)"
                       if traffic is not None else None)
     roofline = None
@@ -612,7 +625,7 @@ def run_ours_backward(args, rank, world, local):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    sp = workloads.spec(args.workload)
+    sp = bench_spec(args)
     if sp.state_complex:  # ~10 GB of inputs: drawn on the device (same recipe, other numbers)
         inp = workloads.generate_on_device(sp, seed=shard_seed(rank), device=device)
     else:
@@ -692,15 +705,18 @@ def run_reference_backward(args, rank, world):
     if rank != 0:
         return None
     from oracle import backward as obwd
-    sp = workloads.spec(args.workload)
-    if sp.state_complex:
-        raise SystemExit("the backward pass is built for real states only")
+    sp = bench_spec(args)
     idx = workloads.generate_idx(sp).numpy()
-    n = 2
+    # complex slices (N = 128, dense N x N products per step) are cut to their first 256 steps
+    n, lcap = (1, 256) if sp.state_complex else (2, sp.seqlen)
     picks = [(i // sp.heads % sp.batch, i % sp.heads) for i in range(n)]
     sls = [workloads.generate_slice(sp, b, h) for b, h in picks]
-    stack = {k: torch.stack([s_[k] for s_ in sls]).double().numpy() for k in sls[0]}
-    dy = torch.randn(n, sp.seqlen, sp.P, generator=torch.Generator().manual_seed(0)).to(sp.out_dtype).double().numpy()
+
+    def np64(t):
+        return (t.to(torch.complex128) if t.is_complex() else t.double()).numpy()
+    stack = {k: np64(torch.stack([s_[k][:lcap] for s_ in sls])) for k in sls[0]}
+    sdt = torch.complex64 if sp.state_complex else torch.float32
+    dy = np64(torch.randn(n, lcap, sp.P, generator=torch.Generator().manual_seed(0), dtype=sdt).to(sp.out_dtype))
 
     def step():
         obwd.scan_backward(stack["logits"], idx, stack["d"], stack["B"], stack["C"], stack["x"], dy, tau=args.tau)
@@ -711,14 +727,16 @@ def run_reference_backward(args, rank, world):
     for _ in range(args.steps):
         step()
     sec = (time.perf_counter() - t0) / args.steps
-    units = n * sp.seqlen
+    units = n * lcap
     value = units / sec
-    sample = (f"each step: {n} whole (batch, head) slices x L={sp.seqlen} of the {sp.recipe} workload "
+    cut = "whole" if lcap == sp.seqlen else f"cut to their first {lcap} steps,"
+    sample = (f"each step: {n} {cut} (batch, head) slices x L={lcap} of the {sp.recipe} workload "
               f"({units} token-heads), dense fp64 backward oracle (numpy, one thread)")
     return {
         "impl": "reference", "metric": BWD_METRIC, "pass": "backward", "value": round(value, 1), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "c128" if sp.state_complex else "f64", "data": "synthetic",
         "config": dict(workload_config(sp, 0, world), tau=args.tau),
         "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -732,7 +750,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     import oracle
-    sp = workloads.spec(args.workload)
+    sp = bench_spec(args)
     cores = oracle.threads()
     idx = workloads.generate_idx(sp)
     n = max(1, cores)
@@ -776,6 +794,10 @@ def main(argv=None):
                     help="skip the other configurations, the original PD-SSM contrast and the projection")
     ap.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward")
     ap.add_argument("--tau", type=float, default=1.0, help="softmax temperature of the backward pass")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (shorter runs for profiling captures; 0 = full)")
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the workload's sequence length (profiling captures; 0 = full)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -795,7 +817,7 @@ def main(argv=None):
         res = run_ours(args, rank, world, local)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
-                res["cpu_baseline"] = cpu_baseline(workloads.spec(args.workload))
+                res["cpu_baseline"] = cpu_baseline(bench_spec(args))
             if world == 1 and not args.no_extras and args.workload == "lm":
                 dev = torch.device("cuda", local)
                 flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
