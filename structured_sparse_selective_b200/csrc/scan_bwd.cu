@@ -33,6 +33,10 @@ namespace {
 
 constexpr int kBT = 512;  // threads per block (two blocks per SM: at most 64 registers a thread)
 constexpr int kTb = 16;   // steps between checkpoints
+static_assert(PDSSM_MAX_N <= 256, "the dictionary is held in shared memory as uint8 row indices");
+static_assert(PDSSM_MAX_K <= 64, "warp 0 holds two selection logits a lane");
+static_assert(PDSSM_MAX_N + 128 <= kBT && PDSSM_MAX_P + 32 <= kBT,
+              "a thread per vector entry; dC uses threads 128.., dx threads 32..");
 
 struct BParams {
   int64_t L, H, N, P, K, nCk;
