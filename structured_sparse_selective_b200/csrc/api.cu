@@ -400,7 +400,7 @@ pdssm_status pdssm_select_proj(const pdssm_problem *pb, int64_t D, const void *u
   if (!mul_ok(pb->batch, pb->seqlen, &rows)) return PDSSM_ERR_UNSUPPORTED;
   if (rows > 0 && (!u || !W || !s)) return PDSSM_ERR_INVALID_ARG;
   if (!aligned(u, 16) || !aligned(W, 16) || !aligned(s, 4) || !aligned(logits, 16)) return PDSSM_ERR_INVALID_ARG;
-  if (!workspace || workspace_bytes < 4) return PDSSM_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < 256) return PDSSM_ERR_WORKSPACE;
   if (!aligned(workspace, 16)) return PDSSM_ERR_INVALID_ARG;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   pdssm_status st = bind_device(cs);

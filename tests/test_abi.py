@@ -247,6 +247,60 @@ def test_backward_validation():
     assert call(ws_bytes=n.value - 1) == 3  # PDSSM_ERR_WORKSPACE
 
 
+def test_dense_selection_validation():
+    """The dictionary hardmax, the fused projection, the soft selection and the scan with
+    per-step transitions reject bad sizes, unsupported shapes, missing or misaligned pointers
+    and small workspaces with a status, before any launch (fake pointers: nothing is read)."""
+    lib, fake, odd = pd._lib, ctypes.c_void_p(4096), ctypes.c_void_p(4098)
+    # pdssm_dict_hardmax(K, N, M, idx, stream)
+    assert lib.pdssm_dict_hardmax(-1, 8, fake, fake, None) == 1
+    assert lib.pdssm_dict_hardmax(4, 0, fake, fake, None) == 1
+    assert lib.pdssm_dict_hardmax(4, 129, fake, fake, None) == 2
+    assert lib.pdssm_dict_hardmax(0, 8, None, None, None) == OK  # nothing to do
+    assert lib.pdssm_dict_hardmax(4, 8, None, fake, None) == 1
+    assert lib.pdssm_dict_hardmax(4, 8, odd, fake, None) == 1
+
+    # pdssm_select_proj(pb, D, u, W, s, logits, workspace, bytes, stream)
+    def proj(D=128, ws_bytes=256, u=fake, W=fake, s_=fake, logits=None, ws=fake, **kw):
+        pb = _pb(**dict(dict(heads=4, K=8), **kw))
+        return lib.pdssm_select_proj(ctypes.byref(pb), D, u, W, s_, logits, ws, ws_bytes, None)
+    assert proj(D=0) == 1 and proj(heads=0) == 1 and proj(K=0) == 1
+    assert proj(K=128) == 2                       # above PDSSM_MAX_K
+    assert proj(K=6) == 2                         # not a power of two
+    assert proj(D=100) == 2                       # not a multiple of 64
+    assert proj(heads=3, K=4) == 2                # heads * K not a multiple of 32
+    assert proj(heads=40, K=8) == 2               # 320: above 256 and not a multiple of it
+    assert proj(u=None) == 1 and proj(W=None) == 1 and proj(s_=None) == 1
+    assert proj(u=odd) == 1 and proj(logits=odd) == 1
+    assert proj(ws_bytes=255) == 3 and proj(ws=None) == 3
+
+    # pdssm_soft_select_workspace_size / pdssm_soft_select(pb, logits, M, tau, idx_steps, ws, bytes, stream)
+    n = ctypes.c_size_t(0)
+    soft = dict(N=64, K=16, logits_t=pd.BF16)
+    assert lib.pdssm_soft_select_workspace_size(ctypes.byref(_pb(**soft)), ctypes.byref(n)) == OK
+    need = n.value
+    assert need >= 256 + 2 * 16 * 64 * 64 * 2  # error word + one dictionary's hi / lo parts
+    assert lib.pdssm_soft_select_workspace_size(ctypes.byref(_pb(N=48, K=16)), ctypes.byref(n)) == 2  # N not 2^k
+    assert lib.pdssm_soft_select_workspace_size(ctypes.byref(_pb(N=8, K=16)), ctypes.byref(n)) == 2   # N < 16
+
+    def softsel(tau=1.0, logits=fake, M=fake, steps=fake, ws=fake, ws_bytes=None):
+        return lib.pdssm_soft_select(ctypes.byref(_pb(**soft)), logits, M, ctypes.c_float(tau), steps, ws,
+                                     need if ws_bytes is None else ws_bytes, None)
+    assert softsel(tau=0.0) == 1 and softsel(tau=float("nan")) == 1
+    assert softsel(logits=None) == 1 and softsel(M=None) == 1 and softsel(steps=None) == 1
+    assert softsel(ws_bytes=need - 1) == 3
+
+    # pdssm_scan_fwd_steps: the fused kernel's shape only (N = P = 64, bf16 inputs, real state)
+    def steps(idx_steps=fake, **kw):
+        pb = _pb(**dict(dict(N=64, P=64, K=16, logits_t=pd.BF16, in_t=pd.BF16, d_t=pd.BF16, out_t=pd.BF16), **kw))
+        return lib.pdssm_scan_fwd_steps(ctypes.byref(pb), idx_steps, fake, fake, fake, fake, None, fake, None,
+                                        None, None, fake, 256, None)
+    assert steps(N=32, P=32) == 2
+    assert steps(in_t=pd.F32, d_t=pd.F32) == 2
+    assert steps(state_t=pd.C64, d_t=pd.C64, out_t=pd.C64) == 2
+    assert steps(idx_steps=None) == 1 and steps(idx_steps=odd) == 1
+
+
 def test_package_refuses_to_load_without_its_cuda_library(tmp_path):
     """No CPU fallback: a copy of the package without libpdssm.so raises on import."""
     import shutil
