@@ -157,3 +157,30 @@ def test_backward_reproduces_the_hand_worked_gradients(cuda_device, name):
 def test_backward_with_per_head_dictionaries(cuda_device, recipe, kw):
     errs = _run(recipe, kw, cuda_device, seed=6, head_dicts=True)
     assert all(v <= TOL for v in errs.values()), errs
+
+
+@pytest.mark.gpu
+def test_backward_full_size_lm_sampled_slices(cuda_device):
+    """The backward pass on the whole LM-layer workload (batch 8, L 2048, heads 32), in the
+    launch configuration the bench times; three sampled (batch, head) slices, the first and
+    the last among them, against the backward oracle (each slice depends on its own inputs
+    only)."""
+    sp = workloads.spec("lm")
+    inp = workloads.generate(sp, seed=12)
+    g = {k: v.to(cuda_device) for k, v in inp.items()}
+    fwd = pd.forward(g["logits"], g["idx"], g["d"], g["B"], g["C"], g["x"], want_s=True, want_prod=False)
+    gen = torch.Generator().manual_seed(112)
+    dy = torch.randn(sp.batch, sp.seqlen, sp.heads, sp.P, generator=gen).to(torch.bfloat16)
+    out = pd.backward(g["logits"], fwd["s"], g["idx"], g["d"], g["B"], g["C"], g["x"], dy.to(cuda_device), tau=0.8)
+    torch.cuda.synchronize(cuda_device)
+    idx = inp["idx"].numpy()
+    for b, h in [(0, 0), (3, 17), (sp.batch - 1, sp.heads - 1)]:
+        sl = {k: _np64(inp[k][b, :, h]) for k in ("logits", "d", "B", "C", "x")}
+        ref = bwd.slice_backward(sl["logits"], idx, sl["d"], sl["B"], sl["C"], sl["x"], _np64(dy[b, :, h]), tau=0.8)
+        assert np.array_equal(fwd["s"][b, :, h].cpu().numpy(), ref["s"])
+        for k in ("dd", "dB", "dC", "dx", "dlogits"):
+            got = _np64(out[k][b, :, h])
+            err = float(np.abs(got - ref[k]).max() / max(np.abs(ref[k]).max(), 1e-30))
+            assert err <= TOL, (b, h, k, err)
+        err = float(np.abs(_np64(out["dh0"][b, h]) - ref["dh0"]).max() / max(np.abs(ref["dh0"]).max(), 1e-30))
+        assert err <= TOL, (b, h, "dh0", err)
