@@ -299,10 +299,14 @@ pdssm_status pdssm_scan_fwd_steps(const pdssm_problem *pb, const uint8_t *idx_st
  * Backward pass: workspace bytes for pdssm_scan_bwd. Checkpoints of the state
  * every 16 steps plus a 16-step scratch per (batch, head) slice:
  * E * N * P * batch * heads * (ceil(L / 16) + 16) bytes (E = 4 for a real state,
- * 8 for a complex one), plus the dictionary's preimage lists.
- * PDSSM_ERR_UNSUPPORTED when one block's shared memory (three N x (P + 1)
- * state buffers and the dictionary) exceeds 227 KiB: every real problem up to
- * N = P = 128, K = 64 fits, and complex ones up to N = 128, P = 64, K = 64.
+ * 8 for a complex one), plus the dictionary's preimage lists. When there are
+ * fewer than about two sequences per SM, a sequence's columns are split over
+ * several blocks (a power of two nb dividing P) and the workspace also holds each
+ * block's share of the sums over columns: nb * batch * seqlen * heads *
+ * (N * (E + 8) + K * 4) bytes.
+ * A block holds three N x (its columns) state buffers and the dictionary in
+ * shared memory; where a whole row does not fit in 227 KiB the columns are split
+ * further, so every problem up to N = P = 128, K = 64 is supported, real or complex.
  */
 pdssm_status pdssm_bwd_workspace_size(const pdssm_problem *pb, size_t *bytes);
 

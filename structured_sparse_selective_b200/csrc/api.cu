@@ -217,16 +217,20 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &plan, const int32_t *
 // Workspace of the backward pass: error word, dictionary preimage lists,
 // checkpoints [Bt][H][nCk][N][P] and the per-slice scratch [Bt][H][16][N][P].
 struct BwdPlan {
-  int64_t Bt, L, H, N, P, K, rows, nCk, Kd, state_size;
-  size_t o_err, o_idx, o_off, o_src, o_ckpt, o_scr, total;
+  int64_t Bt, L, H, N, P, K, rows, nCk, Kd, state_size, nPB;
+  size_t o_err, o_idx, o_off, o_src, o_ckpt, o_scr, o_pdd, o_pdB, o_pdC, o_pdpi, total;
 };
 
 pdssm_status make_bwd_plan(const pdssm_problem *pb, BwdPlan *bp) {
   Plan p;
   pdssm_status st = make_plan(pb, &p, true);
   if (st != PDSSM_OK) return st;
-  if (scan_bwd_smem_bytes(p.N, p.P, p.K, p.cplx) > (size_t)227 * 1024) return PDSSM_ERR_UNSUPPORTED;
   BwdPlan q;
+  q.nPB = scan_bwd_column_blocks(p.Bt * p.H, p.P, p.cplx);
+  // more column blocks (narrower blocks) until one block's shared memory fits
+  while (scan_bwd_smem_bytes(p.N, p.P / q.nPB, p.K, p.cplx) > (size_t)227 * 1024 && p.P % (2 * q.nPB) == 0)
+    q.nPB *= 2;
+  if (scan_bwd_smem_bytes(p.N, p.P / q.nPB, p.K, p.cplx) > (size_t)227 * 1024) return PDSSM_ERR_UNSUPPORTED;
   q.state_size = p.state_size;
   q.Bt = p.Bt; q.L = p.L; q.H = p.H; q.N = p.N; q.P = p.P; q.K = p.K; q.rows = p.rows; q.Kd = p.Kd;
   q.nCk = scan_bwd_checkpoints(p.L);
@@ -241,6 +245,15 @@ pdssm_status make_bwd_plan(const pdssm_problem *pb, BwdPlan *bp) {
   q.o_src = o; o = align256(o + (size_t)(p.Kd * p.N) * 4);
   q.o_ckpt = o; o = align256(o + (size_t)(slices * q.nCk * p.N * p.P) * p.state_size);
   q.o_scr = o; o = align256(o + (size_t)(slices * scan_bwd_scratch_steps() * p.N * p.P) * p.state_size);
+  // the column blocks' shares of the sums over columns (none with one block a sequence)
+  int64_t parts64 = 0, check;
+  if (q.nPB > 1 && (!mul_ok(q.nPB, p.rows, &parts64) || !mul_ok(parts64, (p.N + p.K) * 16, &check)))
+    return PDSSM_ERR_UNSUPPORTED;
+  const size_t parts = (size_t)parts64;
+  q.o_pdd = o; o = align256(o + parts * p.N * p.state_size);
+  q.o_pdB = o; o = align256(o + parts * p.N * 4);
+  q.o_pdC = o; o = align256(o + parts * p.N * 4);
+  q.o_pdpi = o; o = align256(o + parts * p.K * 4);
   q.total = o;
   *bp = q;
   return PDSSM_OK;
@@ -533,6 +546,13 @@ pdssm_status pdssm_scan_bwd(const pdssm_problem *pb, const void *logits, const i
   a.h0 = h0; a.dh_final = dh_final;
   a.ckpt = base + q.o_ckpt;
   a.scratch = base + q.o_scr;
+  a.nPB = q.nPB;
+  if (q.nPB > 1) {
+    a.pdd = base + q.o_pdd;
+    a.pdB = reinterpret_cast<float *>(base + q.o_pdB);
+    a.pdC = reinterpret_cast<float *>(base + q.o_pdC);
+    a.pdpi = reinterpret_cast<float *>(base + q.o_pdpi);
+  }
   a.dlogits = dlogits; a.dd = dd; a.dB = dB; a.dC = dC; a.dx = dx; a.dh0 = dh0;
   a.ws = w;
   st = cuda_status(launch_scan_bwd(a, cs));

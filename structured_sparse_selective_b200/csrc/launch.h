@@ -76,12 +76,18 @@ struct ScanBwdArgs {
   void *dd, *dh0;
   Workspace ws;  // err, idx, csr_off, csr_src
   bool head_dicts = false;  // PDSSM_FLAG_HEAD_DICTS: dictionary entries h * K + k
+  int64_t nPB = 1;          // column blocks per sequence (scan_bwd_column_blocks)
+  void *pdd = nullptr;      // with nPB > 1: the blocks' shares [nPB][rows][N] (state type),
+  float *pdB = nullptr, *pdC = nullptr;  // [nPB][rows][N]
+  float *pdpi = nullptr;                 // [nPB][rows][K]
 };
 // Shared memory of one backward block, checkpoints of a sequence, and the steps
 // between checkpoints (the per-sequence scratch holds that many states).
 size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t K, bool cplx);
 int64_t scan_bwd_checkpoints(int64_t L);
 int64_t scan_bwd_scratch_steps();
+// Blocks a sequence's columns are split over (a power of two dividing P).
+int64_t scan_bwd_column_blocks(int64_t slices, int64_t P, bool cplx);
 cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t st);
 
 }  // namespace pdssm

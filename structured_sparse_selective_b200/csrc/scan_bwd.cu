@@ -31,15 +31,21 @@ namespace pdssm {
 
 namespace {
 
-constexpr int kBT = 512;  // threads per block (two blocks per SM: at most 64 registers a thread)
+// Threads per block: 512 when a block owns all P columns of its sequence, 256 when
+// the columns are split over several blocks (either way at most 64 registers a
+// thread: 2 or 4 blocks an SM).
+constexpr int kBTWhole = 512, kBTSplit = 256;
 constexpr int kTb = 16;   // steps between checkpoints
 static_assert(PDSSM_MAX_N <= 256, "the dictionary is held in shared memory as uint8 row indices");
 static_assert(PDSSM_MAX_K <= 64, "warp 0 holds two selection logits a lane");
-static_assert(PDSSM_MAX_N + 128 <= kBT && PDSSM_MAX_P + 32 <= kBT,
+static_assert(PDSSM_MAX_N + 128 <= kBTSplit && PDSSM_MAX_P + 32 <= kBTSplit,
               "a thread per vector entry; dC uses threads 128.., dx threads 32..");
 
 struct BParams {
   int64_t L, H, N, P, K, nCk;
+  int64_t Pg;    // columns of the state; a block owns P of them (P * nPB >= Pg)
+  int64_t nPB;   // column blocks per sequence
+  int64_t rows;  // batch * seqlen * heads
   float tau;
   int logits_bf16, dy_bf16;
   bool head_dicts;  // idx/off/src hold heads * K entries, head h's from h * K
@@ -49,10 +55,14 @@ struct BParams {
   const int32_t *src;  // [K][N]
   const void *logits, *d, *B, *C, *x, *dy;
   const void *h0, *dh_final;  // state type
-  void *ckpt;     // [Bt*H][nCk][N][P], state type
-  void *scratch;  // [Bt*H][kTb][N][P], state type
+  void *ckpt;     // [Bt*H*nPB][nCk][N][P], state type
+  void *scratch;  // [Bt*H*nPB][kTb][N][P], state type
   float *dlogits, *dB, *dC, *dx;
   void *dd, *dh0;  // state type
+  // with nPB > 1, each column block's share of the sums over columns, [nPB][rows][*]
+  // (the reduction kernel adds them and forms the logits' gradient)
+  void *pdd;
+  float *pdB, *pdC, *pdpi;
   uint32_t *err;
 };
 
@@ -96,19 +106,22 @@ __device__ __forceinline__ void st_run(float2 *p, const float2 (&v)[2]) {
   *reinterpret_cast<float4 *>(p) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
 }
 
-template <bool CPLX, typename TD, typename TIn>
-__global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
+template <bool CPLX, typename TD, typename TIn, int kBT>
+__global__ void __launch_bounds__(kBT, 1024 / kBT) scan_bwd_kernel(BParams a) {
   using NT = Num<CPLX>;
   using T = typename NT::T;
   constexpr int VW = 16 / (int)sizeof(T);  // values per 16-byte run
   extern __shared__ __align__(16) unsigned char smem[];
-  const int N = (int)a.N, P = (int)a.P, K = (int)a.K;
+  const int N = (int)a.N, K = (int)a.K;
+  const int P = (int)min(a.P, a.Pg - (int64_t)(blockIdx.x % a.nPB) * a.P);  // this block's columns
   // Rows hold PV = P rounded up to whole runs (the extra columns stay zero: their
   // x and dy are zero) plus one run of padding, which keeps rows 16-byte aligned
   // and puts consecutive rows 16 bytes apart in the banks.
   const int NR = (P + VW - 1) / VW, PV = NR * VW, PS = PV + VW;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+  const int64_t bh = blockIdx.x / a.nPB, pb = blockIdx.x % a.nPB, b = bh / a.H, h = bh % a.H;
+  const int64_t Pg = a.Pg, c0 = pb * a.P;  // this block's first column
+  const bool split = a.nPB > 1;
 
   T *buf0 = reinterpret_cast<T *>(smem);  // three [N][PS] buffers
   T *buf1 = buf0 + N * PS;
@@ -137,8 +150,8 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
   const T *h0g = static_cast<const T *>(a.h0);
   const T *dhg = static_cast<const T *>(a.dh_final);
   T *ddg = static_cast<T *>(a.dd);
-  T *ck = static_cast<T *>(a.ckpt) + bh * a.nCk * N * P;
-  T *scr = static_cast<T *>(a.scratch) + bh * (int64_t)kTb * N * P;
+  T *ck = static_cast<T *>(a.ckpt) + (int64_t)blockIdx.x * a.nCk * N * a.P;
+  T *scr = static_cast<T *>(a.scratch) + (int64_t)blockIdx.x * kTb * N * a.P;
 
   // loop over the runs of a dense [N][PV] array: thread tid starts at run tid
   const int dr = kBT / NR, dq = kBT - dr * NR;
@@ -175,8 +188,8 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
     }
     if (!rev && tid <= N) v.off = a.off[(kh + v.st) * (N + 1) + tid];
     if (tid < P) {
-      v.x = to_f32(xg[row * P + tid]);
-      if (rev) ld_dy(a.dy, row * P + tid, a.dy_bf16, &v.dy);
+      v.x = to_f32(xg[row * Pg + c0 + tid]);
+      if (rev) ld_dy(a.dy, row * Pg + c0 + tid, a.dy_bf16, &v.dy);
     }
     return v;
   };
@@ -213,34 +226,35 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
       st_run(Hn + i * PS + p0, acc);
     }
   };
-  // [N][P] in global memory <-> [N][PV] rows in shared memory (the padding columns read as zero)
-  auto store_dense = [&](const T *S, T *g) {
+  // [N][P] in global memory (rows ld apart) <-> [N][PV] rows in shared memory (the
+  // padding columns read as zero)
+  auto store_dense = [&](const T *S, T *g, int64_t ld) {
     FOR_RUNS(i, q) {
       const int p0 = q * VW;
       T v[VW];
       ld_run(S + i * PS + p0, v);
 #pragma unroll
       for (int e = 0; e < VW; ++e)
-        if (p0 + e < P) g[i * P + p0 + e] = v[e];
+        if (p0 + e < P) g[i * ld + p0 + e] = v[e];
     }
   };
-  auto load_dense = [&](const T *g, T *S) {
+  auto load_dense = [&](const T *g, T *S, int64_t ld) {
     FOR_RUNS(i, q) {
       const int p0 = q * VW;
       T v[VW];
 #pragma unroll
-      for (int e = 0; e < VW; ++e) v[e] = (g && p0 + e < P) ? g[i * P + p0 + e] : NT::zero();
+      for (int e = 0; e < VW; ++e) v[e] = (g && p0 + e < P) ? g[i * ld + p0 + e] : NT::zero();
       st_run(S + i * PS + p0, v);
     }
   };
 
   // ---- forward sweep: checkpoints every kTb steps
   T *Hc = buf0, *Hn = buf1;
-  load_dense(h0g ? h0g + bh * N * P : nullptr, Hc);
+  load_dense(h0g ? h0g + bh * N * Pg + c0 : nullptr, Hc, Pg);
   Vec nv = fetch(0, false);
   for (int64_t t = 0; t < a.L; ++t) {
     __syncthreads();  // Hc complete; the staged vectors are no longer read
-    if (t % kTb == 0) store_dense(Hc, ck + (t / kTb) * N * P);
+    if (t % kTb == 0) store_dense(Hc, ck + (t / kTb) * N * P, P);
     commit(nv, false);
     if (t + 1 < a.L) nv = fetch(t + 1, false);
     __syncthreads();
@@ -253,7 +267,7 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
   // ---- reverse sweep
   T *Lam = buf2;
   __syncthreads();
-  load_dense(dhg ? dhg + bh * N * P : nullptr, Lam);
+  load_dense(dhg ? dhg + bh * N * Pg + c0 : nullptr, Lam, Pg);
   for (int64_t c = a.nCk - 1; c >= 0; --c) {
     const int64_t t0 = c * kTb, t1 = t0 + kTb < a.L ? t0 + kTb : a.L;
     // recompute the stretch: scratch[t - t0] = H_{t-1}; Hc ends as H_{t1-1}
@@ -261,11 +275,11 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
     Hn = (Lam == buf2) ? buf1 : buf2;
     if (Lam == buf1) Hn = buf2;
     __syncthreads();
-    load_dense(ck + c * N * P, Hc);
+    load_dense(ck + c * N * P, Hc, P);
     nv = fetch(t0, false);
     for (int64_t t = t0; t < t1; ++t) {
       __syncthreads();
-      store_dense(Hc, scr + (t - t0) * N * P);
+      store_dense(Hc, scr + (t - t0) * N * P, P);
       commit(nv, false);
       if (t + 1 < t1) nv = fetch(t + 1, false);
       __syncthreads();
@@ -282,7 +296,7 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
       const int st = rv.st;
       commit(rv, true);
       if (t > t0) rv = fetch(t - 1, true);
-      load_dense(scr + (t - t0) * N * P, Hp);
+      load_dense(scr + (t - t0) * N * P, Hp, P);
       __syncthreads();
       // [B] Lam_t = Lam'_t + C_t dy_t^T
       FOR_RUNS(i, q) {
@@ -296,7 +310,12 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
       }
       __syncthreads();
       // [C] dB_t, dC_t (a thread per row), and per entry k, lanes over j:
-      // q_kj = sum_p Lam_t[idx_k[j]][p] conj(H_{t-1}[j][p]) (dd_t at k = s_t, dpi_t[k])
+      // q_kj = sum_p Lam_t[idx_k[j]][p] conj(H_{t-1}[j][p]) (dd_t at k = s_t, dpi_t[k]).
+      // These sum over the columns: a column block writes its share (sums over its own
+      // columns) to the partial arrays instead.
+      const int64_t prow = split ? pb * a.rows + row : row;  // row of the partial arrays
+      float *dBo = split ? a.pdB : a.dB, *dCo = split ? a.pdC : a.dC;
+      T *ddo = split ? static_cast<T *>(a.pdd) : ddg;
       if (tid < N) {
         float acc = 0.f;
         for (int q = 0; q < NR; ++q) {
@@ -305,7 +324,7 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
 #pragma unroll
           for (int e = 0; e < VW; ++e) acc = fmaf(re_of(v[e]), xsh[q * VW + e], acc);
         }
-        a.dB[row * N + tid] = acc;
+        dBo[prow * N + tid] = acc;
       }
       if (tid >= 128 && tid - 128 < N) {
         const int i = tid - 128;
@@ -316,7 +335,7 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
 #pragma unroll
           for (int e = 0; e < VW; ++e) acc = fma_re_conj(v[e], dysh[q * VW + e], acc);
         }
-        a.dC[row * N + i] = acc;
+        dCo[prow * N + i] = acc;
       }
       for (int k = warp; k < K; k += kBT / 32) {
         float part = 0.f;
@@ -334,17 +353,20 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
             }
           }
           const T qv = NT::add(q0, q1);
-          if (k == st) ddg[row * N + j] = qv;
+          if (k == st) ddo[prow * N + j] = qv;
           part = fma_re_conj(dsh[j], qv, part);  // Re(conj(q) d_j)
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        if (lane == 0) dpi[k] = part;
+        if (lane == 0) {
+          if (split) a.pdpi[prow * K + k] = part;
+          else dpi[k] = part;
+        }
       }
       __syncthreads();
       // [D] logits through the tempered softmax (warp 0); Lam'_{t-1} = A_t^H Lam_t into
       // Hc's buffer; dx_t
-      if (warp == 0 && a.dlogits) {
+      if (warp == 0 && a.dlogits && !split) {
         const float v0 = lane < K ? ld_flag(a.logits, row * K + lane, a.logits_bf16) / a.tau : -INFINITY;
         const float v1 = lane + 32 < K ? ld_flag(a.logits, row * K + lane + 32, a.logits_bf16) / a.tau : -INFINITY;
         float m = fmaxf(v0, v1);
@@ -375,7 +397,7 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
         const int p = tid - 32;
         float acc = 0.f;
         for (int i = 0; i < N; ++i) acc = fmaf(re_of(Lam[i * PS + p]), Bsh[i], acc);
-        a.dx[row * P + p] = acc;
+        a.dx[row * Pg + c0 + p] = acc;
       }
       // rotate: the new adjoint is in Hc's buffer, H_{t-1} becomes the next step's H_t
       T *old = Lam;
@@ -385,8 +407,56 @@ __global__ void __launch_bounds__(kBT, 2) scan_bwd_kernel(BParams a) {
     }
   }
   __syncthreads();
-  if (a.dh0) store_dense(Lam, static_cast<T *>(a.dh0) + bh * N * P);
+  if (a.dh0) store_dense(Lam, static_cast<T *>(a.dh0) + bh * N * Pg + c0, Pg);
 #undef FOR_RUNS
+}
+
+// Column blocks' shares summed in a fixed order (block 0 first): dd, dB, dC, and dpi,
+// which then goes through the tempered softmax's Jacobian into dlogits. One warp a row.
+template <bool CPLX>
+__global__ void __launch_bounds__(256) scan_bwd_reduce_kernel(BParams a) {
+  using NT = Num<CPLX>;
+  using T = typename NT::T;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (row >= a.rows) return;  // whole warps leave together
+  const int N = (int)a.N, K = (int)a.K;
+  const T *pdd = static_cast<const T *>(a.pdd);
+  for (int i = lane; i < N; i += 32) {
+    T dd = NT::zero();
+    float dB = 0.f, dC = 0.f;
+    for (int64_t pb = 0; pb < a.nPB; ++pb) {
+      const int64_t o = (pb * a.rows + row) * N + i;
+      dd = NT::add(dd, pdd[o]);
+      dB += a.pdB[o];
+      dC += a.pdC[o];
+    }
+    static_cast<T *>(a.dd)[row * N + i] = dd;
+    a.dB[row * N + i] = dB;
+    a.dC[row * N + i] = dC;
+  }
+  if (!a.dlogits) return;
+  float g0 = 0.f, g1 = 0.f;
+  for (int64_t pb = 0; pb < a.nPB; ++pb) {
+    const float *pp = a.pdpi + (pb * a.rows + row) * K;
+    if (lane < K) g0 += pp[lane];
+    if (lane + 32 < K) g1 += pp[lane + 32];
+  }
+  const float v0 = lane < K ? ld_flag(a.logits, row * K + lane, a.logits_bf16) / a.tau : -INFINITY;
+  const float v1 = lane + 32 < K ? ld_flag(a.logits, row * K + lane + 32, a.logits_bf16) / a.tau : -INFINITY;
+  float m = fmaxf(v0, v1);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float e0 = lane < K ? expf(v0 - m) : 0.f, e1 = lane + 32 < K ? expf(v1 - m) : 0.f;
+  float sum = e0 + e1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float p0 = e0 / sum, p1 = e1 / sum;
+  float dot = p0 * g0 + p1 * g1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  if (lane < K) a.dlogits[row * K + lane] = p0 * (g0 - dot) / a.tau;
+  if (lane + 32 < K) a.dlogits[row * K + lane + 32] = p1 * (g1 - dot) / a.tau;
 }
 
 }  // namespace
@@ -399,9 +469,20 @@ size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t K, bool cplx) {
 int64_t scan_bwd_checkpoints(int64_t L) { return (L + kTb - 1) / kTb; }
 int64_t scan_bwd_scratch_steps() { return kTb; }
 
+// Column blocks per sequence: doubled while the sequences alone give fewer than two
+// blocks an SM and the halves keep at least one 16-byte run of columns.
+int64_t scan_bwd_column_blocks(int64_t slices, int64_t P, bool cplx) {
+  const int64_t vw = cplx ? 2 : 4;
+  int64_t n = 1;
+  while (slices * n < 2 * 148 && P % (2 * n) == 0 && P / (2 * n) >= vw) n *= 2;
+  return n;
+}
+
 cudaError_t launch_scan_bwd(const ScanBwdArgs &s, cudaStream_t st) {
   BParams a;
-  a.L = s.L; a.H = s.H; a.N = s.N; a.P = s.P; a.K = s.K;
+  a.L = s.L; a.H = s.H; a.N = s.N; a.K = s.K;
+  a.Pg = s.P; a.nPB = s.nPB; a.P = s.P / s.nPB; a.rows = s.Bt * s.L * s.H;
+  a.pdd = s.pdd; a.pdB = s.pdB; a.pdC = s.pdC; a.pdpi = s.pdpi;
   a.nCk = scan_bwd_checkpoints(s.L);
   a.tau = s.tau;
   a.logits_bf16 = s.logits_t == PDSSM_BF16;
@@ -414,19 +495,36 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs &s, cudaStream_t st) {
   a.err = s.ws.err;
   a.head_dicts = s.head_dicts;
   const bool cplx = s.d_t == PDSSM_C64;
-  const size_t smem = scan_bwd_smem_bytes(s.N, s.P, s.K, cplx);
+  const size_t smem = scan_bwd_smem_bytes(s.N, a.P, s.K, cplx);
+  const bool split = s.nPB > 1;
   void (*kern)(BParams);
-  if (cplx)
-    kern = s.in_t == PDSSM_BF16 ? scan_bwd_kernel<true, float2, __nv_bfloat16> : scan_bwd_kernel<true, float2, float>;
-  else if (s.d_t == PDSSM_BF16)
-    kern = s.in_t == PDSSM_BF16 ? scan_bwd_kernel<false, __nv_bfloat16, __nv_bfloat16>
-                                : scan_bwd_kernel<false, __nv_bfloat16, float>;
-  else
-    kern = s.in_t == PDSSM_BF16 ? scan_bwd_kernel<false, float, __nv_bfloat16> : scan_bwd_kernel<false, float, float>;
+#define PDSSM_BWD_KERNEL(BT)                                                                              \
+  if (cplx)                                                                                               \
+    kern = s.in_t == PDSSM_BF16 ? scan_bwd_kernel<true, float2, __nv_bfloat16, BT>                        \
+                                : scan_bwd_kernel<true, float2, float, BT>;                               \
+  else if (s.d_t == PDSSM_BF16)                                                                           \
+    kern = s.in_t == PDSSM_BF16 ? scan_bwd_kernel<false, __nv_bfloat16, __nv_bfloat16, BT>                \
+                                : scan_bwd_kernel<false, __nv_bfloat16, float, BT>;                       \
+  else                                                                                                    \
+    kern = s.in_t == PDSSM_BF16 ? scan_bwd_kernel<false, float, __nv_bfloat16, BT>                        \
+                                : scan_bwd_kernel<false, float, float, BT>;
+  if (split) {
+    PDSSM_BWD_KERNEL(kBTSplit)
+  } else {
+    PDSSM_BWD_KERNEL(kBTWhole)
+  }
+#undef PDSSM_BWD_KERNEL
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if ((e = trace_before(st, "scan_bwd")) != cudaSuccess) return e;
-  kern<<<(unsigned)(s.Bt * s.H), kBT, smem, st>>>(a);
+  kern<<<(unsigned)(s.Bt * s.H * s.nPB), split ? kBTSplit : kBTWhole, smem, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = trace_after(st)) != cudaSuccess) return e;
+  if (!split) return cudaSuccess;
+  if ((e = trace_before(st, "scan_bwd_reduce")) != cudaSuccess) return e;
+  const int64_t warps = a.rows, blocks = (warps * 32 + 255) / 256;
+  if (cplx) scan_bwd_reduce_kernel<true><<<(unsigned)blocks, 256, 0, st>>>(a);
+  else scan_bwd_reduce_kernel<false><<<(unsigned)blocks, 256, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return trace_after(st);
 }

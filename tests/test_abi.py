@@ -215,19 +215,22 @@ def test_default_chunk_keeps_the_workspace_below_the_fixed_chunk_one():
 
 
 def test_backward_validation():
-    """pdssm_scan_bwd rejects a problem whose block does not fit in shared memory, a
-    non-positive temperature, logits without dlogits (and the reverse), missing pointers
-    and a small workspace, before any launch."""
+    """pdssm_bwd_workspace_size serves every shape up to the size limits, and
+    pdssm_scan_bwd rejects a non-positive temperature, logits without dlogits (and the
+    reverse), missing pointers and a small workspace, before any launch."""
     n = ctypes.c_size_t(0)
     cplx = dict(state_t=pd.C64, d_t=pd.C64, out_t=pd.C64)
-    # complex N = 128, P = 64 fits (complex checkpoints: twice the real bytes); P = 128 does not
-    assert pd._lib.pdssm_bwd_workspace_size(ctypes.byref(_pb(N=128, P=64, K=64, **cplx)), ctypes.byref(n)) == OK
-    n_c = n.value
-    assert pd._lib.pdssm_bwd_workspace_size(ctypes.byref(_pb(N=128, P=64, K=64)), ctypes.byref(n)) == OK
-    assert n_c > 1.9 * n.value
-    assert pd._lib.pdssm_bwd_workspace_size(ctypes.byref(_pb(N=128, P=128, K=64, **cplx)),
-                                            ctypes.byref(n)) == 2  # PDSSM_ERR_UNSUPPORTED
-    assert pd._lib.pdssm_bwd_workspace_size(ctypes.byref(_pb(N=128, P=128, K=64)), ctypes.byref(n)) == OK
+    # complex states take twice the checkpoint bytes of real ones; the largest shapes fit
+    # (a block's columns are split until its shared memory does), many sequences or few
+    for kw in (dict(batch=1024, heads=1), dict(batch=2, heads=3)):
+        assert pd._lib.pdssm_bwd_workspace_size(ctypes.byref(_pb(N=128, P=64, K=64, **cplx, **kw)),
+                                                ctypes.byref(n)) == OK
+        n_c = n.value
+        assert pd._lib.pdssm_bwd_workspace_size(ctypes.byref(_pb(N=128, P=64, K=64, **kw)), ctypes.byref(n)) == OK
+        assert n_c > 1.9 * n.value
+        for c in (cplx, {}):
+            assert pd._lib.pdssm_bwd_workspace_size(ctypes.byref(_pb(N=128, P=128, K=64, **c, **kw)),
+                                                    ctypes.byref(n)) == OK
     pb = _pb()
     assert pd._lib.pdssm_bwd_workspace_size(ctypes.byref(pb), ctypes.byref(n)) == OK and n.value > 0
     fake = ctypes.c_void_p(4096)

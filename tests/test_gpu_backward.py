@@ -111,6 +111,20 @@ def test_backward_complex_maximum_sizes(cuda_device):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("recipe,kw", [
+    ("lm", dict(batch=150, seqlen=10, heads=2)),                        # 300 sequences: whole rows
+    ("complex", dict(batch=300, seqlen=12, heads=1, N=16, P=8, K=4)),   # 300 sequences: whole rows
+    ("complex", dict(batch=1, seqlen=10, heads=1, N=128, P=128, K=64)),  # rows split to fit
+])
+def test_backward_whole_and_split_column_blocks(cuda_device, recipe, kw):
+    """With about two sequences per SM or more a block owns whole state rows; with fewer,
+    or when a whole row does not fit in shared memory, a sequence's columns are split over
+    blocks whose shares of the column sums a second kernel adds. Both match the oracle."""
+    errs = _run(recipe, kw, cuda_device, seed=10)
+    assert all(v <= TOL for v in errs.values()), errs
+
+
+@pytest.mark.gpu
 def test_backward_complex_without_initial_state_or_logits(cuda_device):
     errs = _run("complex", dict(batch=1, seqlen=33, heads=2, N=32, P=16, K=8), cuda_device, seed=9,
                 with_h0=False, with_dh=False, with_logits=False)
