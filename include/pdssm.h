@@ -297,9 +297,11 @@ pdssm_status pdssm_scan_fwd_steps(const pdssm_problem *pb, const uint8_t *idx_st
 
 /*
  * Backward pass: workspace bytes for pdssm_scan_bwd. Checkpoints of the state
- * every 16 steps plus a 16-step scratch per (batch, head) slice:
+ * every 16 steps (the carries of the chunked forward scan at chunk length 16, with
+ * their chunk pairs) plus a 16-step scratch per (batch, head) slice:
  * E * N * P * batch * heads * (ceil(L / 16) + 16) bytes (E = 4 for a real state,
- * 8 for a complex one), plus the dictionary's preimage lists. When there are
+ * 8 for a complex one), batch * heads * ceil(L / 16) * N * (4 + E) bytes of pairs,
+ * plus the dictionary's preimage lists. When there are
  * fewer than about two sequences per SM, a sequence's columns are split over
  * several blocks (a power of two nb dividing P) and the workspace also holds each
  * block's share of the sums over columns: nb * batch * seqlen * heads *

@@ -218,7 +218,7 @@ pdssm_status run_scan(const pdssm_problem *pb, const Plan &plan, const int32_t *
 // checkpoints [Bt][H][nCk][N][P] and the per-slice scratch [Bt][H][16][N][P].
 struct BwdPlan {
   int64_t Bt, L, H, N, P, K, rows, nCk, Kd, state_size, nPB;
-  size_t o_err, o_idx, o_off, o_src, o_ckpt, o_scr, o_pdd, o_pdB, o_pdC, o_pdpi, total;
+  size_t o_err, o_idx, o_off, o_src, o_ckpt, o_cidx, o_cval, o_scr, o_pdd, o_pdB, o_pdC, o_pdpi, total;
 };
 
 pdssm_status make_bwd_plan(const pdssm_problem *pb, BwdPlan *bp) {
@@ -243,7 +243,10 @@ pdssm_status make_bwd_plan(const pdssm_problem *pb, BwdPlan *bp) {
   q.o_idx = o; o = align256(o + (size_t)(p.Kd * p.N) * 4);
   q.o_off = o; o = align256(o + (size_t)(p.Kd * (p.N + 1)) * 4);
   q.o_src = o; o = align256(o + (size_t)(p.Kd * p.N) * 4);
+  // checkpoints: the chunked forward's carries at chunk length 16, with its chunk pairs
   q.o_ckpt = o; o = align256(o + (size_t)(slices * q.nCk * p.N * p.P) * p.state_size);
+  q.o_cidx = o; o = align256(o + (size_t)(slices * q.nCk * p.N) * 4);
+  q.o_cval = o; o = align256(o + (size_t)(slices * q.nCk * p.N) * p.state_size);
   q.o_scr = o; o = align256(o + (size_t)(slices * scan_bwd_scratch_steps() * p.N * p.P) * p.state_size);
   // the column blocks' shares of the sums over columns (none with one block a sequence)
   int64_t parts64 = 0, check;
@@ -537,6 +540,23 @@ pdssm_status pdssm_scan_bwd(const pdssm_problem *pb, const void *logits, const i
   }
   st = cuda_status(launch_prep_dict(idx, (int)q.Kd, (int)q.N, w, cs));
   if (st != PDSSM_OK) return st;
+  {
+    // the checkpoints: the states after each 16-step chunk, by phases A and B of the
+    // chunked forward scan (parallel over the chunks)
+    ScanArgs f{};
+    f.Bt = q.Bt; f.L = q.L; f.H = q.H; f.N = q.N; f.P = q.P; f.K = q.K;
+    f.T = scan_bwd_scratch_steps(); f.nC = q.nCk;
+    f.d_t = pb->d_t; f.in_t = pb->in_t; f.out_t = pb->out_t; f.logits_t = pb->logits_t;
+    f.cplx = q.state_size == 8;
+    f.s = s; f.idx = idx; f.d = d; f.B = B; f.C = C; f.x = x; f.h0 = h0;
+    f.ws = w;
+    f.ws.chunk_state = base + q.o_ckpt;
+    f.ws.chunk_idx = reinterpret_cast<int32_t *>(base + q.o_cidx);
+    f.ws.chunk_val = base + q.o_cval;
+    f.head_dicts = (pb->flags & PDSSM_FLAG_HEAD_DICTS) != 0;
+    st = cuda_status(launch_chunked_carries(f, cs));
+    if (st != PDSSM_OK) return st;
+  }
   ScanBwdArgs a;
   a.head_dicts = (pb->flags & PDSSM_FLAG_HEAD_DICTS) != 0;
   a.Bt = q.Bt; a.L = q.L; a.H = q.H; a.N = q.N; a.P = q.P; a.K = q.K;

@@ -47,6 +47,10 @@ bool fused_scan_pointers_ok(const ScanArgs &a);
 cudaError_t launch_fused_scan(const ScanArgs &a, cudaStream_t st);
 // Outputs of an empty sequence (L == 0): h_final = h0 (or 0), prod = identity.
 cudaError_t launch_empty_outputs(const ScanArgs &a, cudaStream_t st);
+// Phases A and B of the chunked scan only: chunk_state[c] ends as the state after
+// chunk c (the carry), h_final / prod_* written when given; no outputs, no y_loc
+// (ws.y_loc may be null).
+cudaError_t launch_chunked_carries(const ScanArgs &a, cudaStream_t st);
 
 // Fused projection and selection on the tensor cores, and dictionary construction
 // by column-wise hardmax (csrc/select_gemm.cu).

@@ -18,13 +18,14 @@
 //   dC_t = Re(H_t conj(dy_t)), dB_t = Re(Lam_t) x_t, dx_t = Re(Lam_t)^T B_t,
 //   dd_t[j] = sum_p Lam_t[idx_{s_t}[j]][p] conj(H_{t-1}[j][p]).
 //
-// One block per (batch, head) sequence. A forward sweep stores the state every
-// kTb steps (O(L N P / kTb) memory, O(L N) for kTb >= P); the reverse sweep
-// recomputes each kTb-step stretch from its checkpoint into a per-sequence
-// scratch and walks it backwards. Three N x P buffers in shared memory hold the
-// adjoint, H_t and H_{t-1}; threads move their rows in 16-byte runs (4 real or 2
-// complex values), so a row's preimage list or dictionary row is read once per
-// run.
+// One block per (batch, head) sequence, or per range of its columns. The
+// checkpoints, the state every kTb steps (O(L N P / kTb) memory), are the carries
+// of the chunked forward scan at chunk length kTb, computed in parallel over the
+// chunks before this kernel; the reverse sweep recomputes each kTb-step stretch
+// from its checkpoint into a per-block scratch and walks it backwards. Three N x P
+// buffers in shared memory hold the adjoint, H_t and H_{t-1}; threads move their
+// rows in 16-byte runs (4 real or 2 complex values), so a row's preimage list or
+// dictionary row is read once per run.
 #include "launch.h"
 
 namespace pdssm {
@@ -55,7 +56,7 @@ struct BParams {
   const int32_t *src;  // [K][N]
   const void *logits, *d, *B, *C, *x, *dy;
   const void *h0, *dh_final;  // state type
-  void *ckpt;     // [Bt*H*nPB][nCk][N][P], state type
+  const void *ckpt;  // [Bt*H][nCk][N][Pg] state type: the state after each 16-step chunk
   void *scratch;  // [Bt*H*nPB][kTb][N][P], state type
   float *dlogits, *dB, *dC, *dx;
   void *dd, *dh0;  // state type
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(kBT, 1024 / kBT) scan_bwd_kernel(BParams a) {
   const T *h0g = static_cast<const T *>(a.h0);
   const T *dhg = static_cast<const T *>(a.dh_final);
   T *ddg = static_cast<T *>(a.dd);
-  T *ck = static_cast<T *>(a.ckpt) + (int64_t)blockIdx.x * a.nCk * N * a.P;
+  const T *ck = static_cast<const T *>(a.ckpt) + bh * a.nCk * N * Pg + c0;  // this block's columns
   T *scr = static_cast<T *>(a.scratch) + (int64_t)blockIdx.x * kTb * N * a.P;
 
   // loop over the runs of a dense [N][PV] array: thread tid starts at run tid
@@ -248,21 +249,11 @@ __global__ void __launch_bounds__(kBT, 1024 / kBT) scan_bwd_kernel(BParams a) {
     }
   };
 
-  // ---- forward sweep: checkpoints every kTb steps
+  // The checkpoints (the state before steps 0, kTb, 2 kTb, ...) are h0 and the
+  // carries of the chunked forward scan (phases A and B at chunk length kTb), which
+  // the caller computes in parallel over the chunks before this kernel.
   T *Hc = buf0, *Hn = buf1;
-  load_dense(h0g ? h0g + bh * N * Pg + c0 : nullptr, Hc, Pg);
-  Vec nv = fetch(0, false);
-  for (int64_t t = 0; t < a.L; ++t) {
-    __syncthreads();  // Hc complete; the staged vectors are no longer read
-    if (t % kTb == 0) store_dense(Hc, ck + (t / kTb) * N * P, P);
-    commit(nv, false);
-    if (t + 1 < a.L) nv = fetch(t + 1, false);
-    __syncthreads();
-    step_fwd(Hc, Hn);
-    T *tmp = Hc;
-    Hc = Hn;
-    Hn = tmp;
-  }
+  Vec nv;
 
   // ---- reverse sweep
   T *Lam = buf2;
@@ -275,7 +266,8 @@ __global__ void __launch_bounds__(kBT, 1024 / kBT) scan_bwd_kernel(BParams a) {
     Hn = (Lam == buf2) ? buf1 : buf2;
     if (Lam == buf1) Hn = buf2;
     __syncthreads();
-    load_dense(ck + c * N * P, Hc, P);
+    if (c == 0) load_dense(h0g ? h0g + bh * N * Pg + c0 : nullptr, Hc, Pg);
+    else load_dense(ck + (c - 1) * N * Pg, Hc, Pg);
     nv = fetch(t0, false);
     for (int64_t t = t0; t < t1; ++t) {
       __syncthreads();

@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(RG * ColRun<typename Num<CPLX>::T>::TPR,
   };
   // output of step t from the warps' parts (fixed order)
   auto finish_y = [&](int64_t t) {
-    if (tid < P) {
+    if (tid < P && yl) {  // no local outputs when only the carries are wanted
       T acc = ysh[tid];
 #pragma unroll
       for (int w = 1; w < NW; ++w) acc = Nm::add(acc, ysh[w * kPB + tid]);
@@ -522,7 +522,8 @@ cudaError_t launch_dyn(Kern kern, const char *name, dim3 grid, int threads, size
   return trace_after(st);
 }
 
-// NMAX bounds N (16, 32, 64 or 128); it sizes every phase's row groups.
+// NMAX bounds N (16, 32, 64 or 128); it sizes every phase's row groups. Without an
+// output (s.y null) only phases A and B run: the carries at the chunk ends.
 template <int NMAX, bool CPLX, typename TD, typename TIn, typename TOut>
 cudaError_t run_chunked_n(const ScanArgs &s, cudaStream_t st) {
   using T = typename Num<CPLX>::T;
@@ -540,7 +541,7 @@ cudaError_t run_chunked_n(const ScanArgs &s, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   e = launch_dyn(phase_b_kernel<RGB, PBB, MRB, CPLX>, "chunked_phase_b", dim3((unsigned)(s.H * k.nPBB), (unsigned)s.Bt), NTB,
                  smem_b, st, k);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || !s.y) return e;
   return launch_dyn(phase_c_kernel<RGA, CPLX, TD, TIn, TOut>, "chunked_phase_c", grid_chunks, NTA, smem_c, st, k);
 }
 
@@ -571,6 +572,14 @@ cudaError_t launch_chunked_scan(const ScanArgs &s, cudaStream_t st) {
   PDSSM_REAL_CASE(PDSSM_BF16, PDSSM_BF16, PDSSM_BF16, __nv_bfloat16, __nv_bfloat16, __nv_bfloat16)
 #undef PDSSM_REAL_CASE
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_chunked_carries(const ScanArgs &s, cudaStream_t st) {
+  // phases A and B only: the output type is not used
+  ScanArgs c = s;
+  c.y = nullptr;
+  c.out_t = c.cplx ? PDSSM_C64 : PDSSM_F32;
+  return launch_chunked_scan(c, st);
 }
 
 cudaError_t launch_empty_outputs(const ScanArgs &s, cudaStream_t st) {
