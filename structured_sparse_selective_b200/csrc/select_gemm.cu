@@ -8,6 +8,7 @@
 //   - dictionary construction: each of the K sparse dictionary matrices is the
 //     column-wise hardmax of a dense trainable matrix, idx[k][j] = argmax_i M[k][i][j].
 #include <algorithm>
+#include <type_traits>
 
 #include "launch.h"
 #include "sm100.cuh"
@@ -222,6 +223,25 @@ __global__ void __launch_bounds__(256) soft_prep_kernel(const float *__restrict_
 //   (r % 8) * 16 + (r / 8) * (K16 * 16) + (k / 8) * 128 + (k % 8) * 2
 // B = dictionary part [K16 x 256 columns (j, i)], MN-major:
 //   (k % 8) * 16 + (k / 8) * 4096 + (n / 8) * 128 + (n % 8) * 2
+// The selection's winner (sel_merge's order: the first NaN, else the maximum, +0 == -0,
+// the lowest index on ties) among CW consecutive values: a maximum and a search for its
+// first occurrence instead of CW sequential merges.
+template <int CW>
+__device__ __forceinline__ void run_winner(const float *v, float &val, int &idx) {
+  float m = v[0];
+  bool nan = false;
+#pragma unroll
+  for (int c = 0; c < CW; ++c) {
+    m = fmaxf(m, v[c]);
+    nan |= v[c] != v[c];
+  }
+  idx = 0;
+#pragma unroll
+  for (int c = CW - 1; c >= 0; --c)
+    if (nan ? v[c] != v[c] : v[c] == m) idx = c;
+  val = nan ? v[idx] : m;
+}
+
 __global__ void __launch_bounds__(kPThreads) soft_select_kernel(SParams a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int aBytes = kSM * a.K16 * 2;             // one pi part
@@ -315,21 +335,34 @@ __global__ void __launch_bounds__(kPThreads) soft_select_kernel(SParams a) {
     }
     ok = __syncthreads_and(ok && pwait(done, nt & 1, a.err));
     tc_fence_after();
-    // columns jj * N + i of this tile: argmax over i for each j
+    // columns jj * N + i of this tile: argmax over i for each j, by runs of CW
+    // consecutive i (the winner of a run merged into the group's)
     float bv = 0.f;
     int bi = INT_MAX;
+    auto runs = [&](auto cw_tag, const float *v, int c0) {
+      constexpr int CW = decltype(cw_tag)::value;
+#pragma unroll
+      for (int h0 = 0; h0 < 32; h0 += CW) {
+        float cv;
+        int ci;
+        run_winner<CW>(v + h0, cv, ci);
+        const int col = c0 + h0, i0 = col & (a.N - 1);
+        if (i0 == 0) {  // a new group: its first run's winner
+          bv = cv;
+          bi = ci;
+        } else {
+          sel_merge(bv, bi, cv, i0 + ci);
+        }
+        if (i0 + CW == a.N && ok && row < a.rows)
+          a.steps[(row * a.H + h) * a.N + nt * groups + col / a.N] = (uint8_t)bi;
+      }
+    };
     for (int c0 = 0; c0 < 256; c0 += 32) {
       float v[32];
       tmem_ld32(tl + c0, v);
       tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int col = c0 + c, i = col & (a.N - 1);
-        if (i == 0) bi = INT_MAX;
-        sel_merge(bv, bi, v[c], i);
-        if (i == a.N - 1 && ok && row < a.rows)
-          a.steps[(row * a.H + h) * a.N + nt * groups + col / a.N] = (uint8_t)bi;
-      }
+      if (a.N == 16) runs(std::integral_constant<int, 16>{}, v, c0);
+      else runs(std::integral_constant<int, 32>{}, v, c0);
     }
     tc_fence_before();
   }
