@@ -55,6 +55,27 @@ __device__ __noinline__ bool pwait(uint64_t *bar, uint32_t parity, uint32_t *err
   return true;
 }
 
+// The selection's winner (sel_merge's order: the first NaN, else the maximum, +0 == -0,
+// the lowest index on ties) among CW consecutive values: a maximum and a search for its
+// first occurrence instead of CW sequential merges.
+template <int CW>
+__device__ __forceinline__ void run_winner(const float *v, float &val, int &idx) {
+  float m = v[0];
+  bool nan = false;
+#pragma unroll
+  for (int c = 0; c < CW; ++c) {
+    m = fmaxf(m, v[c]);
+    nan |= v[c] != v[c];
+  }
+  idx = 0;
+#pragma unroll
+  for (int c = CW - 1; c >= 0; --c)
+    if (nan ? v[c] != v[c] : v[c] == m) idx = c;
+  // the merge looks only at whether a winner is a NaN, so any NaN stands for one (and
+  // no run-time index into v, which would move it to local memory)
+  val = nan ? __int_as_float(0x7fffffff) : m;
+}
+
 // One CTA: rows [row0, row0 + 128) x columns [n0, n0 + ntile) of u W, reduced over
 // D in steps of 64 through two cp.async stages. Stage layouts (no swizzle, 8-row
 // x 16-byte core matrices):
@@ -136,26 +157,47 @@ __global__ void __launch_bounds__(kPThreads) proj_select_kernel(PParams a) {
   const int64_t row = row0 + warp * 32 + lane;
   const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
   const int64_t heads = a.HK / a.K;
-  float bv = 0.f;
-  int bk = INT_MAX;
-  for (int c0 = 0; c0 < a.ntile; c0 += 32) {
-    float v[32];
-    tmem_ld32(tl + c0, v);
-    tmem_wait_ld();
-    if (ok && row < a.rows) {
-      if (a.logits) {
-        float4 *dst = reinterpret_cast<float4 *>(a.logits + row * a.HK + n0 + c0);
+  // each head's K scores by runs of CW = min(K, 32) consecutive columns: the run's
+  // winner, merged into the head's (one instantiation of the loop per CW, so that the
+  // loaded columns stay in registers)
+  auto epilogue = [&](auto cw_tag) {
+    constexpr int CW = decltype(cw_tag)::value;
+    float bv = 0.f;
+    int bk = INT_MAX;
+    for (int c0 = 0; c0 < a.ntile; c0 += 32) {
+      float v[32];
+      tmem_ld32(tl + c0, v);
+      tmem_wait_ld();
+      if (ok && row < a.rows) {
+        if (a.logits) {
+          float4 *dst = reinterpret_cast<float4 *>(a.logits + row * a.HK + n0 + c0);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-      }
+          for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int k = (c0 + c) & (a.K - 1);
-        if (k == 0) bk = INT_MAX;
-        sel_merge(bv, bk, v[c], k);
-        if (k == a.K - 1) a.s[row * heads + (n0 + c0 + c) / a.K] = bk;
+        for (int h0 = 0; h0 < 32; h0 += CW) {
+          float cv;
+          int ci;
+          run_winner<CW>(v + h0, cv, ci);
+          const int k0 = (c0 + h0) & (a.K - 1);
+          if (k0 == 0) {
+            bv = cv;
+            bk = ci;
+          } else {
+            sel_merge(bv, bk, cv, k0 + ci);
+          }
+          if (k0 + CW == a.K) a.s[row * heads + (n0 + c0 + h0) / a.K] = bk;
+        }
       }
     }
+  };
+  switch (a.K) {
+    case 1: epilogue(std::integral_constant<int, 1>{}); break;
+    case 2: epilogue(std::integral_constant<int, 2>{}); break;
+    case 4: epilogue(std::integral_constant<int, 4>{}); break;
+    case 8: epilogue(std::integral_constant<int, 8>{}); break;
+    case 16: epilogue(std::integral_constant<int, 16>{}); break;
+    default: epilogue(std::integral_constant<int, 32>{}); break;
   }
   tc_fence_before();
   __syncthreads();
@@ -223,25 +265,6 @@ __global__ void __launch_bounds__(256) soft_prep_kernel(const float *__restrict_
 //   (r % 8) * 16 + (r / 8) * (K16 * 16) + (k / 8) * 128 + (k % 8) * 2
 // B = dictionary part [K16 x 256 columns (j, i)], MN-major:
 //   (k % 8) * 16 + (k / 8) * 4096 + (n / 8) * 128 + (n % 8) * 2
-// The selection's winner (sel_merge's order: the first NaN, else the maximum, +0 == -0,
-// the lowest index on ties) among CW consecutive values: a maximum and a search for its
-// first occurrence instead of CW sequential merges.
-template <int CW>
-__device__ __forceinline__ void run_winner(const float *v, float &val, int &idx) {
-  float m = v[0];
-  bool nan = false;
-#pragma unroll
-  for (int c = 0; c < CW; ++c) {
-    m = fmaxf(m, v[c]);
-    nan |= v[c] != v[c];
-  }
-  idx = 0;
-#pragma unroll
-  for (int c = CW - 1; c >= 0; --c)
-    if (nan ? v[c] != v[c] : v[c] == m) idx = c;
-  val = nan ? v[idx] : m;
-}
-
 __global__ void __launch_bounds__(kPThreads) soft_select_kernel(SParams a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int aBytes = kSM * a.K16 * 2;             // one pi part
