@@ -100,7 +100,8 @@ __device__ __forceinline__ void st_run(float2 *p, const float2 (&v)[2]) {
 
 // Threads: RG row groups of TPR threads; thread (g, cl) updates rows g, g + RG, ...
 // of columns [cl * VW, cl * VW + VW) of the block's kPB columns.
-template <int RG, bool CPLX, typename TD, typename TIn>
+// kLocalOut: write y_loc (false when only the carries are wanted).
+template <int RG, bool CPLX, typename TD, typename TIn, bool kLocalOut>
 __global__ void __launch_bounds__(RG * ColRun<typename Num<CPLX>::T>::TPR,
                                   CPLX ? 1024 / (RG * ColRun<typename Num<CPLX>::T>::TPR) : 0)
     phase_a_kernel(KParams a) {
@@ -160,7 +161,7 @@ __global__ void __launch_bounds__(RG * ColRun<typename Num<CPLX>::T>::TPR,
   };
   // output of step t from the warps' parts (fixed order)
   auto finish_y = [&](int64_t t) {
-    if (tid < P && yl) {  // no local outputs when only the carries are wanted
+    if (kLocalOut && tid < P) {
       T acc = ysh[tid];
 #pragma unroll
       for (int w = 1; w < NW; ++w) acc = Nm::add(acc, ysh[w * kPB + tid]);
@@ -537,7 +538,10 @@ cudaError_t run_chunked_n(const ScanArgs &s, cudaStream_t st) {
   const size_t smem_b = N * PBB * ts + N * ts + N * 4 + (2 * N + 1) * 4;
   const size_t smem_c = N * kPB * ts + (NTA / 32) * kTG * kPB * ts + 2 * kTG * N * ts + kTG * N * 4 + kTG * 4;
   const dim3 grid_chunks((unsigned)(s.nC * k.nPB), (unsigned)s.H, (unsigned)s.Bt);
-  cudaError_t e = launch_dyn(phase_a_kernel<RGA, CPLX, TD, TIn>, "chunked_phase_a", grid_chunks, NTA, smem_a, st, k);
+  cudaError_t e = s.y ? launch_dyn(phase_a_kernel<RGA, CPLX, TD, TIn, true>, "chunked_phase_a", grid_chunks, NTA,
+                                   smem_a, st, k)
+                      : launch_dyn(phase_a_kernel<RGA, CPLX, TD, TIn, false>, "chunked_phase_a", grid_chunks, NTA,
+                                   smem_a, st, k);
   if (e != cudaSuccess) return e;
   e = launch_dyn(phase_b_kernel<RGB, PBB, MRB, CPLX>, "chunked_phase_b", dim3((unsigned)(s.H * k.nPBB), (unsigned)s.Bt), NTB,
                  smem_b, st, k);
