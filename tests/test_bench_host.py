@@ -37,7 +37,8 @@ def test_traffic_absent_without_summary_or_known_sources(tmp_path, monkeypatch):
     assert bench.recorded_traffic("unknown", "wl") is None
 
 
-@pytest.mark.parametrize("kernel,workload", [("fused_scan", "lm"), ("chunked_phase_a", "long")])
+@pytest.mark.parametrize("kernel,workload", [("fused_scan", "lm"), ("chunked_phase_a", "long"),
+                                             ("chunked_phase_a", "complex")])
 def test_committed_summary_names_known_sources(kernel, workload):
     path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles",
                         f"{kernel}_{workload}.md")
@@ -102,3 +103,26 @@ def test_backward_bytes_per_token_head():
     dd, dB, dC, dx, dlogits (3 x 64 + 64 + 16) x 4 written."""
     import workloads
     assert bench.bwd_bytes_per_token_head(workloads.spec("lm")) == 4 + 32 + 384 + 256 + 272 * 4
+
+
+def test_profiling_overrides_shorten_only_the_named_dimensions():
+    """--batch / --seqlen (profiling captures) replace those sizes of the workload and keep
+    the rest; without them the workload is the full configuration."""
+    import argparse
+    import workloads
+    full = bench.bench_spec(argparse.Namespace(workload="lm", batch=0, seqlen=0))
+    assert full == workloads.spec("lm")
+    short = bench.bench_spec(argparse.Namespace(workload="complex", batch=1, seqlen=0))
+    assert (short.batch, short.seqlen, short.heads, short.N) == (1, 8192, 64, 128)
+    short = bench.bench_spec(argparse.Namespace(workload="lm", batch=0, seqlen=1024))
+    assert (short.batch, short.seqlen, short.heads) == (8, 1024, 32)
+
+
+def test_backward_bytes_cover_complex_gradients():
+    """A complex state's dd is complex: 8 bytes an entry instead of 4."""
+    import workloads
+    sp = workloads.spec("complex")
+    # s, bf16 logits, complex d, bf16 B, C, x, complex dy read; complex dd, fp32 dB, dC, dx, dlogits written
+    reads = 4 + sp.K * 2 + sp.N * 8 + 2 * sp.N * 2 + sp.P * 2 + sp.P * 8
+    assert bench.bwd_bytes_per_token_head(sp) == reads + sp.N * 8 + (2 * sp.N + sp.P + sp.K) * 4
+    assert bench.bwd_bytes_per_token_head(workloads.spec("lm")) == 1764
